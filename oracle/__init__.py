@@ -1,0 +1,135 @@
+"""ctypes wrapper of the fp64 CPU oracle (oracle.cpp).
+
+TEST INFRASTRUCTURE: only tests/, the smoke check and bench.py's CPU-baseline and
+reference legs use it. The CUDA path never imports it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle_tg.so")
+_lib = None
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+I64 = ctypes.c_int64
+F32 = ctypes.c_float
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared",
+                               _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        L.oracle_gate_score.argtypes = [P, ctypes.c_int, I64, ctypes.c_int, P, P, P, F32,
+                                        ctypes.c_int, P, P]
+        L.oracle_gate_score.restype = None
+        L.oracle_select_topk.argtypes = [P, P, P, P, P, ctypes.c_int, P, P]
+        L.oracle_select_topk.restype = I64
+        L.oracle_gather_rows.argtypes = [P, I64, P, I64, P]
+        L.oracle_gather_rows.restype = None
+        L.oracle_gated_attention.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, P, I64, P]
+        L.oracle_gated_attention.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a) -> int:
+    return a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr()
+
+
+def _raw(t: torch.Tensor):
+    """(contiguous CPU tensor, dtype code): f32 -> 0, bf16 -> 1 (bits read as-is)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t, 0
+    if t.dtype == torch.bfloat16:
+        return t, 1
+    raise TypeError(f"oracle: unsupported dtype {t.dtype}")
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _f32(a) -> np.ndarray:
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().float().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def gate_score(x: torch.Tensor, w1: torch.Tensor, b1, w2, b2: float):
+    """s_i = b2 + w2 . GELU(W1 x_i + b1); returns (fp64 scores, fp32 rounding)."""
+    xr, dt = _raw(x)
+    w1r, dt2 = _raw(w1)
+    assert dt == dt2
+    n, d = xr.shape
+    h = w1r.shape[0]
+    assert w1r.shape[1] == d
+    b1a, w2a = _f32(b1), _f32(w2)
+    s64 = np.empty(n, np.float64)
+    s32 = np.empty(n, np.float32)
+    lib().oracle_gate_score(_ptr(xr), dt, n, d, _ptr(w1r), _ptr(b1a), _ptr(w2a), float(b2), h,
+                            _ptr(s64), _ptr(s32))
+    return s64, s32
+
+
+def select_topk(scores, cu_seqlens, doc_begin, doc_end, k_doc):
+    """Returns (kept global row ids, ascending; cu_kept[B+1])."""
+    s = _f32(scores)
+    cu = _i32(cu_seqlens)
+    db, de, kd = _i32(doc_begin), _i32(doc_end), _i32(k_doc)
+    B = len(db)
+    out = np.empty(int(cu[-1]), np.int32)
+    cuk = np.empty(B + 1, np.int32)
+    n = lib().oracle_select_topk(_ptr(s), _ptr(cu), _ptr(db), _ptr(de), _ptr(kd), B, _ptr(out),
+                                 _ptr(cuk))
+    if n < 0:
+        raise ValueError("oracle_select_topk: bad span")
+    return out[:n].copy(), cuk
+
+
+def gather_rows(src: np.ndarray, kept_idx) -> np.ndarray:
+    src = np.ascontiguousarray(src)
+    idx = _i32(kept_idx)
+    row_bytes = src.strides[0]
+    dst = np.empty((len(idx),) + src.shape[1:], src.dtype)
+    lib().oracle_gather_rows(_ptr(src), row_bytes, _ptr(idx), len(idx), _ptr(dst))
+    return dst
+
+
+def gated_attention(q, k, v, s_kept, gain, tau, cu_kept, rows=None) -> np.ndarray:
+    """O [K, hq, dh] fp64 (rows not in `rows` are left as NaN)."""
+    qr, dt = _raw(q)
+    kr, _ = _raw(k)
+    vr, _ = _raw(v)
+    K, hq, dh = qr.shape
+    hkv = kr.shape[1]
+    s, g, t = _f32(s_kept), _f32(gain), _f32(tau)
+    cu = _i32(cu_kept)
+    out = np.full((K, hq, dh), np.nan, np.float64)
+    if rows is None:
+        rp, nr = None, 0
+    else:
+        ra = _i32(rows)
+        rp, nr = _ptr(ra), len(ra)
+    lib().oracle_gated_attention(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(s), _ptr(g), _ptr(t),
+                                 _ptr(cu), len(cu) - 1, hq, hkv, dh, rp, nr, _ptr(out))
+    return out

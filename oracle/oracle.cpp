@@ -1,0 +1,196 @@
+// TokenGate gated-prefill path: plain fp64 CPU oracle.
+//
+// TEST INFRASTRUCTURE. Only the tests, the smoke check and the bench's CPU
+// baseline leg load this library. It shares no code with the CUDA path: no
+// header, helper, table or constant comes from there, and the CUDA path never
+// calls it.
+//
+// Sources: "TokenGate: l'attention gérée par des tokens ..." (MarkTechPost, French
+// translation), sections "Comment TokenGate a-t-il appris le fonctionnement de la
+// réduction des tokens ?" (the three-phase forward pass: gate MLP on the
+// post-attention residual at layer L, top-K selector, layers above L see only the
+// K kept tokens; only the document may be dropped, never the question),
+// "Qu'est-ce que l'attention gérée par des tokens ?" (each kept token's score is
+// a bias on the attention logits, with a learnable per-head gain and a learnable
+// per-head temperature) and "Comment déployer TokenGate ?" (the {state}
+// placeholder marks the droppable document; the budget max_kept_prefill_tokens).
+//
+// Every function is the plain definition of its step, written out as loops in
+// double precision. Readings where the pages are silent:
+//   * gate MLP = two layers d -> h -> 1 with biases and exact (erf) GELU;
+//   * the score is the raw MLP output, used both for ranking and as the bias;
+//   * the temperature divides the q.k term only: z = q.k / (sqrt(dh) tau) + g s;
+//   * ties go to the lower position, -0 equals +0, NaN ranks below -inf;
+//   * every token outside [doc_begin, doc_end) is kept;
+//   * query head hq reads KV head hq / (Hq / Hkv);
+//   * key j is visible to query i iff j <= i in the (position-ordered) kept list.
+// Parity status: gate, select, gather and attention are each pinned by tests
+// (closed forms, brute force, library witnesses, invariants); see tests/.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+// exact widening of the two input storage types
+double load_elem(const void* p, int dtype, int64_t i) {
+  if (dtype == 0) return (double)((const float*)p)[i];
+  uint32_t u = ((uint32_t)((const uint16_t*)p)[i]) << 16;  // bf16 = top half of an f32
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+double gelu(double u) { return 0.5 * u * (1.0 + std::erf(u / std::sqrt(2.0))); }
+
+// total order used by the selector: larger is better; NaN is the worst value and
+// -0 is the same value as +0.
+struct ScoreKey {
+  bool nan;
+  double v;
+};
+ScoreKey score_key(float f) {
+  ScoreKey k;
+  k.nan = std::isnan(f);
+  k.v = k.nan ? 0.0 : (f == 0.0f ? 0.0 : (double)f);
+  return k;
+}
+bool ranks_higher(const ScoreKey& a, const ScoreKey& b) {  // strictly better
+  if (a.nan != b.nan) return b.nan;
+  if (a.nan) return false;
+  return a.v > b.v;
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_version() { return 1; }
+
+// Gate MLP scorer (section "Comment TokenGate a-t-il appris ...": a small MLP
+// scores every token from its residual at layer L):
+//   s_i = b2 + sum_k w2[k] * GELU(b1[k] + sum_c x[i,c] * w1[k,c])
+// x [n, d] and w1 [h, d] (out x in) in `dtype` (0 = f32, 1 = bf16 bits), b1, w2
+// f32, b2 f32. Writes the fp64 value and its fp32 rounding.
+void oracle_gate_score(const void* x, int dtype, int64_t n, int d, const void* w1,
+                       const float* b1, const float* w2, float b2, int h, double* s64,
+                       float* s32) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    double s = (double)b2;
+    for (int k = 0; k < h; ++k) {
+      double u = (double)b1[k];
+      for (int c = 0; c < d; ++c)
+        u += load_elem(x, dtype, i * (int64_t)d + c) * load_elem(w1, dtype, (int64_t)k * d + c);
+      s += (double)w2[k] * gelu(u);
+    }
+    if (s64) s64[i] = s;
+    if (s32) s32[i] = (float)s;
+  }
+}
+
+// Top-K with question protection (sections "Comment TokenGate a-t-il appris ..."
+// and "Comment déployer TokenGate ?"): for sequence b with tokens
+// [cu_seqlens[b], cu_seqlens[b+1]) and droppable span [doc_begin[b], doc_end[b])
+// (local positions), keep the min(k_doc[b], span length) span tokens of highest
+// score (ties to the lower position) and every token outside the span. Writes the
+// kept tokens' global row ids in ascending order and cu_kept[b+1] = running
+// total. Returns the total kept, or -1 on a bad span.
+int64_t oracle_select_topk(const float* scores, const int32_t* cu_seqlens,
+                           const int32_t* doc_begin, const int32_t* doc_end,
+                           const int32_t* k_doc, int batch, int32_t* kept_idx,
+                           int32_t* cu_kept) {
+  int64_t out = 0;
+  if (cu_kept) cu_kept[0] = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int32_t base = cu_seqlens[b];
+    const int32_t len = cu_seqlens[b + 1] - base;
+    const int32_t db = doc_begin[b], de = doc_end[b];
+    if (db < 0 || de < db || de > len) return -1;
+    std::vector<int32_t> doc;
+    for (int32_t p = db; p < de; ++p) doc.push_back(p);
+    // best first; stable_sort keeps equal scores in ascending position order
+    std::stable_sort(doc.begin(), doc.end(), [&](int32_t a, int32_t c) {
+      return ranks_higher(score_key(scores[base + a]), score_key(scores[base + c]));
+    });
+    int64_t take = std::min<int64_t>(std::max<int32_t>(k_doc[b], 0), (int64_t)doc.size());
+    std::vector<char> keep(len, 1);
+    for (int32_t p = db; p < de; ++p) keep[p] = 0;
+    for (int64_t r = 0; r < take; ++r) keep[doc[r]] = 1;
+    for (int32_t p = 0; p < len; ++p)
+      if (keep[p]) {
+        if (kept_idx) kept_idx[out] = base + p;
+        ++out;
+      }
+    if (cu_kept) cu_kept[b + 1] = (int32_t)out;
+  }
+  return out;
+}
+
+// Stable compaction (section "Comment TokenGate a-t-il appris ...": layers above L
+// process only the K kept tokens): dst[r] = src[kept_idx[r]], row_bytes bytes per
+// row.
+void oracle_gather_rows(const void* src, int64_t row_bytes, const int32_t* kept_idx,
+                        int64_t n_kept, void* dst) {
+  for (int64_t r = 0; r < n_kept; ++r)
+    std::memcpy((char*)dst + r * row_bytes, (const char*)src + (int64_t)kept_idx[r] * row_bytes,
+                (size_t)row_bytes);
+}
+
+// Token-gated causal GQA attention over the kept tokens (section "Qu'est-ce que
+// l'attention gérée par des tokens ?"): for sequence b (kept rows
+// [cu_kept[b], cu_kept[b+1])), query head hq, kept query row i:
+//   z_j = (q_i . k_j) / (sqrt(dh) * tau[hq]) + gain[hq] * s_kept[j],  j <= i
+//   O_i = sum_j softmax_j(z) v_j
+// q [K, hq, dh], k/v [K, hkv, dh] in `dtype`; KV head = hq / (n_hq / n_hkv).
+// `rows` (n_rows global kept rows) restricts the computation to those query rows;
+// rows == nullptr computes all. out is [K, hq, dh] fp64; only computed rows are
+// written.
+void oracle_gated_attention(const void* q, const void* k, const void* v, int dtype,
+                            const float* s_kept, const float* gain, const float* tau,
+                            const int32_t* cu_kept, int batch, int n_hq, int n_hkv, int dh,
+                            const int32_t* rows, int64_t n_rows, double* out) {
+  const int64_t total = cu_kept[batch];
+  std::vector<int32_t> all;
+  if (!rows) {
+    for (int64_t r = 0; r < total; ++r) all.push_back((int32_t)r);
+    rows = all.data();
+    n_rows = total;
+  }
+  const int group = n_hq / n_hkv;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+  for (int64_t t = 0; t < n_rows; ++t) {
+    for (int hq = 0; hq < n_hq; ++hq) {
+      const int64_t i = rows[t];
+      int b = 0;
+      while (cu_kept[b + 1] <= i) ++b;
+      const int64_t j0 = cu_kept[b];
+      const int kv = hq / group;
+      const double scale = 1.0 / (std::sqrt((double)dh) * (double)tau[hq]);
+      std::vector<double> z(i - j0 + 1);
+      double zmax = -INFINITY;
+      for (int64_t j = j0; j <= i; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < dh; ++c)
+          dot += load_elem(q, dtype, (i * n_hq + hq) * (int64_t)dh + c) *
+                 load_elem(k, dtype, (j * n_hkv + kv) * (int64_t)dh + c);
+        double zj = dot * scale + (double)gain[hq] * (double)s_kept[j];
+        z[j - j0] = zj;
+        zmax = std::max(zmax, zj);
+      }
+      double denom = 0.0;
+      std::vector<double> acc(dh, 0.0);
+      for (int64_t j = j0; j <= i; ++j) {
+        double w = std::exp(z[j - j0] - zmax);
+        denom += w;
+        for (int c = 0; c < dh; ++c) acc[c] += w * load_elem(v, dtype, (j * n_hkv + kv) * (int64_t)dh + c);
+      }
+      for (int c = 0; c < dh; ++c) out[(i * n_hq + hq) * (int64_t)dh + c] = acc[c] / denom;
+    }
+  }
+}
+
+}  // extern "C"
