@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Gated-prefill benchmark: one gated layer (gate MLP -> question-protected top-K
+-> compaction -> token-gated causal GQA attention) on synthetic inputs shaped like
+the Qwen3-1.7B layer of the TokenGate pages (16k tokens, d=2048, 16/8 heads,
+dh=128, keep 10% of the document).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen16k]
+
+Prints ONE JSON line (rank 0). Multi-GPU runs (torchrun) are independent
+replicas: every rank runs the whole layer on its own copy (no data-path
+collective); the timed region is bracketed by barriers and the slowest rank's
+time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "gated-prefill tokens/s (gate+top-K+attn) at 16k-128k; % of bf16 TC / HBM peak"
+L2_FLUSH_BYTES = 512 << 20      # > 126 MB L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), ws
+    return None, 0, 1
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def _max_over_ranks(dist, v: float) -> float:
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _work(wl):
+    """Algorithmic work of one step (bytes / flops the method must move / do)."""
+    N, d, h, dh, hq = wl.n_tokens, wl.d, wl.h, wl.dh, wl.hq
+    esz = 2 if wl.dtype == "bf16" else 4
+    Ks = wl.kept_counts
+    K = sum(Ks)
+    return {
+        "gate_bytes": esz * N * d + esz * d * h + 4 * N,
+        "gate_flops": 2 * N * d * h,
+        "select_bytes": 4 * N + 8 * K,
+        "compact_bytes": 2 * K * d * esz,
+        "attn_flops": sum(4 * dh * hq * k * (k + 1) // 2 for k in Ks),
+    }
+
+
+def _oracle_sample_time(wl, oracle, n_gate=4096, n_attn_rows=128):
+    """Oracle time for one whole step, extrapolated from a bounded sample: gate on
+    n_gate rows (scaled by N), select and gather in full, attention on n_attn_rows
+    query rows per sequence (scaled by the causal pair count)."""
+    rng = np.random.default_rng(0)
+    N = wl.n_tokens
+    rows = np.sort(rng.choice(N, min(n_gate, N), replace=False))
+    t0 = time.perf_counter()
+    s64, s32 = oracle.gate_score(wl.x[torch.from_numpy(rows)], wl.w1, wl.b1, wl.w2, wl.b2)
+    t_gate = (time.perf_counter() - t0) * N / len(rows)
+    scores = np.zeros(N, np.float32)
+    scores[rows] = s32
+    sel = wl.score_override.numpy() if wl.score_override is not None else scores
+    t0 = time.perf_counter()
+    idx, cu = oracle.select_topk(sel, wl.cu_seqlens, wl.doc_begin, wl.doc_end, wl.k_doc)
+    t_sel = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.gather_rows(wl.x.view(torch.int16).numpy(), idx)
+    t_gather = time.perf_counter() - t0
+    # attention sample: rows spread over each sequence; cost ~ (row index + 1)
+    arows, pairs_sample = [], 0
+    for b in range(wl.batch):
+        a, e = int(cu[b]), int(cu[b + 1])
+        if e <= a:
+            continue
+        r = np.unique(np.linspace(a, e - 1, min(n_attn_rows, e - a)).astype(np.int32))
+        arows.append(r)
+        pairs_sample += int(np.sum(r - a + 1))
+    arows = np.concatenate(arows)
+    pairs_full = sum(k * (k + 1) // 2 for k in wl.kept_counts)
+    t0 = time.perf_counter()
+    oracle.gated_attention(wl.q, wl.k, wl.v, sel[idx], wl.gain, wl.tau, cu, rows=arows)
+    t_attn = (time.perf_counter() - t0) * pairs_full / max(pairs_sample, 1)
+    total = t_gate + t_sel + t_gather + t_attn
+    sample = (f"oracle fp64 on host cores: gate on {len(rows)} of {N} rows (x{N / len(rows):.0f}), "
+              f"select+gather in full, attention on {len(arows)} query rows x {wl.hq} heads "
+              f"(scaled by causal pairs x{pairs_full / max(pairs_sample, 1):.0f})")
+    return total, {"gate": t_gate, "select": t_sel, "compact": t_gather, "attention": t_attn}, sample
+
+
+def _threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
+
+
+def run_reference(args, dist, rank, ws):
+    """The oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    from learned_token_pruning_gemm_b200 import synth
+    oracle.build()
+    wl = synth.WORKLOADS[args.workload]()
+    for _ in range(args.warmup):
+        _oracle_sample_time(wl, oracle, n_gate=64, n_attn_rows=4)
+    times = []
+    sample = ""
+    for _ in range(args.steps):
+        t, _, sample = _oracle_sample_time(wl, oracle)
+        times.append(t)
+    ms = 1e3 * statistics.mean(times)
+    value = wl.n_tokens / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": wl.n_tokens, "kept": wl.total_kept},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, dist, rank, ws):
+    from learned_token_pruning_gemm_b200 import api, pipeline, synth
+    dev_index = torch.cuda.current_device()
+    wl = synth.WORKLOADS[args.workload]()
+    gp = pipeline.GatedPrefill(wl)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    work = _work(wl)
+    peaks, peak_src = _peaks()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        gp.step(stream)
+    torch.cuda.synchronize()
+    assert api.device_status(reset=True) == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev_index)
+    clocks.start()
+    _barrier(dist)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()                     # L2 flush between timed steps (outside the events)
+        gp.step(stream, events=evs[i])
+    torch.cuda.synchronize()
+    _barrier(dist)
+    clk = clocks.stop()
+    status = api.device_status(reset=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} during the timed region")
+
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                for j, name in enumerate(gp.STAGES)}
+    ms = _max_over_ranks(dist, statistics.mean(step_ms))
+    value = ws * wl.n_tokens / (ms / 1e3)
+
+    # dominant kernel and its roofline
+    dom = max(stage_ms, key=stage_ms.get)
+    t = stage_ms[dom] / 1e3
+    tf_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    if dom == "attention":
+        ach, peak, unit, bound = work["attn_flops"] / t / 1e12, tf_peak, "TFLOP/s", "tensor"
+    elif dom == "gate":
+        # at the ridge: report against the binding floor (the larger one)
+        if work["gate_flops"] / (tf_peak * 1e12) >= work["gate_bytes"] / (hbm_peak * 1e9):
+            ach, peak, unit, bound = work["gate_flops"] / t / 1e12, tf_peak, "TFLOP/s", "tensor"
+        else:
+            ach, peak, unit, bound = work["gate_bytes"] / t / 1e9, hbm_peak, "GB/s", "hbm"
+    elif dom == "compact":
+        ach, peak, unit, bound = work["compact_bytes"] / t / 1e9, hbm_peak, "GB/s", "hbm"
+    else:
+        ach, peak, unit, bound = work["select_bytes"] / t / 1e9, hbm_peak, "GB/s", "hbm"
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if os.path.exists(tpath):
+        tr = json.load(open(tpath))
+        ent = tr.get(args.workload, {}).get(dom)
+        if ent and ent.get("kernel_rev") == _kernel_rev():
+            traffic = ent["bytes_per_launch"]
+    roofline = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                "frac": ach / peak, "traffic": traffic, "peak_source": peak_src}
+    stages = {
+        "gate": {"us": stage_ms["gate"] * 1e3,
+                 "tflops": work["gate_flops"] / (stage_ms["gate"] / 1e3) / 1e12,
+                 "gbs": work["gate_bytes"] / (stage_ms["gate"] / 1e3) / 1e9},
+        "select": {"us": stage_ms["select"] * 1e3,
+                   "gbs": work["select_bytes"] / (stage_ms["select"] / 1e3) / 1e9},
+        "compact": {"us": stage_ms["compact"] * 1e3,
+                    "gbs": work["compact_bytes"] / (stage_ms["compact"] / 1e3) / 1e9},
+        "attention": {"us": stage_ms["attention"] * 1e3,
+                      "tflops": work["attn_flops"] / (stage_ms["attention"] / 1e3) / 1e12},
+    }
+    for s in stages.values():
+        if "tflops" in s:
+            s["frac_tc"] = s["tflops"] / tf_peak
+        if "gbs" in s:
+            s["frac_hbm"] = s["gbs"] / hbm_peak
+    sc_bytes = work["select_bytes"] + work["compact_bytes"]
+    stages["select+compact"] = {
+        "us": (stage_ms["select"] + stage_ms["compact"]) * 1e3,
+        "frac_hbm": sc_bytes / ((stage_ms["select"] + stage_ms["compact"]) / 1e3) / 1e9 / hbm_peak}
+
+    # ---- e2e: host buffers in, result out, through the same public calls ----
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.pin_memory() for t in (wl.x, wl.q, wl.k, wl.v)]
+        dev_in = [gp.x, gp.q, gp.k, gp.v]
+        host_out = torch.empty(gp.out.shape, dtype=gp.out.dtype).pin_memory()
+        host_idx = torch.empty(gp.kept_idx.shape, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = host_out.numel() * host_out.element_size() + host_idx.numel() * 4
+
+        def e2e_step():
+            for hsrc, dst in zip(host_in, dev_in):
+                dst.copy_(hsrc, non_blocking=True)
+            gp.step(stream)
+            host_out.copy_(gp.out, non_blocking=True)
+            host_idx.copy_(gp.kept_idx, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        _barrier(dist)
+        for a, b in e_ev:
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        _barrier(dist)
+        e_ms = _max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in e_ev))
+        e2e = {"value": ws * wl.n_tokens / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        t_cpu, parts, sample = _oracle_sample_time(wl, oracle)
+        cpu = {"value": wl.n_tokens / t_cpu, "unit": "tokens/s", "cores": _threads(),
+               "kind": "oracle", "sample": sample,
+               "stage_s": {k: round(v, 4) for k, v in parts.items()}}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "tokens": wl.n_tokens,
+                       "kept": wl.total_kept, "d": wl.d, "gate_hidden": wl.h,
+                       "heads": f"{wl.hq}/{wl.hkv}", "head_dim": wl.dh,
+                       "l2": "flushed between timed steps (512 MB write)",
+                       "parallelism": f"replicas x{ws}"},
+            "stages": stages,
+            "roofline": roofline,
+            "gpu_launches": gp.LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def _kernel_rev() -> str:
+    """Hash of the kernel sources, so stale DRAM-traffic figures are not reported."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "learned_token_pruning_gemm_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen16k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    dist, rank, ws = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist, rank, ws)
+        else:
+            run_ours(args, dist, rank, ws)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * tg.h -- C ABI of the TokenGate gated-prefill path on B200 (sm_100a).
+ *
+ * The path (MarkTechPost page on TokenGate, French translation, section "Comment
+ * TokenGate a-t-il appris le fonctionnement de la réduction des tokens ?"): a small
+ * gate MLP scores every token from its post-attention residual at the gate layer
+ * L; a top-K selector keeps the best-scoring tokens of the droppable document
+ * while the question is always kept; layers above L see only the K kept tokens
+ * and write KV only for them; their attention adds each kept key's score to the
+ * logits through a per-head gain and scales the logits by a per-head temperature
+ * (section "Qu'est-ce que l'attention gérée par des tokens ?").
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless its comment says "host".
+ *     The caller owns every buffer; the library allocates no device memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronises the host, except tg_device_status().
+ *   - Every call returns a tg_status; no exception crosses the ABI. Argument
+ *     errors are detected on the host before any launch. Errors found on the
+ *     device (a bounded wait that ran out, an inconsistent size) are recorded in a
+ *     per-device status word read by tg_device_status(); the kernel then skips the
+ *     remaining work instead of trapping.
+ *   - Rows are token-major and dense: a [rows, cols] array has row stride cols.
+ *   - Ragged batches use cumulative offsets: sequence b owns rows
+ *     [cu[b], cu[b+1]) of a packed array; cu has batch+1 entries, cu[0] = 0.
+ *   - bf16 is IEEE binary32 truncated to its top 16 bits (round to nearest even
+ *     on output).
+ */
+#ifndef TOKENGATE_TG_H_
+#define TOKENGATE_TG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TG_OK = 0,
+  TG_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad span, K mismatch */
+  TG_ERR_UNSUPPORTED = 2,   /* shape outside the kernels' supported set */
+  TG_ERR_MISALIGNED = 3,    /* pointer or row size not 16-byte aligned */
+  TG_ERR_WORKSPACE = 4,     /* caller-provided scratch too small */
+  TG_ERR_CUDA = 5,          /* a CUDA runtime call failed (launch, attribute) */
+  TG_ERR_TIMEOUT = 6,       /* device: a bounded wait ran out (see tg_device_status) */
+  TG_ERR_DEVICE_CHECK = 7   /* device: a size or index check failed, work skipped */
+} tg_status;
+
+typedef enum { TG_F32 = 0, TG_BF16 = 1 } tg_dtype;
+
+typedef struct CUstream_st* tg_stream_t; /* same type as cudaStream_t */
+
+/* Version of this ABI (bumped on any signature change). */
+int tg_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* tg_status_string(tg_status s);
+
+/*
+ * Gate MLP scorer (MarkTechPost page, "Comment TokenGate a-t-il appris ...": an
+ * MLP scores each token from its residual at layer L). For every token i:
+ *     s[i] = b2 + sum_k w2[k] * GELU(b1[k] + sum_c x[i,c] * w1[k,c]),
+ * GELU(u) = u * Phi(u) (exact erf form).
+ *   x       [n_tokens, d]   dtype         residual stream at the gate layer
+ *   w1      [h, d]          dtype         first layer, nn.Linear layout (out x in)
+ *   b1, w2  [h]             f32
+ *   b2                      f32 scalar, by value
+ *   scores  [n_tokens]      f32 output
+ * TG_BF16 (tensor-core path): d % 64 == 0, h in {64, 128, 256}, x and w1 16-byte
+ * aligned. TG_F32 (exact fp32 path, for small checks): 1 <= h <= 1024, d >= 1.
+ * n_tokens == 0 is a no-op.
+ */
+tg_status tg_gate_score(const void* x, tg_dtype dtype, int64_t n_tokens, int d, const void* w1,
+                        const float* b1, const float* w2, float b2, int h, float* scores,
+                        tg_stream_t stream);
+
+/*
+ * Top-K selection with question protection (MarkTechPost page, "Comment TokenGate
+ * a-t-il appris ...": a top-K selector keeps the best-scoring tokens; only the
+ * document part of the prompt can be dropped, never the question; "Comment
+ * déployer TokenGate ?": a {state} placeholder marks the droppable document and
+ * max_kept_prefill_tokens is the budget).
+ * For each sequence b (rows [cu_seqlens[b], cu_seqlens[b+1]) of `scores`), with
+ * droppable span [doc_begin[b], doc_end[b]) in positions local to the sequence:
+ * keep the min(k_doc[b], span length) span tokens of highest score and every
+ * token outside the span. Ties go to the lower position; -0 equals +0; NaN ranks
+ * below -inf; k_doc < 0 counts as 0.
+ *   scores      [total_tokens]  f32
+ *   cu_seqlens  [batch+1]       int32   (device)
+ *   doc_begin, doc_end, k_doc [batch] int32 (device)
+ *   kept_idx    [total_kept]    int32 output: kept rows' global row ids
+ *                                       (indices into `scores`), ascending
+ *   kept_scores [total_kept]    f32 output, may be NULL: scores[kept_idx[r]]
+ *   cu_kept     [batch+1]       int32 output: cumulative kept counts
+ * total_kept must equal sum_b (len_b - span_b + min(max(k_doc_b,0), span_b)); the
+ * caller knows every term, so no device-to-host read is needed to size outputs.
+ * max_seqlen bounds every len_b; max_seqlen <= TG_SELECT_MAX_SEQLEN. A span
+ * outside its sequence or a total that differs from total_kept is found on the
+ * device: the sequence's outputs are skipped and TG_ERR_DEVICE_CHECK recorded.
+ */
+#define TG_SELECT_MAX_SEQLEN 196608
+tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* doc_begin,
+                         const int32_t* doc_end, const int32_t* k_doc, int batch,
+                         int64_t total_tokens, int64_t total_kept, int max_seqlen,
+                         int32_t* kept_idx, float* kept_scores, int32_t* cu_kept,
+                         tg_stream_t stream);
+
+/*
+ * Stable compaction (MarkTechPost page, "Comment TokenGate a-t-il appris ...":
+ * layers above L process only the K kept tokens and never create KV entries for
+ * the dropped ones). For t < n_tensors and r < n_kept:
+ *     dst[t] row r  =  src[t] row kept_idx[r]      (row_bytes[t] bytes per row)
+ *   src, dst    host arrays of n_tensors device pointers (1 <= n_tensors <= 8)
+ *   row_bytes   host array of n_tensors sizes; each a positive multiple of 16
+ *   kept_idx    [n_kept] int32 device, row ids into every src (from tg_select_topk)
+ * Every src/dst pointer must be 16-byte aligned. The caller guarantees that
+ * kept_idx entries are valid rows of every src.
+ */
+tg_status tg_compact_kv(const void* const* src, void* const* dst, const int64_t* row_bytes,
+                        int n_tensors, const int32_t* kept_idx, int64_t n_kept,
+                        tg_stream_t stream);
+
+/*
+ * Token-gated causal GQA attention over the kept tokens (MarkTechPost page,
+ * "Qu'est-ce que l'attention gérée par des tokens ?": each kept token's score is
+ * a bias on the attention logits with a learnable per-head gain; a learnable
+ * per-head temperature corrects for each query seeing fewer keys). For sequence
+ * b (kept rows [cu_kept[b], cu_kept[b+1])), query head hq, kept row i:
+ *     z_j = (q_i . k_j) / (sqrt(head_dim) * tau[hq]) + gain[hq] * s_kept[j],  j <= i
+ *     out_i = sum_j softmax_j(z) * v_j
+ * with KV head hq / (n_hq / n_hkv). Key j is visible to query i iff j <= i in the
+ * position-ordered kept list (the original causal order).
+ *   q    [total_kept, n_hq,  head_dim]  dtype
+ *   k, v [total_kept, n_hkv, head_dim]  dtype
+ *   s_kept [total_kept] f32 (from tg_select_topk), gain, tau [n_hq] f32
+ *   cu_kept [batch+1] int32 device; max_kept >= every cu_kept[b+1]-cu_kept[b]
+ *   out  [total_kept, n_hq, head_dim]  dtype output
+ * TG_BF16 (tensor-core path): head_dim == 128, n_hq % n_hkv == 0, q/k/v/out
+ * 16-byte aligned. TG_F32 (exact fp32 path): head_dim <= 256.
+ */
+tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
+                             const float* s_kept, const float* gain, const float* tau,
+                             const int32_t* cu_kept, int batch, int64_t total_kept, int max_kept,
+                             int n_hq, int n_hkv, int head_dim, void* out, tg_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the first error any kernel recorded on the
+ * current device since the last reset (TG_OK if none). reset != 0 clears it.
+ */
+tg_status tg_device_status(tg_stream_t stream, int reset);
+
+/*
+ * Failure-detection self test: launches one kernel that waits, with the same
+ * bounded wait the other kernels use, on a device flag that nothing sets. After
+ * timeout_ns nanoseconds the wait gives up and records TG_ERR_TIMEOUT in the
+ * status word (read it with tg_device_status). 1000 <= timeout_ns <= 1e10.
+ */
+tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_TG_H_ */

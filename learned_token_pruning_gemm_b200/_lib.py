@@ -1,0 +1,60 @@
+"""ctypes loader for libtokengate.so (the C ABI declared in include/tg.h).
+
+There is no fallback: if the shared library is missing or fails to load, every
+call raises. Build it with `python -m learned_token_pruning_gemm_b200.build`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtokengate.so")
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+I64 = ctypes.c_int64
+F32 = ctypes.c_float
+INT = ctypes.c_int
+
+# (name, restype, argtypes) for every symbol the header declares
+SIGNATURES = {
+    "tg_abi_version": (INT, []),
+    "tg_status_string": (ctypes.c_char_p, [INT]),
+    "tg_gate_score": (INT, [P, INT, I64, INT, P, P, P, F32, INT, P, P]),
+    "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P]),
+    "tg_compact_kv": (INT, [P, P, P, INT, P, I64, P]),
+    "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P]),
+    "tg_device_status": (INT, [P, INT]),
+    "tg_selftest_bounded_wait": (INT, [I64, P]),
+}
+
+_lib = None
+
+
+class TokenGateError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH):
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise TokenGateError(
+                f"{path} not found: build the CUDA library first "
+                "(python -m learned_token_pruning_gemm_b200.build)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        lib.tg_internal_set_attn_variant.restype = None
+        lib.tg_internal_set_attn_variant.argtypes = [INT]
+        _lib = lib
+    return _lib
+
+
+def check(status: int, what: str) -> None:
+    if status != 0:
+        name = load().tg_status_string(status).decode()
+        raise TokenGateError(f"{what} failed: {name} ({status})")

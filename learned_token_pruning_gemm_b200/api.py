@@ -1,0 +1,136 @@
+"""Python binding of the C ABI: argument marshalling over torch CUDA tensors.
+
+Every function here checks shapes/dtypes, passes raw device pointers and the
+current torch stream to libtokengate.so, and raises TokenGateError on a non-OK
+status. All arithmetic happens in the CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import TokenGateError, check
+
+TG_F32, TG_BF16 = 0, 1
+_DT = {torch.float32: TG_F32, torch.bfloat16: TG_BF16}
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TokenGateError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise TokenGateError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TokenGateError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def abi_version() -> int:
+    return _lib.load().tg_abi_version()
+
+
+def gate_score(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: float,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """s = b2 + w2 . GELU(W1 x + b1) per token. x [N, d], w1 [h, d] (same dtype)."""
+    n, d = x.shape
+    h = w1.shape[0]
+    if w1.shape != (h, d) or w1.dtype != x.dtype or x.dtype not in _DT:
+        raise TokenGateError("gate_score: x [N,d] and w1 [h,d] must share a dtype (f32/bf16)")
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=x.device)
+    st = _lib.load().tg_gate_score(_cuda(x, "x"), _DT[x.dtype], n, d, _cuda(w1, "w1"),
+                                   _cuda(b1, "b1", torch.float32), _cuda(w2, "w2", torch.float32),
+                                   float(b2), h, _cuda(out, "scores", torch.float32), _stream(stream))
+    check(st, "tg_gate_score")
+    return out
+
+
+def select_topk(scores: torch.Tensor, cu_seqlens: torch.Tensor, doc_begin: torch.Tensor,
+                doc_end: torch.Tensor, k_doc: torch.Tensor, total_kept: int, max_seqlen: int,
+                kept_idx: Optional[torch.Tensor] = None, kept_scores: Optional[torch.Tensor] = None,
+                cu_kept: Optional[torch.Tensor] = None, want_scores: bool = True, stream=None):
+    """Returns (kept_idx int32 [total_kept], kept_scores f32 [total_kept] or None,
+    cu_kept int32 [B+1])."""
+    B = doc_begin.numel()
+    dev = scores.device
+    if kept_idx is None:
+        kept_idx = torch.empty(total_kept, dtype=torch.int32, device=dev)
+    if kept_scores is None and want_scores:
+        kept_scores = torch.empty(total_kept, dtype=torch.float32, device=dev)
+    if cu_kept is None:
+        cu_kept = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    st = _lib.load().tg_select_topk(
+        _cuda(scores, "scores", torch.float32), _cuda(cu_seqlens, "cu_seqlens", torch.int32),
+        _cuda(doc_begin, "doc_begin", torch.int32), _cuda(doc_end, "doc_end", torch.int32),
+        _cuda(k_doc, "k_doc", torch.int32), B, scores.numel(), int(total_kept), int(max_seqlen),
+        _cuda(kept_idx, "kept_idx", torch.int32),
+        _cuda(kept_scores, "kept_scores", torch.float32) if kept_scores is not None else None,
+        _cuda(cu_kept, "cu_kept", torch.int32), _stream(stream))
+    check(st, "tg_select_topk")
+    return kept_idx, kept_scores, cu_kept
+
+
+def compact_rows(srcs: Sequence[torch.Tensor], kept_idx: torch.Tensor,
+                 outs: Optional[Sequence[torch.Tensor]] = None, stream=None):
+    """dst[t][r] = src[t][kept_idx[r]] for every tensor (rows = first dim)."""
+    n = kept_idx.numel()
+    if outs is None:
+        outs = [torch.empty((n,) + tuple(s.shape[1:]), dtype=s.dtype, device=s.device) for s in srcs]
+    k = len(srcs)
+    src_arr = (ctypes.c_void_p * k)(*[_cuda(s, "src") for s in srcs])
+    dst_arr = (ctypes.c_void_p * k)(*[_cuda(o, "dst") for o in outs])
+    rb = (ctypes.c_int64 * k)(*[math.prod(s.shape[1:]) * s.element_size() for s in srcs])
+    for s, o in zip(srcs, outs):
+        if o.shape[1:] != s.shape[1:] or o.dtype != s.dtype or o.shape[0] != n:
+            raise TokenGateError("compact_rows: output shape/dtype mismatch")
+    st = _lib.load().tg_compact_kv(src_arr, dst_arr, rb, k, _cuda(kept_idx, "kept_idx", torch.int32),
+                                   n, _stream(stream))
+    check(st, "tg_compact_kv")
+    return list(outs)
+
+
+def gated_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s_kept: torch.Tensor,
+                    gain: torch.Tensor, tau: torch.Tensor, cu_kept: torch.Tensor, max_kept: int,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Token-gated causal GQA attention. q [K,Hq,dh], k/v [K,Hkv,dh] (same dtype)."""
+    K, hq, dh = q.shape
+    hkv = k.shape[1]
+    if k.shape != (K, hkv, dh) or v.shape != k.shape or not (q.dtype == k.dtype == v.dtype):
+        raise TokenGateError("gated_attention: q [K,Hq,dh], k/v [K,Hkv,dh] with one dtype")
+    if q.dtype not in _DT:
+        raise TokenGateError(f"gated_attention: unsupported dtype {q.dtype}")
+    if out is None:
+        out = torch.empty_like(q)
+    B = cu_kept.numel() - 1
+    st = _lib.load().tg_gated_attention(
+        _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _DT[q.dtype],
+        _cuda(s_kept, "s_kept", torch.float32), _cuda(gain, "gain", torch.float32),
+        _cuda(tau, "tau", torch.float32), _cuda(cu_kept, "cu_kept", torch.int32), B, K,
+        int(max_kept), hq, hkv, dh, _cuda(out, "out"), _stream(stream))
+    check(st, "tg_gated_attention")
+    return out
+
+
+def device_status(reset: bool = True, stream=None) -> int:
+    """Synchronise the stream and return (then clear) the device status word."""
+    return _lib.load().tg_device_status(_stream(stream), 1 if reset else 0)
+
+
+def selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
+    check(_lib.load().tg_selftest_bounded_wait(int(timeout_ns), _stream(stream)),
+          "tg_selftest_bounded_wait")
+
+
+def set_attention_variant(p_in_tmem: bool) -> None:
+    """Choose how P reaches the PV MMA in the bf16 attention kernel: through
+    shared memory (False, default) or through tensor memory (True)."""
+    _lib.load().tg_internal_set_attn_variant(1 if p_in_tmem else 0)

@@ -1,0 +1,460 @@
+// tg_gated_attention: token-gated causal GQA attention over the kept tokens
+// (MarkTechPost page on TokenGate, section "Qu'est-ce que l'attention gérée par
+// des tokens ?": each kept token's score is a bias on the attention logits,
+// scaled by a learnable per-head gain; a learnable per-head temperature corrects
+// for each query seeing fewer keys).
+//     z_ij = q_i . k_j / (sqrt(dh) tau_h) + g_h s_j,  j <= i;  O_i = softmax_j(z) V
+//
+// bf16 path (dh = 128), one CTA per (128-row query tile, query head, sequence):
+//   warp 0      TMA producer: the Q tile once, then K/V tiles of 128 keys through
+//               a 2-stage mbarrier ring; its 32 lanes also stage the per-key bias
+//               b_j = log2(e) g_h s_j for each tile in shared memory.
+//   warp 1      MMA issuer (one thread): S_{j+1} = Q K_{j+1}^T into one of two
+//               128-column TMEM buffers while the softmax works on S_j, then
+//               O += P_j V_j into a 128-column TMEM accumulator.
+//   warps 4-7   softmax, one query row per thread (TMEM lane = row): loads its row
+//               of S, forms z = S c_h + b_j in the log2 domain (one FFMA,
+//               c_h = log2(e) / (sqrt(dh) tau_h)), masks the diagonal tile, keeps a
+//               running max that is only moved when it grows by more than 2^8
+//               (then O is rescaled in TMEM), writes P in bf16 and its row sum.
+// P goes to the MMA through shared memory (128-byte swizzled, K-major) or through
+// TMEM in place of S (A operand in tensor memory), chosen at compile time.
+// Query tiles are launched longest-first (the last tile of a sequence has the
+// most keys under the causal mask).
+//
+// f32 path: exact fp32 SIMT kernel (one warp per query row and head).
+#include "common.cuh"
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kD = 128;
+constexpr int kStages = 2;
+constexpr int kThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
+
+struct AttnSmem {
+  uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves
+  uint8_t k[kStages][2][kBN * 64 * 2];
+  uint8_t v[kStages][2][kBN * 64 * 2];
+  uint8_t p[2][kBM * 64 * 2];               // P tile (bf16), when P goes through smem
+  float bias[kStages][kBN];
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full;
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// TMEM columns: S buffers at 0 and 128, O at 256 (512 allocated).
+constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
+
+template <bool kPinTmem>
+__global__ void __launch_bounds__(kThreads, 1)
+    gated_attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const float* __restrict__ s_kept, const float* __restrict__ gain,
+                           const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
+                           int n_hq, int n_hkv, __nv_bfloat16* __restrict__ out, int* status) {
+  const int hq = blockIdx.x;
+  const int b = blockIdx.y;
+  const int n_qt_max = gridDim.z;
+  const int t = n_qt_max - 1 - static_cast<int>(blockIdx.z);   // longest tiles first
+  const int seq0 = cu_kept[b];
+  const int len = cu_kept[b + 1] - seq0;
+  if (t * kBM >= len) return;   // uniform: this sequence has no tile t
+  const int kvh = hq / (n_hq / n_hkv);
+  const int nt = t + 1;         // causal: key tiles 0..t
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
+  AttnSmem& S = *reinterpret_cast<AttnSmem*>(smem_raw + pad);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    tg::mbar_init(&S.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tg::mbar_init(&S.kv_full[s], 1 + 32);   // expect_tx arrival + 32 bias lanes
+      tg::mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tg::mbar_init(&S.s_full[s], 1);
+      tg::mbar_init(&S.s_free[s], 128);
+    }
+    tg::mbar_init(&S.p_full, 128);
+    tg::mbar_init(&S.o_done, 1);
+    S.abort_flag = 0;
+    tg::fence_barrier_init();
+  }
+  if (warp == 2) {
+    tg::tmem_alloc(&S.tmem_base, kTmemCols);
+    tg::tmem_relinquish();
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  tg::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer + bias staging ----------------
+    const float gl2 = gain[hq] * kLog2e;
+    int issued = 0;
+    if (lane == 0) {
+      tg::mbar_arrive_expect_tx(&S.q_full, kBM * kD * 2);
+      tg::tma_load_3d(S.q[0], &tm_q, &S.q_full, 0, hq, seq0 + t * kBM);
+      tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
+    }
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % kStages;
+      bool go = true;
+      if (j >= kStages)
+        go = tg::mbar_wait(&S.kv_empty[s], ((j / kStages) - 1) & 1, status, &S.abort_flag);
+      go = __all_sync(0xFFFFFFFFu, go);
+      if (!go) break;
+      if (lane == 0) {
+        tg::mbar_arrive_expect_tx(&S.kv_full[s], 2 * kBN * kD * 2);
+        const int r0 = seq0 + j * kBN;
+        tg::tma_load_3d(S.k[s][0], &tm_k, &S.kv_full[s], 0, kvh, r0);
+        tg::tma_load_3d(S.k[s][1], &tm_k, &S.kv_full[s], 64, kvh, r0);
+        tg::tma_load_3d(S.v[s][0], &tm_v, &S.kv_full[s], 0, kvh, r0);
+        tg::tma_load_3d(S.v[s][1], &tm_v, &S.kv_full[s], 64, kvh, r0);
+      }
+      for (int c = lane; c < kBN; c += 32) {
+        const int kp = j * kBN + c;
+        S.bias[s][c] = kp < len ? gl2 * s_kept[seq0 + kp] : 0.f;
+      }
+      tg::mbar_arrive(&S.kv_full[s]);
+      ++issued;
+    }
+    if (lane == 0 && S.abort_flag) {
+      tg::mbar_wait(&S.q_full, 0, status, nullptr);
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        tg::mbar_wait(&S.kv_full[j % kStages], (j / kStages) & 1, status, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
+      const uint32_t q0 = tg::smem_u32(S.q[0]);
+      bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % kStages;
+        if (!tg::mbar_wait(&S.kv_full[s], (j / kStages) & 1, status, &S.abort_flag)) return false;
+        if (!kPinTmem && j >= 2 &&
+            !tg::mbar_wait(&S.s_free[j & 1], ((j >> 1) - 1) & 1, status, &S.abort_flag))
+          return false;
+        tg::tc_fence_after();
+        const uint32_t k0 = tg::smem_u32(S.k[s][0]);
+        const uint32_t d_s = tmem + kColS0 + 128u * (j & 1);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * (kBN * 64 * 2) + (kk & 3) * 32;
+          tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
+                          tg::smem_desc_sw128(k0 + offk, 16, 1024), idesc_s, kk != 0);
+        }
+        tg::mma_commit(&S.s_full[j & 1]);
+        return true;
+      };
+      if (alive) alive = issue_s(0);
+      for (int j = 0; j < nt && alive; ++j) {
+        if (j + 1 < nt && !issue_s(j + 1)) break;
+        if (!tg::mbar_wait(&S.p_full, j & 1, status, &S.abort_flag)) break;
+        tg::tc_fence_after();
+        const int s = j % kStages;
+        const uint32_t v0 = tg::smem_u32(S.v[s][0]);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // B = V rows 16kk..16kk+15 (MN-major: dh contiguous); the two 64-wide dh
+          // halves are 16 KB apart (LBO), 8-key groups 1024 B apart (SBO)
+          const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
+          if constexpr (kPinTmem) {
+            const uint32_t a_t = tmem + kColS0 + 128u * (j & 1) + kk * 8;
+            tg::mma_bf16_ts(tmem + kColO, a_t, bdesc, idesc_o, (j | kk) != 0);
+          } else {
+            const uint32_t p0 = tg::smem_u32(S.p[0]);
+            const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
+            tg::mma_bf16_ss(tmem + kColO, tg::smem_desc_sw128(p0 + off, 16, 1024), bdesc, idesc_o,
+                            (j | kk) != 0);
+          }
+        }
+        tg::mma_commit(&S.o_done);
+        tg::mma_commit(&S.kv_empty[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- softmax: one query row per thread ----------------
+    const int r = tid - 128;                       // row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool alive = true;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % kStages;
+      alive = tg::mbar_wait(&S.s_full[j & 1], (j >> 1) & 1, status, &S.abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
+      tg::tc_fence_after();
+      float z[kBN];
+      {
+        uint32_t u[32];
+#pragma unroll
+        for (int c = 0; c < kBN; c += 32) {
+          tg::tmem_ld32(tmem + lane_base + kColS0 + 128u * (j & 1) + c, u);
+          tg::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[c + e] = __uint_as_float(u[e]);
+        }
+      }
+      tg::tc_fence_before();
+      tg::mbar_arrive(&S.s_free[j & 1]);
+      // the bias of tile j is visible: kv_full[s] completed before S_j was issued
+      const float* bias = S.bias[s];
+      float mt = -INFINITY;
+      if (j == t) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          z[c] = c <= r ? fmaf(z[c], c_h, bias[c]) : -INFINITY;
+          mt = fmaxf(mt, z[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          z[c] = fmaf(z[c], c_h, bias[c]);
+          mt = fmaxf(mt, z[c]);
+        }
+      }
+      float m_use = m_run, alpha = 1.f;
+      bool rescale = false;
+      if (j == 0 || mt > m_run + kRescaleThreshold) {
+        m_use = fmaxf(m_run, mt);
+        if (j > 0) {
+          alpha = tg::exp2_approx(m_run - m_use);
+          rescale = true;
+        }
+      }
+      float lsum = 0.f;
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) {
+        const float p0 = tg::exp2_approx(z[c] - m_use);
+        const float p1 = tg::exp2_approx(z[c + 1] - m_use);
+        lsum += p0 + p1;
+        pk[c / 2] = tg::pack_bf16x2(p0, p1);
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_use;
+      // O and the P buffer are free once PV_{j-1} has completed
+      if (j > 0) {
+        alive = tg::mbar_wait(&S.o_done, (j - 1) & 1, status, &S.abort_flag);
+        if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
+        tg::tc_fence_after();
+      }
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < kD; c += 32) {
+          tg::tmem_ld32(tmem + lane_base + kColO + c, o);
+          tg::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tg::tmem_st16(tmem + lane_base + kColO + c, o);
+          tg::tmem_st16(tmem + lane_base + kColO + c + 16, o + 16);
+        }
+        tg::tmem_st_wait();
+      }
+      if constexpr (kPinTmem) {
+        const uint32_t pcol = tmem + lane_base + kColS0 + 128u * (j & 1);
+#pragma unroll
+        for (int c = 0; c < kBN / 2; c += 16) tg::tmem_st16(pcol + c, pk + c);
+        tg::tmem_st_wait();
+      } else {
+        // 128-byte swizzle: 16-byte chunk ch of row r sits at chunk ch ^ (r & 7)
+#pragma unroll
+        for (int ch = 0; ch < kBN / 8; ++ch) {
+          uint8_t* base = S.p[ch >> 3] + r * 128 + ((((ch & 7) ^ (r & 7))) << 4);
+          *reinterpret_cast<uint4*>(base) =
+              make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      tg::tc_fence_before();
+      tg::mbar_arrive(&S.p_full);
+    }
+    // ---------------- epilogue: O / l -> bf16 ----------------
+    if (alive) alive = tg::mbar_wait(&S.o_done, (nt - 1) & 1, status, &S.abort_flag);
+    if (__all_sync(0xFFFFFFFFu, alive)) {
+      tg::tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const bool valid = t * kBM + r < len;
+      __nv_bfloat16* orow =
+          out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD;
+      uint32_t o[32];
+#pragma unroll
+      for (int c = 0; c < kD; c += 32) {
+        tg::tmem_ld32(tmem + lane_base + kColO + c, o);
+        tg::tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+            w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            w.z = tg::pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+            w.w = tg::pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + c + e) = w;
+          }
+        }
+      }
+    }
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tg::tc_fence_after();
+    tg::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------- exact fp32 path ----------------
+constexpr int kF32Warps = 4;
+
+__global__ void __launch_bounds__(kF32Warps * 32)
+    gated_attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                          const float* __restrict__ v, const float* __restrict__ s_kept,
+                          const float* __restrict__ gain, const float* __restrict__ tau,
+                          const int32_t* __restrict__ cu_kept, int batch, int64_t total,
+                          int n_hq, int n_hkv, int dh, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kF32Warps + (threadIdx.x >> 5);
+  const int hq = blockIdx.y;
+  if (i >= total) return;
+  int b = 0;
+  while (b + 1 < batch && cu_kept[b + 1] <= i) ++b;
+  const int64_t j0 = cu_kept[b];
+  const int kvh = hq / (n_hq / n_hkv);
+  const float scale = 1.f / (sqrtf(static_cast<float>(dh)) * tau[hq]);
+  const float g = gain[hq];
+  constexpr int kMaxPerLane = 8;   // dh <= 256
+  float qv[kMaxPerLane], acc[kMaxPerLane];
+  const float* qi = q + (i * n_hq + hq) * dh;
+#pragma unroll
+  for (int e = 0; e < kMaxPerLane; ++e) {
+    const int c = lane + 32 * e;
+    qv[e] = c < dh ? qi[c] : 0.f;
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int64_t j = j0; j <= i; ++j) {
+    const float* kj = k + (j * n_hkv + kvh) * dh;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < kMaxPerLane; ++e) {
+      const int c = lane + 32 * e;
+      if (c < dh) dot = fmaf(qv[e], kj[c], dot);
+    }
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+    const float z = dot * scale + g * s_kept[j];
+    const float m_new = fmaxf(m, z);
+    const float a = expf(m - m_new);
+    const float p = expf(z - m_new);
+    l = l * a + p;
+    const float* vj = v + (j * n_hkv + kvh) * dh;
+#pragma unroll
+    for (int e = 0; e < kMaxPerLane; ++e) {
+      const int c = lane + 32 * e;
+      acc[e] = acc[e] * a + (c < dh ? p * vj[c] : 0.f);
+    }
+    m = m_new;
+  }
+  float* oi = out + (i * n_hq + hq) * dh;
+#pragma unroll
+  for (int e = 0; e < kMaxPerLane; ++e) {
+    const int c = lane + 32 * e;
+    if (c < dh) oi[c] = acc[e] / l;
+  }
+}
+
+template <bool kPinTmem>
+tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const float* s_kept,
+                           const float* gain, const float* tau, const int32_t* cu_kept, int batch,
+                           int64_t total, int max_kept, int n_hq, int n_hkv, void* out,
+                           cudaStream_t st) {
+  int* status = tg::status_word();
+  if (!status) return TG_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  const uint64_t dq[3] = {kD, static_cast<uint64_t>(n_hq), static_cast<uint64_t>(total)};
+  const uint64_t sq[2] = {kD * 2, static_cast<uint64_t>(n_hq) * kD * 2};
+  const uint64_t dk[3] = {kD, static_cast<uint64_t>(n_hkv), static_cast<uint64_t>(total)};
+  const uint64_t sk[2] = {kD * 2, static_cast<uint64_t>(n_hkv) * kD * 2};
+  const uint32_t box[3] = {64, 1, kBM};
+  if (!tg::encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dq, sq, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tg::encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dk, sk, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tg::encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dk, sk, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+    return TG_ERR_CUDA;
+  const size_t smem = sizeof(AttnSmem) + 1024;
+  if (cudaFuncSetAttribute(gated_attn_bf16_kernel<kPinTmem>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return TG_ERR_CUDA;
+  const int n_qt = (max_kept + kBM - 1) / kBM;
+  dim3 grid(n_hq, batch, n_qt);
+  gated_attn_bf16_kernel<kPinTmem><<<grid, kThreads, smem, st>>>(
+      tq, tk, tv, s_kept, gain, tau, cu_kept, n_hq, n_hkv, static_cast<__nv_bfloat16*>(out),
+      status);
+  return tg::launch_status();
+}
+
+}  // namespace
+
+// P path of the bf16 kernel: 0 = through shared memory (default), 1 = through TMEM.
+static int g_attn_p_in_tmem = 0;
+extern "C" void tg_internal_set_attn_variant(int p_in_tmem) { g_attn_p_in_tmem = p_in_tmem; }
+
+extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void* v,
+                                        tg_dtype dtype, const float* s_kept, const float* gain,
+                                        const float* tau, const int32_t* cu_kept, int batch,
+                                        int64_t total_kept, int max_kept, int n_hq, int n_hkv,
+                                        int head_dim, void* out, tg_stream_t stream) {
+  if (batch < 0 || total_kept < 0 || max_kept < 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0)
+    return TG_ERR_INVALID_ARG;
+  if (batch == 0 || total_kept == 0 || max_kept == 0) return TG_OK;
+  if (!q || !k || !v || !s_kept || !gain || !tau || !cu_kept || !out) return TG_ERR_INVALID_ARG;
+  if (n_hq % n_hkv != 0) return TG_ERR_INVALID_ARG;
+  if (max_kept > total_kept) return TG_ERR_INVALID_ARG;
+  if (n_hq > 65535 || batch > 65535) return TG_ERR_UNSUPPORTED;
+  if (dtype == TG_BF16) {
+    if (head_dim != kD) return TG_ERR_UNSUPPORTED;
+    if (total_kept > INT32_MAX - kBM || (max_kept + kBM - 1) / kBM > 65535) return TG_ERR_UNSUPPORTED;
+    if (!tg::aligned16(q) || !tg::aligned16(k) || !tg::aligned16(v) || !tg::aligned16(out))
+      return TG_ERR_MISALIGNED;
+    return g_attn_p_in_tmem
+               ? launch_attn_bf16<true>(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept,
+                                        max_kept, n_hq, n_hkv, out, stream)
+               : launch_attn_bf16<false>(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept,
+                                         max_kept, n_hq, n_hkv, out, stream);
+  }
+  if (dtype == TG_F32) {
+    if (head_dim > 256) return TG_ERR_UNSUPPORTED;
+    const int64_t blocks = (total_kept + kF32Warps - 1) / kF32Warps;
+    if (blocks > INT32_MAX) return TG_ERR_UNSUPPORTED;
+    dim3 grid(static_cast<unsigned>(blocks), n_hq);
+    gated_attn_f32_kernel<<<grid, kF32Warps * 32, 0, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        s_kept, gain, tau, cu_kept, batch, total_kept, n_hq, n_hkv, head_dim,
+        static_cast<float*>(out));
+    return tg::launch_status();
+  }
+  return TG_ERR_UNSUPPORTED;
+}

@@ -1,0 +1,234 @@
+// tg_gate_score: the gate MLP scorer (MarkTechPost page on TokenGate, section
+// "Comment TokenGate a-t-il appris le fonctionnement de la réduction des tokens
+// ?": a small MLP scores each token from its post-attention residual at layer L).
+//     s_i = b2 + sum_k w2[k] * GELU(b1[k] + x_i . w1[k,:])
+//
+// bf16 path: one CTA per 128-token tile computes the whole hidden layer
+// (M=128 tokens x N=h units x K=d) with tcgen05.mma (kind::f16, f32 accumulate)
+// into a 128 x h fp32 accumulator in tensor memory. A TMA producer thread streams
+// 128x64 tiles of x and hx64 tiles of w1 (128-byte swizzle) through a 4-stage
+// mbarrier ring; one MMA thread issues 4 K=16 MMAs per stage and frees the stage
+// with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
+// accumulator (warp w: lanes 32*(w%4).., a quarter of the columns), add b1, apply
+// exact erf-GELU and dot with w2; the four column partials are summed in a fixed
+// order, so a token's score depends only on its own row.
+//
+// f32 path: an exact fp32 SIMT kernel (one CTA per token) for small checks.
+#include "common.cuh"
+
+namespace {
+
+constexpr int kBM = 128;      // tokens per tile
+constexpr int kBK = 64;       // reduction columns per stage (128 bytes of bf16)
+constexpr int kStages = 4;
+constexpr int kThreads = 512;
+
+template <int H>
+struct GateSmem {
+  uint8_t a[kStages][kBM * kBK * 2];   // x tiles, 16 KB each
+  uint8_t b[kStages][H * kBK * 2];     // w1 tiles
+  float b1[H];
+  float w2[H];
+  float part[4][kBM];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float gelu_erf(float u) {
+  return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
+}
+
+template <int H>
+__global__ void __launch_bounds__(kThreads, 1)
+    gate_bf16_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                     const float* __restrict__ b1, const float* __restrict__ w2, float b2,
+                     int64_t n_tokens, int d, float* __restrict__ scores, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
+  GateSmem<H>& S = *reinterpret_cast<GateSmem<H>*>(smem_raw + pad);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int nk = d / kBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tg::mbar_init(&S.full[s], 1);
+      tg::mbar_init(&S.empty[s], 1);
+    }
+    tg::mbar_init(&S.acc_full, 1);
+    S.abort_flag = 0;
+    tg::fence_barrier_init();
+  }
+  for (int i = tid; i < H; i += kThreads) {
+    S.b1[i] = b1[i];
+    S.w2[i] = w2[i];
+  }
+  if (warp == 2) {
+    tg::tmem_alloc(&S.tmem_base, H);
+    tg::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tg::tma_prefetch_desc(&tm_x);
+    tg::tma_prefetch_desc(&tm_w);
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  tg::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer ----
+    int issued = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (kb >= kStages &&
+          !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
+        break;
+      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H) * kBK * 2);
+      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, 0);
+      ++issued;
+    }
+    if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
+      for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
+        tg::mbar_wait(&S.full[kb % kStages], (kb / kStages) & 1, status, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ----
+    constexpr uint32_t idesc = tg::idesc_bf16_f32(kBM, H, false, false);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+      tg::tc_fence_after();
+      const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                        tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
+      }
+      tg::mma_commit(&S.empty[s]);
+    }
+    tg::mma_commit(&S.acc_full);
+  }
+  __syncwarp();
+
+  // ---- epilogue: all 16 warps ----
+  constexpr int kCols = H / 4;               // accumulator columns per warp
+  const int lg = warp & 3, cgp = warp >> 2;
+  const int row = lg * 32 + lane;
+  float acc = 0.f;
+  const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
+  if (ok) {
+    tg::tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < kCols; c += 16) {
+      uint32_t r[16];
+      tg::tmem_ld16(tmem + (static_cast<uint32_t>(lg * 32) << 16) + cgp * kCols + c, r);
+      tg::tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int col = cgp * kCols + c + j;
+        acc += S.w2[col] * gelu_erf(__uint_as_float(r[j]) + S.b1[col]);
+      }
+    }
+  }
+  S.part[cgp][row] = acc;
+  tg::tc_fence_before();
+  __syncthreads();
+  if (tid < kBM) {
+    const float s = b2 + ((S.part[0][tid] + S.part[1][tid]) + (S.part[2][tid] + S.part[3][tid]));
+    if (m0 + tid < n_tokens) scores[m0 + tid] = s;
+  }
+  if (warp == 2) {
+    tg::tc_fence_after();
+    tg::tmem_dealloc(tmem, H);
+  }
+}
+
+// Exact fp32 path: one CTA per token, hidden units strided over the threads,
+// fixed-order block reduction.
+constexpr int kF32Threads = 128;
+
+__global__ void __launch_bounds__(kF32Threads)
+    gate_f32_kernel(const float* __restrict__ x, const float* __restrict__ w1,
+                    const float* __restrict__ b1, const float* __restrict__ w2, float b2, int d,
+                    int h, float* __restrict__ scores) {
+  extern __shared__ float xrow[];
+  __shared__ float red[kF32Threads];
+  const int64_t i = blockIdx.x;
+  for (int c = threadIdx.x; c < d; c += kF32Threads) xrow[c] = x[i * d + c];
+  __syncthreads();
+  float part = 0.f;
+  for (int k = threadIdx.x; k < h; k += kF32Threads) {
+    const float* w = w1 + static_cast<int64_t>(k) * d;
+    float u = 0.f;
+    for (int c = 0; c < d; ++c) u = fmaf(xrow[c], w[c], u);
+    part += w2[k] * gelu_erf(u + b1[k]);
+  }
+  red[threadIdx.x] = part;
+  __syncthreads();
+  for (int o = kF32Threads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) scores[i] = b2 + red[0];
+}
+
+template <int H>
+tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, const float* b1,
+                           const float* w2, float b2, float* scores, cudaStream_t st) {
+  int* status = tg::status_word();
+  if (!status) return TG_ERR_CUDA;
+  CUtensorMap tx, tw;
+  const uint64_t dx[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n)};
+  const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
+  const uint32_t bx[2] = {kBK, kBM};
+  const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H)};
+  const uint32_t bw[2] = {kBK, H};
+  if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dx, sx, bx,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w1, dw, sx, bw,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+    return TG_ERR_CUDA;
+  const size_t smem = sizeof(GateSmem<H>) + 1024;
+  if (cudaFuncSetAttribute(gate_bf16_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return TG_ERR_CUDA;
+  const int64_t tiles = (n + kBM - 1) / kBM;
+  gate_bf16_kernel<H><<<static_cast<unsigned>(tiles), kThreads, smem, st>>>(tx, tw, b1, w2, b2, n, d,
+                                                                           scores, status);
+  return tg::launch_status();
+}
+
+}  // namespace
+
+extern "C" tg_status tg_gate_score(const void* x, tg_dtype dtype, int64_t n_tokens, int d,
+                                   const void* w1, const float* b1, const float* w2, float b2,
+                                   int h, float* scores, tg_stream_t stream) {
+  if (n_tokens < 0 || d <= 0 || h <= 0) return TG_ERR_INVALID_ARG;
+  if (n_tokens == 0) return TG_OK;
+  if (!x || !w1 || !b1 || !w2 || !scores) return TG_ERR_INVALID_ARG;
+  if (dtype == TG_BF16) {
+    if (d % kBK != 0 || (h != 64 && h != 128 && h != 256)) return TG_ERR_UNSUPPORTED;
+    if (n_tokens > INT32_MAX - kBM) return TG_ERR_UNSUPPORTED;
+    if (!tg::aligned16(x) || !tg::aligned16(w1)) return TG_ERR_MISALIGNED;
+    switch (h) {
+      case 64: return launch_gate_bf16<64>(x, n_tokens, d, w1, b1, w2, b2, scores, stream);
+      case 128: return launch_gate_bf16<128>(x, n_tokens, d, w1, b1, w2, b2, scores, stream);
+      default: return launch_gate_bf16<256>(x, n_tokens, d, w1, b1, w2, b2, scores, stream);
+    }
+  }
+  if (dtype == TG_F32) {
+    if (h > 1024 || d > 12288) return TG_ERR_UNSUPPORTED;
+    if (n_tokens > INT32_MAX) return TG_ERR_UNSUPPORTED;
+    gate_f32_kernel<<<static_cast<unsigned>(n_tokens), kF32Threads, static_cast<size_t>(d) * 4,
+                      stream>>>(static_cast<const float*>(x), static_cast<const float*>(w1), b1, w2,
+                                b2, d, h, scores);
+    return tg::launch_status();
+  }
+  return TG_ERR_UNSUPPORTED;
+}

@@ -1,0 +1,329 @@
+// tg_select_topk: top-K of the droppable document span with the question always
+// kept (MarkTechPost page on TokenGate, section "Comment TokenGate a-t-il appris
+// le fonctionnement de la réduction des tokens ?": a top-K selector keeps the
+// best-scoring tokens; only the document part may be dropped; section "Comment
+// déployer TokenGate ?": {state} marks the document, max_kept_prefill_tokens the
+// budget).
+//
+// One thread-block cluster of 8 CTAs per sequence, one launch for the whole
+// batch. Each CTA holds a contiguous eighth of the sequence's scores in shared
+// memory as order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass
+// MSB-first radix select (8-bit digits) finds the exact K-th largest document key
+// T: every pass builds warp-aggregated (match_any) histograms, the 8 CTA
+// histograms are summed through distributed shared memory, and the digit that
+// holds the K-th key is found with a block suffix scan. Emission then keeps every
+// token outside the span, every document token with key > T, and the `need`
+// lowest-positioned document tokens with key == T (ties to the lower position);
+// the stable output order comes from warp ballots / popc prefix sums, with the
+// per-warp and per-CTA offsets exchanged the same way. No global scratch memory.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace {
+
+constexpr int kCluster = 8;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunkQuant = kThreads;   // chunk rounded to this -> per-warp segments of 32k
+
+struct SelectSmem {
+  uint32_t whist[kWarps][256];   // per-warp histograms
+  uint32_t hist[2][256];         // this CTA's histogram, by pass parity (read by peers)
+  uint32_t scan[kWarps];
+  uint32_t warp_tot[kWarps];
+  uint32_t warp_off[kWarps];
+  uint32_t cta_eq;               // published to peers
+  uint32_t cta_keep;             // published to peers
+  uint32_t digit;
+  uint32_t remaining;
+  uint32_t cta_eq_off;
+  uint32_t cta_keep_off;
+  uint32_t seq_keep;
+  int64_t out_base;
+  int64_t red[kWarps];
+  // followed by: uint32_t masks[chunk / 32]; uint32_t keys[chunk];
+};
+
+__host__ __device__ inline int select_chunk(int max_len) {
+  int c = (max_len + kCluster - 1) / kCluster;
+  c = (c + kChunkQuant - 1) / kChunkQuant * kChunkQuant;
+  return c < kChunkQuant ? kChunkQuant : c;
+}
+
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;   // NaN ranks lowest
+  if (u == 0x80000000u) u = 0u;                     // -0 is +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// kept count of a sequence from the (possibly hostile) device arrays, clamped
+__device__ __forceinline__ int64_t seq_kept(const int32_t* cu, const int32_t* db,
+                                            const int32_t* de, const int32_t* kd, int b) {
+  int64_t len = (int64_t)cu[b + 1] - cu[b];
+  if (len < 0) len = 0;
+  int64_t s0 = db[b], s1 = de[b];
+  if (s0 < 0) s0 = 0;
+  if (s1 > len) s1 = len;
+  int64_t nd = s1 > s0 ? s1 - s0 : 0;
+  int64_t k = kd[b];
+  if (k < 0) k = 0;
+  if (k > nd) k = nd;
+  return len - nd + k;
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+    select_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ cu_seqlens,
+                       const int32_t* __restrict__ doc_begin, const int32_t* __restrict__ doc_end,
+                       const int32_t* __restrict__ k_doc, int batch, int64_t total_kept,
+                       int chunk, int32_t* __restrict__ kept_idx, float* __restrict__ kept_scores,
+                       int32_t* __restrict__ cu_kept, int* status) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
+  uint32_t* keys = masks + chunk / 32;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned rank = cluster.block_rank();
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned full = 0xFFFFFFFFu;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  // ---- sequence geometry (identical in every CTA of the cluster) ----
+  const int64_t base = cu_seqlens[b];
+  const int64_t len = (int64_t)cu_seqlens[b + 1] - base;
+  const int64_t db = doc_begin[b], de = doc_end[b];
+  const bool bad = len < 0 || len > (int64_t)chunk * kCluster || db < 0 || de < db || de > len;
+  if (bad) {
+    if (rank == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    return;   // uniform across the cluster: nobody reaches a cluster barrier
+  }
+  const int64_t nd = de - db;
+  int64_t k_eff = k_doc[b];
+  if (k_eff < 0) k_eff = 0;
+  if (k_eff > nd) k_eff = nd;
+
+  // output offset of this sequence: sum of kept counts of earlier sequences
+  {
+    int64_t acc = 0;
+    for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
+    if (lane == 0) S.red[warp] = acc;
+    __syncthreads();
+    if (tid == 0) {
+      int64_t t = 0;
+      for (int w = 0; w < kWarps; ++w) t += S.red[w];
+      S.out_base = t;
+    }
+  }
+
+  // ---- load this CTA's slice as keys ----
+  const int64_t c0 = (int64_t)rank * chunk;
+  int64_t n_local = len - c0;
+  if (n_local < 0) n_local = 0;
+  if (n_local > chunk) n_local = chunk;
+  for (int i = tid; i < chunk; i += kThreads)
+    keys[i] = i < n_local ? score_key(scores[base + c0 + i]) : 0u;
+  __syncthreads();
+
+  const int seg = chunk / kWarps;          // multiple of 32
+  const int seg0 = warp * seg;
+
+  // ---- radix select of the k_eff-th largest document key ----
+  uint32_t T, need;
+  if (k_eff == 0) {
+    T = 0xFFFFFFFFu;   // above every key (the largest key, +inf, is 0xFF800000)
+    need = 0;
+  } else if (k_eff == nd) {
+    T = 0u;            // everything is kept
+    need = (uint32_t)nd;
+  } else {
+    uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k_eff;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < kWarps * 256; i += kThreads) (&S.whist[0][0])[i] = 0u;
+      __syncthreads();
+      for (int i = seg0 + lane; i < seg0 + seg; i += 32) {
+        const int64_t pos = c0 + i;
+        const uint32_t key = keys[i];
+        const bool valid = i < n_local && pos >= db && pos < de && (key & pmask) == prefix;
+        const unsigned act = __ballot_sync(full, valid);
+        if (valid) {
+          const uint32_t digit = (key >> shift) & 0xFFu;
+          const unsigned peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&S.whist[warp][digit], (uint32_t)__popc(peers));
+        }
+      }
+      __syncthreads();
+      uint32_t* h = S.hist[pass & 1];
+      if (tid < 256) {
+        uint32_t t = 0;
+        for (int w = 0; w < kWarps; ++w) t += S.whist[w][tid];
+        h[tid] = t;
+      }
+      cluster.sync();
+      // thread t holds digit d = 255 - t; an inclusive prefix over t is the
+      // count of document keys (matching the prefix) with digit >= d
+      uint32_t cnt = 0;
+      if (tid < 256) {
+        const int d = 255 - tid;
+        for (unsigned r = 0; r < kCluster; ++r) cnt += cluster.map_shared_rank(h, r)[d];
+        uint32_t inc = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+          uint32_t y = __shfl_up_sync(full, inc, o);
+          if (lane >= o) inc += y;
+        }
+        if (lane == 31) S.scan[warp] = inc;
+        tg::named_barrier(1, 256);   // warps 0-7 only
+        uint32_t woff = 0;
+        for (int w = 0; w < warp; ++w) woff += S.scan[w];
+        inc += woff;
+        const uint32_t exc = inc - cnt;
+        if (exc < remaining && remaining <= inc) {
+          S.digit = (uint32_t)d;
+          S.remaining = remaining - exc;
+        }
+      }
+      __syncthreads();
+      prefix |= S.digit << shift;
+      pmask |= 0xFFu << shift;
+      remaining = S.remaining;
+      __syncthreads();
+    }
+    T = prefix;
+    need = remaining;
+  }
+
+  // ---- emission, phase A: per-warp counts of document keys equal to T ----
+  {
+    uint32_t cnt = 0;
+    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
+      const int64_t pos = c0 + i;
+      const bool eq = i < n_local && pos >= db && pos < de && keys[i] == T;
+      const unsigned m = __ballot_sync(full, eq);
+      if (lane == 0) masks[wi] = m;
+      cnt += __popc(m);
+    }
+    if (lane == 0) S.warp_tot[warp] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        S.warp_off[w] = t;
+        t += S.warp_tot[w];
+      }
+      S.cta_eq = t;
+    }
+    cluster.sync();
+    if (tid == 0) {
+      uint32_t off = 0;
+      for (unsigned r = 0; r < rank; ++r) off += *cluster.map_shared_rank(&S.cta_eq, r);
+      S.cta_eq_off = off;
+    }
+    __syncthreads();
+  }
+
+  // ---- phase B: keep decisions and per-warp kept counts ----
+  {
+    uint32_t running = S.cta_eq_off + S.warp_off[warp];
+    uint32_t kept = 0;
+    __syncthreads();   // warp_off is rewritten below
+    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
+      const int64_t pos = c0 + i;
+      const uint32_t eqm = masks[wi];
+      bool keep = false;
+      if (i < n_local) {
+        const bool in_doc = pos >= db && pos < de;
+        const uint32_t key = keys[i];
+        const bool eq = (eqm >> lane) & 1u;
+        keep = !in_doc || key > T || (eq && running + __popc(eqm & lt_mask) < need);
+      }
+      running += __popc(eqm);
+      const unsigned km = __ballot_sync(full, keep);
+      __syncwarp();
+      if (lane == 0) masks[wi] = km;
+      kept += __popc(km);
+    }
+    if (lane == 0) S.warp_tot[warp] = kept;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        S.warp_off[w] = t;
+        t += S.warp_tot[w];
+      }
+      S.cta_keep = t;
+    }
+    cluster.sync();
+    if (tid == 0) {
+      uint32_t off = 0, tot = 0;
+      for (unsigned r = 0; r < kCluster; ++r) {
+        const uint32_t v = *cluster.map_shared_rank(&S.cta_keep, r);
+        if (r < rank) off += v;
+        tot += v;
+      }
+      S.cta_keep_off = off;
+      S.seq_keep = tot;
+    }
+    __syncthreads();
+  }
+
+  // ---- phase C: write kept row ids (and their scores), ascending ----
+  const int64_t out_base = S.out_base;
+  const int64_t seq_keep = S.seq_keep;
+  const int64_t expect = len - nd + k_eff;
+  const bool ok = seq_keep == expect && out_base + seq_keep <= total_kept;
+  if (ok) {
+    int64_t running = out_base + S.cta_keep_off + S.warp_off[warp];
+    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
+      const uint32_t km = masks[wi];
+      if ((km >> lane) & 1u) {
+        const int64_t o = running + __popc(km & lt_mask);
+        const int64_t row = base + c0 + i;
+        kept_idx[o] = (int32_t)row;
+        if (kept_scores) kept_scores[o] = scores[row];
+      }
+      running += __popc(km);
+    }
+  }
+  if (rank == 0 && tid == 0) {
+    if (!ok) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    if (b == 0) cu_kept[0] = 0;
+    cu_kept[b + 1] = (int32_t)(out_base + expect);
+    if (b == batch - 1 && out_base + expect != total_kept) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+  }
+  cluster.sync();   // peers may still read this CTA's shared memory until here
+}
+
+}  // namespace
+
+extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens,
+                                    const int32_t* doc_begin, const int32_t* doc_end,
+                                    const int32_t* k_doc, int batch, int64_t total_tokens,
+                                    int64_t total_kept, int max_seqlen, int32_t* kept_idx,
+                                    float* kept_scores, int32_t* cu_kept, tg_stream_t stream) {
+  if (batch < 0 || total_tokens < 0 || total_kept < 0 || max_seqlen < 0) return TG_ERR_INVALID_ARG;
+  if (batch == 0) return TG_OK;
+  if (!cu_seqlens || !doc_begin || !doc_end || !k_doc || !cu_kept) return TG_ERR_INVALID_ARG;
+  if (total_tokens > 0 && !scores) return TG_ERR_INVALID_ARG;
+  if (total_kept > 0 && !kept_idx) return TG_ERR_INVALID_ARG;
+  if (total_kept > total_tokens || total_tokens > INT32_MAX) return TG_ERR_INVALID_ARG;
+  if (max_seqlen > TG_SELECT_MAX_SEQLEN) return TG_ERR_UNSUPPORTED;
+  if (batch > 65535) return TG_ERR_UNSUPPORTED;
+  int* st = tg::status_word();
+  if (!st) return TG_ERR_CUDA;
+  const int chunk = select_chunk(max_seqlen);
+  const size_t smem = sizeof(SelectSmem) + (size_t)chunk / 32 * 4 + (size_t)chunk * 4;
+  if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return TG_ERR_CUDA;
+  dim3 grid(kCluster, batch);
+  select_topk_kernel<<<grid, kThreads, smem, stream>>>(scores, cu_seqlens, doc_begin, doc_end,
+                                                       k_doc, batch, total_kept, chunk, kept_idx,
+                                                       kept_scores, cu_kept, st);
+  return tg::launch_status();
+}

@@ -1,0 +1,88 @@
+"""One gated layer of the prefill path, end to end on the GPU:
+gate scores -> question-protected top-K -> compaction of the residual rows ->
+token-gated causal GQA attention over the kept tokens (MarkTechPost page on
+TokenGate, section "Comment TokenGate a-t-il appris le fonctionnement de la
+réduction des tokens ?").
+
+The attention inputs q/k/v are the kept tokens' projections; the projection
+that would produce them from the compacted residual is outside this path, so
+they are supplied already compacted ([K, H, dh]) and only the key scores come
+from the selection.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import api
+from .synth import Workload
+
+
+class GatedPrefill:
+    """Device-resident buffers for one workload and a `step()` that runs the four
+    stages on one stream (4 kernel launches)."""
+
+    LAUNCHES_PER_STEP = 4
+
+    def __init__(self, wl: Workload, device: str = "cuda", use_score_override: bool = True):
+        dev = torch.device(device)
+        self.wl = wl
+        self.x = wl.x.to(dev)
+        self.w1 = wl.w1.to(dev)
+        self.b1 = wl.b1.to(dev)
+        self.w2 = wl.w2.to(dev)
+        self.b2 = float(wl.b2)
+        self.gain = wl.gain.to(dev)
+        self.tau = wl.tau.to(dev)
+        self.q = wl.q.to(dev)
+        self.k = wl.k.to(dev)
+        self.v = wl.v.to(dev)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.cu_seqlens = torch.tensor(wl.cu_seqlens, **i32)
+        self.doc_begin = torch.tensor(wl.doc_begin, **i32)
+        self.doc_end = torch.tensor(wl.doc_end, **i32)
+        self.k_doc = torch.tensor(wl.k_doc, **i32)
+        self.override = (wl.score_override.to(dev)
+                         if (use_score_override and wl.score_override is not None) else None)
+        self.n_tokens = wl.n_tokens
+        self.total_kept = wl.total_kept
+        self.max_seqlen = max(wl.seqlens)
+        self.max_kept = max(wl.kept_counts)
+        K = self.total_kept
+        self.scores = torch.empty(self.n_tokens, dtype=torch.float32, device=dev)
+        self.kept_idx = torch.empty(K, dtype=torch.int32, device=dev)
+        self.kept_scores = torch.empty(K, dtype=torch.float32, device=dev)
+        self.cu_kept = torch.empty(wl.batch + 1, **i32)
+        self.xc = torch.empty((K, wl.d), dtype=self.x.dtype, device=dev)
+        self.out = torch.empty_like(self.q)
+
+    def stage_gate(self, stream=None):
+        api.gate_score(self.x, self.w1, self.b1, self.w2, self.b2, out=self.scores, stream=stream)
+
+    def stage_select(self, stream=None):
+        sel = self.override if self.override is not None else self.scores
+        api.select_topk(sel, self.cu_seqlens, self.doc_begin, self.doc_end, self.k_doc,
+                        self.total_kept, self.max_seqlen, kept_idx=self.kept_idx,
+                        kept_scores=self.kept_scores, cu_kept=self.cu_kept, stream=stream)
+
+    def stage_compact(self, stream=None):
+        api.compact_rows([self.x], self.kept_idx, outs=[self.xc], stream=stream)
+
+    def stage_attention(self, stream=None):
+        api.gated_attention(self.q, self.k, self.v, self.kept_scores, self.gain, self.tau,
+                            self.cu_kept, self.max_kept, out=self.out, stream=stream)
+
+    STAGES = ("gate", "select", "compact", "attention")
+
+    def step(self, stream=None, events: Optional[list] = None):
+        """Run the four stages. If `events` is a list of 5 CUDA events, they are
+        recorded on the stream before, between and after the stages."""
+        s = stream if stream is not None else torch.cuda.current_stream()
+        fns = (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention)
+        for i, fn in enumerate(fns):
+            if events is not None:
+                events[i].record(s)
+            fn(stream=s)
+        if events is not None:
+            events[4].record(s)

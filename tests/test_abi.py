@@ -1,0 +1,82 @@
+"""The C-ABI library builds, loads and exports every symbol include/tg.h declares;
+host-side argument validation returns status codes without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learned_token_pruning_gemm_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "tg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"tg_gate_score", "tg_select_topk", "tg_compact_kv", "tg_gated_attention"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures cover the header"
+
+
+def test_status_strings(lib):
+    assert lib.tg_abi_version() == 1
+    for code, name in [(0, "TG_OK"), (1, "TG_ERR_INVALID_ARG"), (3, "TG_ERR_MISALIGNED"),
+                       (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (99, "TG_ERR_UNKNOWN")]:
+        assert lib.tg_status_string(code).decode() == name
+
+
+def test_validation_returns_status_without_gpu(lib):
+    INVALID, UNSUP, MIS = 1, 2, 3
+    P = ctypes.c_void_p
+    fake = P(0x10000)      # never dereferenced: validation fails first
+    odd = P(0x10004)       # not 16-byte aligned
+    # gate: null pointers / bad sizes / unsupported h / misalignment
+    assert lib.tg_gate_score(None, 1, 128, 128, fake, fake, fake, 0.0, 64, fake, None) == INVALID
+    assert lib.tg_gate_score(fake, 1, -1, 128, fake, fake, fake, 0.0, 64, fake, None) == INVALID
+    assert lib.tg_gate_score(fake, 1, 0, 128, fake, fake, fake, 0.0, 64, fake, None) == 0
+    assert lib.tg_gate_score(fake, 1, 128, 100, fake, fake, fake, 0.0, 64, fake, None) == UNSUP
+    assert lib.tg_gate_score(fake, 1, 128, 128, fake, fake, fake, 0.0, 96, fake, None) == UNSUP
+    assert lib.tg_gate_score(odd, 1, 128, 128, fake, fake, fake, 0.0, 64, fake, None) == MIS
+    assert lib.tg_gate_score(fake, 7, 128, 128, fake, fake, fake, 0.0, 64, fake, None) == UNSUP
+    # select: K > N, too long, null outputs
+    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 11, 10, fake, None, fake,
+                              None) == INVALID
+    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 5, 300000, fake, None, fake,
+                              None) == UNSUP
+    assert lib.tg_select_topk(fake, None, fake, fake, fake, 1, 10, 5, 10, fake, None, fake,
+                              None) == INVALID
+    assert lib.tg_select_topk(None, None, None, None, None, 0, 0, 0, 0, None, None, None,
+                              None) == 0
+    # compact: row bytes must be a positive multiple of 16, pointers aligned
+    arr = (P * 1)(fake)
+    arr_odd = (P * 1)(odd)
+    rb = (ctypes.c_int64 * 1)(4096)
+    rb_odd = (ctypes.c_int64 * 1)(40)
+    assert lib.tg_compact_kv(arr, arr, rb_odd, 1, fake, 5, None) == MIS
+    assert lib.tg_compact_kv(arr_odd, arr, rb, 1, fake, 5, None) == MIS
+    assert lib.tg_compact_kv(arr, arr, rb, 0, fake, 5, None) == INVALID
+    assert lib.tg_compact_kv(arr, arr, rb, 9, fake, 5, None) == INVALID
+    assert lib.tg_compact_kv(arr, arr, rb, 1, fake, 0, None) == 0
+    # attention: GQA divisibility, head dim, max_kept > total, alignment
+    args = [fake, fake, fake, 1, fake, fake, fake, fake, 1, 256, 256]
+    assert lib.tg_gated_attention(*args, 16, 6, 128, fake, None) == INVALID
+    assert lib.tg_gated_attention(*args, 16, 8, 64, fake, None) == UNSUP
+    assert lib.tg_gated_attention(*args[:-1], 300, 16, 8, 128, fake, None) == INVALID
+    assert lib.tg_gated_attention(*args, 16, 8, 128, odd, None) == MIS
+    assert lib.tg_gated_attention(fake, fake, fake, 1, fake, fake, fake, fake, 1, 256, 256, 16, 8,
+                                  300, fake, None) == UNSUP
+    # self test bounds
+    assert lib.tg_selftest_bounded_wait(10, None) == INVALID
