@@ -68,51 +68,64 @@ def _max_over_ranks(dist, v: float) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during a region."""
+    """SM clock and clock-event reasons, sampled by a background thread through
+    NVML (about every 0.5 ms) while the benchmark runs; `window(t0, t1)` keeps
+    the samples taken inside a host-time window."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, device: int):
+        self.samples = []
+        self._stop = False
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            idx = device
+            if hasattr(torch.cuda, "_get_nvml_device_index"):
+                idx = torch.cuda._get_nvml_device_index(device)
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # noqa: BLE001
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        while not self._stop:
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self._reasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.0005)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+        import threading
+        if self.error is None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join()
+
+    def window(self, t0, t1):
+        if self.error is not None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        where = "timed region"
+        if len(inside) < 3:          # too short a region: widen to the whole loaded run
+            inside, where = self.samples, "warm-up + timed region"
+        mhz = [s[1] for s in inside]
+        reasons = sorted({n for s in inside for bit, n in self.REASONS.items() if s[2] & bit})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "sampled_over": where}
 
 
 def _work(wl):
@@ -215,23 +228,27 @@ def run_ours(args, dist, rank, ws):
     work = _work(wl)
     peaks, peak_src = _peaks()
 
+    clocks = ClockSampler(dev_index)
+    clocks.start()
+    gp.capture()                          # one CUDA graph per stage; replays below
     for _ in range(args.warmup):
         flush.zero_()
-        gp.step(stream)
+        gp.replay()
     torch.cuda.synchronize()
     assert api.device_status(reset=True) == 0
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    clocks = ClockSampler(dev_index)
-    clocks.start()
     _barrier(dist)
     torch.cuda.synchronize()
+    t_host0 = time.perf_counter()
     for i in range(args.steps):
         flush.zero_()                     # L2 flush between timed steps (outside the events)
-        gp.step(stream, events=evs[i])
+        gp.replay(events=evs[i])
     torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
     _barrier(dist)
-    clk = clocks.stop()
+    clocks.stop()
+    clk = clocks.window(t_host0, t_host1)
     status = api.device_status(reset=True)
     if status != 0:
         raise RuntimeError(f"device status {status} during the timed region")
@@ -302,7 +319,7 @@ def run_ours(args, dist, rank, ws):
         def e2e_step():
             for hsrc, dst in zip(host_in, dev_in):
                 dst.copy_(hsrc, non_blocking=True)
-            gp.step(stream)
+            gp.replay()
             host_out.copy_(gp.out, non_blocking=True)
             host_idx.copy_(gp.kept_idx, non_blocking=True)
 
@@ -344,6 +361,7 @@ def run_ours(args, dist, rank, ws):
             "stages": stages,
             "roofline": roofline,
             "gpu_launches": gp.LAUNCHES_PER_STEP * args.steps,
+            "launch": "one CUDA graph per stage, replayed; per-stage CUDA events between them",
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

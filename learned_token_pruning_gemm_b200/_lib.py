@@ -48,8 +48,6 @@ def load(path: str = LIB_PATH):
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
-        lib.tg_internal_set_attn_variant.restype = None
-        lib.tg_internal_set_attn_variant.argtypes = [INT]
         _lib = lib
     return _lib
 

@@ -128,9 +128,3 @@ def device_status(reset: bool = True, stream=None) -> int:
 def selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
     check(_lib.load().tg_selftest_bounded_wait(int(timeout_ns), _stream(stream)),
           "tg_selftest_bounded_wait")
-
-
-def set_attention_variant(p_in_tmem: bool) -> None:
-    """Choose how P reaches the PV MMA in the bf16 attention kernel: through
-    shared memory (False, default) or through tensor memory (True)."""
-    _lib.load().tg_internal_set_attn_variant(1 if p_in_tmem else 0)

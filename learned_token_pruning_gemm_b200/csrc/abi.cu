@@ -63,6 +63,25 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const 
   return r == CUDA_SUCCESS;
 }
 
+bool ensure_smem(const void* fn, int bytes) {
+  struct Entry {
+    int dev;
+    const void* fn;
+    int bytes;
+  };
+  static Entry cache[256];
+  static int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < n; ++i)
+    if (cache[i].dev == dev && cache[i].fn == fn && cache[i].bytes >= bytes) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (n < 256) cache[n++] = Entry{dev, fn, bytes};
+  return true;
+}
+
 tg_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;

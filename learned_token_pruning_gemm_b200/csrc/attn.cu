@@ -8,19 +8,21 @@
 // bf16 path (dh = 128), one CTA per (128-row query tile, query head, sequence):
 //   warp 0      TMA producer: the Q tile once, then K/V tiles of 128 keys through
 //               a 2-stage mbarrier ring; its 32 lanes also stage the per-key bias
-//               b_j = log2(e) g_h s_j for each tile in shared memory.
-//   warp 1      MMA issuer (one thread): S_{j+1} = Q K_{j+1}^T into one of two
-//               128-column TMEM buffers while the softmax works on S_j, then
-//               O += P_j V_j into a 128-column TMEM accumulator.
-//   warps 4-7   softmax, one query row per thread (TMEM lane = row): loads its row
-//               of S, forms z = S c_h + b_j in the log2 domain (one FFMA,
-//               c_h = log2(e) / (sqrt(dh) tau_h)), masks the diagonal tile, keeps a
-//               running max that is only moved when it grows by more than 2^8
-//               (then O is rescaled in TMEM), writes P in bf16 and its row sum.
-// P goes to the MMA through shared memory (128-byte swizzled, K-major) or through
-// TMEM in place of S (A operand in tensor memory), chosen at compile time.
-// Query tiles are launched longest-first (the last tile of a sequence has the
-// most keys under the causal mask).
+//               b_j = log2(e) g_h s_j of each tile in shared memory.
+//   warp 1      MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
+//               S_j = Q K_j^T into one of two 128-column TMEM buffers, and
+//               O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
+//               and V_j as an MN-major shared-memory operand.
+//   warps 4-11  softmax, two threads per query row (TMEM lane = row, each thread
+//               one 64-key half of the tile): z = S c_h + b_j in the log2 domain
+//               (one FFMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile mask,
+//               row max exchanged through shared memory, a running max that only
+//               moves when it grows by more than 2^8 (O is then rescaled in TMEM),
+//               exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA pipe
+//               (own polynomial) for the 4th, P packed to bf16 into TMEM.
+// Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
+// PV_j and S_{j+2}; the only cross-tile wait is the rare O rescale. Query tiles
+// are launched longest-first (the last tile of a sequence has the most keys).
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
 #include "common.cuh"
@@ -31,31 +33,61 @@ constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kD = 128;
 constexpr int kStages = 2;
-constexpr int kThreads = 256;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
+constexpr int kHalf = kBN / 2;                         // keys per softmax thread
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
+constexpr int kPolyEvery = 4;               // every 4th key's exp2 on the FMA pipe
+
+// 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
+// fit_exp2_poly.py in this directory.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+// exp2 on the FMA pipe: n = rint(x) via the 1.5*2^23 shift, 2^f by the polynomial,
+// 2^n added to the exponent field. Inputs below -125 return ~2^-125 (P is bf16;
+// such a weight is zero for every purpose here); inputs are <= 8 by construction.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  const int ni = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(p) + (ni << 23));
+}
 
 struct AttnSmem {
-  uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves
+  uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves (16 KB each)
   uint8_t k[kStages][2][kBN * 64 * 2];
   uint8_t v[kStages][2][kBN * 64 * 2];
-  uint8_t p[2][kBM * 64 * 2];               // P tile (bf16), when P goes through smem
   float bias[kStages][kBN];
+  float red[2][2][kBM];                     // [tile parity][half][row] partial maxima
+  float lsum[2][kBM];                       // [half][row] final partial row sums
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];
-  uint64_t s_free[2];
   uint64_t p_full;
   uint64_t o_done;
+  uint64_t red_full[2][4];                  // [tile parity][row group]: the two halves of a row
+  uint64_t l_full[4];                       // [row group]: final row-sum exchange
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// TMEM columns: S buffers at 0 and 128, O at 256 (512 allocated).
+// TMEM columns: S/P buffers at 0 and 128, O at 256 (512 allocated).
 constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
 
-template <bool kPinTmem>
+__device__ __forceinline__ bool all_alive(bool a) { return __all_sync(0xFFFFFFFFu, a); }
+
+}  // namespace
+
+namespace {
+
 __global__ void __launch_bounds__(kThreads, 1)
     gated_attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -65,8 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            int n_hq, int n_hkv, __nv_bfloat16* __restrict__ out, int* status) {
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
-  const int n_qt_max = gridDim.z;
-  const int t = n_qt_max - 1 - static_cast<int>(blockIdx.z);   // longest tiles first
+  const int t = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);   // longest first
   const int seq0 = cu_kept[b];
   const int len = cu_kept[b + 1] - seq0;
   if (t * kBM >= len) return;   // uniform: this sequence has no tile t
@@ -84,18 +115,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mbar_init(&S.kv_full[s], 1 + 32);   // expect_tx arrival + 32 bias lanes
       tg::mbar_init(&S.kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      tg::mbar_init(&S.s_full[s], 1);
-      tg::mbar_init(&S.s_free[s], 128);
-    }
-    tg::mbar_init(&S.p_full, 128);
+    for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
+    tg::mbar_init(&S.p_full, kSoftmaxWarps * 32);
     tg::mbar_init(&S.o_done, 1);
+    for (int s = 0; s < 2; ++s)
+      for (int g = 0; g < 4; ++g) tg::mbar_init(&S.red_full[s][g], 64);
+    for (int g = 0; g < 4; ++g) tg::mbar_init(&S.l_full[g], 64);
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
   if (warp == 2) {
     tg::tmem_alloc(&S.tmem_base, kTmemCols);
     tg::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tg::tma_prefetch_desc(&tm_q);
+    tg::tma_prefetch_desc(&tm_k);
+    tg::tma_prefetch_desc(&tm_v);
   }
   tg::tc_fence_before();
   __syncthreads();
@@ -116,8 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool go = true;
       if (j >= kStages)
         go = tg::mbar_wait(&S.kv_empty[s], ((j / kStages) - 1) & 1, status, &S.abort_flag);
-      go = __all_sync(0xFFFFFFFFu, go);
-      if (!go) break;
+      if (!all_alive(go)) break;
       if (lane == 0) {
         tg::mbar_arrive_expect_tx(&S.kv_full[s], 2 * kBN * kD * 2);
         const int r0 = seq0 + j * kBN;
@@ -133,39 +168,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mbar_arrive(&S.kv_full[s]);
       ++issued;
     }
-    if (lane == 0 && S.abort_flag) {
+    if (lane == 0 && S.abort_flag) {   // let copies in flight land before the CTA exits
       tg::mbar_wait(&S.q_full, 0, status, nullptr);
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
         tg::mbar_wait(&S.kv_full[j % kStages], (j / kStages) & 1, status, nullptr);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: S_0, S_1, PV_0, S_2, PV_1, ... ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
       const uint32_t q0 = tg::smem_u32(S.q[0]);
-      bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
       auto issue_s = [&](int j) -> bool {
         const int s = j % kStages;
         if (!tg::mbar_wait(&S.kv_full[s], (j / kStages) & 1, status, &S.abort_flag)) return false;
-        if (!kPinTmem && j >= 2 &&
-            !tg::mbar_wait(&S.s_free[j & 1], ((j >> 1) - 1) & 1, status, &S.abort_flag))
-          return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
         const uint32_t d_s = tmem + kColS0 + 128u * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          const uint32_t offk = (kk >> 2) * (kBN * 64 * 2) + (kk & 3) * 32;
           tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
-                          tg::smem_desc_sw128(k0 + offk, 16, 1024), idesc_s, kk != 0);
+                          tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
         tg::mma_commit(&S.s_full[j & 1]);
         return true;
       };
+      bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
       if (alive) alive = issue_s(0);
       for (int j = 0; j < nt && alive; ++j) {
+        // S_{j+1} goes into the buffer that held P_{j-1}; PV_{j-1} was issued before
         if (j + 1 < nt && !issue_s(j + 1)) break;
         if (!tg::mbar_wait(&S.p_full, j & 1, status, &S.abort_flag)) break;
         tg::tc_fence_after();
@@ -173,18 +205,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t v0 = tg::smem_u32(S.v[s][0]);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          // B = V rows 16kk..16kk+15 (MN-major: dh contiguous); the two 64-wide dh
-          // halves are 16 KB apart (LBO), 8-key groups 1024 B apart (SBO)
+          // A = P_j in TMEM (16 keys = 8 packed columns per K step); B = V rows
+          // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
+          // (LBO), 8-key groups 1024 B apart (SBO)
           const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-          if constexpr (kPinTmem) {
-            const uint32_t a_t = tmem + kColS0 + 128u * (j & 1) + kk * 8;
-            tg::mma_bf16_ts(tmem + kColO, a_t, bdesc, idesc_o, (j | kk) != 0);
-          } else {
-            const uint32_t p0 = tg::smem_u32(S.p[0]);
-            const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-            tg::mma_bf16_ss(tmem + kColO, tg::smem_desc_sw128(p0 + off, 16, 1024), bdesc, idesc_o,
-                            (j | kk) != 0);
-          }
+          tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (j & 1) + kk * 8, bdesc, idesc_o,
+                          (j | kk) != 0);
         }
         tg::mma_commit(&S.o_done);
         tg::mma_commit(&S.kv_empty[s]);
@@ -192,46 +218,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- softmax: one query row per thread ----------------
-    const int r = tid - 128;                       // row within the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // ---------------- softmax: two threads per query row ----------------
+    const int g = warp & 3;                        // row group == TMEM lane quarter
+    const int hf = (warp - 4) >> 2;                // which 64-key half of each tile
+    const int r = g * 32 + lane;                   // row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(g * 32) << 16;
     const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_part = 0.f;
     bool alive = true;
     for (int j = 0; j < nt; ++j) {
       const int s = j % kStages;
+      const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (j & 1);
       alive = tg::mbar_wait(&S.s_full[j & 1], (j >> 1) & 1, status, &S.abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
+      // tile j's bias: kv_full[s] completed before S_j was issued and cannot move on
+      // before this thread's p_full(j); waiting makes the producer's stores visible
+      if (alive) alive = tg::mbar_wait(&S.kv_full[s], (j / kStages) & 1, status, &S.abort_flag);
+      if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
-      float z[kBN];
+      float z[kHalf];
       {
-        uint32_t u[32];
+        uint32_t u[kHalf];
+        tg::tmem_ld32(sbuf + hf * kHalf, u);
+        tg::tmem_ld32(sbuf + hf * kHalf + 32, u + 32);
+        tg::tmem_ld_wait();
+        const float4* b4 = reinterpret_cast<const float4*>(S.bias[s] + hf * kHalf);
 #pragma unroll
-        for (int c = 0; c < kBN; c += 32) {
-          tg::tmem_ld32(tmem + lane_base + kColS0 + 128u * (j & 1) + c, u);
-          tg::tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) z[c + e] = __uint_as_float(u[e]);
+        for (int c = 0; c < kHalf; c += 4) {
+          const float4 bb = b4[c / 4];
+          z[c + 0] = fmaf(__uint_as_float(u[c + 0]), c_h, bb.x);
+          z[c + 1] = fmaf(__uint_as_float(u[c + 1]), c_h, bb.y);
+          z[c + 2] = fmaf(__uint_as_float(u[c + 2]), c_h, bb.z);
+          z[c + 3] = fmaf(__uint_as_float(u[c + 3]), c_h, bb.w);
         }
       }
-      tg::tc_fence_before();
-      tg::mbar_arrive(&S.s_free[j & 1]);
-      // the bias of tile j is visible: kv_full[s] completed before S_j was issued
-      const float* bias = S.bias[s];
-      float mt = -INFINITY;
-      if (j == t) {
+      if (j == t) {   // diagonal tile: key hf*64+c is visible to row r iff hf*64+c <= r
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          z[c] = c <= r ? fmaf(z[c], c_h, bias[c]) : -INFINITY;
-          mt = fmaxf(mt, z[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          z[c] = fmaf(z[c], c_h, bias[c]);
-          mt = fmaxf(mt, z[c]);
-        }
+        for (int c = 0; c < kHalf; ++c)
+          if (hf * kHalf + c > r) z[c] = -INFINITY;
       }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = z[i];
+#pragma unroll
+      for (int c = 8; c < kHalf; ++c) mx[c & 7] = fmaxf(mx[c & 7], z[c]);
+      const float mpart = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      S.red[j & 1][hf][r] = mpart;
+      tg::mbar_arrive(&S.red_full[j & 1][g]);
+      alive = tg::mbar_wait(&S.red_full[j & 1][g], (j >> 1) & 1, status, &S.abort_flag);
+      if (!all_alive(alive)) { alive = false; break; }
+      const float mt = fmaxf(S.red[j & 1][0][r], S.red[j & 1][1][r]);
       float m_use = m_run, alpha = 1.f;
       bool rescale = false;
       if (j == 0 || mt > m_run + kRescaleThreshold) {
@@ -241,77 +277,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           rescale = true;
         }
       }
-      float lsum = 0.f;
-      uint32_t pk[kBN / 2];
+      uint32_t pk[kHalf / 2];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = tg::exp2_approx(z[c] - m_use);
-        const float p1 = tg::exp2_approx(z[c + 1] - m_use);
-        lsum += p0 + p1;
-        pk[c / 2] = tg::pack_bf16x2(p0, p1);
+      for (int c = 0; c < kHalf; c += 2) {
+        const float x0 = z[c] - m_use, x1 = z[c + 1] - m_use;
+        const float p0 = (c % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x0) : tg::exp2_approx(x0);
+        const float p1 =
+            ((c + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x1) : tg::exp2_approx(x1);
+        ls[(c >> 1) & 3] += p0 + p1;
+        pk[c >> 1] = tg::pack_bf16x2(p0, p1);
       }
-      l_run = l_run * alpha + lsum;
+      l_part = l_part * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
       m_run = m_use;
-      // O and the P buffer are free once PV_{j-1} has completed
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
+        // O must hold PV_{j-1} before it is scaled (phases <= j-2 are confirmed)
+        alive = tg::mbar_wait(&S.o_done, (j - 1) & 1, status, &S.abort_flag);
+        if (!all_alive(alive)) { alive = false; break; }
+        tg::tc_fence_after();
+        uint32_t o[kHalf];
+        tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf, o);
+        tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf + 32, o + 32);
+        tg::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < kHalf; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+#pragma unroll
+        for (int e = 0; e < kHalf; e += 16) tg::tmem_st16(tmem + lane_base + kColO + hf * kHalf + e, o + e);
+      }
+      // P_j over S_j: this thread's 64 keys -> 32 packed columns (all S reads of the
+      // row finished before the max exchange above)
+      tg::tmem_st16(sbuf + hf * (kHalf / 2), pk);
+      tg::tmem_st16(sbuf + hf * (kHalf / 2) + 16, pk + 16);
+      tg::tmem_st_wait();
+      // confirm PV_{j-1} (keeps the o_done phase tracking exact; normally complete)
       if (j > 0) {
         alive = tg::mbar_wait(&S.o_done, (j - 1) & 1, status, &S.abort_flag);
-        if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
-        tg::tc_fence_after();
-      }
-      if (__any_sync(0xFFFFFFFFu, rescale)) {
-        uint32_t o[32];
-#pragma unroll
-        for (int c = 0; c < kD; c += 32) {
-          tg::tmem_ld32(tmem + lane_base + kColO + c, o);
-          tg::tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tg::tmem_st16(tmem + lane_base + kColO + c, o);
-          tg::tmem_st16(tmem + lane_base + kColO + c + 16, o + 16);
-        }
-        tg::tmem_st_wait();
-      }
-      if constexpr (kPinTmem) {
-        const uint32_t pcol = tmem + lane_base + kColS0 + 128u * (j & 1);
-#pragma unroll
-        for (int c = 0; c < kBN / 2; c += 16) tg::tmem_st16(pcol + c, pk + c);
-        tg::tmem_st_wait();
-      } else {
-        // 128-byte swizzle: 16-byte chunk ch of row r sits at chunk ch ^ (r & 7)
-#pragma unroll
-        for (int ch = 0; ch < kBN / 8; ++ch) {
-          uint8_t* base = S.p[ch >> 3] + r * 128 + ((((ch & 7) ^ (r & 7))) << 4);
-          *reinterpret_cast<uint4*>(base) =
-              make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!all_alive(alive)) { alive = false; break; }
       }
       tg::tc_fence_before();
       tg::mbar_arrive(&S.p_full);
     }
     // ---------------- epilogue: O / l -> bf16 ----------------
+    S.lsum[hf][r] = l_part;
+    tg::mbar_arrive(&S.l_full[g]);
+    if (alive) alive = tg::mbar_wait(&S.l_full[g], 0, status, &S.abort_flag);
     if (alive) alive = tg::mbar_wait(&S.o_done, (nt - 1) & 1, status, &S.abort_flag);
-    if (__all_sync(0xFFFFFFFFu, alive)) {
+    if (all_alive(alive)) {
       tg::tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      const bool valid = t * kBM + r < len;
-      __nv_bfloat16* orow =
-          out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD;
-      uint32_t o[32];
+      const float inv_l = 1.f / (S.lsum[0][r] + S.lsum[1][r]);
+      uint32_t o[kHalf];
+      tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf, o);
+      tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf + 32, o + 32);
+      tg::tmem_ld_wait();
+      if (t * kBM + r < len) {
+        __nv_bfloat16* orow =
+            out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD + hf * kHalf;
 #pragma unroll
-      for (int c = 0; c < kD; c += 32) {
-        tg::tmem_ld32(tmem + lane_base + kColO + c, o);
-        tg::tmem_ld_wait();
-        if (valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 w;
-            w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
-            w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-            w.z = tg::pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
-            w.w = tg::pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c + e) = w;
-          }
+        for (int e = 0; e < kHalf; e += 8) {
+          uint4 w;
+          w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+          w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+          w.z = tg::pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+          w.w = tg::pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+          *reinterpret_cast<uint4*>(orow + e) = w;
         }
       }
     }
@@ -323,6 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::tmem_dealloc(tmem, kTmemCols);
   }
 }
+
+}  // namespace
+
+namespace {
 
 // ---------------- exact fp32 path ----------------
 constexpr int kF32Warps = 4;
@@ -383,7 +415,6 @@ __global__ void __launch_bounds__(kF32Warps * 32)
   }
 }
 
-template <bool kPinTmem>
 tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const float* s_kept,
                            const float* gain, const float* tau, const int32_t* cu_kept, int batch,
                            int64_t total, int max_kept, int n_hq, int n_hkv, void* out,
@@ -404,23 +435,18 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
                        CU_TENSOR_MAP_SWIZZLE_128B))
     return TG_ERR_CUDA;
   const size_t smem = sizeof(AttnSmem) + 1024;
-  if (cudaFuncSetAttribute(gated_attn_bf16_kernel<kPinTmem>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  if (!tg::ensure_smem(reinterpret_cast<const void*>(gated_attn_bf16_kernel),
+                       static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const int n_qt = (max_kept + kBM - 1) / kBM;
   dim3 grid(n_hq, batch, n_qt);
-  gated_attn_bf16_kernel<kPinTmem><<<grid, kThreads, smem, st>>>(
-      tq, tk, tv, s_kept, gain, tau, cu_kept, n_hq, n_hkv, static_cast<__nv_bfloat16*>(out),
-      status);
+  gated_attn_bf16_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, s_kept, gain, tau, cu_kept,
+                                                       n_hq, n_hkv,
+                                                       static_cast<__nv_bfloat16*>(out), status);
   return tg::launch_status();
 }
 
 }  // namespace
-
-// P path of the bf16 kernel: 0 = through shared memory (default), 1 = through TMEM.
-static int g_attn_p_in_tmem = 0;
-extern "C" void tg_internal_set_attn_variant(int p_in_tmem) { g_attn_p_in_tmem = p_in_tmem; }
 
 extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void* v,
                                         tg_dtype dtype, const float* s_kept, const float* gain,
@@ -439,11 +465,8 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
     if (total_kept > INT32_MAX - kBM || (max_kept + kBM - 1) / kBM > 65535) return TG_ERR_UNSUPPORTED;
     if (!tg::aligned16(q) || !tg::aligned16(k) || !tg::aligned16(v) || !tg::aligned16(out))
       return TG_ERR_MISALIGNED;
-    return g_attn_p_in_tmem
-               ? launch_attn_bf16<true>(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept,
-                                        max_kept, n_hq, n_hkv, out, stream)
-               : launch_attn_bf16<false>(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept,
-                                         max_kept, n_hq, n_hkv, out, stream);
+    return launch_attn_bf16(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept, max_kept, n_hq,
+                            n_hkv, out, stream);
   }
   if (dtype == TG_F32) {
     if (head_dim > 256) return TG_ERR_UNSUPPORTED;

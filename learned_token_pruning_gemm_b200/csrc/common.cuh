@@ -278,5 +278,8 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const 
                  CUtensorMapSwizzle swz);
 // map the last CUDA error after a launch to a status
 tg_status launch_status();
+// raise a kernel's dynamic shared memory limit to `bytes` on the current device
+// (cached per device and function)
+bool ensure_smem(const void* fn, int bytes);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 }  // namespace tg

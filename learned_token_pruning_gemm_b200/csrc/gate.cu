@@ -195,8 +195,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
                        CU_TENSOR_MAP_SWIZZLE_128B))
     return TG_ERR_CUDA;
   const size_t smem = sizeof(GateSmem<H>) + 1024;
-  if (cudaFuncSetAttribute(gate_bf16_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const int64_t tiles = (n + kBM - 1) / kBM;
   gate_bf16_kernel<H><<<static_cast<unsigned>(tiles), kThreads, smem, st>>>(tx, tw, b1, w2, b2, n, d,

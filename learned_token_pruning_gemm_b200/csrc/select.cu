@@ -5,13 +5,15 @@
 // déployer TokenGate ?": {state} marks the document, max_kept_prefill_tokens the
 // budget).
 //
-// One thread-block cluster of 8 CTAs per sequence, one launch for the whole
-// batch. Each CTA holds a contiguous eighth of the sequence's scores in shared
-// memory as order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass
-// MSB-first radix select (8-bit digits) finds the exact K-th largest document key
-// T: every pass builds warp-aggregated (match_any) histograms, the 8 CTA
-// histograms are summed through distributed shared memory, and the digit that
-// holds the K-th key is found with a block suffix scan. Emission then keeps every
+// One thread-block cluster per sequence, one launch for the whole batch; the
+// cluster has as many CTAs (1..8) as the longest sequence needs at up to 24576
+// keys per CTA, so a 16k-token sequence runs in one CTA with no cluster traffic.
+// Each CTA holds a contiguous slice of the sequence's scores in shared memory as
+// order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass MSB-first radix
+// select (8-bit digits) finds the exact K-th largest document key T: every pass
+// builds a warp-aggregated (match_any) histogram, the CTA histograms are summed
+// through distributed shared memory, and the digit that holds the K-th key is
+// found with a block suffix scan. Emission then keeps every
 // token outside the span, every document token with key > T, and the `need`
 // lowest-positioned document tokens with key == T (ties to the lower position);
 // the stable output order comes from warp ballots / popc prefix sums, with the
@@ -24,15 +26,14 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int kCluster = 8;
-constexpr int kThreads = 512;
+constexpr int kMaxCluster = 8;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kChunkQuant = kThreads;   // chunk rounded to this -> per-warp segments of 32k
+constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576 keys = 96 KB
 
 struct SelectSmem {
-  uint32_t whist[kWarps][256];   // per-warp histograms
   uint32_t hist[2][256];         // this CTA's histogram, by pass parity (read by peers)
-  uint32_t scan[kWarps];
+  uint32_t scan[8];
   uint32_t warp_tot[kWarps];
   uint32_t warp_off[kWarps];
   uint32_t cta_eq;               // published to peers
@@ -47,10 +48,15 @@ struct SelectSmem {
   // followed by: uint32_t masks[chunk / 32]; uint32_t keys[chunk];
 };
 
-__host__ __device__ inline int select_chunk(int max_len) {
-  int c = (max_len + kCluster - 1) / kCluster;
-  c = (c + kChunkQuant - 1) / kChunkQuant * kChunkQuant;
-  return c < kChunkQuant ? kChunkQuant : c;
+inline int select_cluster(int max_len) {
+  int c = (max_len + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
+  return c < 1 ? 1 : c;
+}
+
+inline int select_chunk(int max_len, int csize) {
+  int c = (max_len + csize - 1) / csize;
+  c = (c + kThreads - 1) / kThreads * kThreads;
+  return c < kThreads ? kThreads : c;
 }
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -75,7 +81,17 @@ __device__ __forceinline__ int64_t seq_kept(const int32_t* cu, const int32_t* db
   return len - nd + k;
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+// exclusive scan of per-warp totals (thread 0), result in warp_off, total returned
+__device__ __forceinline__ uint32_t scan_warp_totals(SelectSmem& S) {
+  uint32_t t = 0;
+  for (int w = 0; w < kWarps; ++w) {
+    S.warp_off[w] = t;
+    t += S.warp_tot[w];
+  }
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     select_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ cu_seqlens,
                        const int32_t* __restrict__ doc_begin, const int32_t* __restrict__ doc_end,
                        const int32_t* __restrict__ k_doc, int batch, int64_t total_kept,
@@ -88,6 +104,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
+  const unsigned csize = cluster.num_blocks();
   const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xFFFFFFFFu;
@@ -97,7 +114,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   const int64_t base = cu_seqlens[b];
   const int64_t len = (int64_t)cu_seqlens[b + 1] - base;
   const int64_t db = doc_begin[b], de = doc_end[b];
-  const bool bad = len < 0 || len > (int64_t)chunk * kCluster || db < 0 || de < db || de > len;
+  const bool bad = len < 0 || len > (int64_t)chunk * csize || db < 0 || de < db || de > len;
   if (bad) {
     if (rank == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
     return;   // uniform across the cluster: nobody reaches a cluster barrier
@@ -107,28 +124,25 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   if (k_eff < 0) k_eff = 0;
   if (k_eff > nd) k_eff = nd;
 
-  // output offset of this sequence: sum of kept counts of earlier sequences
-  {
-    int64_t acc = 0;
-    for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
-    if (lane == 0) S.red[warp] = acc;
-    __syncthreads();
-    if (tid == 0) {
-      int64_t t = 0;
-      for (int w = 0; w < kWarps; ++w) t += S.red[w];
-      S.out_base = t;
-    }
-  }
-
-  // ---- load this CTA's slice as keys ----
+  // ---- load this CTA's slice as keys; meanwhile sum earlier sequences' counts ----
   const int64_t c0 = (int64_t)rank * chunk;
   int64_t n_local = len - c0;
   if (n_local < 0) n_local = 0;
   if (n_local > chunk) n_local = chunk;
   for (int i = tid; i < chunk; i += kThreads)
     keys[i] = i < n_local ? score_key(scores[base + c0 + i]) : 0u;
+  {
+    int64_t acc = 0;
+    for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
+    if (lane == 0) S.red[warp] = acc;
+  }
   __syncthreads();
+  if (tid == 0) {
+    int64_t t = 0;
+    for (int w = 0; w < kWarps; ++w) t += S.red[w];
+    S.out_base = t;
+  }
 
   const int seg = chunk / kWarps;          // multiple of 32
   const int seg0 = warp * seg;
@@ -145,7 +159,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k_eff;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
-      for (int i = tid; i < kWarps * 256; i += kThreads) (&S.whist[0][0])[i] = 0u;
+      uint32_t* h = S.hist[pass & 1];
+      if (tid < 256) h[tid] = 0u;
       __syncthreads();
       for (int i = seg0 + lane; i < seg0 + seg; i += 32) {
         const int64_t pos = c0 + i;
@@ -155,26 +170,19 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         if (valid) {
           const uint32_t digit = (key >> shift) & 0xFFu;
           const unsigned peers = __match_any_sync(act, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&S.whist[warp][digit], (uint32_t)__popc(peers));
+          if (lane == __ffs(peers) - 1) atomicAdd(&h[digit], (uint32_t)__popc(peers));
         }
       }
-      __syncthreads();
-      uint32_t* h = S.hist[pass & 1];
+      cluster.sync();   // every CTA's histogram of this pass is complete
       if (tid < 256) {
-        uint32_t t = 0;
-        for (int w = 0; w < kWarps; ++w) t += S.whist[w][tid];
-        h[tid] = t;
-      }
-      cluster.sync();
-      // thread t holds digit d = 255 - t; an inclusive prefix over t is the
-      // count of document keys (matching the prefix) with digit >= d
-      uint32_t cnt = 0;
-      if (tid < 256) {
+        // thread t holds digit d = 255 - t; an inclusive prefix over t is the
+        // count of matching document keys with digit >= d
         const int d = 255 - tid;
-        for (unsigned r = 0; r < kCluster; ++r) cnt += cluster.map_shared_rank(h, r)[d];
+        uint32_t cnt = 0;
+        for (unsigned r = 0; r < csize; ++r) cnt += cluster.map_shared_rank(h, r)[d];
         uint32_t inc = cnt;
         for (int o = 1; o < 32; o <<= 1) {
-          uint32_t y = __shfl_up_sync(full, inc, o);
+          const uint32_t y = __shfl_up_sync(full, inc, o);
           if (lane >= o) inc += y;
         }
         if (lane == 31) S.scan[warp] = inc;
@@ -192,7 +200,6 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       prefix |= S.digit << shift;
       pmask |= 0xFFu << shift;
       remaining = S.remaining;
-      __syncthreads();
     }
     T = prefix;
     need = remaining;
@@ -210,14 +217,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) S.warp_tot[warp] = cnt;
     __syncthreads();
-    if (tid == 0) {
-      uint32_t t = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        S.warp_off[w] = t;
-        t += S.warp_tot[w];
-      }
-      S.cta_eq = t;
-    }
+    if (tid == 0) S.cta_eq = scan_warp_totals(S);
     cluster.sync();
     if (tid == 0) {
       uint32_t off = 0;
@@ -231,37 +231,27 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   {
     uint32_t running = S.cta_eq_off + S.warp_off[warp];
     uint32_t kept = 0;
-    __syncthreads();   // warp_off is rewritten below
     for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
       const int64_t pos = c0 + i;
       const uint32_t eqm = masks[wi];
       bool keep = false;
       if (i < n_local) {
         const bool in_doc = pos >= db && pos < de;
-        const uint32_t key = keys[i];
         const bool eq = (eqm >> lane) & 1u;
-        keep = !in_doc || key > T || (eq && running + __popc(eqm & lt_mask) < need);
+        keep = !in_doc || keys[i] > T || (eq && running + __popc(eqm & lt_mask) < need);
       }
       running += __popc(eqm);
       const unsigned km = __ballot_sync(full, keep);
-      __syncwarp();
       if (lane == 0) masks[wi] = km;
       kept += __popc(km);
     }
     if (lane == 0) S.warp_tot[warp] = kept;
     __syncthreads();
-    if (tid == 0) {
-      uint32_t t = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        S.warp_off[w] = t;
-        t += S.warp_tot[w];
-      }
-      S.cta_keep = t;
-    }
+    if (tid == 0) S.cta_keep = scan_warp_totals(S);
     cluster.sync();
     if (tid == 0) {
       uint32_t off = 0, tot = 0;
-      for (unsigned r = 0; r < kCluster; ++r) {
+      for (unsigned r = 0; r < csize; ++r) {
         const uint32_t v = *cluster.map_shared_rank(&S.cta_keep, r);
         if (r < rank) off += v;
         tot += v;
@@ -296,7 +286,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     cu_kept[b + 1] = (int32_t)(out_base + expect);
     if (b == batch - 1 && out_base + expect != total_kept) tg::set_status(status, TG_ERR_DEVICE_CHECK);
   }
-  cluster.sync();   // peers may still read this CTA's shared memory until here
+  cluster.sync();   // peers may read this CTA's shared memory until here
 }
 
 }  // namespace
@@ -316,14 +306,26 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   if (batch > 65535) return TG_ERR_UNSUPPORTED;
   int* st = tg::status_word();
   if (!st) return TG_ERR_CUDA;
-  const int chunk = select_chunk(max_seqlen);
+  const int csize = select_cluster(max_seqlen);
+  const int chunk = select_chunk(max_seqlen, csize);
   const size_t smem = sizeof(SelectSmem) + (size_t)chunk / 32 * 4 + (size_t)chunk * 4;
-  if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (!tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem))
     return TG_ERR_CUDA;
-  dim3 grid(kCluster, batch);
-  select_topk_kernel<<<grid, kThreads, smem, stream>>>(scores, cu_seqlens, doc_begin, doc_end,
-                                                       k_doc, batch, total_kept, chunk, kept_idx,
-                                                       kept_scores, cu_kept, st);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize, batch, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, select_topk_kernel, scores, cu_seqlens, doc_begin, doc_end, k_doc,
+                         batch, total_kept, chunk, kept_idx, kept_scores, cu_kept, st) !=
+      cudaSuccess)
+    return TG_ERR_CUDA;
   return tg::launch_status();
 }

@@ -86,3 +86,34 @@ class GatedPrefill:
             fn(stream=s)
         if events is not None:
             events[4].record(s)
+
+    # ------------------------------------------------------------------ graphs
+    def capture(self):
+        """Capture each stage into its own CUDA graph so that replays carry no host
+        launch overhead. One eager step runs first (outside capture) so every
+        lazily initialised piece of the library exists before capture."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step(side)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graphs = []
+        for fn in (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+        return self
+
+    def replay(self, events: Optional[list] = None):
+        """Replay the captured stages on the current stream (same launches as
+        `step`), recording `events` around them like `step` does."""
+        s = torch.cuda.current_stream()
+        for i, g in enumerate(self.graphs):
+            if events is not None:
+                events[i].record(s)
+            g.replay()
+        if events is not None:
+            events[4].record(s)

@@ -198,18 +198,14 @@ def _run_attn(api, q, k, v, s, gain, tau, cu):
                                cu_d, max_kept)
 
 
-@pytest.mark.parametrize("p_in_tmem", [False, True])
-@pytest.mark.parametrize("lens", [[128], [300], [1000], [1868], [513, 1, 129, 700]])
-def test_attention_bf16_vs_oracle(api, orc, lens, p_in_tmem):
-    api.set_attention_variant(p_in_tmem)
-    try:
-        q, k, v, s, gain, tau, cu = _attn_case(sum(lens), lens, 16, 8, 128, torch.bfloat16)
-        out = _run_attn(api, q, k, v, s, gain, tau, cu)
-        rows = sample_rows(cu, 96) if sum(lens) > 1000 else None
-        ref = orc.gated_attention(q, k, v, s, gain, tau, cu, rows=rows)
-        assert_attn_close(out, ref, torch.bfloat16, rows, what=f"lens={lens} tmemP={p_in_tmem}")
-    finally:
-        api.set_attention_variant(False)
+@pytest.mark.parametrize("lens", [[128], [300], [1000], [1868], [513, 1, 129, 700],
+                                  [4000, 260]])
+def test_attention_bf16_vs_oracle(api, orc, lens):
+    q, k, v, s, gain, tau, cu = _attn_case(sum(lens), lens, 16, 8, 128, torch.bfloat16)
+    out = _run_attn(api, q, k, v, s, gain, tau, cu)
+    rows = sample_rows(cu, 96) if sum(lens) > 1000 else None
+    ref = orc.gated_attention(q, k, v, s, gain, tau, cu, rows=rows)
+    assert_attn_close(out, ref, torch.bfloat16, rows, what=f"lens={lens}")
 
 
 def test_attention_bf16_plain_causal_when_gain0_tau1(api, orc):

@@ -84,3 +84,23 @@ def test_gated_layer_matches_oracle(mods, orc, name):
                               rows=arows)
     dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
     assert_attn_close(gp.out, ref, dt, arows, what=name)
+
+
+def test_graph_replay_matches_eager(mods):
+    api, pipeline, synth = mods
+    wl = synth.ragged8()
+    gp = pipeline.GatedPrefill(wl)
+    gp.step()
+    torch.cuda.synchronize()
+    eager = [t.clone() for t in (gp.scores, gp.kept_idx, gp.kept_scores, gp.cu_kept, gp.xc, gp.out)]
+    for t in (gp.scores, gp.kept_scores, gp.out):
+        t.zero_()
+    gp.capture()
+    for t in (gp.scores, gp.kept_scores, gp.out):
+        t.zero_()
+    gp.replay()
+    torch.cuda.synchronize()
+    assert api.device_status(reset=True) == 0
+    got = (gp.scores, gp.kept_idx, gp.kept_scores, gp.cu_kept, gp.xc, gp.out)
+    for a, b in zip(eager, got):
+        assert torch.equal(a, b)
