@@ -6,9 +6,11 @@
 //     z_ij = q_i . k_j / (sqrt(dh) tau_h) + g_h s_j,  j <= i;  O_i = softmax_j(z) V
 //
 // bf16 path (dh = 128), one CTA per (128-row query tile, query head, sequence):
-//   warp 0      TMA producer: the Q tile once, then K/V tiles of 128 keys through
-//               a 2-stage mbarrier ring; its 32 lanes also stage the per-key bias
-//               b_j = log2(e) g_h s_j of each tile in shared memory.
+//   warp 0      TMA producer of Q (once) and of K tiles of 128 keys through a
+//               3-stage ring; its 32 lanes also stage each tile's per-key bias
+//               b_j = log2(e) g_h s_j in shared memory beside the K tile. A K stage
+//               is free once S_j is computed and every softmax warp read the bias.
+//   warp 3      TMA producer of V tiles through a 2-stage ring (free after PV_j).
 //   warp 1      MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
 //               S_j = Q K_j^T into one of two 128-column TMEM buffers, and
 //               O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
@@ -32,7 +34,8 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kD = 128;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
 constexpr int kHalf = kBN / 2;                         // keys per softmax thread
@@ -62,14 +65,16 @@ __device__ __forceinline__ float exp2_fma(float x) {
 
 struct AttnSmem {
   uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves (16 KB each)
-  uint8_t k[kStages][2][kBN * 64 * 2];
-  uint8_t v[kStages][2][kBN * 64 * 2];
-  float bias[kStages][kBN];
+  uint8_t k[kKStages][2][kBN * 64 * 2];
+  uint8_t v[kVStages][2][kBN * 64 * 2];
+  float bias[kKStages][kBN];
   float red[2][2][kBM];                     // [tile parity][half][row] partial maxima
   float lsum[2][kBM];                       // [half][row] final partial row sums
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_empty[kVStages];
   uint64_t s_full[2];
   uint64_t p_full;
   uint64_t o_done;
@@ -111,9 +116,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     tg::mbar_init(&S.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      tg::mbar_init(&S.kv_full[s], 1 + 32);   // expect_tx arrival + 32 bias lanes
-      tg::mbar_init(&S.kv_empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      tg::mbar_init(&S.k_full[s], 1 + 32);                // expect_tx arrival + 32 bias lanes
+      tg::mbar_init(&S.k_empty[s], 1 + kSoftmaxWarps);    // S_j done + bias read by every warp
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      tg::mbar_init(&S.v_full[s], 1);
+      tg::mbar_init(&S.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
     tg::mbar_init(&S.p_full, kSoftmaxWarps * 32);
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0) {
-    // ---------------- TMA producer + bias staging ----------------
+    // ---------------- TMA producer: Q, K tiles + bias staging ----------------
     const float gl2 = gain[hq] * kLog2e;
     int issued = 0;
     if (lane == 0) {
@@ -148,31 +157,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
     }
     for (int j = 0; j < nt; ++j) {
-      const int s = j % kStages;
+      const int s = j % kKStages;
       bool go = true;
-      if (j >= kStages)
-        go = tg::mbar_wait(&S.kv_empty[s], ((j / kStages) - 1) & 1, status, &S.abort_flag);
+      if (j >= kKStages)
+        go = tg::mbar_wait(&S.k_empty[s], ((j / kKStages) - 1) & 1, status, &S.abort_flag);
       if (!all_alive(go)) break;
       if (lane == 0) {
-        tg::mbar_arrive_expect_tx(&S.kv_full[s], 2 * kBN * kD * 2);
+        tg::mbar_arrive_expect_tx(&S.k_full[s], kBN * kD * 2);
         const int r0 = seq0 + j * kBN;
-        tg::tma_load_3d(S.k[s][0], &tm_k, &S.kv_full[s], 0, kvh, r0);
-        tg::tma_load_3d(S.k[s][1], &tm_k, &S.kv_full[s], 64, kvh, r0);
-        tg::tma_load_3d(S.v[s][0], &tm_v, &S.kv_full[s], 0, kvh, r0);
-        tg::tma_load_3d(S.v[s][1], &tm_v, &S.kv_full[s], 64, kvh, r0);
+        tg::tma_load_3d(S.k[s][0], &tm_k, &S.k_full[s], 0, kvh, r0);
+        tg::tma_load_3d(S.k[s][1], &tm_k, &S.k_full[s], 64, kvh, r0);
       }
       for (int c = lane; c < kBN; c += 32) {
         const int kp = j * kBN + c;
         S.bias[s][c] = kp < len ? gl2 * s_kept[seq0 + kp] : 0.f;
       }
-      tg::mbar_arrive(&S.kv_full[s]);
+      tg::mbar_arrive(&S.k_full[s]);
       ++issued;
     }
     if (lane == 0 && S.abort_flag) {   // let copies in flight land before the CTA exits
       tg::mbar_wait(&S.q_full, 0, status, nullptr);
-      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        tg::mbar_wait(&S.kv_full[j % kStages], (j / kStages) & 1, status, nullptr);
+      for (int j = issued > kKStages ? issued - kKStages : 0; j < issued; ++j)
+        tg::mbar_wait(&S.k_full[j % kKStages], (j / kKStages) & 1, status, nullptr);
     }
+  } else if (warp == 3) {
+    // ---------------- TMA producer: V tiles ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kVStages;
+        if (j >= kVStages &&
+            !tg::mbar_wait(&S.v_empty[s], ((j / kVStages) - 1) & 1, status, &S.abort_flag))
+          break;
+        tg::mbar_arrive_expect_tx(&S.v_full[s], kBN * kD * 2);
+        const int r0 = seq0 + j * kBN;
+        tg::tma_load_3d(S.v[s][0], &tm_v, &S.v_full[s], 0, kvh, r0);
+        tg::tma_load_3d(S.v[s][1], &tm_v, &S.v_full[s], 64, kvh, r0);
+        ++issued;
+      }
+      if (S.abort_flag) {
+        for (int j = issued > kVStages ? issued - kVStages : 0; j < issued; ++j)
+          tg::mbar_wait(&S.v_full[j % kVStages], (j / kVStages) & 1, status, nullptr);
+      }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer: S_0, S_1, PV_0, S_2, PV_1, ... ----------------
     if (lane == 0) {
@@ -180,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
       const uint32_t q0 = tg::smem_u32(S.q[0]);
       auto issue_s = [&](int j) -> bool {
-        const int s = j % kStages;
-        if (!tg::mbar_wait(&S.kv_full[s], (j / kStages) & 1, status, &S.abort_flag)) return false;
+        const int s = j % kKStages;
+        if (!tg::mbar_wait(&S.k_full[s], (j / kKStages) & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
         const uint32_t d_s = tmem + kColS0 + 128u * (j & 1);
@@ -192,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
         tg::mma_commit(&S.s_full[j & 1]);
+        tg::mma_commit(&S.k_empty[s]);
         return true;
       };
       bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
@@ -200,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S_{j+1} goes into the buffer that held P_{j-1}; PV_{j-1} was issued before
         if (j + 1 < nt && !issue_s(j + 1)) break;
         if (!tg::mbar_wait(&S.p_full, j & 1, status, &S.abort_flag)) break;
+        const int s = j % kVStages;
+        if (!tg::mbar_wait(&S.v_full[s], (j / kVStages) & 1, status, &S.abort_flag)) break;
         tg::tc_fence_after();
-        const int s = j % kStages;
         const uint32_t v0 = tg::smem_u32(S.v[s][0]);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -213,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (j | kk) != 0);
         }
         tg::mma_commit(&S.o_done);
-        tg::mma_commit(&S.kv_empty[s]);
+        tg::mma_commit(&S.v_empty[s]);
       }
     }
     __syncwarp();
@@ -227,12 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_part = 0.f;
     bool alive = true;
     for (int j = 0; j < nt; ++j) {
-      const int s = j % kStages;
+      const int s = j % kKStages;
       const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (j & 1);
       alive = tg::mbar_wait(&S.s_full[j & 1], (j >> 1) & 1, status, &S.abort_flag);
-      // tile j's bias: kv_full[s] completed before S_j was issued and cannot move on
-      // before this thread's p_full(j); waiting makes the producer's stores visible
-      if (alive) alive = tg::mbar_wait(&S.kv_full[s], (j / kStages) & 1, status, &S.abort_flag);
+      // tile j's bias: k_full[s] completed before S_j was issued and cannot move on
+      // before this warp releases k_empty[s]; waiting makes the producer's stores visible
+      if (alive) alive = tg::mbar_wait(&S.k_full[s], (j / kKStages) & 1, status, &S.abort_flag);
       if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
       float z[kHalf];
@@ -251,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           z[c + 3] = fmaf(__uint_as_float(u[c + 3]), c_h, bb.w);
         }
       }
+      __syncwarp();
+      if (lane == 0) tg::mbar_arrive(&S.k_empty[s]);   // this warp is done with the bias
       if (j == t) {   // diagonal tile: key hf*64+c is visible to row r iff hf*64+c <= r
 #pragma unroll
         for (int c = 0; c < kHalf; ++c)

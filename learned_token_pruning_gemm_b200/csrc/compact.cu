@@ -3,9 +3,9 @@
 // tokens ?": layers above the gate layer process only the K kept tokens).
 //
 // dst[t][r] = src[t][kept_idx[r]] for up to 8 tensors at once. One warp moves one
-// row of every tensor; each lane issues 128-bit non-allocating loads, four in
-// flight before the matching stores, so a 4 KB hidden-state row is 8 fully
-// coalesced 512-byte warp transactions. Pure HBM traffic: 2 * K * row_bytes.
+// row of every tensor; each lane issues 128-bit non-allocating loads, eight in
+// flight before the matching stores, so a 4 KB hidden-state row is one batch of 8
+// fully coalesced 512-byte warp transactions. Pure HBM traffic: 2 * K * row_bytes.
 #include "common.cuh"
 
 namespace {
@@ -41,13 +41,12 @@ __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
       const uint4* s = a.src[t] + sr * nv;
       uint4* d = a.dst[t] + r * nv;
       int64_t v = lane;
-      for (; v + 96 < nv; v += 128) {
-        uint4 x0 = ld_stream(s + v), x1 = ld_stream(s + v + 32);
-        uint4 x2 = ld_stream(s + v + 64), x3 = ld_stream(s + v + 96);
-        d[v] = x0;
-        d[v + 32] = x1;
-        d[v + 64] = x2;
-        d[v + 96] = x3;
+      for (; v + 224 < nv; v += 256) {   // 8 loads in flight per lane before the stores
+        uint4 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = ld_stream(s + v + 32 * u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) d[v + 32 * u] = x[u];
       }
       for (; v < nv; v += 32) d[v] = ld_stream(s + v);
     }

@@ -63,10 +63,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
-  for (int i = tid; i < H; i += kThreads) {
-    S.b1[i] = b1[i];
-    S.w2[i] = w2[i];
-  }
   if (warp == 2) {
     tg::tmem_alloc(&S.tmem_base, H);
     tg::tmem_relinquish();
@@ -113,8 +109,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mma_commit(&S.empty[s]);
     }
     tg::mma_commit(&S.acc_full);
+  } else if (warp >= 2) {
+    // stage the epilogue's constants while the mainloop runs
+    for (int i = tid - 64; i < H; i += kThreads - 64) {
+      S.b1[i] = b1[i];
+      S.w2[i] = w2[i];
+    }
   }
   __syncwarp();
+  tg::named_barrier(1, kThreads);   // b1/w2 staged; producer and MMA loops issued
 
   // ---- epilogue: all 16 warps ----
   constexpr int kCols = H / 4;               // accumulator columns per warp
@@ -124,17 +127,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
   if (ok) {
     tg::tc_fence_after();
+    uint32_t r[kCols];
 #pragma unroll
-    for (int c = 0; c < kCols; c += 16) {
-      uint32_t r[16];
-      tg::tmem_ld16(tmem + (static_cast<uint32_t>(lg * 32) << 16) + cgp * kCols + c, r);
-      tg::tmem_ld_wait();
+    for (int c = 0; c < kCols; c += 16)
+      tg::tmem_ld16(tmem + (static_cast<uint32_t>(lg * 32) << 16) + cgp * kCols + c, r + c);
+    tg::tmem_ld_wait();
+    float a2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int col = cgp * kCols + c + j;
-        acc += S.w2[col] * gelu_erf(__uint_as_float(r[j]) + S.b1[col]);
-      }
+    for (int j = 0; j < kCols; ++j) {
+      const int col = cgp * kCols + j;
+      a2[j & 3] = fmaf(S.w2[col], gelu_erf(__uint_as_float(r[j]) + S.b1[col]), a2[j & 3]);
     }
+    acc = (a2[0] + a2[1]) + (a2[2] + a2[3]);
   }
   S.part[cgp][row] = acc;
   tg::tc_fence_before();

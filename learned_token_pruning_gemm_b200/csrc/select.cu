@@ -11,7 +11,7 @@
 // Each CTA holds a contiguous slice of the sequence's scores in shared memory as
 // order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass MSB-first radix
 // select (8-bit digits) finds the exact K-th largest document key T: every pass
-// builds a warp-aggregated (match_any) histogram, the CTA histograms are summed
+// builds per-warp histograms summed into a CTA histogram, the CTA histograms are summed
 // through distributed shared memory, and the digit that holds the K-th key is
 // found with a block suffix scan. Emission then keeps every
 // token outside the span, every document token with key > T, and the `need`
@@ -32,6 +32,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576 keys = 96 KB
 
 struct SelectSmem {
+  uint32_t whist[kWarps][256];   // per-warp histograms (private: no cross-warp atomics)
   uint32_t hist[2][256];         // this CTA's histogram, by pass parity (read by peers)
   uint32_t scan[8];
   uint32_t warp_tot[kWarps];
@@ -160,18 +161,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       uint32_t* h = S.hist[pass & 1];
-      if (tid < 256) h[tid] = 0u;
-      __syncthreads();
+      uint32_t* wh = S.whist[warp];
+#pragma unroll
+      for (int i = lane; i < 256; i += 32) wh[i] = 0u;
+      __syncwarp();
       for (int i = seg0 + lane; i < seg0 + seg; i += 32) {
         const int64_t pos = c0 + i;
         const uint32_t key = keys[i];
-        const bool valid = i < n_local && pos >= db && pos < de && (key & pmask) == prefix;
-        const unsigned act = __ballot_sync(full, valid);
-        if (valid) {
-          const uint32_t digit = (key >> shift) & 0xFFu;
-          const unsigned peers = __match_any_sync(act, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&h[digit], (uint32_t)__popc(peers));
-        }
+        if (i < n_local && pos >= db && pos < de && (key & pmask) == prefix)
+          atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
+      }
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t c = 0;
+#pragma unroll 8
+        for (int w = 0; w < kWarps; ++w) c += S.whist[w][tid];
+        h[tid] = c;
       }
       cluster.sync();   // every CTA's histogram of this pass is complete
       if (tid < 256) {
