@@ -20,8 +20,9 @@
 //               (one FFMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile mask,
 //               row max exchanged through shared memory, a running max that only
 //               moves when it grows by more than 2^8 (O is then rescaled in TMEM),
-//               exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA pipe
-//               (own polynomial) for the 4th, P packed to bf16 into TMEM.
+//               exp2 on the MUFU pipe for 7 of every 8 keys and on the FMA pipe
+//               (own polynomial) for the 8th, packed f32x2 FMA/ADD for the
+//               scale+bias and the sums, P packed to bf16 into TMEM.
 // Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
 // PV_j and S_{j+2}; the only cross-tile wait is the rare O rescale. Query tiles
 // are launched longest-first (the last tile of a sequence has the most keys).
@@ -41,7 +42,7 @@ constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 s
 constexpr int kHalf = kBN / 2;                         // keys per softmax thread
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
-constexpr int kPolyEvery = 4;               // every 4th key's exp2 on the FMA pipe
+constexpr int kPolyEvery = 8;               // every 8th key's exp2 on the FMA pipe
 
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
 // fit_exp2_poly.py in this directory.
@@ -88,6 +89,29 @@ struct AttnSmem {
 constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
 
 __device__ __forceinline__ bool all_alive(bool a) { return __all_sync(0xFFFFFFFFu, a); }
+
+// packed pair arithmetic (one instruction for two fp32 lanes)
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 }  // namespace
 
@@ -275,10 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kHalf; c += 4) {
           const float4 bb = b4[c / 4];
-          z[c + 0] = fmaf(__uint_as_float(u[c + 0]), c_h, bb.x);
-          z[c + 1] = fmaf(__uint_as_float(u[c + 1]), c_h, bb.y);
-          z[c + 2] = fmaf(__uint_as_float(u[c + 2]), c_h, bb.z);
-          z[c + 3] = fmaf(__uint_as_float(u[c + 3]), c_h, bb.w);
+          ffma2(z[c], z[c + 1], __uint_as_float(u[c]), __uint_as_float(u[c + 1]), c_h, c_h, bb.x,
+                bb.y);
+          ffma2(z[c + 2], z[c + 3], __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]), c_h,
+                c_h, bb.z, bb.w);
         }
       }
       __syncwarp();
@@ -288,13 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kHalf; ++c)
           if (hf * kHalf + c > r) z[c] = -INFINITY;
       }
-      float mx[8];
+      float mx[4] = {z[0], z[1], z[2], z[3]};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = z[i];
-#pragma unroll
-      for (int c = 8; c < kHalf; ++c) mx[c & 7] = fmaxf(mx[c & 7], z[c]);
-      const float mpart = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 4; c < kHalf; c += 8) {
+        mx[0] = fmax3(mx[0], z[c], z[c + 1]);
+        mx[1] = fmax3(mx[1], z[c + 2], z[c + 3]);
+        if (c + 4 < kHalf) {
+          mx[2] = fmax3(mx[2], z[c + 4], z[c + 5]);
+          mx[3] = fmax3(mx[3], z[c + 6], z[c + 7]);
+        }
+      }
+      const float mpart = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
       S.red[j & 1][hf][r] = mpart;
       tg::mbar_arrive(&S.red_full[j & 1][g]);
       alive = tg::mbar_wait(&S.red_full[j & 1][g], (j >> 1) & 1, status, &S.abort_flag);
@@ -311,14 +339,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t pk[kHalf / 2];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nm = -m_use;
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 2) {
-        const float x0 = z[c] - m_use, x1 = z[c + 1] - m_use;
-        const float p0 = (c % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x0) : tg::exp2_approx(x0);
-        const float p1 =
-            ((c + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x1) : tg::exp2_approx(x1);
-        ls[(c >> 1) & 3] += p0 + p1;
+      for (int c = 0; c < kHalf; c += 4) {
+        float x0, x1, x2, x3;
+        fadd2(x0, x1, z[c], z[c + 1], nm, nm);
+        fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
+        const float p0 = (c % kPolyEvery == kPolyEvery - 4) ? exp2_fma(x0) : tg::exp2_approx(x0);
+        const float p1 = tg::exp2_approx(x1);
+        const float p2 = tg::exp2_approx(x2);
+        const float p3 = tg::exp2_approx(x3);
+        const int a = (c >> 2) & 1;
+        fadd2(ls[2 * a], ls[2 * a + 1], ls[2 * a], ls[2 * a + 1], p0, p1);
+        fadd2(ls[2 * a], ls[2 * a + 1], ls[2 * a], ls[2 * a + 1], p2, p3);
         pk[c >> 1] = tg::pack_bf16x2(p0, p1);
+        pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
       }
       l_part = l_part * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
       m_run = m_use;

@@ -8,8 +8,8 @@
 // One thread-block cluster per sequence, one launch for the whole batch; the
 // cluster has as many CTAs (1..8) as the longest sequence needs at up to 24576
 // keys per CTA, so a 16k-token sequence runs in one CTA with no cluster traffic.
-// Each CTA holds a contiguous slice of the sequence's scores in shared memory as
-// order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass MSB-first radix
+// Each CTA holds a contiguous slice of the sequence's scores in shared memory;
+// comparisons use order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass MSB-first radix
 // select (8-bit digits) finds the exact K-th largest document key T: every pass
 // builds per-warp histograms summed into a CTA histogram, the CTA histograms are summed
 // through distributed shared memory, and the digit that holds the K-th key is
@@ -46,7 +46,7 @@ struct SelectSmem {
   uint32_t seq_keep;
   int64_t out_base;
   int64_t red[kWarps];
-  // followed by: uint32_t masks[chunk / 32]; uint32_t keys[chunk];
+  // followed by: uint32_t masks[chunk / 32]; float raw[chunk];
 };
 
 inline int select_cluster(int max_len) {
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
-  uint32_t* keys = masks + chunk / 32;
+  float* raw = reinterpret_cast<float*>(masks + chunk / 32);   // this CTA's scores
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
@@ -130,8 +130,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t n_local = len - c0;
   if (n_local < 0) n_local = 0;
   if (n_local > chunk) n_local = chunk;
-  for (int i = tid; i < chunk; i += kThreads)
-    keys[i] = i < n_local ? score_key(scores[base + c0 + i]) : 0u;
+  for (int i0 = tid; i0 < chunk; i0 += 8 * kThreads) {   // 8 loads in flight per thread
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kThreads;
+      v[u] = i < n_local ? scores[base + c0 + i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kThreads;
+      if (i < chunk) raw[i] = v[u];
+    }
+  }
   {
     int64_t acc = 0;
     for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
@@ -167,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       for (int i = seg0 + lane; i < seg0 + seg; i += 32) {
         const int64_t pos = c0 + i;
-        const uint32_t key = keys[i];
+        const uint32_t key = score_key(raw[i]);
         if (i < n_local && pos >= db && pos < de && (key & pmask) == prefix)
           atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
       }
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t cnt = 0;
     for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
       const int64_t pos = c0 + i;
-      const bool eq = i < n_local && pos >= db && pos < de && keys[i] == T;
+      const bool eq = i < n_local && pos >= db && pos < de && score_key(raw[i]) == T;
       const unsigned m = __ballot_sync(full, eq);
       if (lane == 0) masks[wi] = m;
       cnt += __popc(m);
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i < n_local) {
         const bool in_doc = pos >= db && pos < de;
         const bool eq = (eqm >> lane) & 1u;
-        keep = !in_doc || keys[i] > T || (eq && running + __popc(eqm & lt_mask) < need);
+        keep = !in_doc || score_key(raw[i]) > T || (eq && running + __popc(eqm & lt_mask) < need);
       }
       running += __popc(eqm);
       const unsigned km = __ballot_sync(full, keep);
@@ -280,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t o = running + __popc(km & lt_mask);
         const int64_t row = base + c0 + i;
         kept_idx[o] = (int32_t)row;
-        if (kept_scores) kept_scores[o] = scores[row];
+        if (kept_scores) kept_scores[o] = raw[i];
       }
       running += __popc(km);
     }
