@@ -5,27 +5,29 @@
 // for each query seeing fewer keys).
 //     z_ij = q_i . k_j / (sqrt(dh) tau_h) + g_h s_j,  j <= i;  O_i = softmax_j(z) V
 //
-// bf16 path (dh = 128), one CTA per (128-row query tile, query head, sequence):
-//   warp 0      TMA producer of Q (once) and of K tiles of 128 keys through a
-//               3-stage ring; its 32 lanes also stage each tile's per-key bias
-//               b_j = log2(e) g_h s_j in shared memory beside the K tile. A K stage
-//               is free once S_j is computed and every softmax warp read the bias.
-//   warp 3      TMA producer of V tiles through a 2-stage ring (free after PV_j).
-//   warp 1      MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
-//               S_j = Q K_j^T into one of two 128-column TMEM buffers, and
-//               O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
-//               and V_j as an MN-major shared-memory operand.
-//   warps 4-11  softmax, two threads per query row (TMEM lane = row, each thread
-//               one 64-key half of the tile): z = S c_h + b_j in the log2 domain
-//               (one FFMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile mask,
-//               row max exchanged through shared memory, a running max that only
-//               moves when it grows by more than 2^8 (O is then rescaled in TMEM),
-//               exp2 on the MUFU pipe for 7 of every 8 keys and on the FMA pipe
-//               (own polynomial) for the 8th, packed f32x2 FMA/ADD for the
-//               scale+bias and the sums, P packed to bf16 into TMEM.
+// bf16 path (dh = 128). Causal work grows with the query tile index t (tile t
+// meets t+1 key tiles), so each CTA takes the pair of query tiles t and n-1-t of
+// one (query head, sequence): every CTA then does n+1 key tiles and the grid is
+// balanced. Per CTA, pipelines run across both query tiles:
+//   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
+//                ring; its lanes also stage each tile's per-key bias
+//                b_j = log2(e) g_h s_j beside the K tile. A K stage is free once
+//                S_j is computed and every softmax warp has read the bias.
+//   warp 3       TMA producer of V tiles through a 2-stage ring (free after PV_j).
+//   warp 1       MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
+//                S_j = Q K_j^T into one of two 128-column TMEM buffers, and
+//                O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
+//                and V_j as an MN-major shared-memory operand.
+//   warps 4-19   softmax, four threads per query row (TMEM lane = row, each
+//                thread 32 keys of the tile): z = S c_h + b_j in the log2 domain
+//                (packed f32x2 FMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile
+//                mask, row max exchanged through shared memory, a running max that
+//                moves only when it grows by more than 2^8 (O is then rescaled in
+//                TMEM), exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA
+//                pipe (own polynomial) for the 4th, P packed to bf16 into TMEM.
 // Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
-// PV_j and S_{j+2}; the only cross-tile wait is the rare O rescale. Query tiles
-// are launched longest-first (the last tile of a sequence has the most keys).
+// PV_j and S_{j+2}; the only cross-tile waits are the rare O rescale and, between
+// the two query tiles, the epilogue's read of O before it is overwritten.
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
 #include "common.cuh"
@@ -37,12 +39,12 @@ constexpr int kBN = 128;
 constexpr int kD = 128;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
-constexpr int kHalf = kBN / 2;                         // keys per softmax thread
+constexpr int kSoftmaxWarps = 16;
+constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-19 softmax
+constexpr int kQuarter = kBN / 4;                      // keys per softmax thread
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
-constexpr int kPolyEvery = 8;               // every 8th key's exp2 on the FMA pipe
+constexpr int kPolyEvery = 4;               // every 4th key's exp2 on the FMA pipe
 
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
 // fit_exp2_poly.py in this directory.
@@ -69,9 +71,10 @@ struct AttnSmem {
   uint8_t k[kKStages][2][kBN * 64 * 2];
   uint8_t v[kVStages][2][kBN * 64 * 2];
   float bias[kKStages][kBN];
-  float red[2][2][kBM];                     // [tile parity][half][row] partial maxima
-  float lsum[2][kBM];                       // [half][row] final partial row sums
+  float red[2][4][kBM];                     // [tile parity][quarter][row] partial maxima
+  float lsum[4][kBM];                       // [quarter][row] final partial row sums
   uint64_t q_full;
+  uint64_t q_empty;
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
@@ -79,7 +82,8 @@ struct AttnSmem {
   uint64_t s_full[2];
   uint64_t p_full;
   uint64_t o_done;
-  uint64_t red_full[2][4];                  // [tile parity][row group]: the two halves of a row
+  uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
+  uint64_t red_full[2][4];                  // [tile parity][row group]: the four quarters of a row
   uint64_t l_full[4];                       // [row group]: final row-sum exchange
   uint32_t tmem_base;
   int abort_flag;
@@ -126,12 +130,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                            int n_hq, int n_hkv, __nv_bfloat16* __restrict__ out, int* status) {
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
-  const int t = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);   // longest first
+  const int z = blockIdx.z;
   const int seq0 = cu_kept[b];
   const int len = cu_kept[b + 1] - seq0;
-  if (t * kBM >= len) return;   // uniform: this sequence has no tile t
+  const int n_t = (len + kBM - 1) / kBM;
+  if (2 * z >= n_t) return;     // uniform: this sequence has no pair z
+  // the CTA's query tiles: the long one first, then its partner (if distinct)
+  const int tiles[2] = {n_t - 1 - z, z};
+  const int nq = (tiles[1] < tiles[0]) ? 2 : 1;
   const int kvh = hq / (n_hq / n_hkv);
-  const int nt = t + 1;         // causal: key tiles 0..t
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -140,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     tg::mbar_init(&S.q_full, 1);
+    tg::mbar_init(&S.q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
       tg::mbar_init(&S.k_full[s], 1 + 32);                // expect_tx arrival + 32 bias lanes
       tg::mbar_init(&S.k_empty[s], 1 + kSoftmaxWarps);    // S_j done + bias read by every warp
@@ -149,11 +157,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mbar_init(&S.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
-    tg::mbar_init(&S.p_full, kSoftmaxWarps * 32);
+    tg::mbar_init(&S.p_full, kSoftmaxWarps);
     tg::mbar_init(&S.o_done, 1);
+    tg::mbar_init(&S.o_free, kSoftmaxWarps);
     for (int s = 0; s < 2; ++s)
-      for (int g = 0; g < 4; ++g) tg::mbar_init(&S.red_full[s][g], 64);
-    for (int g = 0; g < 4; ++g) tg::mbar_init(&S.l_full[g], 64);
+      for (int g = 0; g < 4; ++g) tg::mbar_init(&S.red_full[s][g], 4);
+    for (int g = 0; g < 4; ++g) tg::mbar_init(&S.l_full[g], 4);
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
@@ -164,8 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tg::tma_prefetch_desc(&tm_q);
     tg::tma_prefetch_desc(&tm_k);
-    tg::tma_prefetch_desc(&tm_v);
   }
+  if (warp == 3 && lane == 0) tg::tma_prefetch_desc(&tm_v);
   tg::tc_fence_before();
   __syncthreads();
   tg::tc_fence_after();
@@ -174,30 +183,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer: Q, K tiles + bias staging ----------------
     const float gl2 = gain[hq] * kLog2e;
-    int issued = 0;
-    if (lane == 0) {
-      tg::mbar_arrive_expect_tx(&S.q_full, kBM * kD * 2);
-      tg::tma_load_3d(S.q[0], &tm_q, &S.q_full, 0, hq, seq0 + t * kBM);
-      tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
-    }
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % kKStages;
-      bool go = true;
-      if (j >= kKStages)
-        go = tg::mbar_wait(&S.k_empty[s], ((j / kKStages) - 1) & 1, status, &S.abort_flag);
-      if (!all_alive(go)) break;
+    int g = 0, issued = 0;
+    bool go = true;
+    for (int qi = 0; qi < nq && go; ++qi) {
+      const int t = tiles[qi];
+      if (qi > 0) go = all_alive(tg::mbar_wait(&S.q_empty, 0, status, &S.abort_flag));
+      if (!go) break;
       if (lane == 0) {
-        tg::mbar_arrive_expect_tx(&S.k_full[s], kBN * kD * 2);
-        const int r0 = seq0 + j * kBN;
-        tg::tma_load_3d(S.k[s][0], &tm_k, &S.k_full[s], 0, kvh, r0);
-        tg::tma_load_3d(S.k[s][1], &tm_k, &S.k_full[s], 64, kvh, r0);
+        tg::mbar_arrive_expect_tx(&S.q_full, kBM * kD * 2);
+        tg::tma_load_3d(S.q[0], &tm_q, &S.q_full, 0, hq, seq0 + t * kBM);
+        tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
       }
-      for (int c = lane; c < kBN; c += 32) {
-        const int kp = j * kBN + c;
-        S.bias[s][c] = kp < len ? gl2 * s_kept[seq0 + kp] : 0.f;
+      for (int j = 0; j <= t; ++j, ++g) {
+        const int s = g % kKStages;
+        if (g >= kKStages)
+          go = all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
+                                       &S.abort_flag));
+        if (!go) break;
+        if (lane == 0) {
+          tg::mbar_arrive_expect_tx(&S.k_full[s], kBN * kD * 2);
+          const int r0 = seq0 + j * kBN;
+          tg::tma_load_3d(S.k[s][0], &tm_k, &S.k_full[s], 0, kvh, r0);
+          tg::tma_load_3d(S.k[s][1], &tm_k, &S.k_full[s], 64, kvh, r0);
+        }
+        for (int c = lane; c < kBN; c += 32) {
+          const int kp = j * kBN + c;
+          S.bias[s][c] = kp < len ? gl2 * s_kept[seq0 + kp] : 0.f;
+        }
+        tg::mbar_arrive(&S.k_full[s]);
+        ++issued;
       }
-      tg::mbar_arrive(&S.k_full[s]);
-      ++issued;
     }
     if (lane == 0 && S.abort_flag) {   // let copies in flight land before the CTA exits
       tg::mbar_wait(&S.q_full, 0, status, nullptr);
@@ -207,20 +222,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 3) {
     // ---------------- TMA producer: V tiles ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        const int s = j % kVStages;
-        if (j >= kVStages &&
-            !tg::mbar_wait(&S.v_empty[s], ((j / kVStages) - 1) & 1, status, &S.abort_flag))
-          break;
-        tg::mbar_arrive_expect_tx(&S.v_full[s], kBN * kD * 2);
-        const int r0 = seq0 + j * kBN;
-        tg::tma_load_3d(S.v[s][0], &tm_v, &S.v_full[s], 0, kvh, r0);
-        tg::tma_load_3d(S.v[s][1], &tm_v, &S.v_full[s], 64, kvh, r0);
-        ++issued;
+      int g = 0;
+      bool go = true;
+      for (int qi = 0; qi < nq && go; ++qi) {
+        for (int j = 0; j <= tiles[qi]; ++j, ++g) {
+          const int s = g % kVStages;
+          if (g >= kVStages &&
+              !tg::mbar_wait(&S.v_empty[s], ((g / kVStages) - 1) & 1, status, &S.abort_flag)) {
+            go = false;
+            break;
+          }
+          tg::mbar_arrive_expect_tx(&S.v_full[s], kBN * kD * 2);
+          const int r0 = seq0 + j * kBN;
+          tg::tma_load_3d(S.v[s][0], &tm_v, &S.v_full[s], 0, kvh, r0);
+          tg::tma_load_3d(S.v[s][1], &tm_v, &S.v_full[s], 64, kvh, r0);
+        }
       }
       if (S.abort_flag) {
-        for (int j = issued > kVStages ? issued - kVStages : 0; j < issued; ++j)
+        for (int j = g > kVStages ? g - kVStages : 0; j < g; ++j)
           tg::mbar_wait(&S.v_full[j % kVStages], (j / kVStages) & 1, status, nullptr);
       }
     }
@@ -231,176 +250,203 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
       const uint32_t q0 = tg::smem_u32(S.q[0]);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % kKStages;
-        if (!tg::mbar_wait(&S.k_full[s], (j / kKStages) & 1, status, &S.abort_flag)) return false;
+      auto issue_s = [&](int g) -> bool {
+        const int s = g % kKStages;
+        if (!tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
-        const uint32_t d_s = tmem + kColS0 + 128u * (j & 1);
+        const uint32_t d_s = tmem + kColS0 + 128u * (g & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
           tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
                           tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
-        tg::mma_commit(&S.s_full[j & 1]);
+        tg::mma_commit(&S.s_full[g & 1]);
         tg::mma_commit(&S.k_empty[s]);
         return true;
       };
-      bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
-      if (alive) alive = issue_s(0);
-      for (int j = 0; j < nt && alive; ++j) {
-        // S_{j+1} goes into the buffer that held P_{j-1}; PV_{j-1} was issued before
-        if (j + 1 < nt && !issue_s(j + 1)) break;
-        if (!tg::mbar_wait(&S.p_full, j & 1, status, &S.abort_flag)) break;
-        const int s = j % kVStages;
-        if (!tg::mbar_wait(&S.v_full[s], (j / kVStages) & 1, status, &S.abort_flag)) break;
-        tg::tc_fence_after();
-        const uint32_t v0 = tg::smem_u32(S.v[s][0]);
+      bool alive = true;
+      int g0 = 0;
+      for (int qi = 0; qi < nq && alive; ++qi) {
+        const int nt = tiles[qi] + 1;
+        alive = tg::mbar_wait(&S.q_full, qi & 1, status, &S.abort_flag);
+        if (alive) alive = issue_s(g0);
+        for (int j = 0; j < nt && alive; ++j) {
+          const int g = g0 + j;
+          // S_{g+1} goes into the buffer that held P_{g-1}; PV_{g-1} was issued before
+          if (j + 1 < nt) {
+            if (!issue_s(g + 1)) { alive = false; break; }
+          } else {
+            tg::mma_commit(&S.q_empty);   // every S of this query tile is issued
+          }
+          if (!tg::mbar_wait(&S.p_full, g & 1, status, &S.abort_flag)) { alive = false; break; }
+          const int s = g % kVStages;
+          if (!tg::mbar_wait(&S.v_full[s], (g / kVStages) & 1, status, &S.abort_flag)) {
+            alive = false;
+            break;
+          }
+          if (j == 0 && qi > 0 &&
+              !tg::mbar_wait(&S.o_free, (qi - 1) & 1, status, &S.abort_flag)) {
+            alive = false;
+            break;
+          }
+          tg::tc_fence_after();
+          const uint32_t v0 = tg::smem_u32(S.v[s][0]);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = P_j in TMEM (16 keys = 8 packed columns per K step); B = V rows
-          // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
-          // (LBO), 8-key groups 1024 B apart (SBO)
-          const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-          tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (j & 1) + kk * 8, bdesc, idesc_o,
-                          (j | kk) != 0);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // A = P_g in TMEM (16 keys = 8 packed columns per K step); B = V rows
+            // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
+            // (LBO), 8-key groups 1024 B apart (SBO)
+            const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
+            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g & 1) + kk * 8, bdesc,
+                            idesc_o, (j | kk) != 0);
+          }
+          tg::mma_commit(&S.o_done);
+          tg::mma_commit(&S.v_empty[s]);
         }
-        tg::mma_commit(&S.o_done);
-        tg::mma_commit(&S.v_empty[s]);
+        g0 += nt;
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- softmax: two threads per query row ----------------
-    const int g = warp & 3;                        // row group == TMEM lane quarter
-    const int hf = (warp - 4) >> 2;                // which 64-key half of each tile
-    const int r = g * 32 + lane;                   // row within the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(g * 32) << 16;
+    // ---------------- softmax: four threads per query row ----------------
+    const int grp = warp & 3;                      // row group == TMEM lane quarter
+    const int qq = (warp - 4) >> 2;                // which 32-key quarter of each tile
+    const int r = grp * 32 + lane;                 // row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(grp * 32) << 16;
     const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
-    float m_run = -INFINITY, l_part = 0.f;
     bool alive = true;
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % kKStages;
-      const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (j & 1);
-      alive = tg::mbar_wait(&S.s_full[j & 1], (j >> 1) & 1, status, &S.abort_flag);
-      // tile j's bias: k_full[s] completed before S_j was issued and cannot move on
-      // before this warp releases k_empty[s]; waiting makes the producer's stores visible
-      if (alive) alive = tg::mbar_wait(&S.k_full[s], (j / kKStages) & 1, status, &S.abort_flag);
-      if (!all_alive(alive)) { alive = false; break; }
-      tg::tc_fence_after();
-      float z[kHalf];
-      {
-        uint32_t u[kHalf];
-        tg::tmem_ld32(sbuf + hf * kHalf, u);
-        tg::tmem_ld32(sbuf + hf * kHalf + 32, u + 32);
-        tg::tmem_ld_wait();
-        const float4* b4 = reinterpret_cast<const float4*>(S.bias[s] + hf * kHalf);
-#pragma unroll
-        for (int c = 0; c < kHalf; c += 4) {
-          const float4 bb = b4[c / 4];
-          ffma2(z[c], z[c + 1], __uint_as_float(u[c]), __uint_as_float(u[c + 1]), c_h, c_h, bb.x,
-                bb.y);
-          ffma2(z[c + 2], z[c + 3], __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]), c_h,
-                c_h, bb.z, bb.w);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.k_empty[s]);   // this warp is done with the bias
-      if (j == t) {   // diagonal tile: key hf*64+c is visible to row r iff hf*64+c <= r
-#pragma unroll
-        for (int c = 0; c < kHalf; ++c)
-          if (hf * kHalf + c > r) z[c] = -INFINITY;
-      }
-      float mx[4] = {z[0], z[1], z[2], z[3]};
-#pragma unroll
-      for (int c = 4; c < kHalf; c += 8) {
-        mx[0] = fmax3(mx[0], z[c], z[c + 1]);
-        mx[1] = fmax3(mx[1], z[c + 2], z[c + 3]);
-        if (c + 4 < kHalf) {
-          mx[2] = fmax3(mx[2], z[c + 4], z[c + 5]);
-          mx[3] = fmax3(mx[3], z[c + 6], z[c + 7]);
-        }
-      }
-      const float mpart = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-      S.red[j & 1][hf][r] = mpart;
-      tg::mbar_arrive(&S.red_full[j & 1][g]);
-      alive = tg::mbar_wait(&S.red_full[j & 1][g], (j >> 1) & 1, status, &S.abort_flag);
-      if (!all_alive(alive)) { alive = false; break; }
-      const float mt = fmaxf(S.red[j & 1][0][r], S.red[j & 1][1][r]);
-      float m_use = m_run, alpha = 1.f;
-      bool rescale = false;
-      if (j == 0 || mt > m_run + kRescaleThreshold) {
-        m_use = fmaxf(m_run, mt);
-        if (j > 0) {
-          alpha = tg::exp2_approx(m_run - m_use);
-          rescale = true;
-        }
-      }
-      uint32_t pk[kHalf / 2];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      const float nm = -m_use;
-#pragma unroll
-      for (int c = 0; c < kHalf; c += 4) {
-        float x0, x1, x2, x3;
-        fadd2(x0, x1, z[c], z[c + 1], nm, nm);
-        fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
-        const float p0 = (c % kPolyEvery == kPolyEvery - 4) ? exp2_fma(x0) : tg::exp2_approx(x0);
-        const float p1 = tg::exp2_approx(x1);
-        const float p2 = tg::exp2_approx(x2);
-        const float p3 = tg::exp2_approx(x3);
-        const int a = (c >> 2) & 1;
-        fadd2(ls[2 * a], ls[2 * a + 1], ls[2 * a], ls[2 * a + 1], p0, p1);
-        fadd2(ls[2 * a], ls[2 * a + 1], ls[2 * a], ls[2 * a + 1], p2, p3);
-        pk[c >> 1] = tg::pack_bf16x2(p0, p1);
-        pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
-      }
-      l_part = l_part * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-      m_run = m_use;
-      if (__any_sync(0xFFFFFFFFu, rescale)) {
-        // O must hold PV_{j-1} before it is scaled (phases <= j-2 are confirmed)
-        alive = tg::mbar_wait(&S.o_done, (j - 1) & 1, status, &S.abort_flag);
+    int g0 = 0;
+    for (int qi = 0; qi < nq && alive; ++qi) {
+      const int t = tiles[qi];
+      const int nt = t + 1;
+      float m_run = -INFINITY, l_part = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        const int g = g0 + j;
+        const int s = g % kKStages;
+        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g & 1);
+        alive = tg::mbar_wait(&S.s_full[g & 1], (g >> 1) & 1, status, &S.abort_flag);
+        // tile g's bias: k_full[s] completed before S_g was issued and cannot move on
+        // before this warp releases k_empty[s]; waiting makes the producer's stores visible
+        if (alive) alive = tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag);
         if (!all_alive(alive)) { alive = false; break; }
         tg::tc_fence_after();
-        uint32_t o[kHalf];
-        tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf, o);
-        tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf + 32, o + 32);
-        tg::tmem_ld_wait();
+        float z[kQuarter];
+        {
+          uint32_t u[kQuarter];
+          tg::tmem_ld32(sbuf + qq * kQuarter, u);
+          tg::tmem_ld_wait();
+          const float4* b4 = reinterpret_cast<const float4*>(S.bias[s] + qq * kQuarter);
 #pragma unroll
-        for (int e = 0; e < kHalf; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          for (int c = 0; c < kQuarter; c += 4) {
+            const float4 bb = b4[c / 4];
+            ffma2(z[c], z[c + 1], __uint_as_float(u[c]), __uint_as_float(u[c + 1]), c_h, c_h,
+                  bb.x, bb.y);
+            ffma2(z[c + 2], z[c + 3], __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]), c_h,
+                  c_h, bb.z, bb.w);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) tg::mbar_arrive(&S.k_empty[s]);   // this warp is done with the bias
+        if (j == t) {   // diagonal tile: key qq*32+c is visible to row r iff qq*32+c <= r
 #pragma unroll
-        for (int e = 0; e < kHalf; e += 16) tg::tmem_st16(tmem + lane_base + kColO + hf * kHalf + e, o + e);
-      }
-      // P_j over S_j: this thread's 64 keys -> 32 packed columns (all S reads of the
-      // row finished before the max exchange above)
-      tg::tmem_st16(sbuf + hf * (kHalf / 2), pk);
-      tg::tmem_st16(sbuf + hf * (kHalf / 2) + 16, pk + 16);
-      tg::tmem_st_wait();
-      // confirm PV_{j-1} (keeps the o_done phase tracking exact; normally complete)
-      if (j > 0) {
-        alive = tg::mbar_wait(&S.o_done, (j - 1) & 1, status, &S.abort_flag);
+          for (int c = 0; c < kQuarter; ++c)
+            if (qq * kQuarter + c > r) z[c] = -INFINITY;
+        }
+        float mx[4] = {z[0], z[1], z[2], z[3]};
+#pragma unroll
+        for (int c = 4; c < kQuarter; c += 8) {
+          mx[0] = fmax3(mx[0], z[c], z[c + 1]);
+          mx[1] = fmax3(mx[1], z[c + 2], z[c + 3]);
+          if (c + 4 < kQuarter) {
+            mx[2] = fmax3(mx[2], z[c + 4], z[c + 5]);
+            mx[3] = fmax3(mx[3], z[c + 6], z[c + 7]);
+          }
+        }
+        S.red[g & 1][qq][r] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+        __syncwarp();
+        if (lane == 0) tg::mbar_arrive(&S.red_full[g & 1][grp]);
+        alive = tg::mbar_wait(&S.red_full[g & 1][grp], (g >> 1) & 1, status, &S.abort_flag);
         if (!all_alive(alive)) { alive = false; break; }
+        const float mt = fmaxf(fmaxf(S.red[g & 1][0][r], S.red[g & 1][1][r]),
+                               fmaxf(S.red[g & 1][2][r], S.red[g & 1][3][r]));
+        float m_use = m_run, alpha = 1.f;
+        bool rescale = false;
+        if (j == 0 || mt > m_run + kRescaleThreshold) {
+          m_use = fmaxf(m_run, mt);
+          if (j > 0) {
+            alpha = tg::exp2_approx(m_run - m_use);
+            rescale = true;
+          }
+        }
+        uint32_t pk[kQuarter / 2];
+        float ls[2] = {0.f, 0.f};
+        const float nm = -m_use;
+#pragma unroll
+        for (int c = 0; c < kQuarter; c += 4) {
+          float x0, x1, x2, x3;
+          fadd2(x0, x1, z[c], z[c + 1], nm, nm);
+          fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
+          const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
+          const float p1 = tg::exp2_approx(x1);
+          const float p2 = tg::exp2_approx(x2);
+          const float p3 = tg::exp2_approx(x3);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
+          pk[c >> 1] = tg::pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
+        }
+        l_part = l_part * alpha + (ls[0] + ls[1]);
+        m_run = m_use;
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+          // O must hold PV_{g-1} before it is scaled (phases <= g-2 are confirmed)
+          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
+          if (!all_alive(alive)) { alive = false; break; }
+          tg::tc_fence_after();
+          uint32_t o[kQuarter];
+          tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
+          tg::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < kQuarter; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter, o);
+          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter + 16, o + 16);
+        }
+        // P_g over S_g: this thread's 32 keys -> 16 packed columns (every S read of
+        // the row finished before the max exchange above)
+        tg::tmem_st16(sbuf + qq * (kQuarter / 2), pk);
+        tg::tmem_st_wait();
+        // confirm PV_{g-1} (keeps the o_done phase tracking exact; normally complete)
+        if (j > 0) {
+          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
+          if (!all_alive(alive)) { alive = false; break; }
+        }
+        tg::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tg::mbar_arrive(&S.p_full);
       }
-      tg::tc_fence_before();
-      tg::mbar_arrive(&S.p_full);
-    }
-    // ---------------- epilogue: O / l -> bf16 ----------------
-    S.lsum[hf][r] = l_part;
-    tg::mbar_arrive(&S.l_full[g]);
-    if (alive) alive = tg::mbar_wait(&S.l_full[g], 0, status, &S.abort_flag);
-    if (alive) alive = tg::mbar_wait(&S.o_done, (nt - 1) & 1, status, &S.abort_flag);
-    if (all_alive(alive)) {
+      if (!alive) break;
+      // ---------------- epilogue of this query tile: O / l -> bf16 ----------------
+      const int g_last = g0 + nt - 1;
+      S.lsum[qq][r] = l_part;
+      __syncwarp();
+      if (lane == 0) tg::mbar_arrive(&S.l_full[grp]);
+      alive = tg::mbar_wait(&S.l_full[grp], qi & 1, status, &S.abort_flag);
+      if (alive) alive = tg::mbar_wait(&S.o_done, g_last & 1, status, &S.abort_flag);
+      if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
-      const float inv_l = 1.f / (S.lsum[0][r] + S.lsum[1][r]);
-      uint32_t o[kHalf];
-      tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf, o);
-      tg::tmem_ld32(tmem + lane_base + kColO + hf * kHalf + 32, o + 32);
+      const float inv_l = 1.f / ((S.lsum[0][r] + S.lsum[1][r]) + (S.lsum[2][r] + S.lsum[3][r]));
+      uint32_t o[kQuarter];
+      tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
       tg::tmem_ld_wait();
+      tg::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tg::mbar_arrive(&S.o_free);   // O may now be overwritten
       if (t * kBM + r < len) {
         __nv_bfloat16* orow =
-            out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD + hf * kHalf;
+            out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD + qq * kQuarter;
 #pragma unroll
-        for (int e = 0; e < kHalf; e += 8) {
+        for (int e = 0; e < kQuarter; e += 8) {
           uint4 w;
           w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
           w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
@@ -409,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(orow + e) = w;
         }
       }
+      g0 += nt;
     }
   }
   tg::tc_fence_before();
@@ -506,7 +553,7 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
                        static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const int n_qt = (max_kept + kBM - 1) / kBM;
-  dim3 grid(n_hq, batch, n_qt);
+  dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
   gated_attn_bf16_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, s_kept, gain, tau, cu_kept,
                                                        n_hq, n_hkv,
                                                        static_cast<__nv_bfloat16*>(out), status);

@@ -5,10 +5,11 @@
 //
 // bf16 path: one CTA per 128-token tile computes the whole hidden layer
 // (M=128 tokens x N=h units x K=d) with tcgen05.mma (kind::f16, f32 accumulate)
-// into a 128 x h fp32 accumulator in tensor memory. A TMA producer thread streams
-// 128x64 tiles of x and hx64 tiles of w1 (128-byte swizzle) through a 4-stage
-// mbarrier ring; one MMA thread issues 4 K=16 MMAs per stage and frees the stage
-// with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
+// into a 128 x h fp32 accumulator in tensor memory. Two TMA producer threads
+// stream 128x64 tiles of x (from HBM, a deep 6-stage ring so enough bytes are in
+// flight to cover HBM latency) and hx64 tiles of w1 (shared by every CTA, served
+// from L2, 3 stages), both 128-byte swizzled; one MMA thread issues 4 K=16 MMAs
+// per k-block and frees each stage with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
 // accumulator (warp w: lanes 32*(w%4).., a quarter of the columns), add b1, apply
 // exact erf-GELU and dot with w2; the four column partials are summed in a fixed
 // order, so a token's score depends only on its own row.
@@ -20,18 +21,21 @@ namespace {
 
 constexpr int kBM = 128;      // tokens per tile
 constexpr int kBK = 64;       // reduction columns per stage (128 bytes of bf16)
-constexpr int kStages = 4;
+constexpr int kXStages = 6;
+constexpr int kWStages = 3;
 constexpr int kThreads = 512;
 
 template <int H>
 struct GateSmem {
-  uint8_t a[kStages][kBM * kBK * 2];   // x tiles, 16 KB each
-  uint8_t b[kStages][H * kBK * 2];     // w1 tiles
+  uint8_t a[kXStages][kBM * kBK * 2];  // x tiles, 16 KB each
+  uint8_t b[kWStages][H * kBK * 2];    // w1 tiles
   float b1[H];
   float w2[H];
   float part[4][kBM];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t x_full[kXStages];
+  uint64_t x_empty[kXStages];
+  uint64_t w_full[kWStages];
+  uint64_t w_empty[kWStages];
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
@@ -55,9 +59,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = d / kBK;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      tg::mbar_init(&S.full[s], 1);
-      tg::mbar_init(&S.empty[s], 1);
+    for (int s = 0; s < kXStages; ++s) {
+      tg::mbar_init(&S.x_full[s], 1);
+      tg::mbar_init(&S.x_empty[s], 1);
+    }
+    for (int s = 0; s < kWStages; ++s) {
+      tg::mbar_init(&S.w_full[s], 1);
+      tg::mbar_init(&S.w_empty[s], 1);
     }
     tg::mbar_init(&S.acc_full, 1);
     S.abort_flag = 0;
@@ -67,51 +75,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::tmem_alloc(&S.tmem_base, H);
     tg::tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
-    tg::tma_prefetch_desc(&tm_x);
-    tg::tma_prefetch_desc(&tm_w);
-  }
+  if (warp == 0 && lane == 0) tg::tma_prefetch_desc(&tm_x);
+  if (warp == 3 && lane == 0) tg::tma_prefetch_desc(&tm_w);
   tg::tc_fence_before();
   __syncthreads();
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer ----
+    // ---- TMA producer: x tiles ----
     int issued = 0;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      if (kb >= kStages &&
-          !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
+      const int s = kb % kXStages;
+      if (kb >= kXStages &&
+          !tg::mbar_wait(&S.x_empty[s], ((kb / kXStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H) * kBK * 2);
-      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
-      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, 0);
+      tg::mbar_arrive_expect_tx(&S.x_full[s], kBM * kBK * 2);
+      tg::tma_load_2d(S.a[s], &tm_x, &S.x_full[s], kb * kBK, static_cast<int>(m0));
       ++issued;
     }
     if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
-      for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
-        tg::mbar_wait(&S.full[kb % kStages], (kb / kStages) & 1, status, nullptr);
+      for (int kb = issued > kXStages ? issued - kXStages : 0; kb < issued; ++kb)
+        tg::mbar_wait(&S.x_full[kb % kXStages], (kb / kXStages) & 1, status, nullptr);
+    }
+  } else if (warp == 3 && lane == 0) {
+    // ---- TMA producer: w1 tiles ----
+    int issued = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kWStages;
+      if (kb >= kWStages &&
+          !tg::mbar_wait(&S.w_empty[s], ((kb / kWStages) - 1) & 1, status, &S.abort_flag))
+        break;
+      tg::mbar_arrive_expect_tx(&S.w_full[s], H * kBK * 2);
+      tg::tma_load_2d(S.b[s], &tm_w, &S.w_full[s], kb * kBK, 0);
+      ++issued;
+    }
+    if (S.abort_flag) {
+      for (int kb = issued > kWStages ? issued - kWStages : 0; kb < issued; ++kb)
+        tg::mbar_wait(&S.w_full[kb % kWStages], (kb / kWStages) & 1, status, nullptr);
     }
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer ----
     constexpr uint32_t idesc = tg::idesc_bf16_f32(kBM, H, false, false);
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+      const int sx = kb % kXStages, sw = kb % kWStages;
+      if (!tg::mbar_wait(&S.x_full[sx], (kb / kXStages) & 1, status, &S.abort_flag)) break;
+      if (!tg::mbar_wait(&S.w_full[sw], (kb / kWStages) & 1, status, &S.abort_flag)) break;
       tg::tc_fence_after();
-      const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
+      const uint32_t a0 = tg::smem_u32(S.a[sx]), b0 = tg::smem_u32(S.b[sw]);
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
         tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
                         tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
       }
-      tg::mma_commit(&S.empty[s]);
+      tg::mma_commit(&S.x_empty[sx]);
+      tg::mma_commit(&S.w_empty[sw]);
     }
     tg::mma_commit(&S.acc_full);
-  } else if (warp >= 2) {
+  } else if (warp >= 4) {
     // stage the epilogue's constants while the mainloop runs
-    for (int i = tid - 64; i < H; i += kThreads - 64) {
+    for (int i = tid - 128; i < H; i += kThreads - 128) {
       S.b1[i] = b1[i];
       S.w2[i] = w2[i];
     }

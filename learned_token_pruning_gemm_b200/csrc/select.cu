@@ -5,19 +5,22 @@
 // déployer TokenGate ?": {state} marks the document, max_kept_prefill_tokens the
 // budget).
 //
-// One thread-block cluster per sequence, one launch for the whole batch; the
-// cluster has as many CTAs (1..8) as the longest sequence needs at up to 24576
-// keys per CTA, so a 16k-token sequence runs in one CTA with no cluster traffic.
-// Each CTA holds a contiguous slice of the sequence's scores in shared memory;
-// comparisons use order-preserving 32-bit keys (NaN lowest, -0 == +0). A 4-pass MSB-first radix
-// select (8-bit digits) finds the exact K-th largest document key T: every pass
-// builds per-warp histograms summed into a CTA histogram, the CTA histograms are summed
-// through distributed shared memory, and the digit that holds the K-th key is
-// found with a block suffix scan. Emission then keeps every
-// token outside the span, every document token with key > T, and the `need`
-// lowest-positioned document tokens with key == T (ties to the lower position);
-// the stable output order comes from warp ballots / popc prefix sums, with the
-// per-warp and per-CTA offsets exchanged the same way. No global scratch memory.
+// One thread-block cluster per sequence, one launch for the whole batch. The
+// cluster has enough CTAs (1..8) for about 4096 keys each (at most 24576), so the
+// passes below stay short. Each CTA holds a contiguous slice of the sequence in
+// shared memory twice: the raw fp32 scores (for the kept-score output) and
+// order-preserving 32-bit keys (NaN lowest, -0 == +0). Tokens outside the
+// document (and padding) get key 0; their count is subtracted from bin 0 so the
+// histograms see document tokens only.
+//
+// A 4-pass MSB-first radix select (8-bit digits) finds the exact K-th largest
+// document key T: per-warp histograms fed by 128-bit shared loads (4 keys per
+// lane), summed per CTA and across the cluster through distributed shared memory,
+// and the digit holding the K-th key found with a block suffix scan. Emission
+// keeps every token outside the span, every document token with key > T, and the
+// `need` lowest-positioned document tokens with key == T (ties to the lower
+// position); ranks and output offsets come from warp scans, per-warp and per-CTA
+// offsets from block scans and distributed shared memory. No global scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -27,12 +30,14 @@ namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kMaxCluster = 8;
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576 keys = 96 KB
+constexpr int kKeysTarget = 4096;                                    // keys per CTA aimed at
+constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576
+constexpr int kChunkQuant = kWarps * 128;                            // 128 keys per warp step
 
-struct SelectSmem {
-  uint32_t whist[kWarps][256];   // per-warp histograms (private: no cross-warp atomics)
+struct alignas(16) SelectSmem {
+  uint32_t whist[kWarps][256];   // per-warp histograms
   uint32_t hist[2][256];         // this CTA's histogram, by pass parity (read by peers)
   uint32_t scan[8];
   uint32_t warp_tot[kWarps];
@@ -46,18 +51,20 @@ struct SelectSmem {
   uint32_t seq_keep;
   int64_t out_base;
   int64_t red[kWarps];
-  // followed by: uint32_t masks[chunk / 32]; float raw[chunk];
+  // followed by: uint32_t keys[chunk]; float raw[chunk]; uint8_t kmask[chunk / 4];
 };
 
 inline int select_cluster(int max_len) {
-  int c = (max_len + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
-  return c < 1 ? 1 : c;
+  int c = (max_len + kKeysTarget - 1) / kKeysTarget;
+  if (c < 1) c = 1;
+  if (c > kMaxCluster) c = kMaxCluster;
+  return c;
 }
 
 inline int select_chunk(int max_len, int csize) {
   int c = (max_len + csize - 1) / csize;
-  c = (c + kThreads - 1) / kThreads * kThreads;
-  return c < kThreads ? kThreads : c;
+  c = (c + kChunkQuant - 1) / kChunkQuant * kChunkQuant;
+  return c < kChunkQuant ? kChunkQuant : c;
 }
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -82,7 +89,7 @@ __device__ __forceinline__ int64_t seq_kept(const int32_t* cu, const int32_t* db
   return len - nd + k;
 }
 
-// exclusive scan of per-warp totals (thread 0), result in warp_off, total returned
+// exclusive scan of the per-warp totals (one thread), total returned
 __device__ __forceinline__ uint32_t scan_warp_totals(SelectSmem& S) {
   uint32_t t = 0;
   for (int w = 0; w < kWarps; ++w) {
@@ -90,6 +97,19 @@ __device__ __forceinline__ uint32_t scan_warp_totals(SelectSmem& S) {
     t += S.warp_tot[w];
   }
   return t;
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+__device__ __forceinline__ uint32_t key_at(const uint4& k, int e) {
+  return e == 0 ? k.x : e == 1 ? k.y : e == 2 ? k.z : k.w;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -100,8 +120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                        int32_t* __restrict__ cu_kept, int* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
-  uint32_t* masks = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
-  float* raw = reinterpret_cast<float*>(masks + chunk / 32);   // this CTA's scores
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
+  float* raw = reinterpret_cast<float*>(keys + chunk);
+  uint8_t* kmask = reinterpret_cast<uint8_t*>(raw + chunk);   // keep bits, one byte per 4 keys
 
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
@@ -109,7 +130,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xFFFFFFFFu;
-  const unsigned lt_mask = (1u << lane) - 1u;
 
   // ---- sequence geometry (identical in every CTA of the cluster) ----
   const int64_t base = cu_seqlens[b];
@@ -125,12 +145,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (k_eff < 0) k_eff = 0;
   if (k_eff > nd) k_eff = nd;
 
-  // ---- load this CTA's slice as keys; meanwhile sum earlier sequences' counts ----
+  // this CTA's slice [c0, c0 + n_local) and its document part [ld0, ld1) (local)
   const int64_t c0 = (int64_t)rank * chunk;
-  int64_t n_local = len - c0;
-  if (n_local < 0) n_local = 0;
-  if (n_local > chunk) n_local = chunk;
-  for (int i0 = tid; i0 < chunk; i0 += 8 * kThreads) {   // 8 loads in flight per thread
+  const int n_local = (int)(len - c0 < 0 ? 0 : (len - c0 > chunk ? chunk : len - c0));
+  auto clampl = [&](int64_t v) { return (int)(v < 0 ? 0 : (v > n_local ? n_local : v)); };
+  const int ld0 = clampl(db - c0), ld1 = clampl(de - c0);
+  const uint32_t excl_local = (uint32_t)(chunk - (ld1 - ld0));   // keys forced to 0
+
+  // ---- load (8 loads in flight per thread); sum the earlier sequences' counts ----
+  for (int i0 = tid; i0 < chunk; i0 += 8 * kThreads) {
     float v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -140,7 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int i = i0 + u * kThreads;
-      if (i < chunk) raw[i] = v[u];
+      if (i < chunk) {
+        raw[i] = v[u];
+        keys[i] = (i >= ld0 && i < ld1) ? score_key(v[u]) : 0u;
+      }
     }
   }
   {
@@ -156,8 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     S.out_base = t;
   }
 
-  const int seg = chunk / kWarps;          // multiple of 32
+  const int seg = chunk / kWarps;                 // multiple of 128
   const int seg0 = warp * seg;
+  const int nsteps = seg / 128;
+  const uint4* k4 = reinterpret_cast<const uint4*>(keys) + seg0 / 4;
 
   // ---- radix select of the k_eff-th largest document key ----
   uint32_t T, need;
@@ -176,17 +204,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = lane; i < 256; i += 32) wh[i] = 0u;
       __syncwarp();
-      for (int i = seg0 + lane; i < seg0 + seg; i += 32) {
-        const int64_t pos = c0 + i;
-        const uint32_t key = score_key(raw[i]);
-        if (i < n_local && pos >= db && pos < de && (key & pmask) == prefix)
-          atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
+      for (int st = 0; st < nsteps; ++st) {
+        const uint4 kk = k4[st * 32 + lane];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t key = key_at(kk, e);
+          if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
+        }
       }
       __syncthreads();
       if (tid < 256) {
         uint32_t c = 0;
 #pragma unroll 8
         for (int w = 0; w < kWarps; ++w) c += S.whist[w][tid];
+        if (tid == 0 && prefix == 0) c -= excl_local;   // forced-zero keys are not document keys
         h[tid] = c;
       }
       cluster.sync();   // every CTA's histogram of this pass is complete
@@ -196,11 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int d = 255 - tid;
         uint32_t cnt = 0;
         for (unsigned r = 0; r < csize; ++r) cnt += cluster.map_shared_rank(h, r)[d];
-        uint32_t inc = cnt;
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(full, inc, o);
-          if (lane >= o) inc += y;
-        }
+        uint32_t inc = warp_incl_scan(cnt, lane);
         if (lane == 31) S.scan[warp] = inc;
         tg::named_barrier(1, 256);   // warps 0-7 only
         uint32_t woff = 0;
@@ -224,13 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- emission, phase A: per-warp counts of document keys equal to T ----
   {
     uint32_t cnt = 0;
-    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
-      const int64_t pos = c0 + i;
-      const bool eq = i < n_local && pos >= db && pos < de && score_key(raw[i]) == T;
-      const unsigned m = __ballot_sync(full, eq);
-      if (lane == 0) masks[wi] = m;
-      cnt += __popc(m);
+    for (int st = 0; st < nsteps; ++st) {
+      const uint4 kk = k4[st * 32 + lane];
+      const int i4 = seg0 + st * 128 + lane * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cnt += (i4 + e >= ld0 && i4 + e < ld1 && key_at(kk, e) == T);
     }
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(full, cnt, o);
     if (lane == 0) S.warp_tot[warp] = cnt;
     __syncthreads();
     if (tid == 0) S.cta_eq = scan_warp_totals(S);
@@ -243,24 +270,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  // ---- phase B: keep decisions and per-warp kept counts ----
+  // ---- phase B: keep decisions (ties by rank in position order) ----
   {
-    uint32_t running = S.cta_eq_off + S.warp_off[warp];
+    uint32_t running = S.cta_eq_off + S.warp_off[warp];   // T-ties before this warp's segment
     uint32_t kept = 0;
-    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
-      const int64_t pos = c0 + i;
-      const uint32_t eqm = masks[wi];
-      bool keep = false;
-      if (i < n_local) {
-        const bool in_doc = pos >= db && pos < de;
-        const bool eq = (eqm >> lane) & 1u;
-        keep = !in_doc || score_key(raw[i]) > T || (eq && running + __popc(eqm & lt_mask) < need);
+    for (int st = 0; st < nsteps; ++st) {
+      const uint4 kk = k4[st * 32 + lane];
+      const int i4 = seg0 + st * 128 + lane * 4;
+      uint32_t ce = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ce += (i4 + e >= ld0 && i4 + e < ld1 && key_at(kk, e) == T);
+      const uint32_t incl = warp_incl_scan(ce, lane);
+      uint32_t r = running + incl - ce;
+      uint32_t nib = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i4 + e;
+        const bool in_doc = i >= ld0 && i < ld1;
+        const uint32_t key = key_at(kk, e);
+        const bool eq = in_doc && key == T;
+        const bool keep = i < n_local && (!in_doc || key > T || (eq && r < need));
+        r += eq;
+        nib |= (uint32_t)keep << e;
       }
-      running += __popc(eqm);
-      const unsigned km = __ballot_sync(full, keep);
-      if (lane == 0) masks[wi] = km;
-      kept += __popc(km);
+      kmask[i4 / 4] = (uint8_t)nib;
+      kept += __popc(nib);
+      running += __shfl_sync(full, incl, 31);
     }
+    for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(full, kept, o);
     if (lane == 0) S.warp_tot[warp] = kept;
     __syncthreads();
     if (tid == 0) S.cta_keep = scan_warp_totals(S);
@@ -285,15 +322,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool ok = seq_keep == expect && out_base + seq_keep <= total_kept;
   if (ok) {
     int64_t running = out_base + S.cta_keep_off + S.warp_off[warp];
-    for (int i = seg0 + lane, wi = seg0 / 32; i < seg0 + seg; i += 32, ++wi) {
-      const uint32_t km = masks[wi];
-      if ((km >> lane) & 1u) {
-        const int64_t o = running + __popc(km & lt_mask);
-        const int64_t row = base + c0 + i;
-        kept_idx[o] = (int32_t)row;
-        if (kept_scores) kept_scores[o] = raw[i];
+    for (int st = 0; st < nsteps; ++st) {
+      const int i4 = seg0 + st * 128 + lane * 4;
+      const uint32_t nib = kmask[i4 / 4];
+      const uint32_t c = __popc(nib);
+      const uint32_t incl = warp_incl_scan(c, lane);
+      int64_t o = running + incl - c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if ((nib >> e) & 1u) {
+          kept_idx[o] = (int32_t)(base + c0 + i4 + e);
+          if (kept_scores) kept_scores[o] = raw[i4 + e];
+          ++o;
+        }
       }
-      running += __popc(km);
+      running += __shfl_sync(full, incl, 31);
     }
   }
   if (rank == 0 && tid == 0) {
@@ -324,7 +367,8 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   if (!st) return TG_ERR_CUDA;
   const int csize = select_cluster(max_seqlen);
   const int chunk = select_chunk(max_seqlen, csize);
-  const size_t smem = sizeof(SelectSmem) + (size_t)chunk / 32 * 4 + (size_t)chunk * 4;
+  if (chunk > kMaxKeysPerCta) return TG_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(SelectSmem) + (size_t)chunk * 8 + (size_t)chunk / 4;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem))
     return TG_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
