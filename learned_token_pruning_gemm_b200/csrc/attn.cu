@@ -10,9 +10,11 @@
 // one (query head, sequence): every CTA then does n+1 key tiles and the grid is
 // balanced. Per CTA, pipelines run across both query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
-//                ring; its lanes also stage each tile's per-key bias
-//                b_j = log2(e) g_h s_j beside the K tile. A K stage is free once
-//                S_j is computed and every softmax warp has read the bias.
+//                ring. A K stage is free once S_j is computed and every softmax
+//                warp has read its bias.
+//   warp 2       allocates TMEM, then stages each tile's per-key bias
+//                b_j = log2(e) g_h s_j beside the K tile (its global loads stay off
+//                the TMA issue path).
 //   warp 3       TMA producer of V tiles through a 2-stage ring (free after PV_j).
 //   warp 1       MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
 //                S_j = Q K_j^T into one of two 128-column TMEM buffers, and
@@ -131,13 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
   const int z = blockIdx.z;
+  // issued first; the barrier set-up and TMEM allocation below overlap their latency
   const int seq0 = cu_kept[b];
-  const int len = cu_kept[b + 1] - seq0;
-  const int n_t = (len + kBM - 1) / kBM;
-  if (2 * z >= n_t) return;     // uniform: this sequence has no pair z
-  // the CTA's query tiles: the long one first, then its partner (if distinct)
-  const int tiles[2] = {n_t - 1 - z, z};
-  const int nq = (tiles[1] < tiles[0]) ? 2 : 1;
+  const int seq1 = cu_kept[b + 1];
   const int kvh = hq / (n_hq / n_hkv);
 
   extern __shared__ uint8_t smem_raw[];
@@ -180,44 +178,69 @@ __global__ void __launch_bounds__(kThreads, 1)
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
+  const int len = seq1 - seq0;
+  const int n_t = (len + kBM - 1) / kBM;
+  if (2 * z >= n_t) {           // uniform: this sequence has no pair z
+    if (warp == 2) tg::tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
+  // the CTA's query tiles: the long one first, then its partner (if distinct)
+  const int tiles[2] = {n_t - 1 - z, z};
+  const int nq = (tiles[1] < tiles[0]) ? 2 : 1;
+
   if (warp == 0) {
-    // ---------------- TMA producer: Q, K tiles + bias staging ----------------
-    const float gl2 = gain[hq] * kLog2e;
-    int g = 0, issued = 0;
-    bool go = true;
-    for (int qi = 0; qi < nq && go; ++qi) {
-      const int t = tiles[qi];
-      if (qi > 0) go = all_alive(tg::mbar_wait(&S.q_empty, 0, status, &S.abort_flag));
-      if (!go) break;
-      if (lane == 0) {
+    // ---------------- TMA producer: Q and K tiles ----------------
+    if (lane == 0) {
+      int g = 0;
+      bool go = true;
+      for (int qi = 0; qi < nq && go; ++qi) {
+        const int t = tiles[qi];
+        if (qi > 0 && !tg::mbar_wait(&S.q_empty, 0, status, &S.abort_flag)) break;
         tg::mbar_arrive_expect_tx(&S.q_full, kBM * kD * 2);
         tg::tma_load_3d(S.q[0], &tm_q, &S.q_full, 0, hq, seq0 + t * kBM);
         tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
-      }
-      for (int j = 0; j <= t; ++j, ++g) {
-        const int s = g % kKStages;
-        if (g >= kKStages)
-          go = all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
-                                       &S.abort_flag));
-        if (!go) break;
-        if (lane == 0) {
+        for (int j = 0; j <= t; ++j, ++g) {
+          const int s = g % kKStages;
+          if (g >= kKStages &&
+              !tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status, &S.abort_flag)) {
+            go = false;
+            break;
+          }
           tg::mbar_arrive_expect_tx(&S.k_full[s], kBN * kD * 2);
           const int r0 = seq0 + j * kBN;
           tg::tma_load_3d(S.k[s][0], &tm_k, &S.k_full[s], 0, kvh, r0);
           tg::tma_load_3d(S.k[s][1], &tm_k, &S.k_full[s], 64, kvh, r0);
         }
-        for (int c = lane; c < kBN; c += 32) {
-          const int kp = j * kBN + c;
-          S.bias[s][c] = kp < len ? gl2 * s_kept[seq0 + kp] : 0.f;
-        }
-        tg::mbar_arrive(&S.k_full[s]);
-        ++issued;
+      }
+      if (S.abort_flag) {   // let copies in flight land before the CTA exits
+        tg::mbar_wait(&S.q_full, 0, status, nullptr);
+        for (int j = g > kKStages ? g - kKStages : 0; j < g; ++j)
+          tg::mbar_wait(&S.k_full[j % kKStages], (j / kKStages) & 1, status, nullptr);
       }
     }
-    if (lane == 0 && S.abort_flag) {   // let copies in flight land before the CTA exits
-      tg::mbar_wait(&S.q_full, 0, status, nullptr);
-      for (int j = issued > kKStages ? issued - kKStages : 0; j < issued; ++j)
-        tg::mbar_wait(&S.k_full[j % kKStages], (j / kKStages) & 1, status, nullptr);
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------- bias staging (32 arrivals per K stage) ----------------
+    const float gl2 = gain[hq] * kLog2e;
+    int g = 0;
+    bool go = true;
+    for (int qi = 0; qi < nq && go; ++qi) {
+      for (int j = 0; j <= tiles[qi]; ++j, ++g) {
+        const int s = g % kKStages;
+        float v[kBN / 32];
+#pragma unroll
+        for (int u = 0; u < kBN / 32; ++u) {   // loads issued before the slot wait
+          const int kp = j * kBN + lane + 32 * u;
+          v[u] = kp < len ? s_kept[seq0 + kp] : 0.f;
+        }
+        if (g >= kKStages)
+          go = all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
+                                       &S.abort_flag));
+        if (!go) break;
+#pragma unroll
+        for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = gl2 * v[u];
+        tg::mbar_arrive(&S.k_full[s]);
+      }
     }
   } else if (warp == 3) {
     // ---------------- TMA producer: V tiles ----------------

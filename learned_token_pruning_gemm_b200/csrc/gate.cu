@@ -3,13 +3,16 @@
 // ?": a small MLP scores each token from its post-attention residual at layer L).
 //     s_i = b2 + sum_k w2[k] * GELU(b1[k] + x_i . w1[k,:])
 //
-// bf16 path: one CTA per 128-token tile computes the whole hidden layer
-// (M=128 tokens x N=h units x K=d) with tcgen05.mma (kind::f16, f32 accumulate)
-// into a 128 x h fp32 accumulator in tensor memory. Two TMA producer threads
-// stream 128x64 tiles of x (from HBM, a deep 6-stage ring so enough bytes are in
-// flight to cover HBM latency) and hx64 tiles of w1 (shared by every CTA, served
-// from L2, 3 stages), both 128-byte swizzled; one MMA thread issues 4 K=16 MMAs
-// per k-block and frees each stage with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
+// bf16 path: a pair of CTAs (a cluster of 2 on neighbouring SMs) computes 256
+// tokens x h hidden units with the 2-SM tensor-core MMA (tcgen05.mma.cta_group::2,
+// kind::f16, M=256, f32 accumulate): each CTA holds its own 128 x rows and half of
+// the w1 rows in shared memory, and its 128 x h slice of the accumulator in its
+// own tensor memory. Every CTA reads w1 (shared by all, served from L2) at half
+// the rate of a single-SM MMA, so a 6-stage ring of 32 KB stages keeps about 2 us
+// of loads in flight. A TMA producer thread per CTA fills the ring (128-byte
+// swizzle); the odd CTA relays "my half landed" to the even CTA with a remote
+// mbarrier arrive; the even CTA issues 4 K=16 pair MMAs per stage and releases
+// the stage in both CTAs with a multicast tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
 // accumulator (warp w: lanes 32*(w%4).., a quarter of the columns), add b1, apply
 // exact erf-GELU and dot with w2; the four column partials are summed in a fixed
 // order, so a token's score depends only on its own row.
@@ -19,24 +22,22 @@
 
 namespace {
 
-constexpr int kBM = 128;      // tokens per tile
+constexpr int kBM = 128;      // tokens per CTA (256 per CTA pair)
 constexpr int kBK = 64;       // reduction columns per stage (128 bytes of bf16)
-constexpr int kXStages = 6;
-constexpr int kWStages = 3;
+constexpr int kStages = 6;
 constexpr int kThreads = 512;
 
 template <int H>
 struct GateSmem {
-  uint8_t a[kXStages][kBM * kBK * 2];  // x tiles, 16 KB each
-  uint8_t b[kWStages][H * kBK * 2];    // w1 tiles
+  uint8_t a[kStages][kBM * kBK * 2];          // this CTA's 128 x rows, 16 KB
+  uint8_t b[kStages][(H / 2) * kBK * 2];      // this CTA's half of the w1 rows
   float b1[H];
   float w2[H];
   float part[4][kBM];
-  uint64_t x_full[kXStages];
-  uint64_t x_empty[kXStages];
-  uint64_t w_full[kWStages];
-  uint64_t w_empty[kWStages];
-  uint64_t acc_full;
+  uint64_t full[kStages];       // this CTA's copies of the stage landed
+  uint64_t peer_full[kStages];  // (even CTA) the odd CTA's copies of the stage landed
+  uint64_t empty[kStages];      // the pair MMAs of the stage completed (multicast commit)
+  uint64_t acc_full;            // the accumulator is final (multicast commit)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -46,7 +47,7 @@ __device__ __forceinline__ float gelu_erf(float u) {
 }
 
 template <int H>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gate_bf16_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const float* __restrict__ b1, const float* __restrict__ w2, float b2,
                      int64_t n_tokens, int d, float* __restrict__ scores, int* status) {
@@ -55,83 +56,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   GateSmem<H>& S = *reinterpret_cast<GateSmem<H>*>(smem_raw + pad);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = tg::cluster_ctarank();   // 0: issues the pair MMAs
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
   const int nk = d / kBK;
 
   if (tid == 0) {
-    for (int s = 0; s < kXStages; ++s) {
-      tg::mbar_init(&S.x_full[s], 1);
-      tg::mbar_init(&S.x_empty[s], 1);
-    }
-    for (int s = 0; s < kWStages; ++s) {
-      tg::mbar_init(&S.w_full[s], 1);
-      tg::mbar_init(&S.w_empty[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      tg::mbar_init(&S.full[s], 1);
+      tg::mbar_init(&S.peer_full[s], 1);
+      tg::mbar_init(&S.empty[s], 1);
     }
     tg::mbar_init(&S.acc_full, 1);
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
   if (warp == 2) {
-    tg::tmem_alloc(&S.tmem_base, H);
-    tg::tmem_relinquish();
+    tg::tmem_alloc_pair(&S.tmem_base, H);
+    tg::tmem_relinquish_pair();
   }
-  if (warp == 0 && lane == 0) tg::tma_prefetch_desc(&tm_x);
-  if (warp == 3 && lane == 0) tg::tma_prefetch_desc(&tm_w);
+  if (warp == 0 && lane == 0) {
+    tg::tma_prefetch_desc(&tm_x);
+    tg::tma_prefetch_desc(&tm_w);
+  }
   tg::tc_fence_before();
-  __syncthreads();
+  tg::cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA signal
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer: x tiles ----
+    // ---- TMA producer: this CTA's x rows and its half of the w1 rows ----
     int issued = 0;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kXStages;
-      if (kb >= kXStages &&
-          !tg::mbar_wait(&S.x_empty[s], ((kb / kXStages) - 1) & 1, status, &S.abort_flag))
+      const int s = kb % kStages;
+      if (kb >= kStages &&
+          !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.x_full[s], kBM * kBK * 2);
-      tg::tma_load_2d(S.a[s], &tm_x, &S.x_full[s], kb * kBK, static_cast<int>(m0));
+      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H / 2) * kBK * 2);
+      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, static_cast<int>(rank) * (H / 2));
       ++issued;
     }
-    if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
-      for (int kb = issued > kXStages ? issued - kXStages : 0; kb < issued; ++kb)
-        tg::mbar_wait(&S.x_full[kb % kXStages], (kb / kXStages) & 1, status, nullptr);
-    }
-  } else if (warp == 3 && lane == 0) {
-    // ---- TMA producer: w1 tiles ----
-    int issued = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kWStages;
-      if (kb >= kWStages &&
-          !tg::mbar_wait(&S.w_empty[s], ((kb / kWStages) - 1) & 1, status, &S.abort_flag))
-        break;
-      tg::mbar_arrive_expect_tx(&S.w_full[s], H * kBK * 2);
-      tg::tma_load_2d(S.b[s], &tm_w, &S.w_full[s], kb * kBK, 0);
-      ++issued;
-    }
-    if (S.abort_flag) {
-      for (int kb = issued > kWStages ? issued - kWStages : 0; kb < issued; ++kb)
-        tg::mbar_wait(&S.w_full[kb % kWStages], (kb / kWStages) & 1, status, nullptr);
-    }
+    // every stage's last release (a commit the other CTA issued) lands before exit
+    for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
+      tg::mbar_wait(&S.empty[kb % kStages], (kb / kStages) & 1, status, &S.abort_flag);
   } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    constexpr uint32_t idesc = tg::idesc_bf16_f32(kBM, H, false, false);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int sx = kb % kXStages, sw = kb % kWStages;
-      if (!tg::mbar_wait(&S.x_full[sx], (kb / kXStages) & 1, status, &S.abort_flag)) break;
-      if (!tg::mbar_wait(&S.w_full[sw], (kb / kWStages) & 1, status, &S.abort_flag)) break;
-      tg::tc_fence_after();
-      const uint32_t a0 = tg::smem_u32(S.a[sx]), b0 = tg::smem_u32(S.b[sw]);
+    if (rank == 0) {
+      // ---- pair MMA issuer: D[256 x H] += A[256 x 64] * B[H x 64]^T per stage ----
+      constexpr uint32_t idesc = tg::idesc_bf16_f32(2 * kBM, H, false, false);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+        if (!tg::mbar_wait(&S.peer_full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+        tg::tc_fence_after();
+        const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k) {
-        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                        tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
+        for (int k = 0; k < kBK / 16; ++k) {
+          tg::mma_bf16_ss_pair(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                               tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
+        }
+        tg::mma_commit_pair(&S.empty[s], 0x3);
       }
-      tg::mma_commit(&S.x_empty[sx]);
-      tg::mma_commit(&S.w_empty[sw]);
+      tg::mma_commit_pair(&S.acc_full, 0x3);
+    } else {
+      // ---- relay: tell the even CTA when this CTA's half of a stage has landed ----
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+        tg::mbar_arrive_remote(tg::mapa_shared(&S.peer_full[s], 0));
+      }
     }
-    tg::mma_commit(&S.acc_full);
   } else if (warp >= 4) {
     // stage the epilogue's constants while the mainloop runs
     for (int i = tid - 128; i < H; i += kThreads - 128) {
@@ -142,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();
   tg::named_barrier(1, kThreads);   // b1/w2 staged; producer and MMA loops issued
 
-  // ---- epilogue: all 16 warps ----
+  // ---- epilogue: all 16 warps; this CTA's TMEM holds its 128 rows x H ----
   constexpr int kCols = H / 4;               // accumulator columns per warp
   const int lg = warp & 3, cgp = warp >> 2;
   const int row = lg * 32 + lane;
@@ -170,9 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float s = b2 + ((S.part[0][tid] + S.part[1][tid]) + (S.part[2][tid] + S.part[3][tid]));
     if (m0 + tid < n_tokens) scores[m0 + tid] = s;
   }
+  tg::cluster_sync_all();   // neither CTA frees TMEM or exits while the pair is in use
   if (warp == 2) {
     tg::tc_fence_after();
-    tg::tmem_dealloc(tmem, H);
+    tg::tmem_dealloc_pair(tmem, H);
   }
 }
 
@@ -215,7 +209,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
   const uint32_t bx[2] = {kBK, kBM};
   const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H)};
-  const uint32_t bw[2] = {kBK, H};
+  const uint32_t bw[2] = {kBK, H / 2};
   if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dx, sx, bx,
                        CU_TENSOR_MAP_SWIZZLE_128B) ||
       !tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w1, dw, sx, bw,
@@ -224,7 +218,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   const size_t smem = sizeof(GateSmem<H>) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
-  const int64_t tiles = (n + kBM - 1) / kBM;
+  const int64_t tiles = 2 * ((n + 2 * kBM - 1) / (2 * kBM));   // whole CTA pairs
   gate_bf16_kernel<H><<<static_cast<unsigned>(tiles), kThreads, smem, st>>>(tx, tw, b1, w2, b2, n, d,
                                                                            scores, status);
   return tg::launch_status();
