@@ -221,26 +221,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ---------------- bias staging (32 arrivals per K stage) ----------------
+    // A register ring keeps the loads of the next kKStages tiles in flight, so the
+    // staging keeps pace with the K ring instead of waiting one load per tile.
     const float gl2 = gain[hq] * kLog2e;
-    int g = 0;
-    bool go = true;
-    for (int qi = 0; qi < nq && go; ++qi) {
-      for (int j = 0; j <= tiles[qi]; ++j, ++g) {
-        const int s = g % kKStages;
-        float v[kBN / 32];
+    const int n_tiles = (tiles[0] + 1) + (nq > 1 ? tiles[1] + 1 : 0);
+    auto tile_j = [&](int g) { return g <= tiles[0] ? g : g - (tiles[0] + 1); };
+    auto load = [&](int g, float* v) {
 #pragma unroll
-        for (int u = 0; u < kBN / 32; ++u) {   // loads issued before the slot wait
-          const int kp = j * kBN + lane + 32 * u;
-          v[u] = kp < len ? s_kept[seq0 + kp] : 0.f;
-        }
-        if (g >= kKStages)
-          go = all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
-                                       &S.abort_flag));
-        if (!go) break;
-#pragma unroll
-        for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = gl2 * v[u];
-        tg::mbar_arrive(&S.k_full[s]);
+      for (int u = 0; u < kBN / 32; ++u) {
+        const int kp = tile_j(g) * kBN + lane + 32 * u;
+        v[u] = (g < n_tiles && kp < len) ? s_kept[seq0 + kp] : 0.f;
       }
+    };
+    float v0[kBN / 32], v1[kBN / 32], v2[kBN / 32];
+    load(0, v0);
+    load(1, v1);
+    load(2, v2);
+    for (int g = 0; g < n_tiles; ++g) {
+      const int s = g % kKStages;
+      if (g >= kKStages &&
+          !all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
+                                   &S.abort_flag)))
+        break;
+#pragma unroll
+      for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = gl2 * v0[u];
+      tg::mbar_arrive(&S.k_full[s]);
+#pragma unroll
+      for (int u = 0; u < kBN / 32; ++u) {
+        v0[u] = v1[u];
+        v1[u] = v2[u];
+      }
+      load(g + 3, v2);
     }
   } else if (warp == 3) {
     // ---------------- TMA producer: V tiles ----------------

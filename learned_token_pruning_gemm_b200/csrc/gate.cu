@@ -3,16 +3,12 @@
 // ?": a small MLP scores each token from its post-attention residual at layer L).
 //     s_i = b2 + sum_k w2[k] * GELU(b1[k] + x_i . w1[k,:])
 //
-// bf16 path: a pair of CTAs (a cluster of 2 on neighbouring SMs) computes 256
-// tokens x h hidden units with the 2-SM tensor-core MMA (tcgen05.mma.cta_group::2,
-// kind::f16, M=256, f32 accumulate): each CTA holds its own 128 x rows and half of
-// the w1 rows in shared memory, and its 128 x h slice of the accumulator in its
-// own tensor memory. Every CTA reads w1 (shared by all, served from L2) at half
-// the rate of a single-SM MMA, so a 6-stage ring of 32 KB stages keeps about 2 us
-// of loads in flight. A TMA producer thread per CTA fills the ring (128-byte
-// swizzle); the odd CTA relays "my half landed" to the even CTA with a remote
-// mbarrier arrive; the even CTA issues 4 K=16 pair MMAs per stage and releases
-// the stage in both CTAs with a multicast tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
+// bf16 path: one CTA per 128-token tile computes the whole hidden layer
+// (M=128 tokens x N=h units x K=d) with tcgen05.mma (kind::f16, f32 accumulate)
+// into a 128 x h fp32 accumulator in tensor memory. A TMA producer thread streams
+// 128x64 tiles of x and hx64 tiles of w1 (128-byte swizzle) through a 4-stage
+// mbarrier ring; one MMA thread issues 4 K=16 MMAs per stage and frees the stage
+// with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
 // accumulator (warp w: lanes 32*(w%4).., a quarter of the columns), add b1, apply
 // exact erf-GELU and dot with w2; the four column partials are summed in a fixed
 // order, so a token's score depends only on its own row.
@@ -22,22 +18,21 @@
 
 namespace {
 
-constexpr int kBM = 128;      // tokens per CTA (256 per CTA pair)
+constexpr int kBM = 128;      // tokens per tile
 constexpr int kBK = 64;       // reduction columns per stage (128 bytes of bf16)
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;
 
 template <int H>
 struct GateSmem {
-  uint8_t a[kStages][kBM * kBK * 2];          // this CTA's 128 x rows, 16 KB
-  uint8_t b[kStages][(H / 2) * kBK * 2];      // this CTA's half of the w1 rows
+  uint8_t a[kStages][kBM * kBK * 2];   // x tiles, 16 KB each
+  uint8_t b[kStages][H * kBK * 2];     // w1 tiles
   float b1[H];
   float w2[H];
   float part[4][kBM];
-  uint64_t full[kStages];       // this CTA's copies of the stage landed
-  uint64_t peer_full[kStages];  // (even CTA) the odd CTA's copies of the stage landed
-  uint64_t empty[kStages];      // the pair MMAs of the stage completed (multicast commit)
-  uint64_t acc_full;            // the accumulator is final (multicast commit)
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -47,7 +42,7 @@ __device__ __forceinline__ float gelu_erf(float u) {
 }
 
 template <int H>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     gate_bf16_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const float* __restrict__ b1, const float* __restrict__ w2, float b2,
                      int64_t n_tokens, int d, float* __restrict__ scores, int* status) {
@@ -56,14 +51,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   GateSmem<H>& S = *reinterpret_cast<GateSmem<H>*>(smem_raw + pad);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = tg::cluster_ctarank();   // 0: issues the pair MMAs
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
   const int nk = d / kBK;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       tg::mbar_init(&S.full[s], 1);
-      tg::mbar_init(&S.peer_full[s], 1);
       tg::mbar_init(&S.empty[s], 1);
     }
     tg::mbar_init(&S.acc_full, 1);
@@ -71,63 +64,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tg::fence_barrier_init();
   }
   if (warp == 2) {
-    tg::tmem_alloc_pair(&S.tmem_base, H);
-    tg::tmem_relinquish_pair();
+    tg::tmem_alloc(&S.tmem_base, H);
+    tg::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
     tg::tma_prefetch_desc(&tm_x);
     tg::tma_prefetch_desc(&tm_w);
   }
   tg::tc_fence_before();
-  tg::cluster_sync_all();   // both CTAs' barriers exist before any cross-CTA signal
+  __syncthreads();
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer: this CTA's x rows and its half of the w1 rows ----
+    // ---- TMA producer ----
     int issued = 0;
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % kStages;
       if (kb >= kStages &&
           !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H / 2) * kBK * 2);
+      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H) * kBK * 2);
       tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
-      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, static_cast<int>(rank) * (H / 2));
+      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, 0);
       ++issued;
     }
-    // every stage's last release (a commit the other CTA issued) lands before exit
-    for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
-      tg::mbar_wait(&S.empty[kb % kStages], (kb / kStages) & 1, status, &S.abort_flag);
-  } else if (warp == 1 && lane == 0) {
-    if (rank == 0) {
-      // ---- pair MMA issuer: D[256 x H] += A[256 x 64] * B[H x 64]^T per stage ----
-      constexpr uint32_t idesc = tg::idesc_bf16_f32(2 * kBM, H, false, false);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
-        if (!tg::mbar_wait(&S.peer_full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
-        tg::tc_fence_after();
-        const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
-#pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          tg::mma_bf16_ss_pair(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                               tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
-        }
-        tg::mma_commit_pair(&S.empty[s], 0x3);
-      }
-      tg::mma_commit_pair(&S.acc_full, 0x3);
-    } else {
-      // ---- relay: tell the even CTA when this CTA's half of a stage has landed ----
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
-        tg::mbar_arrive_remote(tg::mapa_shared(&S.peer_full[s], 0));
-      }
+    if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
+      for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb)
+        tg::mbar_wait(&S.full[kb % kStages], (kb / kStages) & 1, status, nullptr);
     }
-  } else if (warp >= 4) {
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ----
+    constexpr uint32_t idesc = tg::idesc_bf16_f32(kBM, H, false, false);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+      tg::tc_fence_after();
+      const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                        tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
+      }
+      tg::mma_commit(&S.empty[s]);
+    }
+    tg::mma_commit(&S.acc_full);
+  } else if (warp >= 2) {
     // stage the epilogue's constants while the mainloop runs
-    for (int i = tid - 128; i < H; i += kThreads - 128) {
+    for (int i = tid - 64; i < H; i += kThreads - 64) {
       S.b1[i] = b1[i];
       S.w2[i] = w2[i];
     }
@@ -135,7 +119,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncwarp();
   tg::named_barrier(1, kThreads);   // b1/w2 staged; producer and MMA loops issued
 
-  // ---- epilogue: all 16 warps; this CTA's TMEM holds its 128 rows x H ----
+  // ---- epilogue: all 16 warps ----
   constexpr int kCols = H / 4;               // accumulator columns per warp
   const int lg = warp & 3, cgp = warp >> 2;
   const int row = lg * 32 + lane;
@@ -163,10 +147,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float s = b2 + ((S.part[0][tid] + S.part[1][tid]) + (S.part[2][tid] + S.part[3][tid]));
     if (m0 + tid < n_tokens) scores[m0 + tid] = s;
   }
-  tg::cluster_sync_all();   // neither CTA frees TMEM or exits while the pair is in use
   if (warp == 2) {
     tg::tc_fence_after();
-    tg::tmem_dealloc_pair(tmem, H);
+    tg::tmem_dealloc(tmem, H);
   }
 }
 
@@ -209,7 +192,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
   const uint32_t bx[2] = {kBK, kBM};
   const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H)};
-  const uint32_t bw[2] = {kBK, H / 2};
+  const uint32_t bw[2] = {kBK, H};
   if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dx, sx, bx,
                        CU_TENSOR_MAP_SWIZZLE_128B) ||
       !tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w1, dw, sx, bw,
@@ -218,7 +201,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   const size_t smem = sizeof(GateSmem<H>) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
-  const int64_t tiles = 2 * ((n + 2 * kBM - 1) / (2 * kBM));   // whole CTA pairs
+  const int64_t tiles = (n + kBM - 1) / kBM;
   gate_bf16_kernel<H><<<static_cast<unsigned>(tiles), kThreads, smem, st>>>(tx, tw, b1, w2, b2, n, d,
                                                                            scores, status);
   return tg::launch_status();
