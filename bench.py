@@ -230,20 +230,25 @@ def run_ours(args, dist, rank, ws):
 
     clocks = ClockSampler(dev_index)
     clocks.start()
-    gp.capture()                          # one CUDA graph per stage; replays below
+    gp.capture()                          # the whole layer as one CUDA graph
     for _ in range(args.warmup):
         flush.zero_()
-        gp.replay()
+        gp.replay_step()
     torch.cuda.synchronize()
     assert api.device_status(reset=True) == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # timed region: exactly `steps` whole-layer steps (one graph each), L2 flushed
+    # between them outside the events
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     _barrier(dist)
     torch.cuda.synchronize()
     t_host0 = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()                     # L2 flush between timed steps (outside the events)
-        gp.replay(events=evs[i])
+    for a, b in step_ev:
+        flush.zero_()
+        a.record(stream)
+        gp.replay_step()
+        b.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.perf_counter()
     _barrier(dist)
@@ -252,10 +257,16 @@ def run_ours(args, dist, rank, ws):
     status = api.device_status(reset=True)
     if status != 0:
         raise RuntimeError(f"device status {status} during the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
 
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-                for j, name in enumerate(gp.STAGES)}
+    # per-stage breakdown (separate pass): events recorded inside the step graph
+    per = []
+    for _ in range(args.steps):
+        flush.zero_()
+        gp.replay_step()
+        torch.cuda.synchronize()
+        per.append(gp.stage_times_ms())
+    stage_ms = {name: statistics.mean(p[name] for p in per) for name in gp.STAGES}
     ms = _max_over_ranks(dist, statistics.mean(step_ms))
     value = ws * wl.n_tokens / (ms / 1e3)
 
@@ -319,7 +330,7 @@ def run_ours(args, dist, rank, ws):
         def e2e_step():
             for hsrc, dst in zip(host_in, dev_in):
                 dst.copy_(hsrc, non_blocking=True)
-            gp.replay()
+            gp.replay_step()
             host_out.copy_(gp.out, non_blocking=True)
             host_idx.copy_(gp.kept_idx, non_blocking=True)
 
@@ -361,7 +372,9 @@ def run_ours(args, dist, rank, ws):
             "stages": stages,
             "roofline": roofline,
             "gpu_launches": gp.LAUNCHES_PER_STEP * args.steps,
-            "launch": "one CUDA graph per stage, replayed; per-stage CUDA events between them",
+            "stage_sum_us": sum(stage_ms.values()) * 1e3,
+            "launch": ("timed steps: the whole layer as one CUDA graph (4 kernels), events "
+                       "around each replay; stage times: events recorded inside the graph"),
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

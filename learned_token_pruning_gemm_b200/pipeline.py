@@ -89,31 +89,29 @@ class GatedPrefill:
 
     # ------------------------------------------------------------------ graphs
     def capture(self):
-        """Capture each stage into its own CUDA graph so that replays carry no host
-        launch overhead. One eager step runs first (outside capture) so every
-        lazily initialised piece of the library exists before capture."""
+        """Capture the whole layer (four kernels) as one CUDA graph, with five timing
+        events recorded inside it before, between and after the stages. One eager
+        step runs first (outside capture) so that every lazily initialised piece of
+        the library exists before capture."""
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
             self.step(side)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
-        self.graphs = []
-        for fn in (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fn()
-            self.graphs.append(g)
+        self.stage_events = [torch.cuda.Event(enable_timing=True, external=True)
+                             for _ in range(5)]
+        self.step_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.step_graph):
+            self.step(events=self.stage_events)
         torch.cuda.synchronize()
         return self
 
-    def replay(self, events: Optional[list] = None):
-        """Replay the captured stages on the current stream (same launches as
-        `step`), recording `events` around them like `step` does."""
-        s = torch.cuda.current_stream()
-        for i, g in enumerate(self.graphs):
-            if events is not None:
-                events[i].record(s)
-            g.replay()
-        if events is not None:
-            events[4].record(s)
+    def replay_step(self):
+        """Replay the whole layer (one graph, four kernel launches) on the current stream."""
+        self.step_graph.replay()
+
+    def stage_times_ms(self):
+        """Per-stage device times of the last completed replay (needs a sync first)."""
+        ev = self.stage_events
+        return {n: ev[i].elapsed_time(ev[i + 1]) for i, n in enumerate(self.STAGES)}

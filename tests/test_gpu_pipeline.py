@@ -98,9 +98,11 @@ def test_graph_replay_matches_eager(mods):
     gp.capture()
     for t in (gp.scores, gp.kept_scores, gp.out):
         t.zero_()
-    gp.replay()
+    gp.replay_step()
     torch.cuda.synchronize()
     assert api.device_status(reset=True) == 0
+    st = gp.stage_times_ms()
+    assert all(v > 0 for v in st.values()), st
     got = (gp.scores, gp.kept_idx, gp.kept_scores, gp.cu_kept, gp.xc, gp.out)
     for a, b in zip(eager, got):
         assert torch.equal(a, b)
