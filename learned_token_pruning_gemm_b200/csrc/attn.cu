@@ -133,9 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
   const int z = blockIdx.z;
-  // issued first; the barrier set-up and TMEM allocation below overlap their latency
-  const int seq0 = cu_kept[b];
-  const int seq1 = cu_kept[b + 1];
   const int kvh = hq / (n_hq / n_hkv);
 
   extern __shared__ uint8_t smem_raw[];
@@ -177,8 +174,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();   // global memory only from here on
 
-  const int len = seq1 - seq0;
+  const int seq0 = cu_kept[b];
+  const int len = cu_kept[b + 1] - seq0;
   const int n_t = (len + kBM - 1) / kBM;
   if (2 * z >= n_t) {           // uniform: this sequence has no pair z
     if (warp == 2) tg::tmem_dealloc(tmem, kTmemCols);
@@ -513,6 +513,8 @@ __global__ void __launch_bounds__(kF32Warps * 32)
                           const float* __restrict__ gain, const float* __restrict__ tau,
                           const int32_t* __restrict__ cu_kept, int batch, int64_t total,
                           int n_hq, int n_hkv, int dh, float* __restrict__ out) {
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * kF32Warps + (threadIdx.x >> 5);
   const int hq = blockIdx.y;
@@ -588,10 +590,8 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
     return TG_ERR_CUDA;
   const int n_qt = (max_kept + kBM - 1) / kBM;
   dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
-  gated_attn_bf16_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, s_kept, gain, tau, cu_kept,
-                                                       n_hq, n_hkv,
-                                                       static_cast<__nv_bfloat16*>(out), status);
-  return tg::launch_status();
+  return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv, s_kept,
+                    gain, tau, cu_kept, n_hq, n_hkv, static_cast<__nv_bfloat16*>(out), status);
 }
 
 }  // namespace
@@ -621,11 +621,10 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
     const int64_t blocks = (total_kept + kF32Warps - 1) / kF32Warps;
     if (blocks > INT32_MAX) return TG_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(blocks), n_hq);
-    gated_attn_f32_kernel<<<grid, kF32Warps * 32, 0, stream>>>(
-        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        s_kept, gain, tau, cu_kept, batch, total_kept, n_hq, n_hkv, head_dim,
-        static_cast<float*>(out));
-    return tg::launch_status();
+    return tg::launch(gated_attn_f32_kernel, grid, dim3(kF32Warps * 32), 0, stream, 0,
+                      static_cast<const float*>(q), static_cast<const float*>(k),
+                      static_cast<const float*>(v), s_kept, gain, tau, cu_kept, batch, total_kept,
+                      n_hq, n_hkv, head_dim, static_cast<float*>(out));
   }
   return TG_ERR_UNSUPPORTED;
 }

@@ -244,6 +244,20 @@ __device__ __forceinline__ void tmem_st_wait() {
 }
 
 // ------------------------------------------------------------------------- //
+// programmatic dependent launch                                              //
+// ------------------------------------------------------------------------- //
+
+// Let the next kernel on the stream start launching its CTAs (each CTA of this
+// grid calls it once; a CTA that exits counts as having called it).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the previous kernel on the stream has completed and its memory
+// operations are visible. Every kernel here calls it before its first global
+// memory access, after a prologue that touches only shared and tensor memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------------------------- //
 // misc                                                                       //
 // ------------------------------------------------------------------------- //
 
@@ -281,5 +295,37 @@ tg_status launch_status();
 // raise a kernel's dynamic shared memory limit to `bytes` on the current device
 // (cached per device and function)
 bool ensure_smem(const void* fn, int bytes);
+
+// Launch `kernel` with programmatic dependent launch allowed (the kernel's
+// prologue may overlap the previous kernel's tail; it calls pdl_wait() before
+// touching global memory) and, if cluster_x > 0, a (cluster_x,1,1) cluster.
+template <typename... KArgs, typename... Args>
+tg_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                 int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_CUDA;
+  }
+  return launch_status();
+}
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 }  // namespace tg

@@ -31,6 +31,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
                                                                 const int32_t* __restrict__ idx,
                                                                 int64_t n_kept) {
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
@@ -75,6 +77,6 @@ extern "C" tg_status tg_compact_kv(const void* const* src, void* const* dst,
   const int64_t warps_needed = n_kept;
   int64_t blocks = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  compact_rows_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(a, kept_idx, n_kept);
-  return tg::launch_status();
+  return tg::launch(compact_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
+                    stream, 0, a, kept_idx, n_kept);
 }

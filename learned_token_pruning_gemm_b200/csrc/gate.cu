@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tg::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();   // global memory only from here on
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----
@@ -163,6 +165,8 @@ __global__ void __launch_bounds__(kF32Threads)
                     int h, float* __restrict__ scores) {
   extern __shared__ float xrow[];
   __shared__ float red[kF32Threads];
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();
   const int64_t i = blockIdx.x;
   for (int c = threadIdx.x; c < d; c += kF32Threads) xrow[c] = x[i * d + c];
   __syncthreads();
@@ -202,9 +206,8 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const int64_t tiles = (n + kBM - 1) / kBM;
-  gate_bf16_kernel<H><<<static_cast<unsigned>(tiles), kThreads, smem, st>>>(tx, tw, b1, w2, b2, n, d,
-                                                                           scores, status);
-  return tg::launch_status();
+  return tg::launch(gate_bf16_kernel<H>, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), smem, st,
+                    0, tx, tw, b1, w2, b2, n, d, scores, status);
 }
 
 }  // namespace
@@ -228,10 +231,9 @@ extern "C" tg_status tg_gate_score(const void* x, tg_dtype dtype, int64_t n_toke
   if (dtype == TG_F32) {
     if (h > 1024 || d > 12288) return TG_ERR_UNSUPPORTED;
     if (n_tokens > INT32_MAX) return TG_ERR_UNSUPPORTED;
-    gate_f32_kernel<<<static_cast<unsigned>(n_tokens), kF32Threads, static_cast<size_t>(d) * 4,
-                      stream>>>(static_cast<const float*>(x), static_cast<const float*>(w1), b1, w2,
-                                b2, d, h, scores);
-    return tg::launch_status();
+    return tg::launch(gate_f32_kernel, dim3(static_cast<unsigned>(n_tokens)), dim3(kF32Threads),
+                      static_cast<size_t>(d) * 4, stream, 0, static_cast<const float*>(x),
+                      static_cast<const float*>(w1), b1, w2, b2, d, h, scores);
   }
   return TG_ERR_UNSUPPORTED;
 }

@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* raw = reinterpret_cast<float*>(keys + chunk);
   uint8_t* kmask = reinterpret_cast<uint8_t*>(raw + chunk);   // keep bits, one byte per 4 keys
 
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
   const unsigned csize = cluster.num_blocks();
@@ -371,21 +373,7 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   const size_t smem = sizeof(SelectSmem) + (size_t)chunk * 8 + (size_t)chunk / 4;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem))
     return TG_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(csize, batch, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, select_topk_kernel, scores, cu_seqlens, doc_begin, doc_end, k_doc,
-                         batch, total_kept, chunk, kept_idx, kept_scores, cu_kept, st) !=
-      cudaSuccess)
-    return TG_ERR_CUDA;
-  return tg::launch_status();
+  return tg::launch(select_topk_kernel, dim3(csize, batch, 1), dim3(kThreads), smem, stream, csize,
+                    scores, cu_seqlens, doc_begin, doc_end, k_doc, batch, total_kept, chunk,
+                    kept_idx, kept_scores, cu_kept, st);
 }

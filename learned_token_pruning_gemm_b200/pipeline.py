@@ -89,8 +89,8 @@ class GatedPrefill:
 
     # ------------------------------------------------------------------ graphs
     def capture(self):
-        """Capture the whole layer (four kernels) as one CUDA graph, with five timing
-        events recorded inside it before, between and after the stages. One eager
+        """Capture the whole layer (four kernels) as CUDA graphs: one as launched in
+        production and one with timing events between the stages. One eager
         step runs first (outside capture) so that every lazily initialised piece of
         the library exists before capture."""
         side = torch.cuda.Stream()
@@ -99,10 +99,17 @@ class GatedPrefill:
             self.step(side)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
-        self.stage_events = [torch.cuda.Event(enable_timing=True, external=True)
-                             for _ in range(5)]
+        # the step as launched in production: kernels back to back, each launched with
+        # programmatic dependent launch so its prologue overlaps the previous tail
         self.step_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.step_graph):
+            self.step()
+        # the same step with timing events between the stages (the event nodes turn
+        # the programmatic edges into full dependencies; used for the breakdown only)
+        self.stage_events = [torch.cuda.Event(enable_timing=True, external=True)
+                             for _ in range(5)]
+        self.timed_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.timed_graph):
             self.step(events=self.stage_events)
         torch.cuda.synchronize()
         return self
@@ -111,7 +118,11 @@ class GatedPrefill:
         """Replay the whole layer (one graph, four kernel launches) on the current stream."""
         self.step_graph.replay()
 
+    def replay_timed(self):
+        """Replay the step with timing events between the stages."""
+        self.timed_graph.replay()
+
     def stage_times_ms(self):
-        """Per-stage device times of the last completed replay (needs a sync first)."""
+        """Per-stage device times of the last completed `replay_timed` (sync first)."""
         ev = self.stage_events
         return {n: ev[i].elapsed_time(ev[i + 1]) for i, n in enumerate(self.STAGES)}

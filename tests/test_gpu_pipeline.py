@@ -101,8 +101,13 @@ def test_graph_replay_matches_eager(mods):
     gp.replay_step()
     torch.cuda.synchronize()
     assert api.device_status(reset=True) == 0
+    got1 = [t.clone() for t in (gp.scores, gp.kept_idx, gp.kept_scores, gp.cu_kept, gp.xc, gp.out)]
+    for t in (gp.scores, gp.kept_scores, gp.out):
+        t.zero_()
+    gp.replay_timed()
+    torch.cuda.synchronize()
     st = gp.stage_times_ms()
     assert all(v > 0 for v in st.values()), st
     got = (gp.scores, gp.kept_idx, gp.kept_scores, gp.cu_kept, gp.xc, gp.out)
-    for a, b in zip(eager, got):
-        assert torch.equal(a, b)
+    for a, b, c in zip(eager, got, got1):
+        assert torch.equal(a, b) and torch.equal(a, c)
