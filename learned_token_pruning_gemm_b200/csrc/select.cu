@@ -19,8 +19,11 @@
 // and the digit holding the K-th key found with a block suffix scan. Emission
 // keeps every token outside the span, every document token with key > T, and the
 // `need` lowest-positioned document tokens with key == T (ties to the lower
-// position); ranks and output offsets come from warp scans, per-warp and per-CTA
-// offsets from block scans and distributed shared memory. No global scratch.
+// position). One counting pass gives each warp's tie count and tie-independent
+// kept count; since the ties kept before any point number min(need, ties before
+// it), one exchange of those two counts through distributed shared memory fixes
+// every CTA's and warp's output offset, and a second pass writes the kept rows
+// in order (ranks from warp scans). No global scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -41,7 +44,9 @@ struct alignas(16) SelectSmem {
   uint32_t hist[2][256];         // this CTA's histogram, by pass parity (read by peers)
   uint32_t scan[8];
   uint32_t warp_tot[kWarps];
+  uint32_t warp_base[kWarps];
   uint32_t warp_off[kWarps];
+  uint32_t warp_eq_off[kWarps];
   uint32_t cta_eq;               // published to peers
   uint32_t cta_keep;             // published to peers
   uint32_t digit;
@@ -51,7 +56,7 @@ struct alignas(16) SelectSmem {
   uint32_t seq_keep;
   int64_t out_base;
   int64_t red[kWarps];
-  // followed by: uint32_t keys[chunk]; float raw[chunk]; uint8_t kmask[chunk / 4];
+  // followed by: uint32_t keys[chunk]; float raw[chunk];
 };
 
 inline int select_cluster(int max_len) {
@@ -89,16 +94,6 @@ __device__ __forceinline__ int64_t seq_kept(const int32_t* cu, const int32_t* db
   return len - nd + k;
 }
 
-// exclusive scan of the per-warp totals (one thread), total returned
-__device__ __forceinline__ uint32_t scan_warp_totals(SelectSmem& S) {
-  uint32_t t = 0;
-  for (int w = 0; w < kWarps; ++w) {
-    S.warp_off[w] = t;
-    t += S.warp_tot[w];
-  }
-  return t;
-}
-
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -122,7 +117,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
   float* raw = reinterpret_cast<float*>(keys + chunk);
-  uint8_t* kmask = reinterpret_cast<uint8_t*>(raw + chunk);   // keep bits, one byte per 4 keys
 
   tg::pdl_launch_dependents();
   tg::pdl_wait();
@@ -250,40 +244,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     need = remaining;
   }
 
-  // ---- emission, phase A: per-warp counts of document keys equal to T ----
+  // ---- emission, pass 1: per-warp counts of ties (document keys == T) and of
+  //      tokens kept regardless of ties (outside the document, or key > T) ----
   {
-    uint32_t cnt = 0;
+    uint32_t ceq = 0, cbase = 0;
     for (int st = 0; st < nsteps; ++st) {
       const uint4 kk = k4[st * 32 + lane];
       const int i4 = seg0 + st * 128 + lane * 4;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) cnt += (i4 + e >= ld0 && i4 + e < ld1 && key_at(kk, e) == T);
+      for (int e = 0; e < 4; ++e) {
+        const int i = i4 + e;
+        const bool in_doc = i >= ld0 && i < ld1;
+        const uint32_t key = key_at(kk, e);
+        ceq += in_doc && key == T;
+        cbase += i < n_local && (!in_doc || key > T);
+      }
     }
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(full, cnt, o);
-    if (lane == 0) S.warp_tot[warp] = cnt;
+    for (int o = 16; o > 0; o >>= 1) {
+      ceq += __shfl_xor_sync(full, ceq, o);
+      cbase += __shfl_xor_sync(full, cbase, o);
+    }
+    if (lane == 0) {
+      S.warp_tot[warp] = ceq;
+      S.warp_base[warp] = cbase;
+    }
     __syncthreads();
-    if (tid == 0) S.cta_eq = scan_warp_totals(S);
+    if (tid == 0) {
+      uint32_t te = 0, tb = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        te += S.warp_tot[w];
+        tb += S.warp_base[w];
+      }
+      S.cta_eq = te;
+      S.cta_keep = tb;   // published: this CTA's tie count and tie-independent count
+    }
     cluster.sync();
     if (tid == 0) {
-      uint32_t off = 0;
-      for (unsigned r = 0; r < rank; ++r) off += *cluster.map_shared_rank(&S.cta_eq, r);
-      S.cta_eq_off = off;
+      // ties kept before a point = min(need, ties before it); this gives every
+      // CTA's and every warp's output offset from (tie, tie-independent) counts
+      uint32_t eq_before = 0, keep_before = 0, keep_total = 0;
+      for (unsigned r = 0; r < csize; ++r) {
+        const uint32_t er = *cluster.map_shared_rank(&S.cta_eq, r);
+        const uint32_t br = *cluster.map_shared_rank(&S.cta_keep, r);
+        const uint32_t kr = br + (need > eq_before ? min(need - eq_before, er) : 0u);
+        if (r == rank) {
+          S.cta_eq_off = eq_before;
+          S.cta_keep_off = keep_before;
+        }
+        if (r < rank) keep_before += kr;
+        keep_total += kr;
+        eq_before += er;
+      }
+      S.seq_keep = keep_total;
+      uint32_t e_off = S.cta_eq_off, k_off = S.cta_keep_off;
+      for (int w = 0; w < kWarps; ++w) {
+        const uint32_t ew = S.warp_tot[w];
+        S.warp_eq_off[w] = e_off;
+        S.warp_off[w] = k_off;
+        k_off += S.warp_base[w] + (need > e_off ? min(need - e_off, ew) : 0u);
+        e_off += ew;
+      }
     }
     __syncthreads();
   }
 
-  // ---- phase B: keep decisions (ties by rank in position order) ----
-  {
-    uint32_t running = S.cta_eq_off + S.warp_off[warp];   // T-ties before this warp's segment
-    uint32_t kept = 0;
+  // ---- pass 2: keep decisions and output, ascending ----
+  const int64_t out_base = S.out_base;
+  const int64_t seq_keep = S.seq_keep;
+  const int64_t expect = len - nd + k_eff;
+  const bool ok = seq_keep == expect && out_base + seq_keep <= total_kept;
+  if (ok) {
+    uint32_t run_eq = S.warp_eq_off[warp];
+    int64_t run_out = out_base + S.warp_off[warp];
     for (int st = 0; st < nsteps; ++st) {
       const uint4 kk = k4[st * 32 + lane];
       const int i4 = seg0 + st * 128 + lane * 4;
       uint32_t ce = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) ce += (i4 + e >= ld0 && i4 + e < ld1 && key_at(kk, e) == T);
-      const uint32_t incl = warp_incl_scan(ce, lane);
-      uint32_t r = running + incl - ce;
+      const uint32_t incl_e = warp_incl_scan(ce, lane);
+      uint32_t rk = run_eq + incl_e - ce;
       uint32_t nib = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -291,45 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool in_doc = i >= ld0 && i < ld1;
         const uint32_t key = key_at(kk, e);
         const bool eq = in_doc && key == T;
-        const bool keep = i < n_local && (!in_doc || key > T || (eq && r < need));
-        r += eq;
+        const bool keep = i < n_local && (!in_doc || key > T || (eq && rk < need));
+        rk += eq;
         nib |= (uint32_t)keep << e;
       }
-      kmask[i4 / 4] = (uint8_t)nib;
-      kept += __popc(nib);
-      running += __shfl_sync(full, incl, 31);
-    }
-    for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(full, kept, o);
-    if (lane == 0) S.warp_tot[warp] = kept;
-    __syncthreads();
-    if (tid == 0) S.cta_keep = scan_warp_totals(S);
-    cluster.sync();
-    if (tid == 0) {
-      uint32_t off = 0, tot = 0;
-      for (unsigned r = 0; r < csize; ++r) {
-        const uint32_t v = *cluster.map_shared_rank(&S.cta_keep, r);
-        if (r < rank) off += v;
-        tot += v;
-      }
-      S.cta_keep_off = off;
-      S.seq_keep = tot;
-    }
-    __syncthreads();
-  }
-
-  // ---- phase C: write kept row ids (and their scores), ascending ----
-  const int64_t out_base = S.out_base;
-  const int64_t seq_keep = S.seq_keep;
-  const int64_t expect = len - nd + k_eff;
-  const bool ok = seq_keep == expect && out_base + seq_keep <= total_kept;
-  if (ok) {
-    int64_t running = out_base + S.cta_keep_off + S.warp_off[warp];
-    for (int st = 0; st < nsteps; ++st) {
-      const int i4 = seg0 + st * 128 + lane * 4;
-      const uint32_t nib = kmask[i4 / 4];
       const uint32_t c = __popc(nib);
-      const uint32_t incl = warp_incl_scan(c, lane);
-      int64_t o = running + incl - c;
+      const uint32_t incl_k = warp_incl_scan(c, lane);
+      int64_t o = run_out + incl_k - c;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if ((nib >> e) & 1u) {
@@ -338,7 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++o;
         }
       }
-      running += __shfl_sync(full, incl, 31);
+      run_eq += __shfl_sync(full, incl_e, 31);
+      run_out += __shfl_sync(full, incl_k, 31);
     }
   }
   if (rank == 0 && tid == 0) {
@@ -370,7 +379,7 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   const int csize = select_cluster(max_seqlen);
   const int chunk = select_chunk(max_seqlen, csize);
   if (chunk > kMaxKeysPerCta) return TG_ERR_UNSUPPORTED;
-  const size_t smem = sizeof(SelectSmem) + (size_t)chunk * 8 + (size_t)chunk / 4;
+  const size_t smem = sizeof(SelectSmem) + (size_t)chunk * 8;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem))
     return TG_ERR_CUDA;
   return tg::launch(select_topk_kernel, dim3(csize, batch, 1), dim3(kThreads), smem, stream, csize,
