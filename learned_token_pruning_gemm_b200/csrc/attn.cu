@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto next_k_ready = [&]() -> bool {
           const int gn = g0 + s_issued;
           return s_issued < nt &&
-                 tg::mbar_try_wait(tg::smem_u32(&S.k_full[gn % kKStages]), (gn / kKStages) & 1);
+                 tg::mbar_test(tg::smem_u32(&S.k_full[gn % kKStages]), (gn / kKStages) & 1);
         };
         if (alive) alive = issue_next() && issue_next();
         for (int j = 0; j < nt && alive; ++j) {
