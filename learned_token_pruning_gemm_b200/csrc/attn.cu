@@ -16,10 +16,10 @@
 //                b_j = log2(e) g_h s_j beside the K tile (its global loads stay off
 //                the TMA issue path).
 //   warp 3       TMA producer of V tiles through a 2-stage ring (free after PV_j).
-//   warp 1       MMA issuer (one thread), order S_0, S_1, S_2, PV_0, S_3, PV_1, ...:
-//                S_j = Q K_j^T into one of three 128-column TMEM buffers (two tiles
-//                ahead of the softmax), and O += P_j V_j with P_j read from TMEM (it
-//                overwrites S_j in place) and V_j as an MN-major shared-memory operand.
+//   warp 1       MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
+//                S_j = Q K_j^T into one of two 128-column TMEM buffers, and
+//                O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
+//                and V_j as an MN-major shared-memory operand.
 //   warps 4-19   softmax, four threads per query row (TMEM lane = row, each
 //                thread 32 keys of the tile): z = S c_h + b_j in the log2 domain
 //                (packed f32x2 FMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile
@@ -28,7 +28,7 @@
 //                TMEM), exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA
 //                pipe (own polynomial) for the 4th, P packed to bf16 into TMEM.
 // Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
-// PV_j and S_{j+3}; the only cross-tile waits are the rare O rescale and, between
+// PV_j and S_{j+2}; the only cross-tile waits are the rare O rescale and, between
 // the two query tiles, the epilogue's read of O before it is overwritten.
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
@@ -81,7 +81,7 @@ struct AttnSmem {
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
   uint64_t v_empty[kVStages];
-  uint64_t s_full[3];
+  uint64_t s_full[2];
   uint64_t p_full;
   uint64_t o_done;
   uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
@@ -91,8 +91,8 @@ struct AttnSmem {
   int abort_flag;
 };
 
-// TMEM columns: S/P buffers at 0, 128 and 256, O at 384 (512 allocated).
-constexpr uint32_t kColS0 = 0, kColO = 384, kTmemCols = 512;
+// TMEM columns: S/P buffers at 0 and 128, O at 256 (512 allocated).
+constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
 
 __device__ __forceinline__ bool all_alive(bool a) { return __all_sync(0xFFFFFFFFu, a); }
 
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mbar_init(&S.v_full[s], 1);
       tg::mbar_init(&S.v_empty[s], 1);
     }
-    for (int s = 0; s < 3; ++s) tg::mbar_init(&S.s_full[s], 1);
+    for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
     tg::mbar_init(&S.p_full, kSoftmaxWarps);
     tg::mbar_init(&S.o_done, 1);
     tg::mbar_init(&S.o_free, kSoftmaxWarps);
@@ -289,14 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
-        const uint32_t d_s = tmem + kColS0 + 128u * (g % 3);
+        const uint32_t d_s = tmem + kColS0 + 128u * (g & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
           tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
                           tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
-        tg::mma_commit(&S.s_full[g % 3]);
+        tg::mma_commit(&S.s_full[g & 1]);
         tg::mma_commit(&S.k_empty[s]);
         return true;
       };
@@ -305,25 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int qi = 0; qi < nq && alive; ++qi) {
         const int nt = tiles[qi] + 1;
         alive = tg::mbar_wait(&S.q_full, qi & 1, status, &S.abort_flag);
-        int s_issued = 0;   // S tiles of this query tile issued so far
-        auto issue_next = [&]() -> bool {
-          if (s_issued >= nt) return true;
-          if (!issue_s(g0 + s_issued)) return false;
-          if (++s_issued == nt) tg::mma_commit(&S.q_empty);   // every S of the tile issued
-          return true;
-        };
-        // the next S tile's K has landed (non-blocking check)
-        auto next_k_ready = [&]() -> bool {
-          const int gn = g0 + s_issued;
-          return s_issued < nt &&
-                 tg::mbar_test(tg::smem_u32(&S.k_full[gn % kKStages]), (gn / kKStages) & 1);
-        };
-        if (alive) alive = issue_next() && issue_next();
+        if (alive) alive = issue_s(g0);
         for (int j = 0; j < nt && alive; ++j) {
           const int g = g0 + j;
-          // S_{g+2} goes into the buffer that held P_{g-1} (PV_{g-1} already issued):
-          // issue it before waiting for P_g when its K tile is there, else after PV_g
-          if (s_issued < j + 3 && next_k_ready() && !issue_next()) { alive = false; break; }
+          // S_{g+1} goes into the buffer that held P_{g-1}; PV_{g-1} was issued before
+          if (j + 1 < nt) {
+            if (!issue_s(g + 1)) { alive = false; break; }
+          } else {
+            tg::mma_commit(&S.q_empty);   // every S of this query tile is issued
+          }
           if (!tg::mbar_wait(&S.p_full, g & 1, status, &S.abort_flag)) { alive = false; break; }
           const int s = g % kVStages;
           if (!tg::mbar_wait(&S.v_full[s], (g / kVStages) & 1, status, &S.abort_flag)) {
@@ -343,12 +333,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
             // (LBO), 8-key groups 1024 B apart (SBO)
             const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g % 3) + kk * 8, bdesc,
+            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g & 1) + kk * 8, bdesc,
                             idesc_o, (j | kk) != 0);
           }
           tg::mma_commit(&S.o_done);
           tg::mma_commit(&S.v_empty[s]);
-          if (s_issued < j + 3 && !issue_next()) { alive = false; break; }
         }
         g0 += nt;
       }
@@ -370,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nt; ++j) {
         const int g = g0 + j;
         const int s = g % kKStages;
-        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g % 3);
-        alive = tg::mbar_wait(&S.s_full[g % 3], (g / 3) & 1, status, &S.abort_flag);
+        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g & 1);
+        alive = tg::mbar_wait(&S.s_full[g & 1], (g >> 1) & 1, status, &S.abort_flag);
         // tile g's bias: k_full[s] completed before S_g was issued and cannot move on
         // before this warp releases k_empty[s]; waiting makes the producer's stores visible
         if (alive) alive = tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag);
@@ -412,47 +401,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.red[g & 1][qq][r] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
         __syncwarp();
         if (lane == 0) tg::mbar_arrive(&S.red_full[g & 1][grp]);
-        // exp2(z - m) with m = the running max; for j > 0 this is computed while the
-        // other quarters' maxima are still on their way (speculatively), and redone
-        // only if the row max grew by more than 2^8
-        uint32_t pk[kQuarter / 2];
-        float lsum_t = 0.f;
-        auto exps = [&](float m) {
-          float ls[2] = {0.f, 0.f};
-          const float nm = -m;
-#pragma unroll
-          for (int c = 0; c < kQuarter; c += 4) {
-            float x0, x1, x2, x3;
-            fadd2(x0, x1, z[c], z[c + 1], nm, nm);
-            fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
-            const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
-            const float p1 = tg::exp2_approx(x1);
-            const float p2 = tg::exp2_approx(x2);
-            const float p3 = tg::exp2_approx(x3);
-            fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
-            fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
-            pk[c >> 1] = tg::pack_bf16x2(p0, p1);
-            pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
-          }
-          lsum_t = ls[0] + ls[1];
-        };
-        if (j > 0) exps(m_run);
         alive = tg::mbar_wait(&S.red_full[g & 1][grp], (g >> 1) & 1, status, &S.abort_flag);
         if (!all_alive(alive)) { alive = false; break; }
         const float mt = fmaxf(fmaxf(S.red[g & 1][0][r], S.red[g & 1][1][r]),
                                fmaxf(S.red[g & 1][2][r], S.red[g & 1][3][r]));
-        float alpha = 1.f;
+        float m_use = m_run, alpha = 1.f;
         bool rescale = false;
-        if (j == 0) {
-          m_run = mt;
-          exps(m_run);
-        } else if (mt > m_run + kRescaleThreshold) {
-          alpha = tg::exp2_approx(m_run - mt);
-          m_run = mt;
-          rescale = true;
-          exps(m_run);
+        if (j == 0 || mt > m_run + kRescaleThreshold) {
+          m_use = fmaxf(m_run, mt);
+          if (j > 0) {
+            alpha = tg::exp2_approx(m_run - m_use);
+            rescale = true;
+          }
         }
-        l_part = l_part * alpha + lsum_t;
+        uint32_t pk[kQuarter / 2];
+        float ls[2] = {0.f, 0.f};
+        const float nm = -m_use;
+#pragma unroll
+        for (int c = 0; c < kQuarter; c += 4) {
+          float x0, x1, x2, x3;
+          fadd2(x0, x1, z[c], z[c + 1], nm, nm);
+          fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
+          const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
+          const float p1 = tg::exp2_approx(x1);
+          const float p2 = tg::exp2_approx(x2);
+          const float p3 = tg::exp2_approx(x3);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
+          pk[c >> 1] = tg::pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
+        }
+        l_part = l_part * alpha + (ls[0] + ls[1]);
+        m_run = m_use;
         if (__any_sync(0xFFFFFFFFu, rescale)) {
           // O must hold PV_{g-1} before it is scaled (phases <= g-2 are confirmed)
           alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
