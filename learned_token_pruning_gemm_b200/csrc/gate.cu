@@ -5,7 +5,12 @@
 //
 // bf16 path: one CTA per 128-token tile computes the whole hidden layer
 // (M=128 tokens x N=h units x K=d) with tcgen05.mma (kind::f16, f32 accumulate)
-// into a 128 x h fp32 accumulator in tensor memory. A TMA producer thread streams
+// into two 128 x h fp32 accumulators in tensor memory, one per half of the
+// reduction (d/2 columns each, accumulated in a fixed order). Even CTAs run the
+// first half first, odd CTAs the second, so at any moment only half of the CTAs
+// read the same w1 tile (every CTA reads all of w1, from L2); the epilogue adds
+// the two accumulators in a fixed order, so a token's score does not depend on
+// which CTA computed it. A TMA producer thread streams
 // 128x64 tiles of x and hx64 tiles of w1 (128-byte swizzle) through a 4-stage
 // mbarrier ring; one MMA thread issues 4 K=16 MMAs per stage and frees the stage
 // with tcgen05.commit. The epilogue never leaves fp32: 16 warps read the
@@ -53,6 +58,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
   const int nk = d / kBK;
+  const int half = nk / 2;                               // k-blocks [0, half) -> accumulator 0
+  const int kstart = (blockIdx.x & 1) ? half : 0;       // odd CTAs start with the second half
+  auto kblock = [&](int i) { const int k = i + kstart; return k < nk ? k : k - nk; };
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -64,7 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::fence_barrier_init();
   }
   if (warp == 2) {
-    tg::tmem_alloc(&S.tmem_base, H);
+    tg::tmem_alloc(&S.tmem_base, 2 * H);
     tg::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -87,8 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
       tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H) * kBK * 2);
-      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
-      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, 0);
+      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kblock(kb) * kBK, static_cast<int>(m0));
+      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kblock(kb) * kBK, 0);
       ++issued;
     }
     if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
@@ -103,10 +111,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
       tg::tc_fence_after();
       const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
+      const int kg = kblock(kb);
+      const uint32_t acc = kg < half ? tmem : tmem + H;     // accumulator of this k-block
+      const bool first = (kg == 0) || (kg == half);         // first k-block of its half
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
-        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                        tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
+        tg::mma_bf16_ss(acc, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                        tg::smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, !first || k != 0);
       }
       tg::mma_commit(&S.empty[s]);
     }
@@ -129,16 +140,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
   if (ok) {
     tg::tc_fence_after();
-    uint32_t r[kCols];
+    uint32_t r[kCols], r2[kCols];
+    const uint32_t lrow = static_cast<uint32_t>(lg * 32) << 16;
 #pragma unroll
-    for (int c = 0; c < kCols; c += 16)
-      tg::tmem_ld16(tmem + (static_cast<uint32_t>(lg * 32) << 16) + cgp * kCols + c, r + c);
+    for (int c = 0; c < kCols; c += 16) {
+      tg::tmem_ld16(tmem + lrow + cgp * kCols + c, r + c);
+      tg::tmem_ld16(tmem + H + lrow + cgp * kCols + c, r2 + c);
+    }
     tg::tmem_ld_wait();
     float a2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < kCols; ++j) {
       const int col = cgp * kCols + j;
-      a2[j & 3] = fmaf(S.w2[col], gelu_erf(__uint_as_float(r[j]) + S.b1[col]), a2[j & 3]);
+      // accumulator 0 is empty when there is a single k-block (half == 0)
+      const float u = (half > 0 ? __uint_as_float(r[j]) : 0.f) + __uint_as_float(r2[j]);
+      a2[j & 3] = fmaf(S.w2[col], gelu_erf(u + S.b1[col]), a2[j & 3]);
     }
     acc = (a2[0] + a2[1]) + (a2[2] + a2[3]);
   }
@@ -151,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 2) {
     tg::tc_fence_after();
-    tg::tmem_dealloc(tmem, H);
+    tg::tmem_dealloc(tmem, 2 * H);
   }
 }
 
