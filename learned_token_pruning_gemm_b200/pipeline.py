@@ -56,10 +56,6 @@ class GatedPrefill:
         self.cu_kept = torch.empty(wl.batch + 1, **i32)
         self.xc = torch.empty((K, wl.d), dtype=self.x.dtype, device=dev)
         self.out = torch.empty_like(self.q)
-        # the compaction runs on a side stream, concurrently with the attention
-        self.side = torch.cuda.Stream(device=dev)
-        self._fork = torch.cuda.Event()
-        self._join = torch.cuda.Event()
 
     def stage_gate(self, stream=None):
         api.gate_score(self.x, self.w1, self.b1, self.w2, self.b2, out=self.scores, stream=stream)
@@ -80,27 +76,18 @@ class GatedPrefill:
     STAGES = ("gate", "select", "compact", "attention")
 
     def step(self, stream=None, events: Optional[list] = None):
-        """Run the four stages. Without `events`: gate and select on the stream, then
-        the compaction on a side stream concurrently with the attention (it only
-        needs select's outputs), joined back before returning. With `events` (a list
-        of 5 CUDA events): the stages run one after another on the stream with the
-        events recorded before, between and after them."""
+        """Run the four stages back to back on one stream (each kernel launched with
+        programmatic dependent launch, so its prologue overlaps the previous one's
+        tail). If `events` is a list of 5 CUDA events, they are recorded on the
+        stream before, between and after the stages."""
         s = stream if stream is not None else torch.cuda.current_stream()
-        if events is not None:
-            fns = (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention)
-            for i, fn in enumerate(fns):
+        fns = (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention)
+        for i, fn in enumerate(fns):
+            if events is not None:
                 events[i].record(s)
-                fn(stream=s)
+            fn(stream=s)
+        if events is not None:
             events[4].record(s)
-            return
-        self.stage_gate(stream=s)
-        self.stage_select(stream=s)
-        self._fork.record(s)
-        self.side.wait_event(self._fork)
-        self.stage_compact(stream=self.side)
-        self.stage_attention(stream=s)
-        self._join.record(self.side)
-        s.wait_event(self._join)
 
     # ------------------------------------------------------------------ graphs
     def capture(self):
