@@ -8,33 +8,28 @@
 // bf16 path (dh = 128). Causal work grows with the query tile index t (tile t
 // meets t+1 key tiles), so each CTA takes the pair of query tiles t and n-1-t of
 // one (query head, sequence): every CTA then does n+1 key tiles and the grid is
-// balanced. Within a query tile, two softmax teams take alternate key tiles (team
-// A the even ones, team B the odd ones), each with its own S buffer, O
-// accumulator, running max and row sum in tensor memory; the two partial results
-// are merged in the epilogue. The tensor core alternates between the teams, so
-// one team's softmax runs under the other team's MMAs.
+// balanced. Per CTA, pipelines run across both query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
-//                ring. A K stage is free once S_j is computed and the team that
-//                owns tile j has read its bias.
+//                ring. A K stage is free once S_j is computed and every softmax
+//                warp has read its bias.
 //   warp 2       allocates TMEM, then stages each tile's per-key bias
-//                b_j = log2(e) g_h s_j beside the K tile (a register ring keeps
-//                three tiles of loads in flight).
+//                b_j = log2(e) g_h s_j beside the K tile (its global loads stay off
+//                the TMA issue path).
 //   warp 3       TMA producer of V tiles through a 2-stage ring (free after PV_j).
-//   warp 1       MMA issuer (one thread): S_0 -> S_A, S_1 -> S_B, then for every
-//                key tile j: PV_j (P_j read from TMEM, V_j as an MN-major shared
-//                operand) into the owning team's O, followed by S_{j+2} into the
-//                same team's S buffer.
-//   warps 4-7    softmax team A, warps 8-11 team B; one thread per query row
-//                (TMEM lane = row), which reads its S row twice from TMEM in
-//                32-key chunks: first for the row max of z = S c_h + b_j (log2
-//                domain, packed f32x2 FMA, c_h = log2(e) / (sqrt(dh) tau_h),
-//                diagonal-tile mask), then for exp2(z - m) and the bf16 P, written
-//                over S columns the thread has already consumed. The running max
-//                moves only when it grows by more than 2^8 (the team's O is then
-//                rescaled in TMEM); exp2 runs on the MUFU pipe for 3 of every 4 keys
-//                and on the FMA pipe (own polynomial) for the 4th.
-//   epilogue     all 8 softmax warps: O = (O_A 2^(m_A-M) + O_B 2^(m_B-M)) /
-//                (l_A 2^(m_A-M) + l_B 2^(m_B-M)), M = max(m_A, m_B), to bf16.
+//   warp 1       MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
+//                S_j = Q K_j^T into one of two 128-column TMEM buffers, and
+//                O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
+//                and V_j as an MN-major shared-memory operand.
+//   warps 4-19   softmax, four threads per query row (TMEM lane = row, each
+//                thread 32 keys of the tile): z = S c_h + b_j in the log2 domain
+//                (packed f32x2 FMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile
+//                mask, row max exchanged through shared memory, a running max that
+//                moves only when it grows by more than 2^8 (O is then rescaled in
+//                TMEM), exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA
+//                pipe (own polynomial) for the 4th, P packed to bf16 into TMEM.
+// Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
+// PV_j and S_{j+2}; the only cross-tile waits are the rare O rescale and, between
+// the two query tiles, the epilogue's read of O before it is overwritten.
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
 #include "common.cuh"
@@ -46,11 +41,12 @@ constexpr int kBN = 128;
 constexpr int kD = 128;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kTeamWarps = 4;                          // per softmax team: one thread per row
-constexpr int kSoftmaxWarps = 2 * kTeamWarps;
-constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
+constexpr int kSoftmaxWarps = 16;
+constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-19 softmax
+constexpr int kQuarter = kBN / 4;                      // keys per softmax thread
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
+constexpr int kPolyEvery = 4;               // every 4th key's exp2 on the FMA pipe
 
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
 // fit_exp2_poly.py in this directory.
@@ -77,54 +73,28 @@ struct AttnSmem {
   uint8_t k[kKStages][2][kBN * 64 * 2];
   uint8_t v[kVStages][2][kBN * 64 * 2];
   float bias[kKStages][kBN];
-  float mrow[2][kBM];                       // [team][row] final running max
-  float lsum[2][kBM];                       // [team][row] final row sum
+  float red[2][4][kBM];                     // [tile parity][quarter][row] partial maxima
+  float lsum[4][kBM];                       // [quarter][row] final partial row sums
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
   uint64_t v_full[kVStages];
   uint64_t v_empty[kVStages];
-  uint64_t s_full[2];                       // [team]
-  uint64_t p_full[2];                       // [team]
-  uint64_t o_done[2];                       // [team]: a PV into that team's O completed
-  uint64_t o_free;                          // the epilogue has read both O's
-  uint64_t fin_full;                        // every softmax warp published m and l
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t o_done;
+  uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
+  uint64_t red_full[2][4];                  // [tile parity][row group]: the four quarters of a row
+  uint64_t l_full[4];                       // [row group]: final row-sum exchange
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// TMEM columns: S_A at 0, S_B at 128, O_A at 256, O_B at 384 (512 allocated).
-constexpr uint32_t kColS = 0, kColO = 256, kTmemCols = 512;
+// TMEM columns: S/P buffers at 0 and 128, O at 256 (512 allocated).
+constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
 
 __device__ __forceinline__ bool all_alive(bool a) { return __all_sync(0xFFFFFFFFu, a); }
-
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                      float c0, float c1);
-
-// z = S c + b for one 32-key chunk, in place over the loaded S values (fp32 bits);
-// on the diagonal tile, key c is masked when c > rel_row (its query row, relative
-// to the chunk's first key)
-__device__ __forceinline__ void chunk_z(uint32_t* u, const float* bias, float c, bool diag,
-                                        int rel_row) {
-  const float4* b4 = reinterpret_cast<const float4*>(bias);
-#pragma unroll
-  for (int k = 0; k < 32; k += 4) {
-    const float4 bb = b4[k / 4];
-    float z0, z1, z2, z3;
-    ffma2(z0, z1, __uint_as_float(u[k]), __uint_as_float(u[k + 1]), c, c, bb.x, bb.y);
-    ffma2(z2, z3, __uint_as_float(u[k + 2]), __uint_as_float(u[k + 3]), c, c, bb.z, bb.w);
-    u[k] = __float_as_uint(z0);
-    u[k + 1] = __float_as_uint(z1);
-    u[k + 2] = __float_as_uint(z2);
-    u[k + 3] = __float_as_uint(z3);
-  }
-  if (diag) {
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      if (k > rel_row) u[k] = __float_as_uint(-INFINITY);
-  }
-}
 
 // packed pair arithmetic (one instruction for two fp32 lanes)
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
@@ -148,7 +118,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-
 
 }  // namespace
 
@@ -175,20 +144,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::mbar_init(&S.q_full, 1);
     tg::mbar_init(&S.q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
-      tg::mbar_init(&S.k_full[s], 1 + 32);              // expect_tx arrival + 32 bias lanes
-      tg::mbar_init(&S.k_empty[s], 1 + kTeamWarps);     // S_j done + bias read by its team
+      tg::mbar_init(&S.k_full[s], 1 + 32);                // expect_tx arrival + 32 bias lanes
+      tg::mbar_init(&S.k_empty[s], 1 + kSoftmaxWarps);    // S_j done + bias read by every warp
     }
     for (int s = 0; s < kVStages; ++s) {
       tg::mbar_init(&S.v_full[s], 1);
       tg::mbar_init(&S.v_empty[s], 1);
     }
-    for (int e = 0; e < 2; ++e) {
-      tg::mbar_init(&S.s_full[e], 1);
-      tg::mbar_init(&S.p_full[e], kTeamWarps);
-      tg::mbar_init(&S.o_done[e], 1);
-    }
+    for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
+    tg::mbar_init(&S.p_full, kSoftmaxWarps);
+    tg::mbar_init(&S.o_done, 1);
     tg::mbar_init(&S.o_free, kSoftmaxWarps);
-    tg::mbar_init(&S.fin_full, kSoftmaxWarps);
+    for (int s = 0; s < 2; ++s)
+      for (int g = 0; g < 4; ++g) tg::mbar_init(&S.red_full[s][g], 4);
+    for (int g = 0; g < 4; ++g) tg::mbar_init(&S.l_full[g], 4);
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
@@ -252,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ---------------- bias staging (32 arrivals per K stage) ----------------
-    // A register ring keeps the loads of the next kKStages tiles in flight.
+    // A register ring keeps the loads of the next kKStages tiles in flight, so the
+    // staging keeps pace with the K ring instead of waiting one load per tile.
     const float gl2 = gain[hq] * kLog2e;
     const int n_tiles = (tiles[0] + 1) + (nq > 1 ? tiles[1] + 1 : 0);
     auto tile_j = [&](int g) { return g <= tiles[0] ? g : g - (tiles[0] + 1); };
@@ -309,25 +279,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: S_0, S_1, PV_0, S_2, PV_1, ... ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
       const uint32_t q0 = tg::smem_u32(S.q[0]);
-      int pc[2] = {0, 0};   // PVs issued per team (phase counters of p_full / o_done)
-      auto issue_s = [&](int g, int team) -> bool {
+      auto issue_s = [&](int g) -> bool {
         const int s = g % kKStages;
         if (!tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
-        const uint32_t d_s = tmem + kColS + 128u * team;
+        const uint32_t d_s = tmem + kColS0 + 128u * (g & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
           tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
                           tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
-        tg::mma_commit(&S.s_full[team]);
+        tg::mma_commit(&S.s_full[g & 1]);
         tg::mma_commit(&S.k_empty[s]);
         return true;
       };
@@ -336,17 +305,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int qi = 0; qi < nq && alive; ++qi) {
         const int nt = tiles[qi] + 1;
         alive = tg::mbar_wait(&S.q_full, qi & 1, status, &S.abort_flag);
-        // S_0 -> team A, S_1 -> team B
-        if (alive) alive = issue_s(g0, 0);
-        if (alive && nt > 1) alive = issue_s(g0 + 1, 1);
-        if (alive && nt <= 2) tg::mma_commit(&S.q_empty);   // every S of the tile issued
+        if (alive) alive = issue_s(g0);
         for (int j = 0; j < nt && alive; ++j) {
           const int g = g0 + j;
-          const int team = j & 1;
-          if (!tg::mbar_wait(&S.p_full[team], pc[team] & 1, status, &S.abort_flag)) {
-            alive = false;
-            break;
+          // S_{g+1} goes into the buffer that held P_{g-1}; PV_{g-1} was issued before
+          if (j + 1 < nt) {
+            if (!issue_s(g + 1)) { alive = false; break; }
+          } else {
+            tg::mma_commit(&S.q_empty);   // every S of this query tile is issued
           }
+          if (!tg::mbar_wait(&S.p_full, g & 1, status, &S.abort_flag)) { alive = false; break; }
           const int s = g % kVStages;
           if (!tg::mbar_wait(&S.v_full[s], (g / kVStages) & 1, status, &S.abort_flag)) {
             alive = false;
@@ -359,205 +327,168 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tg::tc_fence_after();
           const uint32_t v0 = tg::smem_u32(S.v[s][0]);
-          const uint32_t acc = (j >= 2) ? 1u : 0u;   // the team's first tile starts its O
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            // A = P_j in TMEM (16 keys = 8 packed columns per K step); B = V rows
+            // A = P_g in TMEM (16 keys = 8 packed columns per K step); B = V rows
             // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
             // (LBO), 8-key groups 1024 B apart (SBO)
             const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-            tg::mma_bf16_ts(tmem + kColO + 128u * team, tmem + kColS + 128u * team + kk * 8,
-                            bdesc, idesc_o, acc | (kk != 0));
+            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g & 1) + kk * 8, bdesc,
+                            idesc_o, (j | kk) != 0);
           }
-          tg::mma_commit(&S.o_done[team]);
+          tg::mma_commit(&S.o_done);
           tg::mma_commit(&S.v_empty[s]);
-          ++pc[team];
-          // S_{j+2} goes into this team's S buffer, which held P_j (PV_j issued above)
-          if (j + 2 < nt) {
-            if (!issue_s(g + 2, team)) { alive = false; break; }
-            if (j + 3 == nt) tg::mma_commit(&S.q_empty);   // every S of the tile issued
-          }
         }
         g0 += nt;
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- softmax teams: one thread per query row ----------------
-    const int team = (warp - 4) / kTeamWarps;     // 0: even key tiles, 1: odd key tiles
+    // ---------------- softmax: four threads per query row ----------------
     const int grp = warp & 3;                      // row group == TMEM lane quarter
+    const int qq = (warp - 4) >> 2;                // which 32-key quarter of each tile
     const int r = grp * 32 + lane;                 // row within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(grp * 32) << 16;
-    const uint32_t sbuf = tmem + lane_base + kColS + 128u * team;
-    const uint32_t obuf = tmem + lane_base + kColO + 128u * team;
     const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
     bool alive = true;
-    int cnt = 0;   // this team's tiles so far (phase counter of s_full / p_full / o_done)
     int g0 = 0;
     for (int qi = 0; qi < nq && alive; ++qi) {
       const int t = tiles[qi];
       const int nt = t + 1;
-      float m_run = -INFINITY, l_run = 0.f;
-      int jt = 0;    // this team's tiles in this query tile
-      for (int j = team; j < nt; j += 2, ++jt, ++cnt) {
+      float m_run = -INFINITY, l_part = 0.f;
+      for (int j = 0; j < nt; ++j) {
         const int g = g0 + j;
         const int s = g % kKStages;
-        const bool diag = j == t;
-        alive = tg::mbar_wait(&S.s_full[team], cnt & 1, status, &S.abort_flag);
+        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g & 1);
+        alive = tg::mbar_wait(&S.s_full[g & 1], (g >> 1) & 1, status, &S.abort_flag);
         // tile g's bias: k_full[s] completed before S_g was issued and cannot move on
-        // before this team releases k_empty[s]; waiting makes the stores visible
+        // before this warp releases k_empty[s]; waiting makes the producer's stores visible
         if (alive) alive = tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag);
         if (!all_alive(alive)) { alive = false; break; }
         tg::tc_fence_after();
-        const float* bias = S.bias[s];
-        auto make_z = [&](uint32_t* u, int c0) { chunk_z(u, bias + c0, c_h, diag, r - c0); };
-        auto zf = [](const uint32_t* u, int c) { return __uint_as_float(u[c]); };
-        // pass 1: the row max of this tile
-        float mt = -INFINITY;
+        float z[kQuarter];
         {
-          uint32_t ua[32], ub[32];
-          tg::tmem_ld32(sbuf, ua);
-          tg::tmem_ld32(sbuf + 32, ub);
+          uint32_t u[kQuarter];
+          tg::tmem_ld32(sbuf + qq * kQuarter, u);
           tg::tmem_ld_wait();
+          const float4* b4 = reinterpret_cast<const float4*>(S.bias[s] + qq * kQuarter);
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t* u = (ch & 1) ? ub : ua;
-            make_z(u, ch * 32);
-            float mx[4] = {zf(u, 0), zf(u, 1), zf(u, 2), zf(u, 3)};
-#pragma unroll
-            for (int c = 4; c < 32; c += 8) {
-              mx[0] = fmax3(mx[0], zf(u, c), zf(u, c + 1));
-              mx[1] = fmax3(mx[1], zf(u, c + 2), zf(u, c + 3));
-              if (c + 4 < 32) {
-                mx[2] = fmax3(mx[2], zf(u, c + 4), zf(u, c + 5));
-                mx[3] = fmax3(mx[3], zf(u, c + 6), zf(u, c + 7));
-              }
-            }
-            mt = fmaxf(mt, fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]));
-            if (ch < 2) tg::tmem_ld32(sbuf + (ch + 2) * 32, u);   // next chunks in flight
-            if (ch == 1) tg::tmem_ld_wait();
-          }
-        }
-        float alpha = 1.f;
-        bool rescale = false;
-        if (jt == 0) {
-          m_run = mt;
-        } else if (mt > m_run + kRescaleThreshold) {
-          alpha = tg::exp2_approx(m_run - mt);
-          m_run = mt;
-          rescale = true;
-        }
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
-          // this team's O must hold its previous PV before it is scaled
-          alive = tg::mbar_wait(&S.o_done[team], (cnt - 1) & 1, status, &S.abort_flag);
-          if (!all_alive(alive)) { alive = false; break; }
-          tg::tc_fence_after();
-          uint32_t o[32];
-#pragma unroll
-          for (int h = 0; h < kD / 32; ++h) {
-            tg::tmem_ld32(obuf + 32 * h, o);
-            tg::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tg::tmem_st16(obuf + 32 * h, o);
-            tg::tmem_st16(obuf + 32 * h + 16, o + 16);
-          }
-        }
-        // pass 2: exp2(z - m) and P, chunk by chunk; P chunk ch lands on packed
-        // columns [16ch, 16ch+16), inside S columns this thread has already read
-        float ls[2] = {0.f, 0.f};
-        const float nm = -m_run;
-        {
-          uint32_t ua[32], ub[32];
-          tg::tmem_ld32(sbuf, ua);
-          tg::tmem_ld32(sbuf + 32, ub);
-          tg::tmem_ld_wait();
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t* u = (ch & 1) ? ub : ua;
-            make_z(u, ch * 32);
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              float x0, x1, x2, x3;
-              fadd2(x0, x1, zf(u, c), zf(u, c + 1), nm, nm);
-              fadd2(x2, x3, zf(u, c + 2), zf(u, c + 3), nm, nm);
-              const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
-              const float p1 = tg::exp2_approx(x1);
-              const float p2 = tg::exp2_approx(x2);
-              const float p3 = tg::exp2_approx(x3);
-              fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
-              fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
-              pk[c >> 1] = tg::pack_bf16x2(p0, p1);
-              pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
-            }
-            if (ch < 2) tg::tmem_ld32(sbuf + (ch + 2) * 32, u);   // next chunks in flight
-            if (ch == 1) tg::tmem_ld_wait();   // chunks 2 and 3 are in registers
-            tg::tmem_st16(sbuf + ch * 16, pk);
+          for (int c = 0; c < kQuarter; c += 4) {
+            const float4 bb = b4[c / 4];
+            ffma2(z[c], z[c + 1], __uint_as_float(u[c]), __uint_as_float(u[c + 1]), c_h, c_h,
+                  bb.x, bb.y);
+            ffma2(z[c + 2], z[c + 3], __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]), c_h,
+                  c_h, bb.z, bb.w);
           }
         }
         __syncwarp();
         if (lane == 0) tg::mbar_arrive(&S.k_empty[s]);   // this warp is done with the bias
-        l_run = l_run * alpha + (ls[0] + ls[1]);
+        if (j == t) {   // diagonal tile: key qq*32+c is visible to row r iff qq*32+c <= r
+#pragma unroll
+          for (int c = 0; c < kQuarter; ++c)
+            if (qq * kQuarter + c > r) z[c] = -INFINITY;
+        }
+        float mx[4] = {z[0], z[1], z[2], z[3]};
+#pragma unroll
+        for (int c = 4; c < kQuarter; c += 8) {
+          mx[0] = fmax3(mx[0], z[c], z[c + 1]);
+          mx[1] = fmax3(mx[1], z[c + 2], z[c + 3]);
+          if (c + 4 < kQuarter) {
+            mx[2] = fmax3(mx[2], z[c + 4], z[c + 5]);
+            mx[3] = fmax3(mx[3], z[c + 6], z[c + 7]);
+          }
+        }
+        S.red[g & 1][qq][r] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+        __syncwarp();
+        if (lane == 0) tg::mbar_arrive(&S.red_full[g & 1][grp]);
+        alive = tg::mbar_wait(&S.red_full[g & 1][grp], (g >> 1) & 1, status, &S.abort_flag);
+        if (!all_alive(alive)) { alive = false; break; }
+        const float mt = fmaxf(fmaxf(S.red[g & 1][0][r], S.red[g & 1][1][r]),
+                               fmaxf(S.red[g & 1][2][r], S.red[g & 1][3][r]));
+        float m_use = m_run, alpha = 1.f;
+        bool rescale = false;
+        if (j == 0 || mt > m_run + kRescaleThreshold) {
+          m_use = fmaxf(m_run, mt);
+          if (j > 0) {
+            alpha = tg::exp2_approx(m_run - m_use);
+            rescale = true;
+          }
+        }
+        uint32_t pk[kQuarter / 2];
+        float ls[2] = {0.f, 0.f};
+        const float nm = -m_use;
+#pragma unroll
+        for (int c = 0; c < kQuarter; c += 4) {
+          float x0, x1, x2, x3;
+          fadd2(x0, x1, z[c], z[c + 1], nm, nm);
+          fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
+          const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
+          const float p1 = tg::exp2_approx(x1);
+          const float p2 = tg::exp2_approx(x2);
+          const float p3 = tg::exp2_approx(x3);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
+          fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
+          pk[c >> 1] = tg::pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
+        }
+        l_part = l_part * alpha + (ls[0] + ls[1]);
+        m_run = m_use;
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+          // O must hold PV_{g-1} before it is scaled (phases <= g-2 are confirmed)
+          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
+          if (!all_alive(alive)) { alive = false; break; }
+          tg::tc_fence_after();
+          uint32_t o[kQuarter];
+          tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
+          tg::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < kQuarter; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter, o);
+          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter + 16, o + 16);
+        }
+        // P_g over S_g: this thread's 32 keys -> 16 packed columns (every S read of
+        // the row finished before the max exchange above)
+        tg::tmem_st16(sbuf + qq * (kQuarter / 2), pk);
         tg::tmem_st_wait();
-        // confirm this team's previous PV (keeps the o_done phase tracking exact)
-        if (jt > 0) {
-          alive = tg::mbar_wait(&S.o_done[team], (cnt - 1) & 1, status, &S.abort_flag);
+        // confirm PV_{g-1} (keeps the o_done phase tracking exact; normally complete)
+        if (j > 0) {
+          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
           if (!all_alive(alive)) { alive = false; break; }
         }
         tg::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tg::mbar_arrive(&S.p_full[team]);
+        if (lane == 0) tg::mbar_arrive(&S.p_full);
       }
       if (!alive) break;
-      // ---------------- epilogue of this query tile: merge the two teams ----------------
-      S.mrow[team][r] = m_run;
-      S.lsum[team][r] = l_run;
-      if (jt > 0) {   // this team's last PV of the tile
-        alive = tg::mbar_wait(&S.o_done[team], (cnt - 1) & 1, status, &S.abort_flag);
-        if (!all_alive(alive)) { alive = false; break; }
-      }
+      // ---------------- epilogue of this query tile: O / l -> bf16 ----------------
+      const int g_last = g0 + nt - 1;
+      S.lsum[qq][r] = l_part;
       __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.fin_full);
-      alive = tg::mbar_wait(&S.fin_full, qi & 1, status, &S.abort_flag);
+      if (lane == 0) tg::mbar_arrive(&S.l_full[grp]);
+      alive = tg::mbar_wait(&S.l_full[grp], qi & 1, status, &S.abort_flag);
+      if (alive) alive = tg::mbar_wait(&S.o_done, g_last & 1, status, &S.abort_flag);
       if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
-      const bool two = nt > 1;                     // team B had tiles
-      const float ma = S.mrow[0][r], mb = two ? S.mrow[1][r] : -INFINITY;
-      const float mm = fmaxf(ma, mb);
-      const float sa = tg::exp2_approx(ma - mm), sb = two ? tg::exp2_approx(mb - mm) : 0.f;
-      const float la = S.lsum[0][r], lb = two ? S.lsum[1][r] : 0.f;
-      const float inv = 1.f / (la * sa + lb * sb);
-      const float fa = sa * inv, fb = sb * inv;
-      const bool row_ok = t * kBM + r < len;
-      __nv_bfloat16* orow = out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD;
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {                // this thread's 64 output columns
-        const int c0 = team * 64 + 16 * h;
-        uint32_t oa[16], ob[16];
-        tg::tmem_ld16(tmem + lane_base + kColO + c0, oa);
-        if (two) tg::tmem_ld16(tmem + lane_base + kColO + 128u + c0, ob);
-        tg::tmem_ld_wait();
-        if (row_ok) {
-#pragma unroll
-          for (int e = 0; e < 16; e += 8) {
-            float y[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              y[u] = two ? fmaf(__uint_as_float(oa[e + u]), fa, __uint_as_float(ob[e + u]) * fb)
-                         : __uint_as_float(oa[e + u]) * fa;
-            uint4 w;
-            w.x = tg::pack_bf16x2(y[0], y[1]);
-            w.y = tg::pack_bf16x2(y[2], y[3]);
-            w.z = tg::pack_bf16x2(y[4], y[5]);
-            w.w = tg::pack_bf16x2(y[6], y[7]);
-            *reinterpret_cast<uint4*>(orow + c0 + e) = w;
-          }
-        }
-      }
+      const float inv_l = 1.f / ((S.lsum[0][r] + S.lsum[1][r]) + (S.lsum[2][r] + S.lsum[3][r]));
+      uint32_t o[kQuarter];
+      tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
+      tg::tmem_ld_wait();
       tg::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.o_free);   // both O's may now be overwritten
+      if (lane == 0) tg::mbar_arrive(&S.o_free);   // O may now be overwritten
+      if (t * kBM + r < len) {
+        __nv_bfloat16* orow =
+            out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD + qq * kQuarter;
+#pragma unroll
+        for (int e = 0; e < kQuarter; e += 8) {
+          uint4 w;
+          w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+          w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+          w.z = tg::pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+          w.w = tg::pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+          *reinterpret_cast<uint4*>(orow + e) = w;
+        }
+      }
       g0 += nt;
     }
   }
