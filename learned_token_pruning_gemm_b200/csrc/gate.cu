@@ -50,16 +50,13 @@ template <int H>
 __global__ void __launch_bounds__(kThreads, 1)
     gate_bf16_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const float* __restrict__ b1, const float* __restrict__ w2, float b2,
-                     int64_t n_tokens, int d, int rows, float* __restrict__ scores, int* status) {
+                     int64_t n_tokens, int d, float* __restrict__ scores, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   GateSmem<H>& S = *reinterpret_cast<GateSmem<H>*>(smem_raw + pad);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // `rows` (a multiple of 8, <= 128) tokens per CTA: fewer than 128 when that
-  // spreads a short sequence over every SM; the MMA still runs M=128 and the rows
-  // past `rows` in the shared-memory tile are never stored
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * rows;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
   const int nk = d / kBK;
   const int half = nk / 2;                               // k-blocks [0, half) -> accumulator 0
   const int kstart = (blockIdx.x & 1) ? half : 0;       // odd CTAs start with the second half
@@ -97,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kb >= kStages &&
           !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.full[s], (rows + H) * kBK * 2);
+      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + H) * kBK * 2);
       tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kblock(kb) * kBK, static_cast<int>(m0));
       tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kblock(kb) * kBK, 0);
       ++issued;
@@ -164,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   S.part[cgp][row] = acc;
   tg::tc_fence_before();
   __syncthreads();
-  if (tid < rows) {
+  if (tid < kBM) {
     const float s = b2 + ((S.part[0][tid] + S.part[1][tid]) + (S.part[2][tid] + S.part[3][tid]));
     if (m0 + tid < n_tokens) scores[m0 + tid] = s;
   }
@@ -210,25 +207,10 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
                            const float* w2, float b2, float* scores, cudaStream_t st) {
   int* status = tg::status_word();
   if (!status) return TG_ERR_CUDA;
-  // tokens per CTA: 128, or fewer (a multiple of 8) when that puts a CTA on every SM
-  static int n_sm[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return TG_ERR_CUDA;
-  if (!n_sm[dev] &&
-      cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return TG_ERR_CUDA;
-  int rows = kBM;
-  if (n <= static_cast<int64_t>(n_sm[dev]) * kBM) {
-    const int64_t per = (n + n_sm[dev] - 1) / n_sm[dev];
-    rows = static_cast<int>((per + 7) / 8 * 8);
-    if (rows < 8) rows = 8;
-    if (rows > kBM) rows = kBM;
-  }
   CUtensorMap tx, tw;
   const uint64_t dx[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n)};
   const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
-  const uint32_t bx[2] = {kBK, static_cast<uint32_t>(rows)};
+  const uint32_t bx[2] = {kBK, kBM};
   const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H)};
   const uint32_t bw[2] = {kBK, H};
   if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dx, sx, bx,
@@ -239,9 +221,9 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
   const size_t smem = sizeof(GateSmem<H>) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
-  const int64_t tiles = (n + rows - 1) / rows;
+  const int64_t tiles = (n + kBM - 1) / kBM;
   return tg::launch(gate_bf16_kernel<H>, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), smem, st,
-                    0, tx, tw, b1, w2, b2, n, d, rows, scores, status);
+                    0, tx, tw, b1, w2, b2, n, d, scores, status);
 }
 
 }  // namespace
