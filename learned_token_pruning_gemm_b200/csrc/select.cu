@@ -6,7 +6,7 @@
 // budget).
 //
 // One thread-block cluster per sequence, one launch for the whole batch. The
-// cluster has enough CTAs (1..8) for about 16384 keys each (at most 24576), so the
+// cluster has enough CTAs (1..8) for about 4096 keys each (at most 24576), so the
 // passes below stay short. Each CTA holds a contiguous slice of the sequence in
 // shared memory twice: the raw fp32 scores (for the kept-score output) and
 // order-preserving 32-bit keys (NaN lowest, -0 == +0). Tokens outside the
@@ -35,7 +35,7 @@ namespace {
 constexpr int kMaxCluster = 8;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kKeysTarget = 16384;                                   // keys per CTA aimed at
+constexpr int kKeysTarget = 4096;                                    // keys per CTA aimed at
 constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576
 constexpr int kChunkQuant = kWarps * 128;                            // 128 keys per warp step
 
