@@ -41,32 +41,6 @@ def _peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def _dist():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    if ws > 1:
-        import torch.distributed as dist
-        import datetime
-        local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        return dist, dist.get_rank(), ws
-    return None, 0, 1
-
-
-def _barrier(dist):
-    if dist is not None:
-        dist.barrier()
-
-
-def _max_over_ranks(dist, v: float) -> float:
-    if dist is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 class ClockSampler:
     """SM clock and clock-event reasons, sampled by a background thread through
     NVML (about every 0.5 ms) while the benchmark runs; `window(t0, t1)` keeps
@@ -188,9 +162,10 @@ def _threads():
     return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
 
 
-def run_reference(args, dist, rank, ws):
-    """The oracle timed as the reference arm (rank 0 only)."""
-    if rank != 0:
+def run_reference(args, rep):
+    """The oracle timed as the reference arm (rank 0 only; other ranks exit)."""
+    ws = rep.world
+    if rep.rank != 0:
         return
     import oracle
     from learned_token_pruning_gemm_b200 import synth
@@ -218,7 +193,8 @@ def run_reference(args, dist, rank, ws):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, dist, rank, ws):
+def run_ours(args, rep):
+    ws, rank = rep.world, rep.rank
     from learned_token_pruning_gemm_b200 import api, pipeline, synth
     dev_index = torch.cuda.current_device()
     wl = synth.WORKLOADS[args.workload]()
@@ -241,7 +217,7 @@ def run_ours(args, dist, rank, ws):
     # between them outside the events
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
-    _barrier(dist)
+    rep.barrier()
     torch.cuda.synchronize()
     t_host0 = time.perf_counter()
     for a, b in step_ev:
@@ -251,7 +227,7 @@ def run_ours(args, dist, rank, ws):
         b.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.perf_counter()
-    _barrier(dist)
+    rep.barrier()
     clocks.stop()
     clk = clocks.window(t_host0, t_host1)
     status = api.device_status(reset=True)
@@ -267,7 +243,7 @@ def run_ours(args, dist, rank, ws):
         torch.cuda.synchronize()
         per.append(gp.stage_times_ms())
     stage_ms = {name: statistics.mean(p[name] for p in per) for name in gp.STAGES}
-    ms = _max_over_ranks(dist, statistics.mean(step_ms))
+    ms = rep.max(statistics.mean(step_ms))
     value = ws * wl.n_tokens / (ms / 1e3)
 
     # dominant kernel and its roofline
@@ -339,14 +315,14 @@ def run_ours(args, dist, rank, ws):
         torch.cuda.synchronize()
         e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
-        _barrier(dist)
+        rep.barrier()
         for a, b in e_ev:
             a.record(stream)
             e2e_step()
             b.record(stream)
         torch.cuda.synchronize()
-        _barrier(dist)
-        e_ms = _max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in e_ev))
+        rep.barrier()
+        e_ms = rep.max(statistics.mean(a.elapsed_time(b) for a, b in e_ev))
         e2e = {"value": ws * wl.n_tokens / (e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
@@ -406,15 +382,15 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    dist, rank, ws = _dist()
+    from learned_token_pruning_gemm_b200.dist import Replicas
+    rep = Replicas()
     try:
         if args.impl == "reference":
-            run_reference(args, dist, rank, ws)
+            run_reference(args, rep)
         else:
-            run_ours(args, dist, rank, ws)
+            run_ours(args, rep)
     finally:
-        if dist is not None:
-            dist.destroy_process_group()
+        rep.close()
 
 
 if __name__ == "__main__":
