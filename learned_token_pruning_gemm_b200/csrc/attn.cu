@@ -10,25 +10,30 @@
 // one (query head, sequence): every CTA then does n+1 key tiles and the grid is
 // balanced. Per CTA, pipelines run across both query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
-//                ring. A K stage is free once S_j is computed and every softmax
-//                warp has read its bias.
+//                ring. A K stage is free as soon as S_j is computed; with S issued
+//                three tiles ahead, each K load has about three tile periods to land.
 //   warp 2       allocates TMEM, then stages each tile's per-key bias
-//                b_j = log2(e) g_h s_j beside the K tile (its global loads stay off
-//                the TMA issue path).
+//                b_j = log2(e) g_h s_j in a 4-stage ring of its own (so the K ring
+//                never waits for the softmax to read a bias).
 //   warp 3       TMA producer of V tiles through a 2-stage ring (free after PV_j).
-//   warp 1       MMA issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
-//                S_j = Q K_j^T into one of two 128-column TMEM buffers, and
-//                O += P_j V_j with P_j read from TMEM (it overwrites S_j in place)
-//                and V_j as an MN-major shared-memory operand.
-//   warps 4-19   softmax, four threads per query row (TMEM lane = row, each
-//                thread 32 keys of the tile): z = S c_h + b_j in the log2 domain
-//                (packed f32x2 FMA, c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile
-//                mask, row max exchanged through shared memory, a running max that
-//                moves only when it grows by more than 2^8 (O is then rescaled in
-//                TMEM), exp2 on the MUFU pipe for 3 of every 4 keys and on the FMA
-//                pipe (own polynomial) for the 4th, P packed to bf16 into TMEM.
+//   warp 1       MMA issuer (one thread), order S_0, S_1, S_2, PV_0, S_3, PV_1,
+//                S_4, ...: S_j = Q K_j^T into one of three 128-column TMEM buffers,
+//                and O += P_j V_j with P_j read from TMEM (it overwrites S_j in
+//                place) and V_j as an MN-major shared-memory operand. S_{j+3} reuses
+//                the buffer of P_j right after PV_j, so the next two S tiles are
+//                already computed whenever a softmax pass ends.
+//   warps 4-11   softmax, one warp per 16 query rows (TMEM lane = row). S is read
+//                in the 16x256b shape, which puts a row's 128 keys in one quad of
+//                four threads (two rows per thread, 64 values), so row maxima and
+//                sums are warp shuffles with no exchange between warps:
+//                z = S c_h + b_j in the log2 domain (packed f32x2 FMA,
+//                c_h = log2(e) / (sqrt(dh) tau_h)), diagonal-tile mask, a running
+//                max that moves only when it grows by more than 2^8 (O is then
+//                rescaled in TMEM), exp2 on the MUFU pipe for 3 of every 4 keys and
+//                on the FMA pipe (own polynomial) for the 4th, P packed to bf16 and
+//                written over S in the 16x128b shape (the A-operand layout of PV).
 // Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
-// PV_j and S_{j+2}; the only cross-tile waits are the rare O rescale and, between
+// PV_j and S_{j+3}; the only cross-tile waits are the rare O rescale and, between
 // the two query tiles, the epilogue's read of O before it is overwritten.
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
@@ -41,12 +46,12 @@ constexpr int kBN = 128;
 constexpr int kD = 128;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kSoftmaxWarps = 16;
-constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-19 softmax
-constexpr int kQuarter = kBN / 4;                      // keys per softmax thread
+constexpr int kSBufs = 3;                              // S/P buffers in TMEM
+constexpr int kBiasStages = 4;                         // per-key bias ring (beside the K ring)
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
-constexpr int kPolyEvery = 4;               // every 4th key's exp2 on the FMA pipe
 
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
 // fit_exp2_poly.py in this directory.
@@ -72,27 +77,25 @@ struct AttnSmem {
   uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves (16 KB each)
   uint8_t k[kKStages][2][kBN * 64 * 2];
   uint8_t v[kVStages][2][kBN * 64 * 2];
-  float bias[kKStages][kBN];
-  float red[2][4][kBM];                     // [tile parity][quarter][row] partial maxima
-  float lsum[4][kBM];                       // [quarter][row] final partial row sums
+  float bias[kBiasStages][kBN];
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[kKStages];
   uint64_t k_empty[kKStages];
+  uint64_t b_full[kBiasStages];
+  uint64_t b_empty[kBiasStages];
   uint64_t v_full[kVStages];
   uint64_t v_empty[kVStages];
-  uint64_t s_full[2];
+  uint64_t s_full[kSBufs];
   uint64_t p_full;
   uint64_t o_done;
   uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
-  uint64_t red_full[2][4];                  // [tile parity][row group]: the four quarters of a row
-  uint64_t l_full[4];                       // [row group]: final row-sum exchange
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// TMEM columns: S/P buffers at 0 and 128, O at 256 (512 allocated).
-constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
+// TMEM columns: S/P buffers at 0, 128 and 256, O at 384 (512 allocated).
+constexpr uint32_t kColS0 = 0, kColO = 384, kTmemCols = 512;
 
 __device__ __forceinline__ bool all_alive(bool a) { return __all_sync(0xFFFFFFFFu, a); }
 
@@ -144,20 +147,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::mbar_init(&S.q_full, 1);
     tg::mbar_init(&S.q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
-      tg::mbar_init(&S.k_full[s], 1 + 32);                // expect_tx arrival + 32 bias lanes
-      tg::mbar_init(&S.k_empty[s], 1 + kSoftmaxWarps);    // S_j done + bias read by every warp
+      tg::mbar_init(&S.k_full[s], 1);    // expect_tx arrival
+      tg::mbar_init(&S.k_empty[s], 1);   // S_j computed
+    }
+    for (int s = 0; s < kBiasStages; ++s) {
+      tg::mbar_init(&S.b_full[s], 32);              // every lane of the staging warp
+      tg::mbar_init(&S.b_empty[s], kSoftmaxWarps);  // read by every softmax warp
     }
     for (int s = 0; s < kVStages; ++s) {
       tg::mbar_init(&S.v_full[s], 1);
       tg::mbar_init(&S.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) tg::mbar_init(&S.s_full[s], 1);
+    for (int s = 0; s < kSBufs; ++s) tg::mbar_init(&S.s_full[s], 1);
     tg::mbar_init(&S.p_full, kSoftmaxWarps);
     tg::mbar_init(&S.o_done, 1);
     tg::mbar_init(&S.o_free, kSoftmaxWarps);
-    for (int s = 0; s < 2; ++s)
-      for (int g = 0; g < 4; ++g) tg::mbar_init(&S.red_full[s][g], 4);
-    for (int g = 0; g < 4; ++g) tg::mbar_init(&S.l_full[g], 4);
     S.abort_flag = 0;
     tg::fence_barrier_init();
   }
@@ -238,14 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     load(1, v1);
     load(2, v2);
     for (int g = 0; g < n_tiles; ++g) {
-      const int s = g % kKStages;
-      if (g >= kKStages &&
-          !all_alive(tg::mbar_wait(&S.k_empty[s], ((g / kKStages) - 1) & 1, status,
+      const int s = g % kBiasStages;
+      if (g >= kBiasStages &&
+          !all_alive(tg::mbar_wait(&S.b_empty[s], ((g / kBiasStages) - 1) & 1, status,
                                    &S.abort_flag)))
         break;
 #pragma unroll
       for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = gl2 * v0[u];
-      tg::mbar_arrive(&S.k_full[s]);
+      tg::mbar_arrive(&S.b_full[s]);
 #pragma unroll
       for (int u = 0; u < kBN / 32; ++u) {
         v0[u] = v1[u];
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer: S_0, S_1, PV_0, S_2, PV_1, ... ----------------
+    // ---------------- MMA issuer: S_0, S_1, S_2, PV_0, S_3, PV_1, ... ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
@@ -289,14 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
         const uint32_t k0 = tg::smem_u32(S.k[s][0]);
-        const uint32_t d_s = tmem + kColS0 + 128u * (g & 1);
+        const uint32_t d_s = tmem + kColS0 + 128u * (g % kSBufs);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
           tg::mma_bf16_ss(d_s, tg::smem_desc_sw128(q0 + off, 16, 1024),
                           tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
         }
-        tg::mma_commit(&S.s_full[g & 1]);
+        tg::mma_commit(&S.s_full[g % kSBufs]);
         tg::mma_commit(&S.k_empty[s]);
         return true;
       };
@@ -305,15 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int qi = 0; qi < nq && alive; ++qi) {
         const int nt = tiles[qi] + 1;
         alive = tg::mbar_wait(&S.q_full, qi & 1, status, &S.abort_flag);
-        if (alive) alive = issue_s(g0);
+        for (int j = 0; j < kSBufs && j < nt && alive; ++j) alive = issue_s(g0 + j);
+        if (alive && nt <= kSBufs) tg::mma_commit(&S.q_empty);   // every S of the tile issued
         for (int j = 0; j < nt && alive; ++j) {
           const int g = g0 + j;
-          // S_{g+1} goes into the buffer that held P_{g-1}; PV_{g-1} was issued before
-          if (j + 1 < nt) {
-            if (!issue_s(g + 1)) { alive = false; break; }
-          } else {
-            tg::mma_commit(&S.q_empty);   // every S of this query tile is issued
-          }
           if (!tg::mbar_wait(&S.p_full, g & 1, status, &S.abort_flag)) { alive = false; break; }
           const int s = g % kVStages;
           if (!tg::mbar_wait(&S.v_full[s], (g / kVStages) & 1, status, &S.abort_flag)) {
@@ -333,122 +332,151 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 16kk..16kk+15, MN-major: the two 64-wide dh halves are 16 KB apart
             // (LBO), 8-key groups 1024 B apart (SBO)
             const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g & 1) + kk * 8, bdesc,
+            tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g % kSBufs) + kk * 8, bdesc,
                             idesc_o, (j | kk) != 0);
           }
           tg::mma_commit(&S.o_done);
           tg::mma_commit(&S.v_empty[s]);
+          // S_{g+3} goes into the buffer that held P_g (PV_g is ahead of it in the pipe)
+          if (j + kSBufs < nt) {
+            if (!issue_s(g + kSBufs)) { alive = false; break; }
+            if (j + kSBufs + 1 == nt) tg::mma_commit(&S.q_empty);   // every S of the tile issued
+          }
         }
         g0 += nt;
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- softmax: four threads per query row ----------------
-    const int grp = warp & 3;                      // row group == TMEM lane quarter
-    const int qq = (warp - 4) >> 2;                // which 32-key quarter of each tile
-    const int r = grp * 32 + lane;                 // row within the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(grp * 32) << 16;
+    // ---------------- softmax: one warp per 16 query rows ----------------
+    // Warp w reaches TMEM lanes 32(w%4)..+31 and the two warps of a lane quarter
+    // take its two 16-lane halves. In the 16x256b shape thread l holds rows
+    // ra = l/4 and rb = l/4 + 8 of its half at columns 8i + 2(l%4) + {0,1}, i < 16:
+    // a row's 128 keys sit in one quad, so its max and sum are two shuffles.
+    const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int row0 = quarter * 32 + half * 16;
+    const int ra = row0 + (lane >> 2), rb = ra + 8;   // rows within the tile == TMEM lanes
+    const int cq = 2 * (lane & 3);                    // first column within each group of 8
+    const uint32_t lane_base = static_cast<uint32_t>(row0) << 16;
     const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
     bool alive = true;
     int g0 = 0;
     for (int qi = 0; qi < nq && alive; ++qi) {
       const int t = tiles[qi];
       const int nt = t + 1;
-      float m_run = -INFINITY, l_part = 0.f;
+      float ma = -INFINITY, mb = -INFINITY;   // running maxima of rows ra, rb
+      float la = 0.f, lb = 0.f;               // this thread's share of their sums
       for (int j = 0; j < nt; ++j) {
         const int g = g0 + j;
-        const int s = g % kKStages;
-        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g & 1);
-        alive = tg::mbar_wait(&S.s_full[g & 1], (g >> 1) & 1, status, &S.abort_flag);
-        // tile g's bias: k_full[s] completed before S_g was issued and cannot move on
-        // before this warp releases k_empty[s]; waiting makes the producer's stores visible
-        if (alive) alive = tg::mbar_wait(&S.k_full[s], (g / kKStages) & 1, status, &S.abort_flag);
+        const int s = g % kBiasStages;
+        const uint32_t sbuf = tmem + lane_base + kColS0 + 128u * (g % kSBufs);
+        alive = tg::mbar_wait(&S.s_full[g % kSBufs], (g / kSBufs) & 1, status, &S.abort_flag);
+        if (alive) alive = tg::mbar_wait(&S.b_full[s], (g / kBiasStages) & 1, status, &S.abort_flag);
         if (!all_alive(alive)) { alive = false; break; }
         tg::tc_fence_after();
-        float z[kQuarter];
+        float z[64];
         {
-          uint32_t u[kQuarter];
-          tg::tmem_ld32(sbuf + qq * kQuarter, u);
+          uint32_t u[64];
+          tg::tmem_ld_16x256b_x16(sbuf, u);
           tg::tmem_ld_wait();
-          const float4* b4 = reinterpret_cast<const float4*>(S.bias[s] + qq * kQuarter);
+          const float* bias = S.bias[s] + cq;
 #pragma unroll
-          for (int c = 0; c < kQuarter; c += 4) {
-            const float4 bb = b4[c / 4];
-            ffma2(z[c], z[c + 1], __uint_as_float(u[c]), __uint_as_float(u[c + 1]), c_h, c_h,
-                  bb.x, bb.y);
-            ffma2(z[c + 2], z[c + 3], __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]), c_h,
-                  c_h, bb.z, bb.w);
+          for (int i = 0; i < 16; ++i) {
+            const float2 bb = *reinterpret_cast<const float2*>(bias + 8 * i);
+            ffma2(z[4 * i], z[4 * i + 1], __uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]),
+                  c_h, c_h, bb.x, bb.y);
+            ffma2(z[4 * i + 2], z[4 * i + 3], __uint_as_float(u[4 * i + 2]),
+                  __uint_as_float(u[4 * i + 3]), c_h, c_h, bb.x, bb.y);
           }
         }
         __syncwarp();
-        if (lane == 0) tg::mbar_arrive(&S.k_empty[s]);   // this warp is done with the bias
-        if (j == t) {   // diagonal tile: key qq*32+c is visible to row r iff qq*32+c <= r
+        if (lane == 0) tg::mbar_arrive(&S.b_empty[s]);   // this warp is done with the bias
+        if (j == t) {   // diagonal tile: key column c is visible to row r iff c <= r
 #pragma unroll
-          for (int c = 0; c < kQuarter; ++c)
-            if (qq * kQuarter + c > r) z[c] = -INFINITY;
-        }
-        float mx[4] = {z[0], z[1], z[2], z[3]};
+          for (int i = 0; i < 16; ++i) {
 #pragma unroll
-        for (int c = 4; c < kQuarter; c += 8) {
-          mx[0] = fmax3(mx[0], z[c], z[c + 1]);
-          mx[1] = fmax3(mx[1], z[c + 2], z[c + 3]);
-          if (c + 4 < kQuarter) {
-            mx[2] = fmax3(mx[2], z[c + 4], z[c + 5]);
-            mx[3] = fmax3(mx[3], z[c + 6], z[c + 7]);
+            for (int e = 0; e < 2; ++e) {
+              const int c = 8 * i + cq + e;
+              if (c > ra) z[4 * i + e] = -INFINITY;
+              if (c > rb) z[4 * i + 2 + e] = -INFINITY;
+            }
           }
         }
-        S.red[g & 1][qq][r] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-        __syncwarp();
-        if (lane == 0) tg::mbar_arrive(&S.red_full[g & 1][grp]);
-        alive = tg::mbar_wait(&S.red_full[g & 1][grp], (g >> 1) & 1, status, &S.abort_flag);
-        if (!all_alive(alive)) { alive = false; break; }
-        const float mt = fmaxf(fmaxf(S.red[g & 1][0][r], S.red[g & 1][1][r]),
-                               fmaxf(S.red[g & 1][2][r], S.red[g & 1][3][r]));
-        float m_use = m_run, alpha = 1.f;
+        float a0 = fmaxf(z[0], z[1]), a1 = fmaxf(z[4], z[5]);
+        float b0 = fmaxf(z[2], z[3]), b1 = fmaxf(z[6], z[7]);
+#pragma unroll
+        for (int i = 2; i < 16; i += 2) {
+          a0 = fmax3(a0, z[4 * i], z[4 * i + 1]);
+          a1 = fmax3(a1, z[4 * i + 4], z[4 * i + 5]);
+          b0 = fmax3(b0, z[4 * i + 2], z[4 * i + 3]);
+          b1 = fmax3(b1, z[4 * i + 6], z[4 * i + 7]);
+        }
+        float mta = fmaxf(a0, a1), mtb = fmaxf(b0, b1);
+        mta = fmaxf(mta, __shfl_xor_sync(0xFFFFFFFFu, mta, 1));
+        mtb = fmaxf(mtb, __shfl_xor_sync(0xFFFFFFFFu, mtb, 1));
+        mta = fmaxf(mta, __shfl_xor_sync(0xFFFFFFFFu, mta, 2));
+        mtb = fmaxf(mtb, __shfl_xor_sync(0xFFFFFFFFu, mtb, 2));
+        // the running max of a row moves only when the tile max exceeds it by > 2^8
+        float alpha_a = 1.f, alpha_b = 1.f;
         bool rescale = false;
-        if (j == 0 || mt > m_run + kRescaleThreshold) {
-          m_use = fmaxf(m_run, mt);
-          if (j > 0) {
-            alpha = tg::exp2_approx(m_run - m_use);
+        if (j == 0) {
+          ma = mta;
+          mb = mtb;
+        } else {
+          if (mta > ma + kRescaleThreshold) {
+            alpha_a = tg::exp2_approx(ma - mta);
+            ma = mta;
+            rescale = true;
+          }
+          if (mtb > mb + kRescaleThreshold) {
+            alpha_b = tg::exp2_approx(mb - mtb);
+            mb = mtb;
             rescale = true;
           }
         }
-        uint32_t pk[kQuarter / 2];
-        float ls[2] = {0.f, 0.f};
-        const float nm = -m_use;
+        uint32_t pk[32];
+        float sa[2] = {0.f, 0.f}, sb[2] = {0.f, 0.f};
+        const float nma = -ma, nmb = -mb;
 #pragma unroll
-        for (int c = 0; c < kQuarter; c += 4) {
+        for (int i = 0; i < 16; ++i) {
           float x0, x1, x2, x3;
-          fadd2(x0, x1, z[c], z[c + 1], nm, nm);
-          fadd2(x2, x3, z[c + 2], z[c + 3], nm, nm);
+          fadd2(x0, x1, z[4 * i], z[4 * i + 1], nma, nma);
+          fadd2(x2, x3, z[4 * i + 2], z[4 * i + 3], nmb, nmb);
           const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
           const float p1 = tg::exp2_approx(x1);
           const float p2 = tg::exp2_approx(x2);
           const float p3 = tg::exp2_approx(x3);
-          fadd2(ls[0], ls[1], ls[0], ls[1], p0, p1);
-          fadd2(ls[0], ls[1], ls[0], ls[1], p2, p3);
-          pk[c >> 1] = tg::pack_bf16x2(p0, p1);
-          pk[(c >> 1) + 1] = tg::pack_bf16x2(p2, p3);
+          fadd2(sa[0], sa[1], sa[0], sa[1], p0, p1);
+          fadd2(sb[0], sb[1], sb[0], sb[1], p2, p3);
+          pk[2 * i] = tg::pack_bf16x2(p0, p1);       // row ra, packed column 4i + l%4
+          pk[2 * i + 1] = tg::pack_bf16x2(p2, p3);   // row rb, the same column
         }
-        l_part = l_part * alpha + (ls[0] + ls[1]);
-        m_run = m_use;
+        la = la * alpha_a + (sa[0] + sa[1]);
+        lb = lb * alpha_b + (sb[0] + sb[1]);
         if (__any_sync(0xFFFFFFFFu, rescale)) {
           // O must hold PV_{g-1} before it is scaled (phases <= g-2 are confirmed)
           alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
           if (!all_alive(alive)) { alive = false; break; }
           tg::tc_fence_after();
-          uint32_t o[kQuarter];
-          tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
-          tg::tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < kQuarter; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter, o);
-          tg::tmem_st16(tmem + lane_base + kColO + qq * kQuarter + 16, o + 16);
+          for (int hh = 0; hh < 2; ++hh) {   // O columns 64hh .. 64hh+63 of rows ra, rb
+            uint32_t o[32];
+            const uint32_t oaddr = tmem + lane_base + kColO + 64u * hh;
+            tg::tmem_ld_16x256b_x8(oaddr, o);
+            tg::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              o[4 * i] = __float_as_uint(__uint_as_float(o[4 * i]) * alpha_a);
+              o[4 * i + 1] = __float_as_uint(__uint_as_float(o[4 * i + 1]) * alpha_a);
+              o[4 * i + 2] = __float_as_uint(__uint_as_float(o[4 * i + 2]) * alpha_b);
+              o[4 * i + 3] = __float_as_uint(__uint_as_float(o[4 * i + 3]) * alpha_b);
+            }
+            tg::tmem_st_16x256b_x8(oaddr, o);
+          }
         }
-        // P_g over S_g: this thread's 32 keys -> 16 packed columns (every S read of
-        // the row finished before the max exchange above)
-        tg::tmem_st16(sbuf + qq * (kQuarter / 2), pk);
+        // P_g over S_g: packed bf16 pairs, 64 columns (every S read of these rows is done)
+        tg::tmem_st_16x128b_x16(sbuf, pk);
         tg::tmem_st_wait();
         // confirm PV_{g-1} (keeps the o_done phase tracking exact; normally complete)
         if (j > 0) {
@@ -461,33 +489,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!alive) break;
       // ---------------- epilogue of this query tile: O / l -> bf16 ----------------
+      la += __shfl_xor_sync(0xFFFFFFFFu, la, 1);
+      lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 1);
+      la += __shfl_xor_sync(0xFFFFFFFFu, la, 2);
+      lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 2);
       const int g_last = g0 + nt - 1;
-      S.lsum[qq][r] = l_part;
-      __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.l_full[grp]);
-      alive = tg::mbar_wait(&S.l_full[grp], qi & 1, status, &S.abort_flag);
-      if (alive) alive = tg::mbar_wait(&S.o_done, g_last & 1, status, &S.abort_flag);
+      alive = tg::mbar_wait(&S.o_done, g_last & 1, status, &S.abort_flag);
       if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
-      const float inv_l = 1.f / ((S.lsum[0][r] + S.lsum[1][r]) + (S.lsum[2][r] + S.lsum[3][r]));
-      uint32_t o[kQuarter];
-      tg::tmem_ld32(tmem + lane_base + kColO + qq * kQuarter, o);
+      uint32_t o[64];
+      tg::tmem_ld_16x256b_x16(tmem + lane_base + kColO, o);
       tg::tmem_ld_wait();
       tg::tc_fence_before();
       __syncwarp();
       if (lane == 0) tg::mbar_arrive(&S.o_free);   // O may now be overwritten
-      if (t * kBM + r < len) {
-        __nv_bfloat16* orow =
-            out + (static_cast<int64_t>(seq0 + t * kBM + r) * n_hq + hq) * kD + qq * kQuarter;
+      const float ia = 1.f / la, ib = 1.f / lb;
+      const int ga = t * kBM + ra, gb = t * kBM + rb;
+      if (ga < len) {
+        uint32_t* orow = reinterpret_cast<uint32_t*>(
+            out + (static_cast<int64_t>(seq0 + ga) * n_hq + hq) * kD + cq);
 #pragma unroll
-        for (int e = 0; e < kQuarter; e += 8) {
-          uint4 w;
-          w.x = tg::pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
-          w.y = tg::pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-          w.z = tg::pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
-          w.w = tg::pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(orow + e) = w;
-        }
+        for (int i = 0; i < 16; ++i)
+          orow[4 * i] = tg::pack_bf16x2(__uint_as_float(o[4 * i]) * ia,
+                                        __uint_as_float(o[4 * i + 1]) * ia);
+      }
+      if (gb < len) {
+        uint32_t* orow = reinterpret_cast<uint32_t*>(
+            out + (static_cast<int64_t>(seq0 + gb) * n_hq + hq) * kD + cq);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          orow[4 * i] = tg::pack_bf16x2(__uint_as_float(o[4 * i + 2]) * ib,
+                                        __uint_as_float(o[4 * i + 3]) * ib);
       }
       g0 += nt;
     }
