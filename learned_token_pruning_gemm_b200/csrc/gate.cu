@@ -203,6 +203,156 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// 256-token variant, used when there are more 128-token tiles than SMs: every
+// CTA streams all of w1, so a CTA that owns two row tiles halves the w1 bytes per
+// token. Each stage holds two 128x64 x tiles and one hx64 w1 tile; per K=16 step
+// the MMA thread issues one MMA per row tile into its own 128 x h accumulator (2h
+// TMEM columns in all), both with the same w1 operand. Every accumulator is
+// summed over d in one fixed order, so a token's score depends only on its row.
+constexpr int kPairSmemBudget = 196608;   // bytes of x + w1 stages
+
+template <int H>
+struct GatePair {
+  static constexpr int kStageBytes = 2 * kBM * kBK * 2 + H * kBK * 2;
+  static constexpr int kStages = kPairSmemBudget / kStageBytes > 6 ? 6 : kPairSmemBudget / kStageBytes;
+};
+
+template <int H>
+struct GatePairSmem {
+  uint8_t a[GatePair<H>::kStages][2][kBM * kBK * 2];   // two x tiles, 16 KB each
+  uint8_t b[GatePair<H>::kStages][H * kBK * 2];        // w1 tile
+  float b1[H];
+  float w2[H];
+  float part[2][4][kBM];
+  uint64_t full[GatePair<H>::kStages];
+  uint64_t empty[GatePair<H>::kStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int H>
+__global__ void __launch_bounds__(kThreads, 1)
+    gate_bf16_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
+                          const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ b1,
+                          const float* __restrict__ w2, float b2, int64_t n_tokens, int d,
+                          float* __restrict__ scores, int* status) {
+  constexpr int kS = GatePair<H>::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
+  GatePairSmem<H>& S = *reinterpret_cast<GatePairSmem<H>*>(smem_raw + pad);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * (2 * kBM);
+  const int nk = d / kBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kS; ++s) {
+      tg::mbar_init(&S.full[s], 1);
+      tg::mbar_init(&S.empty[s], 1);
+    }
+    tg::mbar_init(&S.acc_full, 1);
+    S.abort_flag = 0;
+    tg::fence_barrier_init();
+  }
+  if (warp == 2) {
+    tg::tmem_alloc(&S.tmem_base, 2 * H);
+    tg::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tg::tma_prefetch_desc(&tm_x);
+    tg::tma_prefetch_desc(&tm_w);
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  tg::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();   // global memory only from here on
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer: two x tiles and the shared w1 tile per stage ----
+    int issued = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kS;
+      if (kb >= kS && !tg::mbar_wait(&S.empty[s], ((kb / kS) - 1) & 1, status, &S.abort_flag))
+        break;
+      tg::mbar_arrive_expect_tx(&S.full[s], GatePair<H>::kStageBytes);
+      tg::tma_load_2d(S.a[s][0], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+      tg::tma_load_2d(S.a[s][1], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0 + kBM));
+      tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, 0);
+      ++issued;
+    }
+    if (S.abort_flag) {   // let copies already in flight land before the CTA can exit
+      for (int kb = issued > kS ? issued - kS : 0; kb < issued; ++kb)
+        tg::mbar_wait(&S.full[kb % kS], (kb / kS) & 1, status, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer: per K=16 step one MMA per row tile, same w1 operand ----
+    constexpr uint32_t idesc = tg::idesc_bf16_f32(kBM, H, false, false);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kS;
+      if (!tg::mbar_wait(&S.full[s], (kb / kS) & 1, status, &S.abort_flag)) break;
+      tg::tc_fence_after();
+      const uint32_t a0 = tg::smem_u32(S.a[s][0]), a1 = tg::smem_u32(S.a[s][1]);
+      const uint32_t b0 = tg::smem_u32(S.b[s]);
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        const uint64_t bdesc = tg::smem_desc_sw128(b0 + 32 * k, 16, 1024);
+        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * k, 16, 1024), bdesc, idesc, acc);
+        tg::mma_bf16_ss(tmem + H, tg::smem_desc_sw128(a1 + 32 * k, 16, 1024), bdesc, idesc, acc);
+      }
+      tg::mma_commit(&S.empty[s]);
+    }
+    tg::mma_commit(&S.acc_full);
+  } else if (warp >= 2) {
+    for (int i = tid - 64; i < H; i += kThreads - 64) {
+      S.b1[i] = b1[i];
+      S.w2[i] = w2[i];
+    }
+  }
+  __syncwarp();
+  tg::named_barrier(1, kThreads);   // b1/w2 staged; producer and MMA loops issued
+
+  // ---- epilogue: all 16 warps, the two row tiles one after the other ----
+  constexpr int kCols = H / 4;
+  const int lg = warp & 3, cgp = warp >> 2;
+  const int row = lg * 32 + lane;
+  const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
+  if (ok) tg::tc_fence_after();
+  const uint32_t lrow = static_cast<uint32_t>(lg * 32) << 16;
+#pragma unroll 1
+  for (int rt = 0; rt < 2; ++rt) {
+    float acc = 0.f;
+    if (ok) {
+      uint32_t r[kCols];
+#pragma unroll
+      for (int c = 0; c < kCols; c += 16) tg::tmem_ld16(tmem + rt * H + lrow + cgp * kCols + c, r + c);
+      tg::tmem_ld_wait();
+      float a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) {
+        const int col = cgp * kCols + j;
+        a2[j & 3] = fmaf(S.w2[col], gelu_as(__uint_as_float(r[j]) + S.b1[col]), a2[j & 3]);
+      }
+      acc = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+    }
+    S.part[rt][cgp][row] = acc;
+  }
+  tg::tc_fence_before();
+  __syncthreads();
+  if (tid < 2 * kBM) {
+    const int rt = tid / kBM, rr = tid % kBM;
+    const float s = b2 + ((S.part[rt][0][rr] + S.part[rt][1][rr]) + (S.part[rt][2][rr] + S.part[rt][3][rr]));
+    if (m0 + tid < n_tokens) scores[m0 + tid] = s;
+  }
+  if (warp == 2) {
+    tg::tc_fence_after();
+    tg::tmem_dealloc(tmem, 2 * H);
+  }
+}
+
 // Exact fp32 path: one CTA per token, hidden units strided over the threads,
 // fixed-order block reduction.
 constexpr int kF32Threads = 128;
@@ -250,10 +400,22 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
       !tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w1, dw, sx, bw,
                        CU_TENSOR_MAP_SWIZZLE_128B))
     return TG_ERR_CUDA;
+  const int64_t tiles = (n + kBM - 1) / kBM;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return TG_ERR_CUDA;
+  if (tiles > sms) {   // more tiles than SMs: two row tiles per CTA, w1 streamed once for both
+    const size_t smem = sizeof(GatePairSmem<H>) + 1024;
+    if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_pair_kernel<H>),
+                         static_cast<int>(smem)))
+      return TG_ERR_CUDA;
+    return tg::launch(gate_bf16_pair_kernel<H>, dim3(static_cast<unsigned>((tiles + 1) / 2)),
+                      dim3(kThreads), smem, st, 0, tx, tw, b1, w2, b2, n, d, scores, status);
+  }
   const size_t smem = sizeof(GateSmem<H>) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gate_bf16_kernel<H>), static_cast<int>(smem)))
     return TG_ERR_CUDA;
-  const int64_t tiles = (n + kBM - 1) / kBM;
   return tg::launch(gate_bf16_kernel<H>, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), smem, st,
                     0, tx, tw, b1, w2, b2, n, d, scores, status);
 }

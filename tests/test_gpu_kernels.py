@@ -35,8 +35,11 @@ def _gen(seed):
 
 # ------------------------------------------------------------------ gate ----
 
+# the last three have more 128-token tiles than the GPU has SMs (148 on B200), so
+# they run the 256-token kernel (two row tiles per CTA), ragged tails included
 @pytest.mark.parametrize("n,d,h", [(300, 128, 64), (129, 256, 128), (1000, 2048, 256),
-                                   (128, 64, 256), (255, 192, 64)])
+                                   (128, 64, 256), (255, 192, 64), (19100, 256, 256),
+                                   (40001, 128, 128), (18945, 192, 64)])
 def test_gate_bf16_vs_oracle(api, orc, n, d, h):
     g = _gen(n + d + h)
     x = torch.randn(n, d, generator=g).to(torch.bfloat16)
@@ -61,12 +64,14 @@ def test_gate_f32_vs_oracle(api, orc):
     assert np.abs(s.cpu().double().numpy() - s64).max() <= GATE_ATOL
 
 
-def test_gate_duplicate_rows_bit_identical(api):
+@pytest.mark.parametrize("n", [1024, 20000])
+def test_gate_duplicate_rows_bit_identical(api, n):
+    # copies in other tiles, in the other row tile of the same CTA, and across CTAs
     g = _gen(4)
-    n, d, h = 1024, 512, 256
+    d, h = 512, 256
     x = torch.randn(n, d, generator=g).to(torch.bfloat16)
-    src = torch.tensor([3, 200, 511, 900])
-    dst = torch.tensor([700, 5, 1023, 128])
+    src = torch.tensor([3, 200, 511, 900, 10, n - 3])    # disjoint from dst
+    dst = torch.tensor([700, 5, 1023, 128, 130, n // 2 + 7])
     x[dst] = x[src]
     w1 = (torch.randn(h, d, generator=g) / math.sqrt(d)).to(torch.bfloat16)
     b1, w2 = torch.randn(h, generator=g) * 0.05, torch.randn(h, generator=g) * 0.06
