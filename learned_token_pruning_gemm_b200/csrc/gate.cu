@@ -19,6 +19,10 @@
 // order, so a token's score depends only on its own row. The GELU's erf is the
 // Abramowitz-Stegun 7.1.26 form (|error| <= 1.5e-7), branch-free.
 //
+// When there are more 128-token tiles than SMs, a 256-token variant runs instead:
+// two row tiles per CTA share every w1 stage (two MMAs per K step into two
+// accumulators), which halves the w1 bytes each token costs.
+//
 // f32 path: an exact fp32 SIMT kernel (one CTA per token) for small checks.
 #include "common.cuh"
 
