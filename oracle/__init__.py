@@ -47,6 +47,10 @@ def lib():
         L.oracle_gated_attention.argtypes = [P, P, P, ctypes.c_int, P, P, P, P, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, P, I64, P]
         L.oracle_gated_attention.restype = None
+        L.oracle_qkv_rope.argtypes = [P, ctypes.c_int, I64, ctypes.c_int, P, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P, I64, P,
+                                      P, P]
+        L.oracle_qkv_rope.restype = None
         _lib = L
     return _lib
 
@@ -133,3 +137,27 @@ def gated_attention(q, k, v, s_kept, gain, tau, cu_kept, rows=None) -> np.ndarra
     lib().oracle_gated_attention(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(s), _ptr(g), _ptr(t),
                                  _ptr(cu), len(cu) - 1, hq, hkv, dh, rp, nr, _ptr(out))
     return out
+
+
+def qkv_rope(xc: torch.Tensor, w: torch.Tensor, hq: int, hkv: int, dh: int, base: float, pos,
+             rows=None):
+    """(q [n,hq,dh], k [n,hkv,dh], v [n,hkv,dh]) fp64: y = W xc split per head, q and k
+    rotated at pos (rotate-half RoPE). Rows not in `rows` are left as NaN."""
+    xr, dt = _raw(xc)
+    wr, dt2 = _raw(w)
+    assert dt == dt2
+    n, d = xr.shape
+    assert wr.shape == ((hq + 2 * hkv) * dh, d)
+    pa = _i32(pos)
+    assert len(pa) == n
+    q = np.full((n, hq, dh), np.nan)
+    k = np.full((n, hkv, dh), np.nan)
+    v = np.full((n, hkv, dh), np.nan)
+    if rows is None:
+        rp, nr = None, 0
+    else:
+        ra = _i32(rows)
+        rp, nr = _ptr(ra), len(ra)
+    lib().oracle_qkv_rope(_ptr(xr), dt, n, d, _ptr(wr), hq, hkv, dh, float(base), _ptr(pa), rp,
+                          nr, _ptr(q), _ptr(k), _ptr(v))
+    return q, k, v

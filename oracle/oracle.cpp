@@ -24,8 +24,12 @@
 //   * every token outside [doc_begin, doc_end) is kept;
 //   * query head hq reads KV head hq / (Hq / Hkv);
 //   * key j is visible to query i iff j <= i in the (position-ordered) kept list.
-// Parity status: gate, select, gather and attention are each pinned by tests
-// (closed forms, brute force, library witnesses, invariants); see tests/.
+//   * the kept tokens' q/k/v projections use the rotary embedding of the Qwen
+//     models the pages evaluate (rotate-half pairing, base given by the caller),
+//     applied at each token's original position (the pages do not describe it).
+// Parity status: gate, select, gather, attention and the q/k/v projection are each
+// pinned by tests (closed forms, brute force, library witnesses, invariants); see
+// tests/.
 
 #include <algorithm>
 #include <cmath>
@@ -189,6 +193,53 @@ void oracle_gated_attention(const void* q, const void* k, const void* v, int dty
         for (int c = 0; c < dh; ++c) acc[c] += w * load_elem(v, dtype, (j * n_hkv + kv) * (int64_t)dh + c);
       }
       for (int c = 0; c < dh; ++c) out[(i * n_hq + hq) * (int64_t)dh + c] = acc[c] / denom;
+    }
+  }
+}
+
+// The kept tokens' projections for the layers above the gate layer (only the K
+// kept tokens get a KV-cache entry: MarkTechPost page, section "Comment TokenGate
+// a-t-il appris le fonctionnement de la réduction des tokens ?"). Plain definition:
+//   y[r] = W xc[r]            W = [Wq; Wk; Wv] of shape [(hq + 2 hkv) dh, d]
+// split per head into q [n, hq, dh], k [n, hkv, dh], v [n, hkv, dh]; q and k heads
+// are rotated at the token's ORIGINAL position p = pos[r] (rotary embedding,
+// rotate-half pairing): for i < dh/2, theta_i = base^(-2i/dh), a = p theta_i,
+//   out[i]        = y[i] cos a - y[i + dh/2] sin a
+//   out[i + dh/2] = y[i + dh/2] cos a + y[i] sin a
+// v is not rotated. Rows listed in `rows` (all rows when rows == nullptr) are
+// computed; the others are left untouched.
+void oracle_qkv_rope(const void* xc, int dtype, int64_t n, int d, const void* w, int hq,
+                     int hkv, int dh, double base, const int32_t* pos, const int32_t* rows,
+                     int64_t n_sel, double* q, double* k, double* v) {
+  const int nh = hq + 2 * hkv;
+  const int64_t cnt = rows ? n_sel : n;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t s = 0; s < cnt; ++s) {
+    const int64_t r = rows ? rows[s] : s;
+    std::vector<double> y((size_t)nh * dh);
+    for (int o = 0; o < nh * dh; ++o) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c)
+        acc += load_elem(w, dtype, (int64_t)o * d + c) * load_elem(xc, dtype, r * d + c);
+      y[o] = acc;
+    }
+    for (int h = 0; h < nh; ++h) {
+      const double* yh = &y[(size_t)h * dh];
+      double* out = h < hq ? q + (r * hq + h) * dh
+                  : h < hq + hkv ? k + (r * hkv + (h - hq)) * dh
+                                 : v + (r * hkv + (h - hq - hkv)) * dh;
+      if (h >= hq + hkv) {   // value heads: no rotation
+        for (int i = 0; i < dh; ++i) out[i] = yh[i];
+        continue;
+      }
+      const int half = dh / 2;
+      for (int i = 0; i < half; ++i) {
+        const double theta = std::pow(base, -2.0 * i / dh);
+        const double a = (double)pos[r] * theta;
+        const double c = std::cos(a), sn = std::sin(a);
+        out[i] = yh[i] * c - yh[i + half] * sn;
+        out[i + half] = yh[i + half] * c + yh[i] * sn;
+      }
     }
   }
 }
