@@ -145,6 +145,27 @@ tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dty
                              int n_hq, int n_hkv, int head_dim, void* out, tg_stream_t stream);
 
 /*
+ * The kept tokens' q/k/v projections for the layers above the gate layer, so the
+ * KV cache is written for the kept tokens only (MarkTechPost page, section
+ * "Comment TokenGate a-t-il appris le fonctionnement de la réduction des tokens
+ * ?": layers above the gate layer process only the K kept tokens). For every row r:
+ *     y = W xc[r],  W = [Wq; Wk; Wv]  [(n_hq + 2 n_hkv) head_dim, d]  (nn.Linear layout)
+ * split per head; q and k heads are rotated at pos[r] (rotary embedding with the
+ * rotate-half pairing (i, i + head_dim/2) and theta_i = rope_base^(-2i/head_dim), the
+ * convention of the Qwen models the pages evaluate; the pages do not describe it),
+ * v heads are copied. The angle pos * theta_i is formed in fp64 and reduced modulo
+ * 2 pi before an fp32 sine and cosine.
+ *   xc  [n_rows, d] bf16: the compacted residual rows (tg_compact_kv)
+ *   pos [n_rows] int32 device, >= 0: original positions within each sequence
+ *   q [n_rows, n_hq, head_dim], k and v [n_rows, n_hkv, head_dim] bf16 outputs
+ * head_dim == 128, n_hq + 2 n_hkv even, d % 64 == 0, rope_base > 1, every pointer
+ * 16-byte aligned; the caller owns every buffer.
+ */
+tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const void* w_qkv, int n_hq,
+                      int n_hkv, int head_dim, float rope_base, const int32_t* pos, void* q,
+                      void* k, void* v, tg_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the first error any kernel recorded on the
  * current device since the last reset (TG_OK if none). reset != 0 clears it.
  */

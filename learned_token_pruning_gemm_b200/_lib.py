@@ -25,6 +25,7 @@ SIGNATURES = {
     "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P]),
     "tg_compact_kv": (INT, [P, P, P, INT, P, I64, P]),
     "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P]),
+    "tg_qkv_rope": (INT, [P, I64, INT, P, INT, INT, INT, F32, P, P, P, P, P]),
     "tg_device_status": (INT, [P, INT]),
     "tg_selftest_bounded_wait": (INT, [I64, P]),
 }

@@ -120,6 +120,28 @@ def gated_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s_kept: t
     return out
 
 
+def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: torch.Tensor,
+             rope_base: float = 1e6, out=None, stream=None):
+    """The kept rows' projections: (q [K,Hq,dh], k [K,Hkv,dh], v [K,Hkv,dh]) bf16 from
+    xc [K,d] bf16 and w_qkv [(Hq+2Hkv)*dh, d] bf16, q/k rotated at pos [K] int32."""
+    K, d = xc.shape
+    n_out = w_qkv.shape[0]
+    if (n_out % (n_hq + 2 * n_hkv)) or w_qkv.shape[1] != d or xc.dtype != w_qkv.dtype:
+        raise TokenGateError("qkv_rope: w_qkv [(Hq+2Hkv)*dh, d] with the dtype of xc")
+    dh = n_out // (n_hq + 2 * n_hkv)
+    if out is None:
+        out = (torch.empty(K, n_hq, dh, dtype=xc.dtype, device=xc.device),
+               torch.empty(K, n_hkv, dh, dtype=xc.dtype, device=xc.device),
+               torch.empty(K, n_hkv, dh, dtype=xc.dtype, device=xc.device))
+    q, k, v = out
+    st = _lib.load().tg_qkv_rope(_cuda(xc, "xc", torch.bfloat16), K, d,
+                                 _cuda(w_qkv, "w_qkv", torch.bfloat16), n_hq, n_hkv, dh,
+                                 float(rope_base), _cuda(pos, "pos", torch.int32), _cuda(q, "q"),
+                                 _cuda(k, "k"), _cuda(v, "v"), _stream(stream))
+    check(st, "tg_qkv_rope")
+    return q, k, v
+
+
 def device_status(reset: bool = True, stream=None) -> int:
     """Synchronise the stream and return (then clear) the device status word."""
     return _lib.load().tg_device_status(_stream(stream), 1 if reset else 0)

@@ -80,3 +80,19 @@ def test_validation_returns_status_without_gpu(lib):
                                   300, fake, None) == UNSUP
     # self test bounds
     assert lib.tg_selftest_bounded_wait(10, None) == INVALID
+    # q/k/v projection: head_dim 128 only, even head total, d % 64, rope_base > 1,
+    # null pointers, alignment; zero rows is a no-op
+    assert lib.tg_qkv_rope(fake, 100, 2048, fake, 16, 8, 64, 1e6, fake, fake, fake, fake,
+                           None) == UNSUP
+    assert lib.tg_qkv_rope(fake, 100, 2048, fake, 15, 8, 128, 1e6, fake, fake, fake, fake,
+                           None) == UNSUP
+    assert lib.tg_qkv_rope(fake, 100, 2000, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+                           None) == UNSUP
+    assert lib.tg_qkv_rope(fake, 100, 2048, fake, 16, 8, 128, 1.0, fake, fake, fake, fake,
+                           None) == INVALID
+    assert lib.tg_qkv_rope(fake, 100, 2048, None, 16, 8, 128, 1e6, fake, fake, fake, fake,
+                           None) == INVALID
+    assert lib.tg_qkv_rope(fake, 100, 2048, fake, 16, 8, 128, 1e6, fake, odd, fake, fake,
+                           None) == MIS
+    assert lib.tg_qkv_rope(None, 0, 2048, None, 16, 8, 128, 1e6, None, None, None, None,
+                           None) == 0
