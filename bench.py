@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -302,6 +303,44 @@ def run_ours(args, rep):
         "us": (stage_ms["select"] + stage_ms["compact"]) * 1e3,
         "frac_hbm": sc_bytes / ((stage_ms["select"] + stage_ms["compact"]) / 1e3) / 1e9 / hbm_peak}
 
+    # ---- the next step on the path, measured on its own (not part of the metric
+    #      above): the kept rows' q/k/v projections with the rotary embedding at
+    #      their original positions, from the compacted residual rows ----
+    next_step = None
+    nh = wl.hq + 2 * wl.hkv
+    if wl.dtype == "bf16" and wl.dh == 128 and nh % 2 == 0:
+        gw = torch.Generator().manual_seed(11)
+        w_qkv = (torch.randn(nh * wl.dh, wl.d, generator=gw) / math.sqrt(wl.d)).to(
+            torch.bfloat16).cuda()
+        kept = gp.kept_idx.cpu().numpy().astype(np.int64)
+        starts = np.repeat(np.asarray(wl.cu_seqlens[:-1], np.int64),
+                           np.diff(gp.cu_kept.cpu().numpy()))
+        pos = torch.from_numpy((kept - starts).astype(np.int32)).cuda()
+        K = gp.xc.shape[0]
+        outs = (torch.empty(K, wl.hq, wl.dh, dtype=torch.bfloat16, device="cuda"),
+                torch.empty(K, wl.hkv, wl.dh, dtype=torch.bfloat16, device="cuda"),
+                torch.empty(K, wl.hkv, wl.dh, dtype=torch.bfloat16, device="cuda"))
+        q_ms = []
+        for i in range(args.steps + 3):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            api.qkv_rope(gp.xc, w_qkv, wl.hq, wl.hkv, pos, rope_base=1e6, out=outs)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                q_ms.append(a.elapsed_time(b))
+        if api.device_status(reset=True) != 0:
+            raise RuntimeError("device status set by the q/k/v projection")
+        t_q = statistics.median(q_ms) / 1e3
+        flops = 2.0 * K * wl.d * nh * wl.dh
+        nbytes = 2.0 * K * wl.d + 2.0 * nh * wl.dh * wl.d + 2.0 * K * nh * wl.dh
+        next_step = {"kept_qkv_rope": {
+            "us": t_q * 1e6, "tflops": flops / t_q / 1e12, "frac_tc": flops / t_q / 1e12 / tf_peak,
+            "gbs": nbytes / t_q / 1e9, "rows": K, "d": wl.d, "heads": f"{wl.hq}/{wl.hkv}",
+            "note": "y = W xc, q/k rotated at the kept tokens' original positions (rotate-half, "
+                    "base 1e6), v copied; CUDA events around one launch, L2 flushed before each"}}
+
     # ---- e2e: host buffers in, result out, through the same public calls ----
     e2e = None
     if not args.no_e2e:
@@ -363,6 +402,7 @@ def run_ours(args, rep):
                        "a second graph with events between the stages"),
             "clocks": clk,
             "e2e": e2e,
+            "next_step": next_step,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
