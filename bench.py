@@ -278,7 +278,7 @@ def run_ours(args, rep):
     if os.path.exists(tpath):
         tr = json.load(open(tpath))
         ent = tr.get(args.workload, {}).get(dom)
-        if ent and ent.get("kernel_rev") == _kernel_rev():
+        if ent and ent.get("kernel_rev") == _kernel_rev(dom):
             traffic = ent["bytes_per_launch"]
     roofline = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
                 "frac": ach / peak, "traffic": traffic, "peak_source": peak_src}
@@ -408,14 +408,18 @@ def run_ours(args, rep):
         print(json.dumps(line), flush=True)
 
 
-def _kernel_rev() -> str:
-    """Hash of the kernel sources, so stale DRAM-traffic figures are not reported."""
+_STAGE_SRC = {"gate": "gate.cu", "select": "select.cu", "compact": "compact.cu",
+              "attention": "attn.cu", "compact+attention": "attn.cu"}
+
+
+def _kernel_rev(stage: str) -> str:
+    """Hash of one stage's kernel source and the shared header, so DRAM-traffic
+    figures are reported only while that kernel is the one they were taken on."""
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "learned_token_pruning_gemm_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in ("common.cuh", _STAGE_SRC[stage]):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 
 
