@@ -5,13 +5,15 @@
 //     y = W xc[r], W = [Wq; Wk; Wv];  q, k rotated at pos[r] (rotate-half pairs
 //     (i, i + dh/2), theta_i = base^(-2i/dh));  v copied.
 //
-// One CTA per 128 rows x 256 output columns (two whole heads): a TMA producer
-// thread streams 128x64 tiles of xc and 256x64 tiles of W (128-byte swizzle)
-// through a 4-stage mbarrier ring; one thread issues 4 tcgen05.mma (M=128, N=256,
-// K=16, bf16 -> fp32) per stage into one 256-column TMEM accumulator. Epilogue,
-// all 16 warps: warp w reads TMEM lanes 32*(w%4).. and, of head (w/4)/2 of the
-// tile, the pairs i in [32*((w/4)%2), +32) and i + 64, so every rotate-half pair is
-// in one thread. The angle p*theta_i is formed in fp64 and reduced modulo 2 pi
+// One CTA per 256 rows x 256 output columns (two whole heads): a TMA producer
+// thread streams, per stage, two 128x64 tiles of xc and one 256x64 tile of W
+// (128-byte swizzle) through a 3-stage mbarrier ring; one thread issues, per K=16
+// step, one tcgen05.mma (M=128, N=256, bf16 -> fp32) per row tile into its own
+// 256-column TMEM accumulator (512 columns in all), both with the same W operand,
+// so W is streamed once per 256 rows. Epilogue, all 16 warps, one row tile after
+// the other: warp w reads TMEM lanes 32*(w%4).. and, of head (w/4)/2 of the tile,
+// the pairs i in [32*((w/4)%2), +32) and i + 64, so every rotate-half pair is in
+// one thread. The angle p*theta_i is formed in fp64 and reduced modulo 2 pi
 // (positions reach 1e5 and more, where an fp32 product alone is off by ~1e-2 rad),
 // then the fp32 sine and cosine of the reduced angle (MUFU, absolute error about
 // 2^-21 on [-pi, pi]); the rotation and the bf16 rounding are fp32.
@@ -19,16 +21,16 @@
 
 namespace {
 
-constexpr int kBM = 128;      // rows per tile
+constexpr int kBM = 128;      // rows per row tile (two row tiles per CTA)
 constexpr int kBN = 256;      // output columns per tile: two heads of 128
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 512;
 constexpr int kDh = 128;
 constexpr int kHalf = kDh / 2;
 
 struct QkvSmem {
-  uint8_t a[kStages][kBM * kBK * 2];   // xc tiles, 16 KB
+  uint8_t a[kStages][2][kBM * kBK * 2];   // two xc tiles, 16 KB each
   uint8_t b[kStages][kBN * kBK * 2];   // W tiles, 32 KB
   double theta[kHalf];                 // base^(-2i/dh)
   uint64_t full[kStages];
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   QkvSmem& S = *reinterpret_cast<QkvSmem*>(smem_raw + pad);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * (2 * kBM);
   const int n0 = blockIdx.y * kBN;   // first output column (= 128 * first head)
   const int nk = d / kBK;
 
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::fence_barrier_init();
   }
   if (warp == 2) {
-    tg::tmem_alloc(&S.tmem_base, kBN);
+    tg::tmem_alloc(&S.tmem_base, 2 * kBN);
     tg::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -88,8 +90,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kb >= kStages &&
           !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.full[s], (kBM + kBN) * kBK * 2);
-      tg::tma_load_2d(S.a[s], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+      tg::mbar_arrive_expect_tx(&S.full[s], (2 * kBM + kBN) * kBK * 2);
+      tg::tma_load_2d(S.a[s][0], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+      tg::tma_load_2d(S.a[s][1], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0 + kBM));
       tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, n0);
       ++issued;
     }
@@ -104,28 +107,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = kb % kStages;
       if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
       tg::tc_fence_after();
-      const uint32_t a0 = tg::smem_u32(S.a[s]), b0 = tg::smem_u32(S.b[s]);
+      const uint32_t a0 = tg::smem_u32(S.a[s][0]), a1 = tg::smem_u32(S.a[s][1]);
+      const uint32_t b0 = tg::smem_u32(S.b[s]);
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk)
-        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * kk, 16, 1024),
-                        tg::smem_desc_sw128(b0 + 32 * kk, 16, 1024), idesc,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kBK / 16; ++kk) {
+        const uint64_t bdesc = tg::smem_desc_sw128(b0 + 32 * kk, 16, 1024);
+        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+        tg::mma_bf16_ss(tmem, tg::smem_desc_sw128(a0 + 32 * kk, 16, 1024), bdesc, idesc, acc);
+        tg::mma_bf16_ss(tmem + kBN, tg::smem_desc_sw128(a1 + 32 * kk, 16, 1024), bdesc, idesc,
+                        acc);
+      }
       tg::mma_commit(&S.empty[s]);
     }
     tg::mma_commit(&S.acc_full);
   }
   __syncwarp();
 
-  // ---- epilogue: all 16 warps ----
+  // ---- epilogue: all 16 warps, the two row tiles one after the other ----
   const int lg = warp & 3, cg = warp >> 2;
   const int hh = cg >> 1;                 // head within the tile
   const int i0 = (cg & 1) * 32;           // this thread's pairs: i0 .. i0+31 and +64
-  const int64_t r = m0 + lg * 32 + lane;  // row == TMEM lane
   const int gh = n0 / kDh + hh;           // global head index in [q heads, k heads, v heads]
-  if (tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag)) {
-    tg::tc_fence_after();
+  const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
+  if (ok) tg::tc_fence_after();
+#pragma unroll 1
+  for (int rt = 0; rt < 2 && ok; ++rt) {
+    const int64_t r = m0 + rt * kBM + lg * 32 + lane;   // row; TMEM lane lg*32 + lane
     uint32_t ya[32], yb[32];
-    const uint32_t base = tmem + (static_cast<uint32_t>(lg * 32) << 16) + hh * kDh + i0;
+    const uint32_t base =
+        tmem + (static_cast<uint32_t>(lg * 32) << 16) + rt * kBN + hh * kDh + i0;
     tg::tmem_ld32(base, ya);
     tg::tmem_ld32(base + kHalf, yb);
     tg::tmem_ld_wait();
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 2) {
     tg::tc_fence_after();
-    tg::tmem_dealloc(tmem, kBN);
+    tg::tmem_dealloc(tmem, 2 * kBN);
   }
 }
 
@@ -214,7 +224,8 @@ extern "C" tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const vo
   const size_t smem = sizeof(QkvSmem) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(qkv_rope_kernel), static_cast<int>(smem)))
     return TG_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>((n_rows + kBM - 1) / kBM), static_cast<unsigned>(n_out / kBN));
+  const dim3 grid(static_cast<unsigned>((n_rows + 2 * kBM - 1) / (2 * kBM)),
+                  static_cast<unsigned>(n_out / kBN));
   return tg::launch(qkv_rope_kernel, grid, dim3(kThreads), smem, stream, 0, tx, tw, n_rows, d, n_hq,
                     n_hkv, log(static_cast<double>(rope_base)), pos,
                     static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
