@@ -110,53 +110,41 @@ def _work(wl):
     esz = 2 if wl.dtype == "bf16" else 4
     Ks = wl.kept_counts
     K = sum(Ks)
+    nh = wl.hq + 2 * wl.hkv
     return {
         "gate_bytes": esz * N * d + esz * d * h + 4 * N,
         "gate_flops": 2 * N * d * h,
         "select_bytes": 4 * N + 8 * K,
         "compact_bytes": 2 * K * d * esz,
         "attn_flops": sum(4 * dh * hq * k * (k + 1) // 2 for k in Ks),
+        "project_flops": 2 * K * d * nh * dh,
     }
 
 
-def _oracle_sample_time(wl, oracle, n_gate=4096, n_attn_rows=128):
-    """Oracle time for one whole step, extrapolated from a bounded sample: gate on
-    n_gate rows (scaled by N), select and gather in full, attention on n_attn_rows
-    query rows per sequence (scaled by the causal pair count)."""
-    rng = np.random.default_rng(0)
-    N = wl.n_tokens
-    rows = np.sort(rng.choice(N, min(n_gate, N), replace=False))
+def _oracle_step(wl, oracle):
+    """One whole step of the fp64 oracle on the host cores: gate on every row, select,
+    gather, and attention on every kept query row and head. Returns (seconds, per-stage
+    seconds)."""
     t0 = time.perf_counter()
-    s64, s32 = oracle.gate_score(wl.x[torch.from_numpy(rows)], wl.w1, wl.b1, wl.w2, wl.b2)
-    t_gate = (time.perf_counter() - t0) * N / len(rows)
-    scores = np.zeros(N, np.float32)
-    scores[rows] = s32
-    sel = wl.score_override.numpy() if wl.score_override is not None else scores
-    t0 = time.perf_counter()
+    _, s32 = oracle.gate_score(wl.x, wl.w1, wl.b1, wl.w2, wl.b2)
+    t1 = time.perf_counter()
+    sel = wl.score_override.numpy() if wl.score_override is not None else s32
     idx, cu = oracle.select_topk(sel, wl.cu_seqlens, wl.doc_begin, wl.doc_end, wl.k_doc)
-    t_sel = time.perf_counter() - t0
-    t0 = time.perf_counter()
+    t2 = time.perf_counter()
     oracle.gather_rows(wl.x.view(torch.int16).numpy(), idx)
-    t_gather = time.perf_counter() - t0
-    # attention sample: rows spread over each sequence; cost ~ (row index + 1)
-    arows, pairs_sample = [], 0
-    for b in range(wl.batch):
-        a, e = int(cu[b]), int(cu[b + 1])
-        if e <= a:
-            continue
-        r = np.unique(np.linspace(a, e - 1, min(n_attn_rows, e - a)).astype(np.int32))
-        arows.append(r)
-        pairs_sample += int(np.sum(r - a + 1))
-    arows = np.concatenate(arows)
-    pairs_full = sum(k * (k + 1) // 2 for k in wl.kept_counts)
-    t0 = time.perf_counter()
-    oracle.gated_attention(wl.q, wl.k, wl.v, sel[idx], wl.gain, wl.tau, cu, rows=arows)
-    t_attn = (time.perf_counter() - t0) * pairs_full / max(pairs_sample, 1)
-    total = t_gate + t_sel + t_gather + t_attn
-    sample = (f"oracle fp64 on host cores: gate on {len(rows)} of {N} rows (x{N / len(rows):.0f}), "
-              f"select+gather in full, attention on {len(arows)} query rows x {wl.hq} heads "
-              f"(scaled by causal pairs x{pairs_full / max(pairs_sample, 1):.0f})")
-    return total, {"gate": t_gate, "select": t_sel, "compact": t_gather, "attention": t_attn}, sample
+    t3 = time.perf_counter()
+    oracle.gated_attention(wl.q, wl.k, wl.v, sel[idx], wl.gain, wl.tau, cu)
+    t4 = time.perf_counter()
+    return t4 - t0, {"gate": t1 - t0, "select": t2 - t1, "compact": t3 - t2, "attention": t4 - t3}
+
+
+def _oracle_warm(wl, oracle):
+    """A small untimed pass over the same code (threads started, pages touched)."""
+    rows = torch.arange(min(256, wl.n_tokens))
+    oracle.gate_score(wl.x[rows], wl.w1, wl.b1, wl.w2, wl.b2)
+    cu = np.array([0, min(64, wl.total_kept)], np.int32)
+    oracle.gated_attention(wl.q[:cu[1]], wl.k[:cu[1]], wl.v[:cu[1]], np.zeros(cu[1], np.float32),
+                           wl.gain, wl.tau, cu)
 
 
 def _threads():
@@ -164,8 +152,20 @@ def _threads():
     return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
 
 
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def run_reference(args, rep):
-    """The oracle timed as the reference arm (rank 0 only; other ranks exit)."""
+    """The oracle timed as the reference arm (rank 0 only; other ranks exit): each
+    timed step is one whole step of the workload (no sampling, no extrapolation)."""
     ws = rep.world
     if rep.rank != 0:
         return
@@ -174,93 +174,113 @@ def run_reference(args, rep):
     oracle.build()
     wl = synth.WORKLOADS[args.workload]()
     for _ in range(args.warmup):
-        _oracle_sample_time(wl, oracle, n_gate=64, n_attn_rows=4)
-    times = []
-    sample = ""
-    for _ in range(args.steps):
-        t, _, sample = _oracle_sample_time(wl, oracle)
-        times.append(t)
+        _oracle_warm(wl, oracle)
+    times = [_oracle_step(wl, oracle)[0] for _ in range(args.steps)]
     ms = 1e3 * statistics.mean(times)
     value = wl.n_tokens / (ms / 1e3)
+    sample = (f"the whole {args.workload} step ({wl.n_tokens} tokens, K={wl.total_kept}): gate on "
+              f"every row, select, gather, attention on every kept row and head; fp64 oracle")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "tokens": wl.n_tokens, "kept": wl.total_kept},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(),
+                         "cpu_model": _cpu_model(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, rep):
-    ws, rank = rep.world, rep.rank
-    from learned_token_pruning_gemm_b200 import api, pipeline, synth
-    dev_index = torch.cuda.current_device()
-    wl = synth.WORKLOADS[args.workload]()
-    gp = pipeline.GatedPrefill(wl)
-    stream = torch.cuda.current_stream()
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device="cuda")
+class _Flush:
+    """Evict the inputs from L2 between timed steps: write a buffer larger than L2,
+    then read another one, so the lines left behind are clean (otherwise the first
+    kernel of the next step pays for writing back the flush buffer's dirty lines)."""
 
-    def flush_l2():
-        # evict the inputs (write a buffer larger than L2), then read another buffer
-        # larger than L2 so the lines left behind are clean: otherwise the first
-        # kernel of the step pays for writing back the flush buffer's dirty lines
-        flush.zero_()
-        clean.sum()
-    work = _work(wl)
-    peaks, peak_src = _peaks()
+    def __init__(self):
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        self.clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device="cuda")
 
-    clocks = ClockSampler(dev_index)
-    clocks.start()
-    gp.capture()                          # the whole layer as one CUDA graph
-    for _ in range(args.warmup):
-        flush_l2()
+    def __call__(self):
+        self.flush.zero_()
+        self.clean.sum()
+
+
+def _time_layer(gp, steps, warmup, rep, flush, stream, clocks=None):
+    """Capture the layer as a CUDA graph, run `warmup` untimed steps, then time exactly
+    `steps` steps (CUDA events on the launching stream around each replay, L2 flushed
+    before each, outside the events), bracketed by barriers. Then a second pass with
+    events between the stages for the per-stage breakdown. Returns (max over ranks of
+    the mean step ms, per-stage ms, clock window)."""
+    from learned_token_pruning_gemm_b200 import api
+    gp.capture()
+    for _ in range(warmup):
+        flush()
         gp.replay_step()
     torch.cuda.synchronize()
-    assert api.device_status(reset=True) == 0
-
-    # timed region: exactly `steps` whole-layer steps (one graph each), L2 flushed
-    # between them outside the events
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
+    if api.device_status(reset=True) != 0:
+        raise RuntimeError("device status set during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
     rep.barrier()
     torch.cuda.synchronize()
-    t_host0 = time.perf_counter()
-    for a, b in step_ev:
-        flush_l2()
+    t0 = time.perf_counter()
+    for a, b in ev:
+        flush()
         a.record(stream)
         gp.replay_step()
         b.record(stream)
     torch.cuda.synchronize()
-    t_host1 = time.perf_counter()
+    t1 = time.perf_counter()
     rep.barrier()
-    clocks.stop()
-    clk = clocks.window(t_host0, t_host1)
-    status = api.device_status(reset=True)
-    if status != 0:
-        raise RuntimeError(f"device status {status} during the timed region")
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-
-    # per-stage breakdown (separate pass): events recorded inside the step graph
+    clk = clocks.window(t0, t1) if clocks is not None else None
+    if api.device_status(reset=True) != 0:
+        raise RuntimeError("device status set during the timed region")
+    step_ms = rep.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
     per = []
-    for _ in range(args.steps):
-        flush_l2()
+    for _ in range(steps):
+        flush()
         gp.replay_timed()
         torch.cuda.synchronize()
         per.append(gp.stage_times_ms())
-    stage_ms = {name: statistics.mean(p[name] for p in per) for name in gp.STAGES}
-    ms = rep.max(statistics.mean(step_ms))
-    value = ws * wl.n_tokens / (ms / 1e3)
+    stage_ms = {n: statistics.mean(p[n] for p in per) for n in gp.STAGES}
+    return step_ms, stage_ms, clk
 
-    # dominant kernel and its roofline
-    dom = max(stage_ms, key=stage_ms.get)
+
+def _stages_report(work, stage_ms, tf_peak, hbm_peak):
+    st = {}
+    for name, ms in stage_ms.items():
+        t = ms / 1e3
+        e = {"us": ms * 1e3}
+        if name == "gate":
+            e["tflops"] = work["gate_flops"] / t / 1e12
+            e["gbs"] = work["gate_bytes"] / t / 1e9
+        elif name == "select":
+            e["gbs"] = work["select_bytes"] / t / 1e9
+        elif name == "compact":
+            e["gbs"] = work["compact_bytes"] / t / 1e9
+        elif name == "attention":
+            e["tflops"] = work["attn_flops"] / t / 1e12
+        elif name == "project":
+            e["tflops"] = work["project_flops"] / t / 1e12
+        if "tflops" in e:
+            e["frac_tc"] = e["tflops"] / tf_peak
+        if "gbs" in e:
+            e["frac_hbm"] = e["gbs"] / hbm_peak
+        st[name] = e
+    if "select" in stage_ms and "compact" in stage_ms:
+        t = (stage_ms["select"] + stage_ms["compact"]) / 1e3
+        st["select+compact"] = {
+            "us": t * 1e6,
+            "frac_hbm": (work["select_bytes"] + work["compact_bytes"]) / t / 1e9 / hbm_peak}
+    return st
+
+
+def _roofline(work, stage_ms, tf_peak, hbm_peak, peak_src, workload):
+    """The dominant kernel of the step against its bound."""
+    dom = max((n for n in stage_ms if n != "project"), key=stage_ms.get)
     t = stage_ms[dom] / 1e3
-    tf_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     if dom == "attention":
         ach, peak, unit, bound = work["attn_flops"] / t / 1e12, tf_peak, "TFLOP/s", "tensor"
     elif dom == "gate":
@@ -276,70 +296,62 @@ def run_ours(args, rep):
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if os.path.exists(tpath):
-        tr = json.load(open(tpath))
-        ent = tr.get(args.workload, {}).get(dom)
+        ent = json.load(open(tpath)).get(workload, {}).get(dom)
         if ent and ent.get("kernel_rev") == _kernel_rev(dom):
             traffic = ent["bytes_per_launch"]
-    roofline = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                "frac": ach / peak, "traffic": traffic, "peak_source": peak_src}
-    stages = {
-        "gate": {"us": stage_ms["gate"] * 1e3,
-                 "tflops": work["gate_flops"] / (stage_ms["gate"] / 1e3) / 1e12,
-                 "gbs": work["gate_bytes"] / (stage_ms["gate"] / 1e3) / 1e9},
-        "select": {"us": stage_ms["select"] * 1e3,
-                   "gbs": work["select_bytes"] / (stage_ms["select"] / 1e3) / 1e9},
-        "compact": {"us": stage_ms["compact"] * 1e3,
-                    "gbs": work["compact_bytes"] / (stage_ms["compact"] / 1e3) / 1e9},
-        "attention": {"us": stage_ms["attention"] * 1e3,
-                      "tflops": work["attn_flops"] / (stage_ms["attention"] / 1e3) / 1e12},
-    }
-    for s in stages.values():
-        if "tflops" in s:
-            s["frac_tc"] = s["tflops"] / tf_peak
-        if "gbs" in s:
-            s["frac_hbm"] = s["gbs"] / hbm_peak
-    sc_bytes = work["select_bytes"] + work["compact_bytes"]
-    stages["select+compact"] = {
-        "us": (stage_ms["select"] + stage_ms["compact"]) * 1e3,
-        "frac_hbm": sc_bytes / ((stage_ms["select"] + stage_ms["compact"]) / 1e3) / 1e9 / hbm_peak}
+    return {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+            "frac": ach / peak, "traffic": traffic, "peak_source": peak_src}
 
-    # ---- the next step on the path, measured on its own (not part of the metric
-    #      above): the kept rows' q/k/v projections with the rotary embedding at
-    #      their original positions, from the compacted residual rows ----
-    next_step = None
-    nh = wl.hq + 2 * wl.hkv
-    if wl.dtype == "bf16" and wl.dh == 128 and nh % 2 == 0:
-        gw = torch.Generator().manual_seed(11)
-        w_qkv = (torch.randn(nh * wl.dh, wl.d, generator=gw) / math.sqrt(wl.d)).to(
-            torch.bfloat16).cuda()
-        kept = gp.kept_idx.cpu().numpy().astype(np.int64)
-        starts = np.repeat(np.asarray(wl.cu_seqlens[:-1], np.int64),
-                           np.diff(gp.cu_kept.cpu().numpy()))
-        pos = torch.from_numpy((kept - starts).astype(np.int32)).cuda()
-        K = gp.xc.shape[0]
-        outs = (torch.empty(K, wl.hq, wl.dh, dtype=torch.bfloat16, device="cuda"),
-                torch.empty(K, wl.hkv, wl.dh, dtype=torch.bfloat16, device="cuda"),
-                torch.empty(K, wl.hkv, wl.dh, dtype=torch.bfloat16, device="cuda"))
-        q_ms = []
-        for i in range(args.steps + 3):
-            flush_l2()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            api.qkv_rope(gp.xc, w_qkv, wl.hq, wl.hkv, pos, rope_base=1e6, out=outs)
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                q_ms.append(a.elapsed_time(b))
-        if api.device_status(reset=True) != 0:
-            raise RuntimeError("device status set by the q/k/v projection")
-        t_q = statistics.median(q_ms) / 1e3
-        flops = 2.0 * K * wl.d * nh * wl.dh
-        nbytes = 2.0 * K * wl.d + 2.0 * nh * wl.dh * wl.d + 2.0 * K * nh * wl.dh
-        next_step = {"kept_qkv_rope": {
-            "us": t_q * 1e6, "tflops": flops / t_q / 1e12, "frac_tc": flops / t_q / 1e12 / tf_peak,
-            "gbs": nbytes / t_q / 1e9, "rows": K, "d": wl.d, "heads": f"{wl.hq}/{wl.hkv}",
-            "note": "y = W xc, q/k rotated at the kept tokens' original positions (rotate-half, "
-                    "base 1e6), v copied; CUDA events around one launch, L2 flushed before each"}}
+
+def run_ours(args, rep):
+    ws, rank = rep.world, rep.rank
+    from learned_token_pruning_gemm_b200 import pipeline, synth
+    dev_index = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    flush = _Flush()
+    peaks, peak_src = _peaks()
+    tf_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+
+    wl = synth.WORKLOADS[args.workload]()
+    gp = pipeline.GatedPrefill(wl)
+    work = _work(wl)
+    clocks = ClockSampler(dev_index)
+    clocks.start()
+    ms, stage_ms, clk = _time_layer(gp, args.steps, args.warmup, rep, flush, stream, clocks)
+    value = ws * wl.n_tokens / (ms / 1e3)
+    stages = _stages_report(work, stage_ms, tf_peak, hbm_peak)
+    roofline = _roofline(work, stage_ms, tf_peak, hbm_peak, peak_src, args.workload)
+
+    # ---- the same layer with the kept rows' q/k/v projections computed on the path
+    #      (rotary embedding at each kept token's position): the KV entries of the
+    #      layer above the gate exist for the kept tokens only ----
+    with_proj = None
+    if wl.dtype == "bf16" and wl.dh == 128 and (wl.hq + 2 * wl.hkv) % 2 == 0:
+        gpp = pipeline.GatedPrefill(wl, project=True)
+        pms, pstage, _ = _time_layer(gpp, args.steps, args.warmup, rep, flush, stream)
+        with_proj = {"value": ws * wl.n_tokens / (pms / 1e3), "unit": "tokens/s",
+                     "ms_per_step": pms, "launches_per_step": gpp.LAUNCHES_PER_STEP,
+                     "stages": _stages_report(work, pstage, tf_peak, hbm_peak)}
+        del gpp
+
+    # ---- the other single-GPU workloads of the metric (16k-128k): same measurement ----
+    others = {}
+    for name in ([] if args.no_extra_workloads else args.extra_workloads.split(",")):
+        if not name or name == args.workload:
+            continue
+        owl = synth.WORKLOADS[name]()
+        ogp = pipeline.GatedPrefill(owl)
+        owork = _work(owl)
+        oms, ostage, _ = _time_layer(ogp, args.steps, args.warmup, rep, flush, stream)
+        others[name] = {
+            "value": ws * owl.n_tokens / (oms / 1e3), "unit": "tokens/s", "ms_per_step": oms,
+            "tokens": owl.n_tokens, "kept": owl.total_kept, "batch": owl.batch,
+            "stages": _stages_report(owork, ostage, tf_peak, hbm_peak),
+            "roofline": _roofline(owork, ostage, tf_peak, hbm_peak, peak_src, name)}
+        del ogp, owl
+        torch.cuda.empty_cache()
+    clocks.stop()
 
     # ---- e2e: host buffers in, result out, through the same public calls ----
     e2e = None
@@ -378,9 +390,13 @@ def run_ours(args, rep):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        t_cpu, parts, sample = _oracle_sample_time(wl, oracle)
+        _oracle_warm(wl, oracle)
+        t_cpu, parts = _oracle_step(wl, oracle)
         cpu = {"value": wl.n_tokens / t_cpu, "unit": "tokens/s", "cores": _threads(),
-               "kind": "oracle", "sample": sample,
+               "cpu_model": _cpu_model(), "kind": "oracle",
+               "sample": (f"one whole {args.workload} step timed once: gate on all "
+                          f"{wl.n_tokens} rows, select, gather, attention on all {wl.total_kept} "
+                          f"kept rows x {wl.hq} heads (fp64, OpenMP over the host cores)"),
                "stage_s": {k: round(v, 4) for k, v in parts.items()}}
 
     if rank == 0:
@@ -397,19 +413,20 @@ def run_ours(args, rep):
             "roofline": roofline,
             "gpu_launches": gp.LAUNCHES_PER_STEP * args.steps,
             "stage_sum_us": sum(stage_ms.values()) * 1e3,
-            "launch": ("timed steps: the whole layer as one CUDA graph of 4 kernels chained by "
-                       "programmatic dependent launch, events around each replay; stage times: "
-                       "a second graph with events between the stages"),
+            "launch": (f"timed steps: the whole layer as one CUDA graph of {gp.LAUNCHES_PER_STEP} "
+                       "kernels chained by programmatic dependent launch, events around each "
+                       "replay; stage times: a second graph with events between the stages"),
             "clocks": clk,
             "e2e": e2e,
-            "next_step": next_step,
+            "with_projection": with_proj,
+            "workloads": others,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
 
 
 _STAGE_SRC = {"gate": "gate.cu", "select": "select.cu", "compact": "compact.cu",
-              "attention": "attn.cu", "compact+attention": "attn.cu"}
+              "attention": "attn.cu", "project": "qkv.cu"}
 
 
 def _kernel_rev(stage: str) -> str:
@@ -432,6 +449,9 @@ def main():
     ap.add_argument("--workload", default="qwen16k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra-workloads", default="long128k,ragged8",
+                    help="other workloads measured the same way, reported under 'workloads'")
+    ap.add_argument("--no-extra-workloads", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -92,19 +92,25 @@ tg_status tg_gate_score(const void* x, tg_dtype dtype, int64_t n_tokens, int d, 
  *   kept_idx    [total_kept]    int32 output: kept rows' global row ids
  *                                       (indices into `scores`), ascending
  *   kept_scores [total_kept]    f32 output, may be NULL: scores[kept_idx[r]]
+ *   kept_pos    [total_kept]    int32 output, may be NULL: the kept rows'
+ *                                       positions within their own sequence
+ *                                       (kept_idx[r] - cu_seqlens[b])
  *   cu_kept     [batch+1]       int32 output: cumulative kept counts
  * total_kept must equal sum_b (len_b - span_b + min(max(k_doc_b,0), span_b)); the
  * caller knows every term, so no device-to-host read is needed to size outputs.
- * max_seqlen bounds every len_b; max_seqlen <= TG_SELECT_MAX_SEQLEN. A span
- * outside its sequence or a total that differs from total_kept is found on the
- * device: the sequence's outputs are skipped and TG_ERR_DEVICE_CHECK recorded.
+ * max_seqlen bounds every len_b; max_seqlen <= TG_SELECT_MAX_SEQLEN; the
+ * scores of sequence b must lie inside [0, total_tokens). A sequence whose rows or
+ * span fall outside these bounds, or a total that differs from total_kept, is
+ * found on the device: TG_ERR_DEVICE_CHECK is recorded, the sequence's output
+ * rows get row id -1 (score 0, position -1), and cu_kept still advances by its
+ * clamped count, clipped to total_kept, so every offset stays inside the outputs.
  */
 #define TG_SELECT_MAX_SEQLEN 196608
 tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* doc_begin,
                          const int32_t* doc_end, const int32_t* k_doc, int batch,
                          int64_t total_tokens, int64_t total_kept, int max_seqlen,
-                         int32_t* kept_idx, float* kept_scores, int32_t* cu_kept,
-                         tg_stream_t stream);
+                         int32_t* kept_idx, float* kept_scores, int32_t* kept_pos,
+                         int32_t* cu_kept, tg_stream_t stream);
 
 /*
  * Stable compaction (MarkTechPost page, "Comment TokenGate a-t-il appris ...":
@@ -114,12 +120,13 @@ tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const i
  *   src, dst    host arrays of n_tensors device pointers (1 <= n_tensors <= 8)
  *   row_bytes   host array of n_tensors sizes; each a positive multiple of 16
  *   kept_idx    [n_kept] int32 device, row ids into every src (from tg_select_topk)
- * Every src/dst pointer must be 16-byte aligned. The caller guarantees that
- * kept_idx entries are valid rows of every src.
+ *   n_src_rows  rows of every src: an index outside [0, n_src_rows) is skipped
+ *               (that dst row is left as it was) and TG_ERR_DEVICE_CHECK recorded
+ * Every src/dst pointer must be 16-byte aligned.
  */
 tg_status tg_compact_kv(const void* const* src, void* const* dst, const int64_t* row_bytes,
                         int n_tensors, const int32_t* kept_idx, int64_t n_kept,
-                        tg_stream_t stream);
+                        int64_t n_src_rows, tg_stream_t stream);
 
 /*
  * Token-gated causal GQA attention over the kept tokens (MarkTechPost page,
@@ -136,6 +143,9 @@ tg_status tg_compact_kv(const void* const* src, void* const* dst, const int64_t*
  *   s_kept [total_kept] f32 (from tg_select_topk), gain, tau [n_hq] f32
  *   cu_kept [batch+1] int32 device; max_kept >= every cu_kept[b+1]-cu_kept[b]
  *   out  [total_kept, n_hq, head_dim]  dtype output
+ * A sequence whose kept range is not inside [0, total_kept] or is longer than
+ * max_kept is skipped (its out rows are left as they were) and TG_ERR_DEVICE_CHECK
+ * is recorded.
  * TG_BF16 (tensor-core path): head_dim == 128, n_hq % n_hkv == 0, q/k/v/out
  * 16-byte aligned. TG_F32 (exact fp32 path): head_dim <= 256.
  */

@@ -22,8 +22,8 @@ SIGNATURES = {
     "tg_abi_version": (INT, []),
     "tg_status_string": (ctypes.c_char_p, [INT]),
     "tg_gate_score": (INT, [P, INT, I64, INT, P, P, P, F32, INT, P, P]),
-    "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P]),
-    "tg_compact_kv": (INT, [P, P, P, INT, P, I64, P]),
+    "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P, P]),
+    "tg_compact_kv": (INT, [P, P, P, INT, P, I64, I64, P]),
     "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P]),
     "tg_qkv_rope": (INT, [P, I64, INT, P, INT, INT, INT, F32, P, P, P, P, P]),
     "tg_device_status": (INT, [P, INT]),

@@ -34,6 +34,18 @@ def _cuda(t: torch.Tensor, name: str, dtype=None) -> int:
     return t.data_ptr()
 
 
+def _numel(t: torch.Tensor, n: int, name: str) -> None:
+    if t.numel() != n:
+        raise TokenGateError(f"{name} must have {n} elements, got {t.numel()}")
+
+
+def _shape(t: torch.Tensor, shape, name: str, dtype=None) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise TokenGateError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TokenGateError(f"{name} must be {dtype}, got {t.dtype}")
+
+
 def abi_version() -> int:
     return _lib.load().tg_abi_version()
 
@@ -45,8 +57,11 @@ def gate_score(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Te
     h = w1.shape[0]
     if w1.shape != (h, d) or w1.dtype != x.dtype or x.dtype not in _DT:
         raise TokenGateError("gate_score: x [N,d] and w1 [h,d] must share a dtype (f32/bf16)")
+    _numel(b1, h, "b1")
+    _numel(w2, h, "w2")
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=x.device)
+    _numel(out, n, "scores")
     st = _lib.load().tg_gate_score(_cuda(x, "x"), _DT[x.dtype], n, d, _cuda(w1, "w1"),
                                    _cuda(b1, "b1", torch.float32), _cuda(w2, "w2", torch.float32),
                                    float(b2), h, _cuda(out, "scores", torch.float32), _stream(stream))
@@ -57,25 +72,42 @@ def gate_score(x: torch.Tensor, w1: torch.Tensor, b1: torch.Tensor, w2: torch.Te
 def select_topk(scores: torch.Tensor, cu_seqlens: torch.Tensor, doc_begin: torch.Tensor,
                 doc_end: torch.Tensor, k_doc: torch.Tensor, total_kept: int, max_seqlen: int,
                 kept_idx: Optional[torch.Tensor] = None, kept_scores: Optional[torch.Tensor] = None,
-                cu_kept: Optional[torch.Tensor] = None, want_scores: bool = True, stream=None):
+                cu_kept: Optional[torch.Tensor] = None, want_scores: bool = True,
+                kept_pos: Optional[torch.Tensor] = None, want_pos: bool = False, stream=None):
     """Returns (kept_idx int32 [total_kept], kept_scores f32 [total_kept] or None,
-    cu_kept int32 [B+1])."""
+    cu_kept int32 [B+1]); with want_pos (or kept_pos given) also kept_pos int32
+    [total_kept], the kept rows' positions within their sequences, as a 4th item."""
     B = doc_begin.numel()
     dev = scores.device
+    total_kept = int(total_kept)
+    _numel(cu_seqlens, B + 1, "cu_seqlens")
+    _numel(doc_end, B, "doc_end")
+    _numel(k_doc, B, "k_doc")
     if kept_idx is None:
         kept_idx = torch.empty(total_kept, dtype=torch.int32, device=dev)
     if kept_scores is None and want_scores:
         kept_scores = torch.empty(total_kept, dtype=torch.float32, device=dev)
+    if kept_pos is None and want_pos:
+        kept_pos = torch.empty(total_kept, dtype=torch.int32, device=dev)
     if cu_kept is None:
         cu_kept = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    _numel(kept_idx, total_kept, "kept_idx")
+    if kept_scores is not None:
+        _numel(kept_scores, total_kept, "kept_scores")
+    if kept_pos is not None:
+        _numel(kept_pos, total_kept, "kept_pos")
+    _numel(cu_kept, B + 1, "cu_kept")
     st = _lib.load().tg_select_topk(
         _cuda(scores, "scores", torch.float32), _cuda(cu_seqlens, "cu_seqlens", torch.int32),
         _cuda(doc_begin, "doc_begin", torch.int32), _cuda(doc_end, "doc_end", torch.int32),
-        _cuda(k_doc, "k_doc", torch.int32), B, scores.numel(), int(total_kept), int(max_seqlen),
+        _cuda(k_doc, "k_doc", torch.int32), B, scores.numel(), total_kept, int(max_seqlen),
         _cuda(kept_idx, "kept_idx", torch.int32),
         _cuda(kept_scores, "kept_scores", torch.float32) if kept_scores is not None else None,
+        _cuda(kept_pos, "kept_pos", torch.int32) if kept_pos is not None else None,
         _cuda(cu_kept, "cu_kept", torch.int32), _stream(stream))
     check(st, "tg_select_topk")
+    if kept_pos is not None:
+        return kept_idx, kept_scores, cu_kept, kept_pos
     return kept_idx, kept_scores, cu_kept
 
 
@@ -83,17 +115,22 @@ def compact_rows(srcs: Sequence[torch.Tensor], kept_idx: torch.Tensor,
                  outs: Optional[Sequence[torch.Tensor]] = None, stream=None):
     """dst[t][r] = src[t][kept_idx[r]] for every tensor (rows = first dim)."""
     n = kept_idx.numel()
+    if not srcs:
+        raise TokenGateError("compact_rows: at least one source tensor")
     if outs is None:
         outs = [torch.empty((n,) + tuple(s.shape[1:]), dtype=s.dtype, device=s.device) for s in srcs]
     k = len(srcs)
-    src_arr = (ctypes.c_void_p * k)(*[_cuda(s, "src") for s in srcs])
-    dst_arr = (ctypes.c_void_p * k)(*[_cuda(o, "dst") for o in outs])
-    rb = (ctypes.c_int64 * k)(*[math.prod(s.shape[1:]) * s.element_size() for s in srcs])
+    if len(outs) != k:
+        raise TokenGateError("compact_rows: one output per source")
     for s, o in zip(srcs, outs):
         if o.shape[1:] != s.shape[1:] or o.dtype != s.dtype or o.shape[0] != n:
             raise TokenGateError("compact_rows: output shape/dtype mismatch")
+    src_arr = (ctypes.c_void_p * k)(*[_cuda(s, "src") for s in srcs])
+    dst_arr = (ctypes.c_void_p * k)(*[_cuda(o, "dst") for o in outs])
+    rb = (ctypes.c_int64 * k)(*[math.prod(s.shape[1:]) * s.element_size() for s in srcs])
+    n_src = min(s.shape[0] for s in srcs)
     st = _lib.load().tg_compact_kv(src_arr, dst_arr, rb, k, _cuda(kept_idx, "kept_idx", torch.int32),
-                                   n, _stream(stream))
+                                   n, n_src, _stream(stream))
     check(st, "tg_compact_kv")
     return list(outs)
 
@@ -108,8 +145,14 @@ def gated_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s_kept: t
         raise TokenGateError("gated_attention: q [K,Hq,dh], k/v [K,Hkv,dh] with one dtype")
     if q.dtype not in _DT:
         raise TokenGateError(f"gated_attention: unsupported dtype {q.dtype}")
+    _numel(s_kept, K, "s_kept")
+    _numel(gain, hq, "gain")
+    _numel(tau, hq, "tau")
+    if cu_kept.numel() < 1:
+        raise TokenGateError("cu_kept must have batch+1 >= 1 elements")
     if out is None:
         out = torch.empty_like(q)
+    _shape(out, q.shape, "out", q.dtype)
     B = cu_kept.numel() - 1
     st = _lib.load().tg_gated_attention(
         _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _DT[q.dtype],
@@ -129,11 +172,15 @@ def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: 
     if (n_out % (n_hq + 2 * n_hkv)) or w_qkv.shape[1] != d or xc.dtype != w_qkv.dtype:
         raise TokenGateError("qkv_rope: w_qkv [(Hq+2Hkv)*dh, d] with the dtype of xc")
     dh = n_out // (n_hq + 2 * n_hkv)
+    _numel(pos, K, "pos")
     if out is None:
         out = (torch.empty(K, n_hq, dh, dtype=xc.dtype, device=xc.device),
                torch.empty(K, n_hkv, dh, dtype=xc.dtype, device=xc.device),
                torch.empty(K, n_hkv, dh, dtype=xc.dtype, device=xc.device))
     q, k, v = out
+    _shape(q, (K, n_hq, dh), "q", xc.dtype)
+    _shape(k, (K, n_hkv, dh), "k", xc.dtype)
+    _shape(v, (K, n_hkv, dh), "v", xc.dtype)
     st = _lib.load().tg_qkv_rope(_cuda(xc, "xc", torch.bfloat16), K, d,
                                  _cuda(w_qkv, "w_qkv", torch.bfloat16), n_hq, n_hkv, dh,
                                  float(rope_base), _cuda(pos, "pos", torch.int32), _cuda(q, "q"),

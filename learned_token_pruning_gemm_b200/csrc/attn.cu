@@ -53,8 +53,8 @@ constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 s
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
 
-// 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5); fitted by
-// fit_exp2_poly.py in this directory.
+// 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by a
+// Remez exchange on the relative error (equi-oscillating error at 5 points).
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tm_v,
                            const float* __restrict__ s_kept, const float* __restrict__ gain,
                            const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
-                           int n_hq, int n_hkv, __nv_bfloat16* __restrict__ out, int* status) {
+                           int total, int max_kept, int n_hq, int n_hkv,
+                           __nv_bfloat16* __restrict__ out, int* status) {
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
   const int z = blockIdx.z;
@@ -182,7 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tg::pdl_wait();   // global memory only from here on
 
   const int seq0 = cu_kept[b];
-  const int len = cu_kept[b + 1] - seq0;
+  const int seq1 = cu_kept[b + 1];
+  // a kept range outside [0, total] or longer than max_kept (the grid covers
+  // max_kept rows per sequence) is not attended: record it and skip the sequence
+  const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
+  if (bad && z == 0 && hq == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+  const int len = bad ? 0 : seq1 - seq0;
   const int n_t = (len + kBM - 1) / kBM;
   if (2 * z >= n_t) {           // uniform: this sequence has no pair z
     if (warp == 2) tg::tmem_dealloc(tmem, kTmemCols);
@@ -544,7 +550,7 @@ __global__ void __launch_bounds__(kF32Warps * 32)
                           const float* __restrict__ v, const float* __restrict__ s_kept,
                           const float* __restrict__ gain, const float* __restrict__ tau,
                           const int32_t* __restrict__ cu_kept, int batch, int64_t total,
-                          int n_hq, int n_hkv, int dh, float* __restrict__ out) {
+                          int n_hq, int n_hkv, int dh, float* __restrict__ out, int* status) {
   tg::pdl_launch_dependents();
   tg::pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -554,6 +560,10 @@ __global__ void __launch_bounds__(kF32Warps * 32)
   int b = 0;
   while (b + 1 < batch && cu_kept[b + 1] <= i) ++b;
   const int64_t j0 = cu_kept[b];
+  if (j0 < 0 || j0 > i) {   // row i is not inside sequence b's kept range
+    if (lane == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    return;
+  }
   const int kvh = hq / (n_hq / n_hkv);
   const float scale = 1.f / (sqrtf(static_cast<float>(dh)) * tau[hq]);
   const float g = gain[hq];
@@ -623,7 +633,8 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
   const int n_qt = (max_kept + kBM - 1) / kBM;
   dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
   return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv, s_kept,
-                    gain, tau, cu_kept, n_hq, n_hkv, static_cast<__nv_bfloat16*>(out), status);
+                    gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
+                    static_cast<__nv_bfloat16*>(out), status);
 }
 
 }  // namespace
@@ -633,6 +644,7 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
                                         const float* tau, const int32_t* cu_kept, int batch,
                                         int64_t total_kept, int max_kept, int n_hq, int n_hkv,
                                         int head_dim, void* out, tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_gated_attention");
   if (batch < 0 || total_kept < 0 || max_kept < 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0)
     return TG_ERR_INVALID_ARG;
   if (batch == 0 || total_kept == 0 || max_kept == 0) return TG_OK;
@@ -652,11 +664,13 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
     if (head_dim > 256) return TG_ERR_UNSUPPORTED;
     const int64_t blocks = (total_kept + kF32Warps - 1) / kF32Warps;
     if (blocks > INT32_MAX) return TG_ERR_UNSUPPORTED;
+    int* status = tg::status_word();
+    if (!status) return TG_ERR_CUDA;
     dim3 grid(static_cast<unsigned>(blocks), n_hq);
     return tg::launch(gated_attn_f32_kernel, grid, dim3(kF32Warps * 32), 0, stream, 0,
                       static_cast<const float*>(q), static_cast<const float*>(k),
                       static_cast<const float*>(v), s_kept, gain, tau, cu_kept, batch, total_kept,
-                      n_hq, n_hkv, head_dim, static_cast<float*>(out));
+                      n_hq, n_hkv, head_dim, static_cast<float*>(out), status);
   }
   return TG_ERR_UNSUPPORTED;
 }

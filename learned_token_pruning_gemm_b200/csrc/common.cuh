@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "tg.h"
@@ -404,4 +405,14 @@ tg_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return launch_status();
 }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range named after the entry point, open for the whole call (host side:
+// argument checks, tensor-map encoding, launch). Without a profiler attached the
+// push and pop are a check of a null function pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 }  // namespace tg

@@ -2,7 +2,8 @@
 // section "Comment TokenGate a-t-il appris le fonctionnement de la réduction des
 // tokens ?": layers above the gate layer process only the K kept tokens).
 //
-// dst[t][r] = src[t][kept_idx[r]] for up to 8 tensors at once. One warp moves one
+// dst[t][r] = src[t][kept_idx[r]] for up to 8 tensors at once (an index outside
+// [0, n_src_rows) is skipped and recorded as a device-check error). One warp moves one
 // row of every tensor; each lane issues 128-bit non-allocating loads, eight in
 // flight before the matching stores, so a 4 KB hidden-state row is one batch of 8
 // fully coalesced 512-byte warp transactions. Pure HBM traffic: 2 * K * row_bytes.
@@ -30,7 +31,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 
 __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
                                                                 const int32_t* __restrict__ idx,
-                                                                int64_t n_kept) {
+                                                                int64_t n_kept, int64_t n_src,
+                                                                int* status) {
   tg::pdl_launch_dependents();
   tg::pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -38,6 +40,10 @@ __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
   for (int64_t r = warp; r < n_kept; r += nwarps) {
     const int64_t sr = idx[r];
+    if (sr < 0 || sr >= n_src) {   // not a row of the sources: skip it, record the error
+      if (lane == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+      continue;
+    }
     for (int t = 0; t < a.n; ++t) {
       const int64_t nv = a.vecs[t];
       const uint4* s = a.src[t] + sr * nv;
@@ -59,8 +65,11 @@ __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
 
 extern "C" tg_status tg_compact_kv(const void* const* src, void* const* dst,
                                    const int64_t* row_bytes, int n_tensors,
-                                   const int32_t* kept_idx, int64_t n_kept, tg_stream_t stream) {
-  if (!src || !dst || !row_bytes || n_tensors < 1 || n_tensors > kMaxTensors || n_kept < 0)
+                                   const int32_t* kept_idx, int64_t n_kept, int64_t n_src_rows,
+                                   tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_compact_kv");
+  if (!src || !dst || !row_bytes || n_tensors < 1 || n_tensors > kMaxTensors || n_kept < 0 ||
+      n_src_rows < 0)
     return TG_ERR_INVALID_ARG;
   if (n_kept == 0) return TG_OK;
   if (!kept_idx) return TG_ERR_INVALID_ARG;
@@ -74,9 +83,11 @@ extern "C" tg_status tg_compact_kv(const void* const* src, void* const* dst,
     a.dst[t] = static_cast<uint4*>(dst[t]);
     a.vecs[t] = row_bytes[t] / 16;
   }
+  int* st = tg::status_word();
+  if (!st) return TG_ERR_CUDA;
   const int64_t warps_needed = n_kept;
   int64_t blocks = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
   if (blocks > 148 * 16) blocks = 148 * 16;
   return tg::launch(compact_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0,
-                    stream, 0, a, kept_idx, n_kept);
+                    stream, 0, a, kept_idx, n_kept, n_src_rows, st);
 }

@@ -429,6 +429,7 @@ tg_status launch_gate_bf16(const void* x, int64_t n, int d, const void* w1, cons
 extern "C" tg_status tg_gate_score(const void* x, tg_dtype dtype, int64_t n_tokens, int d,
                                    const void* w1, const float* b1, const float* w2, float b2,
                                    int h, float* scores, tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_gate_score");
   if (n_tokens < 0 || d <= 0 || h <= 0) return TG_ERR_INVALID_ARG;
   if (n_tokens == 0) return TG_OK;
   if (!x || !w1 || !b1 || !w2 || !scores) return TG_ERR_INVALID_ARG;

@@ -197,6 +197,7 @@ extern "C" tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const vo
                                  int n_hq, int n_hkv, int head_dim, float rope_base,
                                  const int32_t* pos, void* q, void* k, void* v,
                                  tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_qkv_rope");
   if (n_rows < 0 || d <= 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0) return TG_ERR_INVALID_ARG;
   if (!(rope_base > 1.0f)) return TG_ERR_INVALID_ARG;
   if (n_rows == 0) return TG_OK;

@@ -23,7 +23,8 @@
 // kept count; since the ties kept before any point number min(need, ties before
 // it), one exchange of those two counts through distributed shared memory fixes
 // every CTA's and warp's output offset, and a second pass writes the kept rows
-// in order (ranks from warp scans). No global scratch.
+// in order (ranks from warp scans), with their scores and their positions within
+// the sequence. No global scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -110,9 +111,10 @@ __device__ __forceinline__ uint32_t key_at(const uint4& k, int e) {
 __global__ void __launch_bounds__(kThreads, 1)
     select_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ cu_seqlens,
                        const int32_t* __restrict__ doc_begin, const int32_t* __restrict__ doc_end,
-                       const int32_t* __restrict__ k_doc, int batch, int64_t total_kept,
-                       int chunk, int32_t* __restrict__ kept_idx, float* __restrict__ kept_scores,
-                       int32_t* __restrict__ cu_kept, int* status) {
+                       const int32_t* __restrict__ k_doc, int batch, int64_t total_tokens,
+                       int64_t total_kept, int chunk, int32_t* __restrict__ kept_idx, float* __restrict__ kept_scores,
+                       int32_t* __restrict__ kept_pos, int32_t* __restrict__ cu_kept,
+                       int* status) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
@@ -127,13 +129,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xFFFFFFFFu;
 
+  // ---- output offset: the earlier sequences' kept counts (clamped the same way
+  //      for every sequence, so a rejected sequence still has a defined extent) ----
+  {
+    int64_t acc = 0;
+    for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
+    if (lane == 0) S.red[warp] = acc;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int64_t t = 0;
+    for (int w = 0; w < kWarps; ++w) t += S.red[w];
+    S.out_base = t;
+  }
+  __syncthreads();
+  const int64_t out_base = S.out_base;
+
+  // Rejected sequence (or an inconsistent total found below): its output rows
+  // get row id -1, score 0 and position -1, and cu_kept still advances by the
+  // clamped count, clipped to total_kept, so the kernels that read these outputs
+  // next see in-range offsets and an index the compaction rejects.
+  auto reject = [&](int64_t count) {
+    const int64_t o0 = out_base < total_kept ? out_base : total_kept;
+    const int64_t o1 = out_base + count < total_kept ? out_base + count : total_kept;
+    for (int64_t r = o0 + (int64_t)rank * kThreads + tid; r < o1; r += (int64_t)csize * kThreads) {
+      kept_idx[r] = -1;
+      if (kept_scores) kept_scores[r] = 0.f;
+      if (kept_pos) kept_pos[r] = -1;
+    }
+    if (rank == 0 && tid == 0) {
+      tg::set_status(status, TG_ERR_DEVICE_CHECK);
+      if (b == 0) cu_kept[0] = 0;
+      cu_kept[b + 1] = (int32_t)o1;
+    }
+  };
+
   // ---- sequence geometry (identical in every CTA of the cluster) ----
   const int64_t base = cu_seqlens[b];
   const int64_t len = (int64_t)cu_seqlens[b + 1] - base;
   const int64_t db = doc_begin[b], de = doc_end[b];
-  const bool bad = len < 0 || len > (int64_t)chunk * csize || db < 0 || de < db || de > len;
+  const bool bad = base < 0 || len < 0 || base + len > total_tokens ||
+                   len > (int64_t)chunk * csize || db < 0 || de < db || de > len;
   if (bad) {
-    if (rank == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    reject(seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, b));
     return;   // uniform across the cluster: nobody reaches a cluster barrier
   }
   const int64_t nd = de - db;
@@ -148,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ld0 = clampl(db - c0), ld1 = clampl(de - c0);
   const uint32_t excl_local = (uint32_t)(chunk - (ld1 - ld0));   // keys forced to 0
 
-  // ---- load (8 loads in flight per thread); sum the earlier sequences' counts ----
+  // ---- load (8 loads in flight per thread) ----
   for (int i0 = tid; i0 < chunk; i0 += 8 * kThreads) {
     float v[8];
 #pragma unroll
@@ -165,18 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  {
-    int64_t acc = 0;
-    for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
-    if (lane == 0) S.red[warp] = acc;
-  }
   __syncthreads();
-  if (tid == 0) {
-    int64_t t = 0;
-    for (int w = 0; w < kWarps; ++w) t += S.red[w];
-    S.out_base = t;
-  }
 
   const int seg = chunk / kWarps;                 // multiple of 128
   const int seg0 = warp * seg;
@@ -309,7 +337,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- pass 2: keep decisions and output, ascending ----
-  const int64_t out_base = S.out_base;
   const int64_t seq_keep = S.seq_keep;
   const int64_t expect = len - nd + k_eff;
   const bool ok = seq_keep == expect && out_base + seq_keep <= total_kept;
@@ -343,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((nib >> e) & 1u) {
           kept_idx[o] = (int32_t)(base + c0 + i4 + e);
           if (kept_scores) kept_scores[o] = raw[i4 + e];
+          if (kept_pos) kept_pos[o] = (int32_t)(c0 + i4 + e);
           ++o;
         }
       }
@@ -350,8 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       run_out += __shfl_sync(full, incl_k, 31);
     }
   }
-  if (rank == 0 && tid == 0) {
-    if (!ok) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+  if (!ok) {
+    reject(expect);
+  } else if (rank == 0 && tid == 0) {
     if (b == 0) cu_kept[0] = 0;
     cu_kept[b + 1] = (int32_t)(out_base + expect);
     if (b == batch - 1 && out_base + expect != total_kept) tg::set_status(status, TG_ERR_DEVICE_CHECK);
@@ -365,7 +394,9 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
                                     const int32_t* doc_begin, const int32_t* doc_end,
                                     const int32_t* k_doc, int batch, int64_t total_tokens,
                                     int64_t total_kept, int max_seqlen, int32_t* kept_idx,
-                                    float* kept_scores, int32_t* cu_kept, tg_stream_t stream) {
+                                    float* kept_scores, int32_t* kept_pos, int32_t* cu_kept,
+                                    tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_select_topk");
   if (batch < 0 || total_tokens < 0 || total_kept < 0 || max_seqlen < 0) return TG_ERR_INVALID_ARG;
   if (batch == 0) return TG_OK;
   if (!cu_seqlens || !doc_begin || !doc_end || !k_doc || !cu_kept) return TG_ERR_INVALID_ARG;
@@ -383,6 +414,7 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   if (!tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem))
     return TG_ERR_CUDA;
   return tg::launch(select_topk_kernel, dim3(csize, batch, 1), dim3(kThreads), smem, stream, csize,
-                    scores, cu_seqlens, doc_begin, doc_end, k_doc, batch, total_kept, chunk,
-                    kept_idx, kept_scores, cu_kept, st);
+                    scores, cu_seqlens, doc_begin, doc_end, k_doc, batch, total_tokens,
+                    total_kept, chunk,
+                    kept_idx, kept_scores, kept_pos, cu_kept, st);
 }

@@ -4,10 +4,13 @@ token-gated causal GQA attention over the kept tokens (MarkTechPost page on
 TokenGate, section "Comment TokenGate a-t-il appris le fonctionnement de la
 réduction des tokens ?").
 
-The attention inputs q/k/v are the kept tokens' projections; the projection
-that would produce them from the compacted residual is outside this path, so
-they are supplied already compacted ([K, H, dh]) and only the key scores come
-from the selection.
+Two modes. By default the attention inputs q/k/v are supplied already compacted
+([K, H, dh], drawn for the kept rows), and only the key scores come from the
+selection: this is the measured metric (gate + top-K + attention). With
+`project=True` the layer above the gate layer computes them itself: the kept
+residual rows' q/k/v projections with the rotary embedding at each kept token's
+original position (tg_qkv_rope on the compacted rows), so the KV entries exist
+for the kept tokens only, and attention reads those.
 """
 from __future__ import annotations
 
@@ -20,14 +23,16 @@ from .synth import Workload
 
 
 class GatedPrefill:
-    """Device-resident buffers for one workload and a `step()` that runs the four
-    stages (4 kernel launches)."""
+    """Device-resident buffers for one workload and a `step()` that runs the stages
+    (one kernel launch each)."""
 
-    LAUNCHES_PER_STEP = 4
-
-    def __init__(self, wl: Workload, device: str = "cuda", use_score_override: bool = True):
+    def __init__(self, wl: Workload, device: str = "cuda", use_score_override: bool = True,
+                 project: bool = False, w_qkv: Optional[torch.Tensor] = None,
+                 rope_base: float = 1e6):
         dev = torch.device(device)
         self.wl = wl
+        self.project = project
+        self.rope_base = rope_base
         self.x = wl.x.to(dev)
         self.w1 = wl.w1.to(dev)
         self.b1 = wl.b1.to(dev)
@@ -56,6 +61,20 @@ class GatedPrefill:
         self.cu_kept = torch.empty(wl.batch + 1, **i32)
         self.xc = torch.empty((K, wl.d), dtype=self.x.dtype, device=dev)
         self.out = torch.empty_like(self.q)
+        if project:
+            from .synth import qkv_weights
+            self.w_qkv = (w_qkv if w_qkv is not None else qkv_weights(wl)).to(dev)
+            self.kept_pos = torch.empty(K, **i32)
+            # the kept rows' projections replace the supplied q/k/v
+            self.q = torch.empty((K, wl.hq, wl.dh), dtype=self.x.dtype, device=dev)
+            self.k = torch.empty((K, wl.hkv, wl.dh), dtype=self.x.dtype, device=dev)
+            self.v = torch.empty((K, wl.hkv, wl.dh), dtype=self.x.dtype, device=dev)
+        else:
+            self.w_qkv = None
+            self.kept_pos = None
+        self.STAGES = (("gate", "select", "compact", "project", "attention") if project
+                       else ("gate", "select", "compact", "attention"))
+        self.LAUNCHES_PER_STEP = len(self.STAGES)
 
     def stage_gate(self, stream=None):
         api.gate_score(self.x, self.w1, self.b1, self.w2, self.b2, out=self.scores, stream=stream)
@@ -64,34 +83,37 @@ class GatedPrefill:
         sel = self.override if self.override is not None else self.scores
         api.select_topk(sel, self.cu_seqlens, self.doc_begin, self.doc_end, self.k_doc,
                         self.total_kept, self.max_seqlen, kept_idx=self.kept_idx,
-                        kept_scores=self.kept_scores, cu_kept=self.cu_kept, stream=stream)
+                        kept_scores=self.kept_scores, cu_kept=self.cu_kept,
+                        kept_pos=self.kept_pos, stream=stream)
 
     def stage_compact(self, stream=None):
         api.compact_rows([self.x], self.kept_idx, outs=[self.xc], stream=stream)
+
+    def stage_project(self, stream=None):
+        api.qkv_rope(self.xc, self.w_qkv, self.wl.hq, self.wl.hkv, self.kept_pos,
+                     rope_base=self.rope_base, out=(self.q, self.k, self.v), stream=stream)
 
     def stage_attention(self, stream=None):
         api.gated_attention(self.q, self.k, self.v, self.kept_scores, self.gain, self.tau,
                             self.cu_kept, self.max_kept, out=self.out, stream=stream)
 
-    STAGES = ("gate", "select", "compact", "attention")
-
     def step(self, stream=None, events: Optional[list] = None):
-        """Run the four stages back to back on one stream (each kernel launched with
+        """Run the stages back to back on one stream (each kernel launched with
         programmatic dependent launch, so its prologue overlaps the previous one's
-        tail). If `events` is a list of 5 CUDA events, they are recorded on the
-        stream before, between and after the stages."""
+        tail). If `events` is a list of len(STAGES)+1 CUDA events, they are recorded
+        on the stream before, between and after the stages."""
         s = stream if stream is not None else torch.cuda.current_stream()
-        fns = (self.stage_gate, self.stage_select, self.stage_compact, self.stage_attention)
+        fns = [getattr(self, "stage_" + n) for n in self.STAGES]
         for i, fn in enumerate(fns):
             if events is not None:
                 events[i].record(s)
             fn(stream=s)
         if events is not None:
-            events[4].record(s)
+            events[len(fns)].record(s)
 
     # ------------------------------------------------------------------ graphs
     def capture(self):
-        """Capture the whole layer (four kernels) as CUDA graphs: one as launched in
+        """Capture the whole layer as CUDA graphs: one as launched in
         production and one with timing events between the stages. One eager
         step runs first (outside capture) so that every lazily initialised piece of
         the library exists before capture."""
@@ -109,7 +131,7 @@ class GatedPrefill:
         # the same step with timing events between the stages (the event nodes turn
         # the programmatic edges into full dependencies; used for the breakdown only)
         self.stage_events = [torch.cuda.Event(enable_timing=True, external=True)
-                             for _ in range(5)]
+                             for _ in range(len(self.STAGES) + 1)]
         self.timed_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.timed_graph):
             self.step(events=self.stage_events)
@@ -117,7 +139,7 @@ class GatedPrefill:
         return self
 
     def replay_step(self):
-        """Replay the whole layer (one graph, four kernel launches) on the current stream."""
+        """Replay the whole layer (one graph, one launch per stage) on the current stream."""
         self.step_graph.replay()
 
     def replay_timed(self):

@@ -76,6 +76,7 @@ class Workload:
     planted: Optional[np.ndarray] = None            # global rows of planted clusters
     duplicates: Optional[np.ndarray] = None         # [n,2] (copied-from, copied-to)
     keep_ratio: Optional[float] = None
+    v_dist: str = "normal"
 
     @property
     def n_tokens(self) -> int:
@@ -110,18 +111,22 @@ def _weights(seed, dtype, d, h, hq):
             torch.from_numpy(gain), torch.from_numpy(tau))
 
 
-def _qkv(seed, dtype, K, hq, hkv, dh):
-    # Q, K ~ N(0,1) (unit-variance projections of a unit-variance residual);
-    # V ~ U(-sqrt3, sqrt3): unit variance and bounded by 1.74, so the bf16 rounding
-    # of an output row (a convex mix of V rows) stays below 2^-8.
+def _qkv(seed, dtype, K, hq, hkv, dh, v_dist="normal"):
+    # Q, K, V ~ N(0,1): what a projection with N(0,1)/sqrt(fan_in) weights makes of a
+    # unit-variance residual. v_dist="uniform" draws V from U(-sqrt3, sqrt3) instead
+    # (unit variance, bounded by 1.74), for extra cases that keep |O| below 2.
     q = _rng(seed, "q").standard_normal((K, hq, dh))
     k = _rng(seed, "k").standard_normal((K, hkv, dh))
-    v = _rng(seed, "v").uniform(-math.sqrt(3.0), math.sqrt(3.0), (K, hkv, dh))
+    if v_dist == "uniform":
+        v = _rng(seed, "v").uniform(-math.sqrt(3.0), math.sqrt(3.0), (K, hkv, dh))
+    else:
+        v = _rng(seed, "v").standard_normal((K, hkv, dh))
     return _as_dtype(q, dtype), _as_dtype(k, dtype), _as_dtype(v, dtype)
 
 
 def make_workload(name: str, dtype: str, seed: int, seqlens, q_lens, keep_ratio=None,
-                  k_doc=None, d=2048, h=256, hq=16, hkv=8, dh=128) -> Workload:
+                  k_doc=None, d=2048, h=256, hq=16, hkv=8, dh=128,
+                  v_dist="normal") -> Workload:
     """Generic builder: per sequence the droppable span is [0, n - q_len) and the
     protected question is the last q_len tokens."""
     seqlens = [int(n) for n in seqlens]
@@ -133,9 +138,10 @@ def make_workload(name: str, dtype: str, seed: int, seqlens, q_lens, keep_ratio=
     x = _as_dtype(_rng(seed, "x").standard_normal((N, d)), dtype)
     w1, b1, w2, b2, gain, tau = _weights(seed, dtype, d, h, hq)
     K = sum(kept_total(seqlens, doc_begin, doc_end, k_doc))
-    q, k, v = _qkv(seed, dtype, K, hq, hkv, dh)
+    q, k, v = _qkv(seed, dtype, K, hq, hkv, dh, v_dist)
     return Workload(name, dtype, seed, seqlens, doc_begin, doc_end, list(k_doc), d, h, hq,
-                    hkv, dh, x, w1, b1, w2, b2, gain, tau, q, k, v, keep_ratio=keep_ratio)
+                    hkv, dh, x, w1, b1, w2, b2, gain, tau, q, k, v, keep_ratio=keep_ratio,
+                    v_dist=v_dist)
 
 
 # --------------------------------------------------------------------------- #
@@ -224,12 +230,28 @@ WORKLOADS = {
 
 
 def small_case(seed: int, seqlens, q_lens, k_doc, dtype="bf16", d=128, h=64, hq=4, hkv=2,
-               dh=128, doc_begin=None) -> Workload:
+               dh=128, doc_begin=None, v_dist="normal") -> Workload:
     """A small workload for parity tests, with an arbitrary droppable span."""
     wl = make_workload(f"small_{seed}", dtype, seed, seqlens, q_lens, k_doc=k_doc, d=d, h=h,
-                       hq=hq, hkv=hkv, dh=dh)
+                       hq=hq, hkv=hkv, dh=dh, v_dist=v_dist)
     if doc_begin is not None:
         wl.doc_begin = list(doc_begin)
         K = sum(kept_total(wl.seqlens, wl.doc_begin, wl.doc_end, wl.k_doc))
-        wl.q, wl.k, wl.v = _qkv(seed, dtype, K, hq, hkv, dh)
+        wl.q, wl.k, wl.v = _qkv(seed, dtype, K, hq, hkv, dh, v_dist)
     return wl
+
+
+def uniform_v(wl: Workload) -> Workload:
+    """The same workload with V redrawn from U(-sqrt3, sqrt3) (the other arrays unchanged)."""
+    K = wl.total_kept
+    _, _, wl.v = _qkv(wl.seed, wl.dtype, K, wl.hq, wl.hkv, wl.dh, "uniform")
+    wl.v_dist = "uniform"
+    return wl
+
+
+def qkv_weights(wl: Workload, seed: int = 11) -> torch.Tensor:
+    """W = [Wq; Wk; Wv] [(hq + 2 hkv) dh, d] ~ N(0,1)/sqrt(d), in the workload's dtype: the
+    projection weights of the layer above the gate layer, for the kept rows' q/k/v."""
+    g = np.random.Generator(np.random.Philox(key=[wl.seed, 100 + seed]))
+    n = (wl.hq + 2 * wl.hkv) * wl.dh
+    return _as_dtype(g.standard_normal((n, wl.d)) / math.sqrt(wl.d), wl.dtype)

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.tg_abi_version() == 1
+    assert lib.tg_abi_version() == 2
     for code, name in [(0, "TG_OK"), (1, "TG_ERR_INVALID_ARG"), (3, "TG_ERR_MISALIGNED"),
                        (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (99, "TG_ERR_UNKNOWN")]:
         assert lib.tg_status_string(code).decode() == name
@@ -52,24 +52,25 @@ def test_validation_returns_status_without_gpu(lib):
     assert lib.tg_gate_score(odd, 1, 128, 128, fake, fake, fake, 0.0, 64, fake, None) == MIS
     assert lib.tg_gate_score(fake, 7, 128, 128, fake, fake, fake, 0.0, 64, fake, None) == UNSUP
     # select: K > N, too long, null outputs
-    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 11, 10, fake, None, fake,
-                              None) == INVALID
-    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 5, 300000, fake, None, fake,
-                              None) == UNSUP
-    assert lib.tg_select_topk(fake, None, fake, fake, fake, 1, 10, 5, 10, fake, None, fake,
-                              None) == INVALID
+    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 11, 10, fake, None, None,
+                              fake, None) == INVALID
+    assert lib.tg_select_topk(fake, fake, fake, fake, fake, 1, 10, 5, 300000, fake, None, None,
+                              fake, None) == UNSUP
+    assert lib.tg_select_topk(fake, None, fake, fake, fake, 1, 10, 5, 10, fake, None, None,
+                              fake, None) == INVALID
     assert lib.tg_select_topk(None, None, None, None, None, 0, 0, 0, 0, None, None, None,
-                              None) == 0
+                              None, None) == 0
     # compact: row bytes must be a positive multiple of 16, pointers aligned
     arr = (P * 1)(fake)
     arr_odd = (P * 1)(odd)
     rb = (ctypes.c_int64 * 1)(4096)
     rb_odd = (ctypes.c_int64 * 1)(40)
-    assert lib.tg_compact_kv(arr, arr, rb_odd, 1, fake, 5, None) == MIS
-    assert lib.tg_compact_kv(arr_odd, arr, rb, 1, fake, 5, None) == MIS
-    assert lib.tg_compact_kv(arr, arr, rb, 0, fake, 5, None) == INVALID
-    assert lib.tg_compact_kv(arr, arr, rb, 9, fake, 5, None) == INVALID
-    assert lib.tg_compact_kv(arr, arr, rb, 1, fake, 0, None) == 0
+    assert lib.tg_compact_kv(arr, arr, rb_odd, 1, fake, 5, 10, None) == MIS
+    assert lib.tg_compact_kv(arr_odd, arr, rb, 1, fake, 5, 10, None) == MIS
+    assert lib.tg_compact_kv(arr, arr, rb, 0, fake, 5, 10, None) == INVALID
+    assert lib.tg_compact_kv(arr, arr, rb, 9, fake, 5, 10, None) == INVALID
+    assert lib.tg_compact_kv(arr, arr, rb, 1, fake, 5, -1, None) == INVALID
+    assert lib.tg_compact_kv(arr, arr, rb, 1, fake, 0, 10, None) == 0
     # attention: GQA divisibility, head dim, max_kept > total, alignment
     args = [fake, fake, fake, 1, fake, fake, fake, fake, 1, 256, 256]
     assert lib.tg_gated_attention(*args, 16, 6, 128, fake, None) == INVALID
@@ -96,3 +97,82 @@ def test_validation_returns_status_without_gpu(lib):
                            None) == MIS
     assert lib.tg_qkv_rope(None, 0, 2048, None, 16, 8, 128, 1e6, None, None, None, None,
                            None) == 0
+
+
+# ---- the Python binding checks every tensor's size against the sizes it passes
+#      to the C ABI, before any call (so a CPU tensor reaches none of them) ----
+
+def _raises(fn, match):
+    from learned_token_pruning_gemm_b200._lib import TokenGateError
+    with pytest.raises(TokenGateError, match=match):
+        fn()
+
+
+def test_binding_gate_checks_lengths():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    x, w1 = torch.zeros(8, 64), torch.zeros(16, 64)
+    ok = torch.zeros(16)
+    _raises(lambda: api.gate_score(x, w1, torch.zeros(15), ok, 0.0), "b1 must have 16")
+    _raises(lambda: api.gate_score(x, w1, ok, torch.zeros(17), 0.0), "w2 must have 16")
+    _raises(lambda: api.gate_score(x, w1, ok, ok, 0.0, out=torch.zeros(7)), "scores must have 8")
+    _raises(lambda: api.gate_score(x, torch.zeros(16, 32), ok, ok, 0.0), "share a dtype")
+
+
+def test_binding_select_checks_lengths():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    i32 = lambda n: torch.zeros(n, dtype=torch.int32)
+    s = torch.zeros(100)
+    args = (s, i32(3), i32(2), i32(2), i32(2), 40, 60)
+    _raises(lambda: api.select_topk(s, i32(2), i32(2), i32(2), i32(2), 40, 60),
+            "cu_seqlens must have 3")
+    _raises(lambda: api.select_topk(s, i32(3), i32(2), i32(1), i32(2), 40, 60),
+            "doc_end must have 2")
+    _raises(lambda: api.select_topk(s, i32(3), i32(2), i32(2), i32(3), 40, 60), "k_doc must have 2")
+    _raises(lambda: api.select_topk(*args, kept_idx=i32(39)), "kept_idx must have 40")
+    _raises(lambda: api.select_topk(*args, kept_scores=torch.zeros(41)), "kept_scores must have 40")
+    _raises(lambda: api.select_topk(*args, kept_pos=i32(1)), "kept_pos must have 40")
+    _raises(lambda: api.select_topk(*args, cu_kept=i32(2)), "cu_kept must have 3")
+
+
+def test_binding_compact_checks_shapes():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    idx = torch.zeros(4, dtype=torch.int32)
+    x = torch.zeros(10, 8)
+    _raises(lambda: api.compact_rows([x], idx, outs=[torch.zeros(5, 8)]), "shape/dtype mismatch")
+    _raises(lambda: api.compact_rows([x], idx, outs=[torch.zeros(4, 7)]), "shape/dtype mismatch")
+    _raises(lambda: api.compact_rows([x, x], idx, outs=[torch.zeros(4, 8)]), "one output per")
+    _raises(lambda: api.compact_rows([], idx), "at least one source")
+
+
+def test_binding_attention_checks_lengths():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    K, hq, hkv, dh = 10, 4, 2, 64
+    q, k = torch.zeros(K, hq, dh), torch.zeros(K, hkv, dh)
+    cu = torch.tensor([0, K], dtype=torch.int32)
+    g = torch.zeros(hq)
+    _raises(lambda: api.gated_attention(q, k, k, torch.zeros(K - 1), g, g, cu, K),
+            "s_kept must have 10")
+    _raises(lambda: api.gated_attention(q, k, k, torch.zeros(K), torch.zeros(3), g, cu, K),
+            "gain must have 4")
+    _raises(lambda: api.gated_attention(q, k, k, torch.zeros(K), g, torch.zeros(5), cu, K),
+            "tau must have 4")
+    _raises(lambda: api.gated_attention(q, k, k, torch.zeros(K), g, g, cu, K,
+                                        out=torch.zeros(K, hq, dh - 1)), "out must have shape")
+    _raises(lambda: api.gated_attention(q, k, torch.zeros(K, hkv, dh + 1), torch.zeros(K), g, g,
+                                        cu, K), "q \\[K,Hq,dh\\]")
+
+
+def test_binding_qkv_rope_checks_lengths():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    xc = torch.zeros(6, 64, dtype=torch.bfloat16)
+    w = torch.zeros(4 * 128, 64, dtype=torch.bfloat16)
+    _raises(lambda: api.qkv_rope(xc, w, 2, 1, torch.zeros(5, dtype=torch.int32)), "pos must have 6")
+    bad = (torch.zeros(6, 2, 128, dtype=torch.bfloat16), torch.zeros(6, 1, 128, dtype=torch.bfloat16),
+           torch.zeros(6, 2, 128, dtype=torch.bfloat16))
+    _raises(lambda: api.qkv_rope(xc, w, 2, 1, torch.zeros(6, dtype=torch.int32), out=bad),
+            "v must have shape")

@@ -26,7 +26,12 @@ def test_tiny_workload_shapes_and_determinism():
     assert torch.equal(a.x, b.x) and torch.equal(a.v, b.v) and a.b2 == b.b2
     assert float(a.gain.min()) >= 0 and float(a.gain.max()) <= 1
     assert float(a.tau.min()) >= 0.8 and float(a.tau.max()) <= 1.5
-    assert float(a.v.abs().max()) <= math.sqrt(3.0)
+    # Q/K/V ~ N(0,1) as the tiny configuration states: moments and a heavy-ish tail
+    for t in (a.q, a.k, a.v):
+        assert abs(float(t.mean())) < 0.05 and abs(float(t.std()) - 1.0) < 0.05
+    assert float(a.v.abs().max()) > math.sqrt(3.0)      # not the bounded uniform draw
+    u = synth.uniform_v(synth.tiny_f32())
+    assert float(u.v.abs().max()) <= math.sqrt(3.0) and torch.equal(u.q, a.q)
 
 
 def test_ragged_workload():
@@ -57,3 +62,11 @@ def test_planted_clusters_outrank_the_rest(orc):
     assert s64[:n_doc][mask].min() > s64[:n_doc][~mask].max()
     idx, _ = orc.select_topk(s32, wl.cu_seqlens, wl.doc_begin, wl.doc_end, wl.k_doc)
     assert len(idx) == 1868 and np.isin(wl.planted, idx).all()
+
+
+def test_qkv_weights_are_seeded_and_scaled():
+    wl = synth.tiny_f32()
+    w = synth.qkv_weights(wl)
+    assert w.shape == ((wl.hq + 2 * wl.hkv) * wl.dh, wl.d) and w.dtype == wl.x.dtype
+    assert torch.equal(w, synth.qkv_weights(synth.tiny_f32()))
+    assert abs(float(w.std()) * math.sqrt(wl.d) - 1.0) < 0.05
