@@ -51,6 +51,10 @@ def lib():
                                       ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P, I64, P,
                                       P, P]
         L.oracle_qkv_rope.restype = None
+        L.oracle_gated_decode.argtypes = [P, P, P, ctypes.c_int, P, P, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          P, P, P]
+        L.oracle_gated_decode.restype = None
         _lib = L
     return _lib
 
@@ -161,3 +165,23 @@ def qkv_rope(xc: torch.Tensor, w: torch.Tensor, hq: int, hkv: int, dh: int, base
     lib().oracle_qkv_rope(_ptr(xr), dt, n, d, _ptr(wr), hq, hkv, dh, float(base), _ptr(pa), rp,
                           nr, _ptr(q), _ptr(k), _ptr(v))
     return q, k, v
+
+
+def gated_decode(q, k_cache, v_cache, s_cache, cache_len, gain, tau) -> np.ndarray:
+    """One query row per sequence over its cache rows j < cache_len[b]:
+    q [B, hq, dh], k/v cache [B, cap, hkv, dh], s cache [B, cap] -> O [B, hq, dh] fp64."""
+    qr, dt = _raw(q)
+    kr, dt2 = _raw(k_cache)
+    vr, dt3 = _raw(v_cache)
+    assert dt == dt2 == dt3
+    B, hq, dh = qr.shape
+    Bk, cap, hkv, dh2 = kr.shape
+    assert Bk == B and dh2 == dh and tuple(vr.shape) == tuple(kr.shape)
+    s = _f32(s_cache).reshape(B, cap)
+    ln = _i32(cache_len)
+    assert len(ln) == B and (ln <= cap).all()
+    g, t = _f32(gain), _f32(tau)
+    out = np.empty((B, hq, dh), np.float64)
+    lib().oracle_gated_decode(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(s), _ptr(ln), B, cap, hq,
+                              hkv, dh, _ptr(g), _ptr(t), _ptr(out))
+    return out

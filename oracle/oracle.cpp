@@ -244,4 +244,52 @@ void oracle_qkv_rope(const void* xc, int dtype, int64_t n, int d, const void* w,
   }
 }
 
+// Decode over the compacted cache (MarkTechPost page, section "Comment déployer
+// TokenGate ?": generation runs on the cache the pruned prefill left behind, with
+// max_kept_prefill_tokens bounding it; section "Qu'est-ce que l'attention gérée
+// par des tokens ?" for the logits). One new query row per sequence b attends
+// over that sequence's cache rows j < cache_len[b] (the new token's own row is in
+// the cache already, so the causal rule "key position <= query position" keeps
+// every cached row):
+//   z_j = (q_b . k_j) / (sqrt(dh) * tau[hq]) + gain[hq] * s_j,  O_b = sum_j softmax_j(z) v_j
+// q [B, hq, dh]; k/v cache [B, cap, hkv, dh] in `dtype`; s cache [B, cap] f32;
+// KV head = hq / (n_hq / n_hkv). out [B, hq, dh] fp64. A sequence with an empty
+// cache gets zeros.
+void oracle_gated_decode(const void* q, const void* kc, const void* vc, int dtype,
+                         const float* sc, const int32_t* cache_len, int batch, int cap,
+                         int n_hq, int n_hkv, int dh, const float* gain, const float* tau,
+                         double* out) {
+  const int group = n_hq / n_hkv;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < batch; ++b) {
+    for (int hq = 0; hq < n_hq; ++hq) {
+      const int kv = hq / group;
+      const int64_t n = cache_len[b];
+      double* o = out + ((int64_t)b * n_hq + hq) * dh;
+      for (int c = 0; c < dh; ++c) o[c] = 0.0;
+      if (n <= 0) continue;
+      const double scale = 1.0 / (std::sqrt((double)dh) * (double)tau[hq]);
+      std::vector<double> z(n);
+      double zmax = -INFINITY;
+      for (int64_t j = 0; j < n; ++j) {
+        const int64_t row = ((int64_t)b * cap + j) * n_hkv + kv;
+        double dot = 0.0;
+        for (int c = 0; c < dh; ++c)
+          dot += load_elem(q, dtype, ((int64_t)b * n_hq + hq) * dh + c) *
+                 load_elem(kc, dtype, row * dh + c);
+        z[j] = dot * scale + (double)gain[hq] * (double)sc[(int64_t)b * cap + j];
+        zmax = std::max(zmax, z[j]);
+      }
+      double denom = 0.0;
+      for (int64_t j = 0; j < n; ++j) {
+        const double w = std::exp(z[j] - zmax);
+        denom += w;
+        const int64_t row = ((int64_t)b * cap + j) * n_hkv + kv;
+        for (int c = 0; c < dh; ++c) o[c] += w * load_elem(vc, dtype, row * dh + c);
+      }
+      for (int c = 0; c < dh; ++c) o[c] /= denom;
+    }
+  }
+}
+
 }  // extern "C"

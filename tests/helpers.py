@@ -5,6 +5,15 @@ Tolerances (fixed by the project's accuracy targets):
   kept indices             bit-exact given identical scores
   attention, fp32 path     max-abs <= 1e-4
   attention, bf16 path     max-abs <= 1e-2 and relative L2 <= 5e-3
+
+The bf16 output format itself: a bf16 value in [2^e, 2^(e+1)) is a multiple of
+2^(e-7), so rounding the exact output to bf16 alone can move it by half of that.
+Below |O| = 4 half a spacing is at most 2^-8 (about 0.0039, at |O| in [2, 4)), so
+the 1e-2 bar measures the kernel. At |O| >= 4 half a spacing is 2^-6 = 0.0156 >
+1e-2: no bf16 output can meet 1e-2 there, whatever computed it. Elements with
+|O| >= 4 (rows dominated by one key with |v| >= 4, which V ~ N(0,1) draws) are
+therefore held to 1e-2 plus their own half spacing, i.e. the bar applies to the
+value before its final rounding; every other element to 1e-2 exactly.
 """
 import numpy as np
 import torch
@@ -29,14 +38,30 @@ def attn_errors(gpu_out: torch.Tensor, ref: np.ndarray, rows=None):
     return max_abs, rl2
 
 
+def bf16_half_spacing(a: np.ndarray) -> np.ndarray:
+    """Half the distance between adjacent bf16 values at magnitude |a| (normal range)."""
+    e = np.floor(np.log2(np.maximum(np.abs(a), 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
 def assert_attn_close(gpu_out, ref, dtype, rows=None, what=""):
     max_abs, rl2 = attn_errors(gpu_out, ref, rows)
-    max_o = float(np.abs(ref if rows is None else ref[rows]).max())
+    r = ref if rows is None else ref[rows]
+    max_o = float(np.abs(r).max()) if r.size else 0.0
     if dtype == torch.float32:
         assert max_abs <= ATTN_F32_ATOL, f"{what}: max_abs {max_abs:.3e} (max|O| {max_o:.3f})"
     else:
-        assert max_abs <= ATTN_BF16_ATOL and rl2 <= ATTN_BF16_RL2, (
-            f"{what}: max_abs {max_abs:.3e} rel_l2 {rl2:.3e} (max|O| {max_o:.3f})")
+        g = to_np64(gpu_out)
+        if rows is not None:
+            g = g[rows]
+        err = np.abs(g - r)
+        big = np.abs(r) >= 4.0
+        allowed = np.where(big, ATTN_BF16_ATOL + bf16_half_spacing(r), ATTN_BF16_ATOL)
+        worst = float((err - allowed).max()) if err.size else 0.0
+        small_max = float(err[~big].max()) if (~big).any() else 0.0
+        assert worst <= 0 and rl2 <= ATTN_BF16_RL2, (
+            f"{what}: max_abs {max_abs:.3e} (|O|<4: {small_max:.3e}) rel_l2 {rl2:.3e} "
+            f"(max|O| {max_o:.3f}, {int(big.sum())} elements with |O| >= 4)")
     return max_abs, rl2
 
 
