@@ -303,6 +303,76 @@ def _roofline(work, stage_ms, tf_peak, hbm_peak, peak_src, workload):
             "frac": ach / peak, "traffic": traffic, "peak_source": peak_src}
 
 
+def _time_decode(gp, wl, steps, warmup, rep, flush, stream, hbm_peak):
+    """One decode step per sequence over the compacted cache of the measured prefill:
+    the kept rows' k, v and scores are the cache (batch-major, capacity K_b + 64); a
+    step appends one new token (tg_cache_append) and attends over the cache
+    (tg_gated_decode), captured as one CUDA graph (three launches). The cache
+    length is reset before every step (outside the events), so every step reads the
+    same number of rows."""
+    from learned_token_pruning_gemm_b200 import api
+    counts = wl.kept_counts
+    B, cap = wl.batch, max(counts) + 64
+    dev = gp.q.device
+    kc = torch.zeros(B, cap, wl.hkv, wl.dh, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    sc = torch.zeros(B, cap, device=dev)
+    cu = gp.cu_kept.cpu().tolist()
+    for b in range(B):
+        n = cu[b + 1] - cu[b]
+        kc[b, :n] = gp.k[cu[b]:cu[b + 1]]
+        vc[b, :n] = gp.v[cu[b]:cu[b + 1]]
+        sc[b, :n] = gp.kept_scores[cu[b]:cu[b + 1]]
+    base_len = torch.tensor(counts, dtype=torch.int32, device=dev)
+    ln = base_len.clone()
+    g = torch.Generator(device="cpu").manual_seed(3)
+    qn = torch.randn(B, wl.hq, wl.dh, generator=g).to(torch.bfloat16).to(dev)
+    kn = torch.randn(B, wl.hkv, wl.dh, generator=g).to(torch.bfloat16).to(dev)
+    vn = torch.randn(B, wl.hkv, wl.dh, generator=g).to(torch.bfloat16).to(dev)
+    sn = torch.randn(B, generator=g).to(dev)
+    out = torch.empty(B, wl.hq, wl.dh, dtype=torch.bfloat16, device=dev)
+    max_len = cap
+    ws = torch.empty(api.decode_workspace_size(B, wl.hq, wl.dh, max_len), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        api.cache_append(kn, vn, sn, kc, vc, sc, ln)
+        api.gated_decode(qn, kc, vc, sc, ln, gp.gain, gp.tau, max_len, out=out, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    ln.copy_(base_len)
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        ln.copy_(base_len)
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    rep.barrier()
+    for a, b in ev:
+        ln.copy_(base_len)
+        flush()
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    rep.barrier()
+    if api.device_status(reset=True) != 0:
+        raise RuntimeError("device status set by the decode step")
+    ms = rep.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
+    rows = sum(counts) + B
+    nbytes = rows * wl.hkv * wl.dh * 2 * 2 + rows * 4 + 2 * B * wl.hq * wl.dh * 2
+    return {"us": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "batch": B,
+            "cache_rows": rows, "gbs": nbytes / (ms / 1e3) / 1e9,
+            "frac_hbm": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "launches_per_step": 3,
+            "note": "append + split-KV decode + combine, one CUDA graph; bytes = the cache's "
+                    "K, V and scores read once, q and out"}
+
+
 def run_ours(args, rep):
     ws, rank = rep.world, rep.rank
     from learned_token_pruning_gemm_b200 import pipeline, synth
@@ -335,6 +405,12 @@ def run_ours(args, rep):
                      "stages": _stages_report(work, pstage, tf_peak, hbm_peak)}
         del gpp
 
+    # ---- decode over the compacted cache the prefill leaves (one new token per
+    #      sequence: append its k/v/score, then attend over the cache) ----
+    decode = None
+    if wl.dtype == "bf16" and wl.dh == 128 and not args.no_decode:
+        decode = _time_decode(gp, wl, args.steps, args.warmup, rep, flush, stream, hbm_peak)
+
     # ---- the other single-GPU workloads of the metric (16k-128k): same measurement ----
     others = {}
     for name in ([] if args.no_extra_workloads else args.extra_workloads.split(",")):
@@ -349,6 +425,9 @@ def run_ours(args, rep):
             "tokens": owl.n_tokens, "kept": owl.total_kept, "batch": owl.batch,
             "stages": _stages_report(owork, ostage, tf_peak, hbm_peak),
             "roofline": _roofline(owork, ostage, tf_peak, hbm_peak, peak_src, name)}
+        if not args.no_decode and owl.dtype == "bf16" and owl.dh == 128:
+            others[name]["decode"] = _time_decode(ogp, owl, args.steps, args.warmup, rep, flush,
+                                                  stream, hbm_peak)
         del ogp, owl
         torch.cuda.empty_cache()
     clocks.stop()
@@ -419,6 +498,7 @@ def run_ours(args, rep):
             "clocks": clk,
             "e2e": e2e,
             "with_projection": with_proj,
+            "decode": decode,
             "workloads": others,
             "cpu_baseline": cpu,
         }
@@ -452,6 +532,7 @@ def main():
     ap.add_argument("--extra-workloads", default="long128k,ragged8",
                     help="other workloads measured the same way, reported under 'workloads'")
     ap.add_argument("--no-extra-workloads", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

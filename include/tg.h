@@ -12,7 +12,8 @@
  *
  * Conventions shared by every entry point
  *   - Every pointer argument is a DEVICE pointer unless its comment says "host".
- *     The caller owns every buffer; the library allocates no device memory.
+ *     The caller owns every buffer (scratch included, sized by the matching
+ *     *_workspace_size query); the library allocates no device memory.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and never synchronises the host, except tg_device_status().
  *   - Every call returns a tg_status; no exception crosses the ABI. Argument
@@ -174,6 +175,49 @@ tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dty
 tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const void* w_qkv, int n_hq,
                       int n_hkv, int head_dim, float rope_base, const int32_t* pos, void* q,
                       void* k, void* v, tg_stream_t stream);
+
+/*
+ * Decode over the compacted cache (MarkTechPost page on TokenGate, section
+ * "Comment déployer TokenGate ?": generation runs on the cache the pruned prefill
+ * leaves, bounded by max_kept_prefill_tokens; section "Qu'est-ce que l'attention
+ * gérée par des tokens ?": the key-score bias with per-head gain, and the per-head
+ * temperature). The cache of sequence b is rows [b*cap, b*cap + cache_len[b]) of
+ *   k_cache, v_cache  [batch, cap, n_hkv, head_dim] bf16 (dense, token-major)
+ *   s_cache           [batch, cap] f32            (each cached key's gate score)
+ * as left by the prefill's compaction (tg_compact_kv of the kept rows) and grown by
+ * tg_cache_append. In the layers up to the gate layer (no score bias) pass
+ * gain = 0 and tau = 1: the same call is then plain causal attention.
+ *
+ * tg_cache_append: for every sequence b, writes k_new[b], v_new[b] ([batch, n_hkv,
+ * head_dim] bf16) and s_new[b] (f32) into row cache_len[b] of its cache and adds
+ * one to cache_len[b] (int32 [batch], device). A full cache (cache_len[b] >= cap)
+ * is left unchanged and TG_ERR_DEVICE_CHECK recorded. head_dim == 128.
+ */
+tg_status tg_cache_append(const void* k_new, const void* v_new, const float* s_new, int batch,
+                          int cap, int n_hkv, int head_dim, void* k_cache, void* v_cache,
+                          float* s_cache, int32_t* cache_len, tg_stream_t stream);
+
+/*
+ * tg_gated_decode: one new query row per sequence (q [batch, n_hq, head_dim] bf16,
+ * its own k/v already appended) attends over cache rows j < cache_len[b]:
+ *     z_j = q . k_j / (sqrt(head_dim) * tau[hq]) + gain[hq] * s_j
+ *     out[b, hq] = sum_j softmax_j(z) v_j          (bf16 [batch, n_hq, head_dim])
+ * with KV head hq / (n_hq / n_hkv). max_len (host) bounds every cache_len[b] and
+ * sizes the launch; max_len <= cap. head_dim == 128, n_hq / n_hkv <= 8; q, the
+ * caches, out and workspace 16-byte aligned. An empty cache gives zeros. A length
+ * outside [0, min(cap, max_len)] leaves that row of out unchanged and records
+ * TG_ERR_DEVICE_CHECK.
+ * workspace: caller-owned device scratch of at least
+ * tg_gated_decode_workspace_size(batch, n_hq, head_dim, max_len) bytes (per-chunk
+ * partial results; no initial value needed; calls that overlap on the GPU must not
+ * share it). Too small a workspace returns TG_ERR_WORKSPACE.
+ */
+size_t tg_gated_decode_workspace_size(int batch, int n_hq, int head_dim, int max_len);
+tg_status tg_gated_decode(const void* q, const void* k_cache, const void* v_cache,
+                          const float* s_cache, const int32_t* cache_len, int batch, int cap,
+                          int max_len, int n_hq, int n_hkv, int head_dim, const float* gain,
+                          const float* tau, void* out, void* workspace, size_t workspace_bytes,
+                          tg_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns the first error any kernel recorded on the

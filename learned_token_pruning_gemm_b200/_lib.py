@@ -26,6 +26,10 @@ SIGNATURES = {
     "tg_compact_kv": (INT, [P, P, P, INT, P, I64, I64, P]),
     "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P]),
     "tg_qkv_rope": (INT, [P, I64, INT, P, INT, INT, INT, F32, P, P, P, P, P]),
+    "tg_cache_append": (INT, [P, P, P, INT, INT, INT, INT, P, P, P, P, P]),
+    "tg_gated_decode_workspace_size": (ctypes.c_size_t, [INT, INT, INT, INT]),
+    "tg_gated_decode": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P,
+                              ctypes.c_size_t, P]),
     "tg_device_status": (INT, [P, INT]),
     "tg_selftest_bounded_wait": (INT, [I64, P]),
 }

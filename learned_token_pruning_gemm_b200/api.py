@@ -189,6 +189,64 @@ def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: 
     return q, k, v
 
 
+def cache_append(k_new: torch.Tensor, v_new: torch.Tensor, s_new: torch.Tensor,
+                 k_cache: torch.Tensor, v_cache: torch.Tensor, s_cache: torch.Tensor,
+                 cache_len: torch.Tensor, stream=None) -> None:
+    """Row cache_len[b] of sequence b's cache gets k_new[b], v_new[b], s_new[b];
+    cache_len[b] += 1. Caches [B, cap, Hkv, dh] bf16 and [B, cap] f32."""
+    B, cap, hkv, dh = k_cache.shape
+    _shape(v_cache, k_cache.shape, "v_cache", k_cache.dtype)
+    _shape(k_new, (B, hkv, dh), "k_new", k_cache.dtype)
+    _shape(v_new, (B, hkv, dh), "v_new", k_cache.dtype)
+    _shape(s_new, (B,), "s_new", torch.float32)
+    _shape(s_cache, (B, cap), "s_cache", torch.float32)
+    _shape(cache_len, (B,), "cache_len", torch.int32)
+    st = _lib.load().tg_cache_append(
+        _cuda(k_new, "k_new", torch.bfloat16), _cuda(v_new, "v_new", torch.bfloat16),
+        _cuda(s_new, "s_new"), B, cap, hkv, dh, _cuda(k_cache, "k_cache", torch.bfloat16),
+        _cuda(v_cache, "v_cache", torch.bfloat16), _cuda(s_cache, "s_cache"),
+        _cuda(cache_len, "cache_len"), _stream(stream))
+    check(st, "tg_cache_append")
+
+
+def decode_workspace_size(batch: int, n_hq: int, head_dim: int, max_len: int) -> int:
+    return int(_lib.load().tg_gated_decode_workspace_size(batch, n_hq, head_dim, max_len))
+
+
+def gated_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 s_cache: torch.Tensor, cache_len: torch.Tensor, gain: torch.Tensor,
+                 tau: torch.Tensor, max_len: int, out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One query row per sequence (q [B, Hq, dh] bf16) over its cache rows
+    j < cache_len[b]; returns out [B, Hq, dh] bf16."""
+    B, hq, dh = q.shape
+    Bc, cap, hkv, dh2 = k_cache.shape
+    if Bc != B or dh2 != dh:
+        raise TokenGateError("gated_decode: q [B,Hq,dh] and caches [B,cap,Hkv,dh]")
+    _shape(v_cache, k_cache.shape, "v_cache", k_cache.dtype)
+    _shape(s_cache, (B, cap), "s_cache", torch.float32)
+    _shape(cache_len, (B,), "cache_len", torch.int32)
+    _numel(gain, hq, "gain")
+    _numel(tau, hq, "tau")
+    if out is None:
+        out = torch.empty_like(q)
+    _shape(out, q.shape, "out", q.dtype)
+    need = decode_workspace_size(B, hq, dh, max(int(max_len), 1))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise TokenGateError(f"gated_decode: workspace needs {need} bytes")
+    st = _lib.load().tg_gated_decode(
+        _cuda(q, "q", torch.bfloat16), _cuda(k_cache, "k_cache", torch.bfloat16),
+        _cuda(v_cache, "v_cache", torch.bfloat16), _cuda(s_cache, "s_cache"),
+        _cuda(cache_len, "cache_len"), B, cap, int(max_len), hq, hkv, dh,
+        _cuda(gain, "gain", torch.float32), _cuda(tau, "tau", torch.float32), _cuda(out, "out"),
+        _cuda(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    check(st, "tg_gated_decode")
+    return out
+
+
 def device_status(reset: bool = True, stream=None) -> int:
     """Synchronise the stream and return (then clear) the device status word."""
     return _lib.load().tg_device_status(_stream(stream), 1 if reset else 0)

@@ -99,6 +99,44 @@ def test_validation_returns_status_without_gpu(lib):
                            None) == 0
 
 
+
+def test_decode_validation_without_gpu(lib):
+    INVALID, UNSUP, MIS, WS = 1, 2, 3, 4
+    P = ctypes.c_void_p
+    fake, odd = P(0x10000), P(0x10004)
+    ws_size = lib.tg_gated_decode_workspace_size
+    # partials of (dh + 2) fp32 per (sequence, query head, 64-key chunk)
+    assert ws_size(2, 16, 128, 1868) == 2 * 16 * 30 * 130 * 4
+    assert ws_size(1, 16, 64, 100) == 0 and ws_size(0, 16, 128, 100) == 0
+    need = ws_size(1, 16, 128, 1000)
+
+    def dec(hq=16, hkv=8, dh=128, cap=1000, max_len=1000, ws=fake, ws_bytes=None, q=fake,
+            batch=1):
+        return lib.tg_gated_decode(q, fake, fake, fake, fake, batch, cap, max_len, hq, hkv, dh,
+                                   fake, fake, fake, ws, need if ws_bytes is None else ws_bytes,
+                                   None)
+    assert dec(hkv=6) == INVALID
+    assert dec(dh=64) == UNSUP
+    assert dec(hq=32, hkv=2) == UNSUP            # more than 8 query heads per KV head
+    assert dec(max_len=1001) == INVALID
+    assert dec(ws_bytes=need - 4) == WS
+    assert dec(ws=None) == WS
+    assert dec(q=odd) == MIS
+    assert dec(ws=odd) == MIS
+    assert dec(batch=0) == 0
+    assert lib.tg_gated_decode(None, fake, fake, fake, fake, 1, 10, 10, 16, 8, 128, fake, fake,
+                               fake, fake, need, None) == INVALID
+    # append: null pointers, head_dim, alignment
+    assert lib.tg_cache_append(None, fake, fake, 1, 10, 8, 128, fake, fake, fake, fake,
+                               None) == INVALID
+    assert lib.tg_cache_append(fake, fake, fake, 1, 10, 8, 64, fake, fake, fake, fake,
+                               None) == UNSUP
+    assert lib.tg_cache_append(fake, odd, fake, 1, 10, 8, 128, fake, fake, fake, fake,
+                               None) == MIS
+    assert lib.tg_cache_append(None, None, None, 0, 10, 8, 128, None, None, None, None,
+                               None) == 0
+
+
 # ---- the Python binding checks every tensor's size against the sizes it passes
 #      to the C ABI, before any call (so a CPU tensor reaches none of them) ----
 
@@ -176,3 +214,19 @@ def test_binding_qkv_rope_checks_lengths():
            torch.zeros(6, 2, 128, dtype=torch.bfloat16))
     _raises(lambda: api.qkv_rope(xc, w, 2, 1, torch.zeros(6, dtype=torch.int32), out=bad),
             "v must have shape")
+
+
+def test_binding_decode_checks_shapes():
+    import torch
+    from learned_token_pruning_gemm_b200 import api
+    q = torch.zeros(2, 4, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(2, 50, 2, 128, dtype=torch.bfloat16)
+    sc, ln, g = torch.zeros(2, 50), torch.zeros(2, dtype=torch.int32), torch.zeros(4)
+    _raises(lambda: api.gated_decode(q, kc, kc, torch.zeros(2, 49), ln, g, g, 50), "s_cache must")
+    _raises(lambda: api.gated_decode(q, kc, kc, sc, torch.zeros(3, dtype=torch.int32), g, g, 50),
+            "cache_len must")
+    _raises(lambda: api.gated_decode(q, kc, kc[:, :, :1].contiguous(), sc, ln, g, g, 50),
+            "v_cache must")
+    _raises(lambda: api.gated_decode(q, kc, kc, sc, ln, torch.zeros(3), g, 50), "gain must have 4")
+    _raises(lambda: api.cache_append(kc[:, 0], kc[:, 0], torch.zeros(3), kc, kc, sc, ln),
+            "s_new must")
