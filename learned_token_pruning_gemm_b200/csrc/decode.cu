@@ -195,14 +195,23 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Merge one row's chunk partials in chunk order; thread d writes dimension d.
+// Merge one row's chunk partials in chunk order; thread d writes dimension d. The
+// chunks' maxima and sums are read by all threads at once into shared memory
+// (weights 2^(m_c - M) there), then every thread sums its dimension over the
+// chunks with independent loads (eight in flight), so no step waits on a chain
+// of global loads.
+constexpr int kCombineMaxChunks = 4096;   // shared-memory weights; longer caches loop in blocks
+
 __global__ void __launch_bounds__(kThreads)
     decode_combine_kernel(const float* __restrict__ partial, const int32_t* __restrict__ cache_len,
                           int cap, int max_len, int n_hq, int n_split,
                           __nv_bfloat16* __restrict__ out, int* status) {
+  __shared__ float w[kCombineMaxChunks];
+  __shared__ float red[kThreads / 32 + 1];   // block partials; red[0] keeps the max across blocks
   tg::pdl_launch_dependents();
   tg::pdl_wait();
   const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int lane = d & 31, warp = d >> 5;
   const int len = cache_len[b];
   __nv_bfloat16* o = out + (static_cast<int64_t>(b) * n_hq + hq) * kDh;
   if (len < 0 || len > cap || len > max_len) {
@@ -215,13 +224,53 @@ __global__ void __launch_bounds__(kThreads)
   }
   const int nc = (len + kChunk - 1) / kChunk;
   const float* pr = partial + (static_cast<int64_t>(b) * n_hq + hq) * n_split * kPartial;
-  float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, pr[c * kPartial + kDh]);
-  float L = 0.f, acc = 0.f;
-  for (int c = 0; c < nc; ++c) {
-    const float w = tg::exp2_approx(pr[c * kPartial + kDh] - M);
-    L = fmaf(w, pr[c * kPartial + kDh + 1], L);
-    acc = fmaf(w, pr[c * kPartial + d], acc);
+  auto block_reduce = [&](float v, bool is_max) {
+    for (int off = 16; off > 0; off >>= 1) {
+      const float x = __shfl_xor_sync(0xFFFFFFFFu, v, off);
+      v = is_max ? fmaxf(v, x) : v + x;
+    }
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    v = red[0];
+    for (int i = 1; i < kThreads / 32; ++i) v = is_max ? fmaxf(v, red[i]) : v + red[i];
+    return v;
+  };
+  float acc = 0.f, L = 0.f;
+  for (int c0 = 0; c0 < nc; c0 += kCombineMaxChunks) {
+    const int cn = min(kCombineMaxChunks, nc - c0);
+    // the overall max first (over every chunk, so the weights of all blocks agree)
+    float mloc = -INFINITY;
+    if (c0 == 0)
+      for (int c = d; c < nc; c += kThreads) mloc = fmaxf(mloc, pr[c * kPartial + kDh]);
+    const float M = c0 == 0 ? block_reduce(mloc, true) : red[0];
+    if (c0 == 0) {
+      __syncthreads();
+      if (d == 0) red[0] = M;   // kept for the later blocks
+    }
+    float lloc = 0.f;
+    for (int c = d; c < cn; c += kThreads) {
+      const float* pc = pr + (c0 + c) * kPartial;
+      const float wc = tg::exp2_approx(pc[kDh] - M);
+      w[c] = wc;
+      lloc = fmaf(wc, pc[kDh + 1], lloc);
+    }
+    __syncthreads();   // weights in shared memory
+    // block sums of l in a fixed order: warp shuffles, then warps in index order
+    for (int off = 16; off > 0; off >>= 1) lloc += __shfl_xor_sync(0xFFFFFFFFu, lloc, off);
+    if (lane == 0) red[1 + warp] = lloc;   // red[0] holds M
+    __syncthreads();
+    for (int i = 0; i < kThreads / 32; ++i) L += red[1 + i];
+    int c = 0;
+    for (; c + 8 <= cn; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = pr[(c0 + c + u) * kPartial + d];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc = fmaf(w[c + u], v[u], acc);
+    }
+    for (; c < cn; ++c) acc = fmaf(w[c], pr[(c0 + c) * kPartial + d], acc);
+    __syncthreads();   // w and red are rewritten by the next block
   }
   o[d] = __float2bfloat16_rn(acc / L);
 }

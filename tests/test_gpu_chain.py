@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_attn_close, sample_rows
+from helpers import assert_attn_close, assert_chain_close, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -81,8 +81,7 @@ def test_projected_layer_matches_oracle_chain(mods, orc, name):
         to_bf16 = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)
         ref_chain = orc.gated_attention(to_bf16(q64), to_bf16(k64), to_bf16(v64),
                                         gp.kept_scores.cpu(), wl.gain, wl.tau, cu_kept)
-        max_abs, rl2 = assert_attn_close(gp.out, ref_chain, torch.bfloat16,
-                                         what=f"{name} oracle chain")
+        max_abs, rl2 = assert_chain_close(gp.out, ref_chain, what=f"{name} oracle chain")
         print(f"{name} chain vs oracle chain: max_abs {max_abs:.2e} rel_l2 {rl2:.2e}")
 
 

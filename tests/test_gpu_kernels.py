@@ -221,6 +221,19 @@ def test_attention_bf16_vs_oracle(api, orc, lens, v_dist):
           f" max_abs {max_abs:.2e} rel_l2 {rl2:.2e}")
 
 
+@pytest.mark.parametrize("hq,hkv,lens", [
+    (16, 8, [700, 1, 300]),      # groups of two: two heads per CTA
+    (16, 2, [513]),              # groups of eight: four head pairs per KV head
+    (8, 8, [700, 300]),          # groups of one: one head per CTA
+    (12, 4, [257, 640]),         # groups of three: one head per CTA
+])
+def test_attention_bf16_head_groups(api, orc, hq, hkv, lens):
+    q, k, v, s, gain, tau, cu = _attn_case(hq * 100 + hkv, lens, hq, hkv, 128, torch.bfloat16)
+    out = _run_attn(api, q, k, v, s, gain, tau, cu)
+    ref = orc.gated_attention(q, k, v, s, gain, tau, cu)
+    assert_attn_close(out, ref, torch.bfloat16, what=f"heads {hq}/{hkv} lens={lens}")
+
+
 def test_attention_bf16_16k_shape_all_rows_normal_v(api, orc):
     # the 16k layer's attention shape (K = 1868, 16/8 heads) with V ~ N(0,1), every row
     q, k, v, s, gain, tau, cu = _attn_case(1868, [1868], 16, 8, 128, torch.bfloat16)
