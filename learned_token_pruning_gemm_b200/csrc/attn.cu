@@ -819,9 +819,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBN; ++i)
           if (i > row) z[i] = -INFINITY;
       }
-      float mx[4] = {z[0], z[1], z[2], z[3]};
+      float mx[4] = {fmaxf(z[0], z[1]), fmaxf(z[2], z[3]), fmaxf(z[4], z[5]), fmaxf(z[6], z[7])};
 #pragma unroll
-      for (int i = 4; i < kBN; i += 8) {
+      for (int i = 8; i < kBN; i += 8) {   // z[8..127]
         mx[0] = fmax3(mx[0], z[i], z[i + 1]);
         mx[1] = fmax3(mx[1], z[i + 2], z[i + 3]);
         mx[2] = fmax3(mx[2], z[i + 4], z[i + 5]);
