@@ -116,6 +116,10 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
+// the two bf16 halves of a packed pair, widened exactly to fp32
+__device__ __forceinline__ float bf16x2_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16x2_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -453,10 +457,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p1 = tg::exp2_approx(x1);
           const float p2 = tg::exp2_approx(x2);
           const float p3 = tg::exp2_approx(x3);
-          fadd2(sa[0], sa[1], sa[0], sa[1], p0, p1);
-          fadd2(sb[0], sb[1], sb[0], sb[1], p2, p3);
           pk[2 * i] = tg::pack_bf16x2(p0, p1);       // row ra, packed column 4i + l%4
           pk[2 * i + 1] = tg::pack_bf16x2(p2, p3);   // row rb, the same column
+          // the row sums add the bf16 weights that the PV MMA multiplies: numerator
+          // and denominator then carry the same rounding, so a key that dominates
+          // its row contributes its v exactly, whatever weight the lagging max left it
+          fadd2(sa[0], sa[1], sa[0], sa[1], bf16x2_lo(pk[2 * i]), bf16x2_hi(pk[2 * i]));
+          fadd2(sb[0], sb[1], sb[0], sb[1], bf16x2_lo(pk[2 * i + 1]), bf16x2_hi(pk[2 * i + 1]));
         }
         la = la * alpha_a + (sa[0] + sa[1]);
         lb = lb * alpha_b + (sb[0] + sb[1]);
@@ -850,9 +857,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p1 = tg::exp2_approx(x1);
         const float p2 = tg::exp2_approx(x2);
         const float p3 = tg::exp2_approx(x3);
-        fadd2(sa, sb, sa, sb, p0 + p2, p1 + p3);
         pk[i / 2] = tg::pack_bf16x2(p0, p1);
         pk[i / 2 + 1] = tg::pack_bf16x2(p2, p3);
+        // the row sum adds the bf16 weights the PV MMA multiplies (numerator and
+        // denominator then carry the same rounding)
+        fadd2(sa, sb, sa, sb, bf16x2_lo(pk[i / 2]) + bf16x2_lo(pk[i / 2 + 1]),
+              bf16x2_hi(pk[i / 2]) + bf16x2_hi(pk[i / 2 + 1]));
       }
       l = l * alpha + (sa + sb);
       if (__any_sync(0xFFFFFFFFu, rescale)) {
