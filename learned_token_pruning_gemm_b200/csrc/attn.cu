@@ -804,35 +804,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (alive) alive = tg::mbar_wait(&S.b_full[st], (j / kBiasStages) & 1, status, &S.abort_flag);
       if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
       tg::tc_fence_after();
-      float z[kBN];
-      {
-        uint32_t u[kBN];
-        tg::tmem_ld32x64(s_addr, u);
-        tg::tmem_ld32x64(s_addr + 64, u + 64);
+      const float* bias = S.bias[st][x];
+      const bool diag = (j == tq);   // diagonal tile: key column i is visible to row r iff i <= r
+      // The row is read from TMEM twice, 64 columns at a time: first for its max,
+      // then for the weights, so that at most 64 logits and 32 packed weights are
+      // live per thread (a whole row at once spills).
+      // pass 1: z = S c_h + b (log2 domain) and the tile's row max
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t u[64];
+        tg::tmem_ld32x64(s_addr + 64u * hh, u);
         tg::tmem_ld_wait();
-        const float* bias = S.bias[st][x];
 #pragma unroll
-        for (int i = 0; i < kBN; i += 4) {
-          const float4 bb = *reinterpret_cast<const float4*>(bias + i);
-          ffma2(z[i], z[i + 1], __uint_as_float(u[i]), __uint_as_float(u[i + 1]), c_h, c_h, bb.x, bb.y);
-          ffma2(z[i + 2], z[i + 3], __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]), c_h, c_h,
-                bb.z, bb.w);
+        for (int i = 0; i < 64; i += 4) {
+          const float4 bb = *reinterpret_cast<const float4*>(bias + 64 * hh + i);
+          float z0, z1, z2, z3;
+          ffma2(z0, z1, __uint_as_float(u[i]), __uint_as_float(u[i + 1]), c_h, c_h, bb.x, bb.y);
+          ffma2(z2, z3, __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]), c_h, c_h, bb.z, bb.w);
+          const int c0 = 64 * hh + i;
+          if (diag) {
+            if (c0 > row) z0 = -INFINITY;
+            if (c0 + 1 > row) z1 = -INFINITY;
+            if (c0 + 2 > row) z2 = -INFINITY;
+            if (c0 + 3 > row) z3 = -INFINITY;
+          }
+          mx[(i >> 2) & 1] = fmax3(mx[(i >> 2) & 1], z0, z1);
+          mx[2 + ((i >> 2) & 1)] = fmax3(mx[2 + ((i >> 2) & 1)], z2, z3);
         }
-      }
-      __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.b_empty[st]);
-      if (j == tq) {   // diagonal tile: key column i is visible to row r iff i <= r
-#pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i > row) z[i] = -INFINITY;
-      }
-      float mx[4] = {fmaxf(z[0], z[1]), fmaxf(z[2], z[3]), fmaxf(z[4], z[5]), fmaxf(z[6], z[7])};
-#pragma unroll
-      for (int i = 8; i < kBN; i += 8) {   // z[8..127]
-        mx[0] = fmax3(mx[0], z[i], z[i + 1]);
-        mx[1] = fmax3(mx[1], z[i + 2], z[i + 3]);
-        mx[2] = fmax3(mx[2], z[i + 4], z[i + 5]);
-        mx[3] = fmax3(mx[3], z[i + 6], z[i + 7]);
       }
       const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // the running max moves only when the tile's max exceeds it by more than 2^8
@@ -845,24 +844,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mt;
         rescale = true;
       }
-      uint32_t pk[kBN / 2];
+      // pass 2: weights 2^(z - m), packed to bf16 over S (columns 0..63: half hh of
+      // the row goes to columns 32hh..32hh+31, which the first half has already
+      // left); the row sum adds the bf16 weights the PV MMA multiplies, so
+      // numerator and denominator carry the same rounding
       float sa = 0.f, sb = 0.f;
       const float nm = -m;
 #pragma unroll
-      for (int i = 0; i < kBN; i += 4) {
-        float x0, x1, x2, x3;
-        fadd2(x0, x1, z[i], z[i + 1], nm, nm);
-        fadd2(x2, x3, z[i + 2], z[i + 3], nm, nm);
-        const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
-        const float p1 = tg::exp2_approx(x1);
-        const float p2 = tg::exp2_approx(x2);
-        const float p3 = tg::exp2_approx(x3);
-        pk[i / 2] = tg::pack_bf16x2(p0, p1);
-        pk[i / 2 + 1] = tg::pack_bf16x2(p2, p3);
-        // the row sum adds the bf16 weights the PV MMA multiplies (numerator and
-        // denominator then carry the same rounding)
-        fadd2(sa, sb, sa, sb, bf16x2_lo(pk[i / 2]) + bf16x2_lo(pk[i / 2 + 1]),
-              bf16x2_hi(pk[i / 2]) + bf16x2_hi(pk[i / 2 + 1]));
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t u[64];
+        tg::tmem_ld32x64(s_addr + 64u * hh, u);
+        tg::tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 64; i += 4) {
+          const float4 bb = *reinterpret_cast<const float4*>(bias + 64 * hh + i);
+          float z0, z1, z2, z3;
+          ffma2(z0, z1, __uint_as_float(u[i]), __uint_as_float(u[i + 1]), c_h, c_h, bb.x, bb.y);
+          ffma2(z2, z3, __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]), c_h, c_h, bb.z, bb.w);
+          const int c0 = 64 * hh + i;
+          if (diag) {
+            if (c0 > row) z0 = -INFINITY;
+            if (c0 + 1 > row) z1 = -INFINITY;
+            if (c0 + 2 > row) z2 = -INFINITY;
+            if (c0 + 3 > row) z3 = -INFINITY;
+          }
+          float x0, x1, x2, x3;
+          fadd2(x0, x1, z0, z1, nm, nm);
+          fadd2(x2, x3, z2, z3, nm, nm);
+          const float p0 = tg::exp2_approx(x0);
+          const float p1 = tg::exp2_approx(x1);
+          const float p2 = tg::exp2_approx(x2);
+          const float p3 = tg::exp2_approx(x3);
+          pk[i / 2] = tg::pack_bf16x2(p0, p1);
+          pk[i / 2 + 1] = tg::pack_bf16x2(p2, p3);
+          fadd2(sa, sb, sa, sb, bf16x2_lo(pk[i / 2]) + bf16x2_lo(pk[i / 2 + 1]),
+                bf16x2_hi(pk[i / 2]) + bf16x2_hi(pk[i / 2 + 1]));
+        }
+        tg::tmem_st32(s_addr + 32u * hh, pk);
       }
       l = l * alpha + (sa + sb);
       if (__any_sync(0xFFFFFFFFu, rescale)) {
@@ -879,9 +898,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tg::tmem_st32(oaddr + 32, o + 32);
         }
       }
-      // P_x(j) over S_x(j): packed bf16 pairs, columns 0..63 (the whole row was read)
-      tg::tmem_st32(s_addr, pk);
-      tg::tmem_st32(s_addr + 32, pk + 32);
       tg::tmem_st_wait();
       tg::tc_fence_before();
       __syncwarp();
