@@ -883,6 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tg::tmem_st32(s_addr + 32u * hh, pk);
       }
+      __syncwarp();
+      if (lane == 0) tg::mbar_arrive(&S.b_empty[st]);   // this warp is done with the biases
       l = l * alpha + (sa + sb);
       if (__any_sync(0xFFFFFFFFu, rescale)) {
         // PV_x(j-1) is complete (S_x(j) was issued after it): scale this row of O_x
