@@ -547,418 +547,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-namespace pair {
-
-// ---- Two query heads of one GQA group per CTA (even group sizes) ----
-// The CTA takes one query tile t of a sequence and two query heads A, B that read
-// the same KV head: both streams meet the same key tiles 0..t, so each K and V
-// tile is loaded once for both, and the two streams keep the tensor core busy in
-// turn (while stream A's softmax runs, the tensor core does B's PV and next S,
-// and the other way round). Query tiles go longest first (blockIdx.y counts down
-// from the last tile), so the grid's long CTAs start in the first wave.
-//   warps 0-3    softmax of stream A, warps 4-7 of stream B: one thread per query
-//                row (TMEM lane), the whole 128-key row of S in registers
-//                (32x32b loads), so row maxima and sums need no exchange.
-//   warp 8       TMA producer of both Q tiles and the K ring (2 stages).
-//   warp 9       MMA issuer: S_A(0), S_B(0), then per key tile j PV_A(j),
-//                S_A(j+1), PV_B(j), S_B(j+1). P_X(j) overwrites S_X(j) in TMEM
-//                (packed bf16, 64 columns), and S_X(j+1) is issued after PV_X(j), so
-//                the commit that signals S_X(j+1) also proves PV_X(j) is complete:
-//                a softmax pass can rescale O_X without any further wait.
-//   warp 10      TMA producer of the V ring (2 stages).
-//   warp 11      TMEM allocation, then each key tile's per-head biases
-//                log2(e) g_h s_j for both streams (4-stage ring).
-// TMEM: S_A at column 0, S_B at 128, O_A at 256, O_B at 384 (all 512 columns).
-// Epilogue: O / l in bf16 is written into the stream's own Q buffer (free after
-// its last S) in the tensor map's swizzled layout and stored by TMA; a tile that
-// ends past its sequence (the last, partial one) is stored row by row instead.
-constexpr int kBM = 128, kBN = 128, kD = 128;
-constexpr int kKStages = 2, kVStages = 2, kBiasStages = 4;
-constexpr int kThreads = 384;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;
-__device__ __forceinline__ uint32_t col_s(int x) { return 128u * x; }          // S/P of stream x
-__device__ __forceinline__ uint32_t col_o(int x) { return 256u + 128u * x; }   // O of stream x
-constexpr uint32_t kTmemCols = 512;
-
-struct Smem {
-  uint8_t q[2][2][kBM * 64 * 2];        // [stream][dh half], 16 KB each; then the output tile
-  uint8_t k[kKStages][2][kBN * 64 * 2];
-  uint8_t v[kVStages][2][kBN * 64 * 2];
-  float bias[kBiasStages][2][kBN];
-  uint64_t q_full;
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t b_full[kBiasStages], b_empty[kBiasStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
-  uint32_t tmem_base;
-  int abort_flag;
-};
-
-__global__ void __launch_bounds__(kThreads, 1)
-    gated_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
-                           const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v,
-                           const __grid_constant__ CUtensorMap tm_o,
-                           const float* __restrict__ s_kept, const float* __restrict__ gain,
-                           const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
-                           int total, int max_kept, int n_hq, int n_hkv,
-                           __nv_bfloat16* __restrict__ out, int* status) {
-  const int hp = blockIdx.x;                       // head pair: heads 2hp, 2hp + 1
-  const int tq = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);
-  const int b = blockIdx.z;
-  const int head[2] = {2 * hp, 2 * hp + 1};
-  const int kvh = head[0] / (n_hq / n_hkv);        // the group size is even: same KV head
-
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw + pad);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  if (tid == 0) {
-    tg::mbar_init(&S.q_full, 1);
-    for (int i = 0; i < kKStages; ++i) {
-      tg::mbar_init(&S.k_full[i], 1);
-      tg::mbar_init(&S.k_empty[i], 1);
-    }
-    for (int i = 0; i < kVStages; ++i) {
-      tg::mbar_init(&S.v_full[i], 1);
-      tg::mbar_init(&S.v_empty[i], 1);
-    }
-    for (int i = 0; i < kBiasStages; ++i) {
-      tg::mbar_init(&S.b_full[i], 32);   // every lane of the staging warp
-      tg::mbar_init(&S.b_empty[i], 8);   // every softmax warp
-    }
-    for (int x = 0; x < 2; ++x) {
-      tg::mbar_init(&S.s_full[x], 1);
-      tg::mbar_init(&S.p_full[x], 4);    // the stream's four softmax warps
-      tg::mbar_init(&S.o_done[x], 1);
-    }
-    S.abort_flag = 0;
-    tg::fence_barrier_init();
-  }
-  if (warp == 11) {
-    tg::tmem_alloc(&S.tmem_base, kTmemCols);
-    tg::tmem_relinquish();
-  }
-  if (warp == 8 && lane == 0) {
-    tg::tma_prefetch_desc(&tm_q);
-    tg::tma_prefetch_desc(&tm_k);
-    tg::tma_prefetch_desc(&tm_o);
-  }
-  if (warp == 10 && lane == 0) tg::tma_prefetch_desc(&tm_v);
-  tg::tc_fence_before();
-  __syncthreads();
-  tg::tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
-  tg::pdl_launch_dependents();
-  tg::pdl_wait();   // global memory only from here on
-
-  const int seq0 = cu_kept[b];
-  const int seq1 = cu_kept[b + 1];
-  const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
-  if (bad && tq == static_cast<int>(gridDim.y) - 1 && hp == 0 && tid == 0)
-    tg::set_status(status, TG_ERR_DEVICE_CHECK);
-  const int len = bad ? 0 : seq1 - seq0;
-  if (tq * kBM >= len) {   // uniform: this sequence has no query tile tq
-    if (warp == 11) tg::tmem_dealloc(tmem, kTmemCols);
-    return;
-  }
-  const int nt = tq + 1;   // key tiles 0..tq
-
-  if (warp == 8) {
-    // ---------------- TMA producer: Q (both heads) and the K ring ----------------
-    if (lane == 0) {
-      tg::mbar_arrive_expect_tx(&S.q_full, 2 * kBM * kD * 2);
-      for (int x = 0; x < 2; ++x) {
-        tg::tma_load_3d(S.q[x][0], &tm_q, &S.q_full, 0, head[x], seq0 + tq * kBM);
-        tg::tma_load_3d(S.q[x][1], &tm_q, &S.q_full, 64, head[x], seq0 + tq * kBM);
-      }
-      int j = 0;
-      for (; j < nt; ++j) {
-        const int st = j % kKStages;
-        if (j >= kKStages &&
-            !tg::mbar_wait(&S.k_empty[st], ((j / kKStages) - 1) & 1, status, &S.abort_flag))
-          break;
-        tg::mbar_arrive_expect_tx(&S.k_full[st], kBN * kD * 2);
-        tg::tma_load_3d(S.k[st][0], &tm_k, &S.k_full[st], 0, kvh, seq0 + j * kBN);
-        tg::tma_load_3d(S.k[st][1], &tm_k, &S.k_full[st], 64, kvh, seq0 + j * kBN);
-      }
-      if (S.abort_flag) {   // let the copies in flight land before the CTA exits
-        tg::mbar_wait(&S.q_full, 0, status, nullptr);
-        for (int i = j > kKStages ? j - kKStages : 0; i < j; ++i)
-          tg::mbar_wait(&S.k_full[i % kKStages], (i / kKStages) & 1, status, nullptr);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 10) {
-    // ---------------- TMA producer: the V ring ----------------
-    if (lane == 0) {
-      int j = 0;
-      for (; j < nt; ++j) {
-        const int st = j % kVStages;
-        if (j >= kVStages &&
-            !tg::mbar_wait(&S.v_empty[st], ((j / kVStages) - 1) & 1, status, &S.abort_flag))
-          break;
-        tg::mbar_arrive_expect_tx(&S.v_full[st], kBN * kD * 2);
-        tg::tma_load_3d(S.v[st][0], &tm_v, &S.v_full[st], 0, kvh, seq0 + j * kBN);
-        tg::tma_load_3d(S.v[st][1], &tm_v, &S.v_full[st], 64, kvh, seq0 + j * kBN);
-      }
-      if (S.abort_flag) {
-        for (int i = j > kVStages ? j - kVStages : 0; i < j; ++i)
-          tg::mbar_wait(&S.v_full[i % kVStages], (i / kVStages) & 1, status, nullptr);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 11) {
-    // ---------------- per-key biases of both heads (32 arrivals per stage) ----------------
-    const float ga = gain[head[0]] * kLog2e, gb = gain[head[1]] * kLog2e;
-    auto load = [&](int j, float* v) {
-#pragma unroll
-      for (int u = 0; u < kBN / 32; ++u) {
-        const int kp = j * kBN + lane + 32 * u;
-        v[u] = (j < nt && kp < len) ? s_kept[seq0 + kp] : 0.f;
-      }
-    };
-    float v0[kBN / 32], v1[kBN / 32];
-    load(0, v0);
-    load(1, v1);
-    for (int j = 0; j < nt; ++j) {
-      const int st = j % kBiasStages;
-      if (j >= kBiasStages &&
-          !__all_sync(0xFFFFFFFFu, tg::mbar_wait(&S.b_empty[st], ((j / kBiasStages) - 1) & 1,
-                                                 status, &S.abort_flag)))
-        break;
-#pragma unroll
-      for (int u = 0; u < kBN / 32; ++u) {
-        S.bias[st][0][lane + 32 * u] = ga * v0[u];
-        S.bias[st][1][lane + 32 * u] = gb * v0[u];
-        v0[u] = v1[u];
-      }
-      tg::mbar_arrive(&S.b_full[st]);
-      load(j + 2, v1);
-    }
-  } else if (warp == 9) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
-      constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBM, kD, false, true);
-      bool alive = tg::mbar_wait(&S.q_full, 0, status, &S.abort_flag);
-      auto issue_s = [&](int x, int j) -> bool {
-        const int st = j % kKStages;
-        if (x == 0 && !tg::mbar_wait(&S.k_full[st], (j / kKStages) & 1, status, &S.abort_flag))
-          return false;
-        tg::tc_fence_after();
-        const uint32_t q0 = tg::smem_u32(S.q[x][0]), k0 = tg::smem_u32(S.k[st][0]);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          tg::mma_bf16_ss(tmem + col_s(x), tg::smem_desc_sw128(q0 + off, 16, 1024),
-                          tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
-        }
-        tg::mma_commit(&S.s_full[x]);
-        if (x == 1) tg::mma_commit(&S.k_empty[st]);   // both streams' S of this key tile issued
-        return true;
-      };
-      auto issue_pv = [&](int x, int j) -> bool {
-        const int st = j % kVStages;
-        if (!tg::mbar_wait(&S.p_full[x], j & 1, status, &S.abort_flag)) return false;
-        if (x == 0 && !tg::mbar_wait(&S.v_full[st], (j / kVStages) & 1, status, &S.abort_flag))
-          return false;
-        tg::tc_fence_after();
-        const uint32_t v0 = tg::smem_u32(S.v[st][0]);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = P_x(j) in TMEM (8 packed columns per K=16 step); B = V rows
-          // 16kk..16kk+15, MN-major (dh halves 16 KB apart, 8-key groups 1 KB apart)
-          const uint64_t bdesc = tg::smem_desc_sw128(v0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-          tg::mma_bf16_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, bdesc, idesc_o, (j | kk) != 0);
-        }
-        if (x == 1) tg::mma_commit(&S.v_empty[st]);
-        if (j == nt - 1) tg::mma_commit(&S.o_done[x]);
-        return true;
-      };
-      if (alive) alive = issue_s(0, 0);
-      if (alive) alive = issue_s(1, 0);
-      for (int j = 0; j < nt && alive; ++j) {
-        alive = issue_pv(0, j);
-        if (alive && j + 1 < nt) alive = issue_s(0, j + 1);
-        if (alive) alive = issue_pv(1, j);
-        if (alive && j + 1 < nt) alive = issue_s(1, j + 1);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---------------- softmax: warps 0-3 stream A, 4-7 stream B ----------------
-    const int x = warp >> 2;
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;              // query row in the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + col_s(x);
-    const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[head[x]]);
-    float m = -INFINITY, l = 0.f;
-    bool alive = true;
-    for (int j = 0; j < nt; ++j) {
-      const int st = j % kBiasStages;
-      alive = tg::mbar_wait(&S.s_full[x], j & 1, status, &S.abort_flag);
-      if (alive) alive = tg::mbar_wait(&S.b_full[st], (j / kBiasStages) & 1, status, &S.abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
-      tg::tc_fence_after();
-      const float* bias = S.bias[st][x];
-      const bool diag = (j == tq);   // diagonal tile: key column i is visible to row r iff i <= r
-      // The row is read from TMEM twice, 64 columns at a time: first for its max,
-      // then for the weights, so that at most 64 logits and 32 packed weights are
-      // live per thread (a whole row at once spills).
-      // pass 1: z = S c_h + b (log2 domain) and the tile's row max
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t u[64];
-        tg::tmem_ld32x64(s_addr + 64u * hh, u);
-        tg::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          const float4 bb = *reinterpret_cast<const float4*>(bias + 64 * hh + i);
-          float z0, z1, z2, z3;
-          ffma2(z0, z1, __uint_as_float(u[i]), __uint_as_float(u[i + 1]), c_h, c_h, bb.x, bb.y);
-          ffma2(z2, z3, __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]), c_h, c_h, bb.z, bb.w);
-          const int c0 = 64 * hh + i;
-          if (diag) {
-            if (c0 > row) z0 = -INFINITY;
-            if (c0 + 1 > row) z1 = -INFINITY;
-            if (c0 + 2 > row) z2 = -INFINITY;
-            if (c0 + 3 > row) z3 = -INFINITY;
-          }
-          mx[(i >> 2) & 1] = fmax3(mx[(i >> 2) & 1], z0, z1);
-          mx[2 + ((i >> 2) & 1)] = fmax3(mx[2 + ((i >> 2) & 1)], z2, z3);
-        }
-      }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      // the running max moves only when the tile's max exceeds it by more than 2^8
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m = mt;
-      } else if (mt > m + kRescaleThreshold) {
-        alpha = tg::exp2_approx(m - mt);
-        m = mt;
-        rescale = true;
-      }
-      // pass 2: weights 2^(z - m), packed to bf16 over S (columns 0..63: half hh of
-      // the row goes to columns 32hh..32hh+31, which the first half has already
-      // left); the row sum adds the bf16 weights the PV MMA multiplies, so
-      // numerator and denominator carry the same rounding
-      float sa = 0.f, sb = 0.f;
-      const float nm = -m;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t u[64];
-        tg::tmem_ld32x64(s_addr + 64u * hh, u);
-        tg::tmem_ld_wait();
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          const float4 bb = *reinterpret_cast<const float4*>(bias + 64 * hh + i);
-          float z0, z1, z2, z3;
-          ffma2(z0, z1, __uint_as_float(u[i]), __uint_as_float(u[i + 1]), c_h, c_h, bb.x, bb.y);
-          ffma2(z2, z3, __uint_as_float(u[i + 2]), __uint_as_float(u[i + 3]), c_h, c_h, bb.z, bb.w);
-          const int c0 = 64 * hh + i;
-          if (diag) {
-            if (c0 > row) z0 = -INFINITY;
-            if (c0 + 1 > row) z1 = -INFINITY;
-            if (c0 + 2 > row) z2 = -INFINITY;
-            if (c0 + 3 > row) z3 = -INFINITY;
-          }
-          float x0, x1, x2, x3;
-          fadd2(x0, x1, z0, z1, nm, nm);
-          fadd2(x2, x3, z2, z3, nm, nm);
-          const float p0 = tg::exp2_approx(x0);
-          const float p1 = tg::exp2_approx(x1);
-          const float p2 = tg::exp2_approx(x2);
-          const float p3 = tg::exp2_approx(x3);
-          pk[i / 2] = tg::pack_bf16x2(p0, p1);
-          pk[i / 2 + 1] = tg::pack_bf16x2(p2, p3);
-          fadd2(sa, sb, sa, sb, bf16x2_lo(pk[i / 2]) + bf16x2_lo(pk[i / 2 + 1]),
-                bf16x2_hi(pk[i / 2]) + bf16x2_hi(pk[i / 2 + 1]));
-        }
-        tg::tmem_st32(s_addr + 32u * hh, pk);
-      }
-      __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.b_empty[st]);   // this warp is done with the biases
-      l = l * alpha + (sa + sb);
-      if (__any_sync(0xFFFFFFFFu, rescale)) {
-        // PV_x(j-1) is complete (S_x(j) was issued after it): scale this row of O_x
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t o[64];
-          const uint32_t oaddr = tmem + lane_base + col_o(x) + 64u * hh;
-          tg::tmem_ld32x64(oaddr, o);
-          tg::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tg::tmem_st32(oaddr, o);
-          tg::tmem_st32(oaddr + 32, o + 32);
-        }
-      }
-      tg::tmem_st_wait();
-      tg::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tg::mbar_arrive(&S.p_full[x]);
-    }
-    // ---------------- epilogue: O / l -> bf16 ----------------
-    if (alive) alive = tg::mbar_wait(&S.o_done[x], 0, status, &S.abort_flag);
-    const bool full_tile = (tq + 1) * kBM <= len;   // uniform across the CTA
-    uint8_t* stage = S.q[x][0];   // 32 KB: two [128 rows][128 B] halves, 128-byte swizzle
-    if (__all_sync(0xFFFFFFFFu, alive)) {
-      tg::tc_fence_after();
-      const float il = 1.f / l;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t o[64];
-        tg::tmem_ld32x64(tmem + lane_base + col_o(x) + 64u * hh, o);
-        tg::tmem_ld_wait();
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          w[i] = tg::pack_bf16x2(__uint_as_float(o[2 * i]) * il, __uint_as_float(o[2 * i + 1]) * il);
-        if (full_tile) {
-          uint8_t* rowp = stage + hh * (kBM * 128) + row * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7)) << 4)) =
-                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        } else if (tq * kBM + row < len) {
-          uint4* dst = reinterpret_cast<uint4*>(
-              out + (static_cast<int64_t>(seq0 + tq * kBM + row) * n_hq + head[x]) * kD + 64 * hh);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        }
-      }
-    }
-    if (full_tile) {
-      // every warp of the stream reaches this barrier, whether or not it wrote its
-      // rows: a warp that gave up after a bounded wait has set the abort flag first,
-      // and then nothing is stored
-      tg::fence_proxy_async_shared();
-      tg::named_barrier(1 + x, 128);   // the stream's 128 threads have written the tile
-      if (quarter == 0 && lane == 0 && S.abort_flag == 0) {
-        tg::tma_store_3d(&tm_o, stage, 0, head[x], seq0 + tq * kBM);
-        tg::tma_store_3d(&tm_o, stage + kBM * 128, 64, head[x], seq0 + tq * kBM);
-        tg::bulk_commit();
-        tg::bulk_wait_read_all();   // shared memory must outlive the stores' reads
-      }
-    }
-  }
-  tg::tc_fence_before();
-  __syncthreads();
-  if (warp == 11) {
-    tg::tc_fence_after();
-    tg::tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-}  // namespace pair
-
 namespace {
 
 // ---------------- exact fp32 path ----------------
@@ -1045,21 +633,6 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
       !tg::encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dk, sk, box,
                        CU_TENSOR_MAP_SWIZZLE_128B))
     return TG_ERR_CUDA;
-  if ((n_hq / n_hkv) % 2 == 0) {   // two query heads of one group per CTA
-    CUtensorMap to;
-    if (!tg::encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dq, sq, box,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-      return TG_ERR_CUDA;
-    const size_t psmem = sizeof(pair::Smem) + 1024;
-    if (!tg::ensure_smem(reinterpret_cast<const void*>(pair::gated_attn_pair_kernel),
-                         static_cast<int>(psmem)))
-      return TG_ERR_CUDA;
-    const int n_qt = (max_kept + kBM - 1) / kBM;
-    dim3 grid(n_hq / 2, n_qt, batch);   // y counts query tiles down: longest first
-    return tg::launch(pair::gated_attn_pair_kernel, grid, dim3(pair::kThreads), psmem, st, 0, tq,
-                      tk, tv, to, s_kept, gain, tau, cu_kept, static_cast<int>(total), max_kept,
-                      n_hq, n_hkv, static_cast<__nv_bfloat16*>(out), status);
-  }
   const size_t smem = sizeof(AttnSmem) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(gated_attn_bf16_kernel),
                        static_cast<int>(smem)))
