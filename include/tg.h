@@ -220,6 +220,33 @@ tg_status tg_gated_decode(const void* q, const void* k_cache, const void* v_cach
                           tg_stream_t stream);
 
 /*
+ * tg_gated_decode_noalloc: tg_gated_decode without a caller-provided workspace.
+ * There is no counterpart on the pages; this is a convenience of this library.
+ * It is for callers that cannot allocate device memory where they decode: a host
+ * program whose device memory all belongs to another runtime's pool (a library may
+ * not, or cannot, call cudaMalloc behind it), or a token-by-token generation loop
+ * that must not allocate because cudaMalloc and cudaFree can synchronise the whole
+ * device. The per-chunk partials go to a fixed array in the library's own device
+ * memory, TG_DECODE_NOALLOC_SCRATCH_BYTES large, which every device that loads the
+ * library holds until the process exits. Arguments, outputs and checks are those
+ * of tg_gated_decode; a call whose partials would need more than the array
+ * (tg_gated_decode_workspace_size(batch, n_hq, head_dim, max_len) >
+ * TG_DECODE_NOALLOC_SCRATCH_BYTES) returns TG_ERR_WORKSPACE and launches nothing.
+ * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. All calls share the one array and it keeps what the last
+ * call left there (nothing in it needs to start at zero): calls whose kernels
+ * overlap on the GPU (different streams, or different host threads) race on it.
+ */
+#define TG_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+tg_status tg_gated_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                  const float* s_cache, const int32_t* cache_len, int batch,
+                                  int cap, int max_len, int n_hq, int n_hkv, int head_dim,
+                                  const float* gain, const float* tau, void* out,
+                                  tg_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the first error any kernel recorded on the
  * current device since the last reset (TG_OK if none). reset != 0 clears it.
  */

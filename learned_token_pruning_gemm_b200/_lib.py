@@ -30,6 +30,7 @@ SIGNATURES = {
     "tg_gated_decode_workspace_size": (ctypes.c_size_t, [INT, INT, INT, INT]),
     "tg_gated_decode": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P,
                               ctypes.c_size_t, P]),
+    "tg_gated_decode_noalloc": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P]),
     "tg_device_status": (INT, [P, INT]),
     "tg_selftest_bounded_wait": (INT, [I64, P]),
 }

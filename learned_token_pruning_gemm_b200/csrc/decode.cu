@@ -20,6 +20,8 @@
 // to a caller-provided workspace. A second kernel merges a row's partials in
 // chunk order (a fixed order: the result does not depend on timing) and writes
 // O = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c in bf16.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -380,4 +382,60 @@ extern "C" tg_status tg_gated_decode(const void* q, const void* k_cache, const v
   return tg::launch(decode_combine_kernel, dim3(n_hq, batch), dim3(kThreads), 0, stream, 0,
                     static_cast<const float*>(part), cache_len, cap, max_len, n_hq, ns,
                     static_cast<__nv_bfloat16*>(out), st);
+}
+
+// ---- decode with library-owned scratch, for callers that cannot allocate ----
+//
+// tg_gated_decode needs a caller-provided workspace for its per-chunk partial
+// results. Some callers cannot allocate one where they call decode: a host
+// program whose device memory all belongs to another runtime's pool (so a
+// library may not, or cannot, call cudaMalloc behind it), or a token-by-token
+// generation loop that must not allocate at all because cudaMalloc and cudaFree
+// can synchronise the whole device. tg_gated_decode_noalloc serves them from a
+// fixed array in the library's own device memory instead. Every device that
+// loads the library holds that array (TG_DECODE_NOALLOC_SCRATCH_BYTES) until the
+// process exits, whether or not this entry point is ever called.
+static __device__ __align__(256) float g_decode_scratch[TG_DECODE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+float* g_scratch_addr[kMaxScratchDevices];   // device address of the array, per device
+std::mutex g_scratch_mu;
+
+// In host code g_decode_scratch names a host-side stand-in, not device memory: the
+// array's address on the current device comes from the runtime, looked up once
+// per device (with that device current) and kept.
+float* decode_scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" tg_status tg_gated_decode_noalloc(const void* q, const void* k_cache,
+                                             const void* v_cache, const float* s_cache,
+                                             const int32_t* cache_len, int batch, int cap,
+                                             int max_len, int n_hq, int n_hkv, int head_dim,
+                                             const float* gain, const float* tau, void* out,
+                                             tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_gated_decode_noalloc");
+  if (batch > 0 && n_hq > 0 && head_dim > 0) {
+    const size_t need = tg_gated_decode_workspace_size(batch, n_hq, head_dim, max_len > 0 ? max_len : 1);
+    if (need > TG_DECODE_NOALLOC_SCRATCH_BYTES) return TG_ERR_WORKSPACE;   // beyond the fixed array
+  }
+  float* scratch = nullptr;
+  if (batch > 0) {
+    scratch = decode_scratch_on_current_device();
+    if (!scratch) return TG_ERR_CUDA;
+  }
+  return tg_gated_decode(q, k_cache, v_cache, s_cache, cache_len, batch, cap, max_len, n_hq, n_hkv,
+                         head_dim, gain, tau, out, scratch, TG_DECODE_NOALLOC_SCRATCH_BYTES, stream);
 }
