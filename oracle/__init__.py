@@ -55,6 +55,10 @@ def lib():
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           P, P, P]
         L.oracle_gated_decode.restype = None
+        L.oracle_gated_attention_bwd.argtypes = [P, P, P, P, ctypes.c_int, P, P, P, P,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, P, P, P, P, P, P]
+        L.oracle_gated_attention_bwd.restype = None
         _lib = L
     return _lib
 
@@ -185,3 +189,27 @@ def gated_decode(q, k_cache, v_cache, s_cache, cache_len, gain, tau) -> np.ndarr
     lib().oracle_gated_decode(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(s), _ptr(ln), B, cap, hq,
                               hkv, dh, _ptr(g), _ptr(t), _ptr(out))
     return out
+
+
+def gated_attention_bwd(q, k, v, dout, s_kept, gain, tau, cu_kept):
+    """Gradients of the gated attention for upstream dout: returns fp64
+    (dq [K,hq,dh], dk [K,hkv,dh], dv [K,hkv,dh], ds [K], dgain [hq], dtau [hq])."""
+    qr, dt = _raw(q)
+    kr, dt2 = _raw(k)
+    vr, dt3 = _raw(v)
+    dr, dt4 = _raw(dout)
+    assert dt == dt2 == dt3 == dt4
+    K, hq, dh = qr.shape
+    hkv = kr.shape[1]
+    s, g, t = _f32(s_kept), _f32(gain), _f32(tau)
+    cu = _i32(cu_kept)
+    dq = np.empty((K, hq, dh))
+    dk = np.empty((K, hkv, dh))
+    dv = np.empty((K, hkv, dh))
+    ds = np.empty(K)
+    dg = np.empty(hq)
+    dtau = np.empty(hq)
+    lib().oracle_gated_attention_bwd(_ptr(qr), _ptr(kr), _ptr(vr), _ptr(dr), dt, _ptr(s), _ptr(g),
+                                     _ptr(t), _ptr(cu), len(cu) - 1, hq, hkv, dh, _ptr(dq),
+                                     _ptr(dk), _ptr(dv), _ptr(ds), _ptr(dg), _ptr(dtau))
+    return dq, dk, dv, ds, dg, dtau

@@ -244,6 +244,76 @@ void oracle_qkv_rope(const void* xc, int dtype, int64_t n, int d, const void* w,
   }
 }
 
+// Backward of the token-gated attention (MarkTechPost page, section "Qu'est-ce que
+// l'attention gérée par des tokens ?": the key score is a logit bias precisely so
+// that gradients reach the scorer; the gain and the temperature are learned).
+// Given dO = dL/dO for the forward above, for sequence b, query head hq (KV head
+// kv), kept rows i and keys j <= i, with c = 1 / (sqrt(dh) tau[hq]):
+//   z_ij = c q_i.k_j + gain s_j,  P_ij = softmax_j(z_ij),  dP_ij = dO_i . v_j
+//   D_i = sum_j P_ij dP_ij,       dZ_ij = P_ij (dP_ij - D_i)
+//   dq_i += c sum_j dZ_ij k_j     dk_j += c dZ_ij q_i      dv_j += P_ij dO_i
+//   ds_j += gain dZ_ij            dgain += dZ_ij s_j
+//   dtau += dZ_ij dz_ij/dtau = dZ_ij (-(q_i.k_j) / (sqrt(dh) tau^2))
+// (dk, dv and ds sum over every query head that reads the key; dgain and dtau are
+// per query head). q, k, v, dout in `dtype`; every output fp64 and overwritten.
+void oracle_gated_attention_bwd(const void* q, const void* k, const void* v, const void* dout,
+                                int dtype, const float* s_kept, const float* gain,
+                                const float* tau, const int32_t* cu_kept, int batch, int n_hq,
+                                int n_hkv, int dh, double* dq, double* dk, double* dv,
+                                double* ds, double* dgain, double* dtau) {
+  const int64_t total = cu_kept[batch];
+  const int group = n_hq / n_hkv;
+  for (int64_t t = 0; t < total * n_hq * dh; ++t) dq[t] = 0.0;
+  for (int64_t t = 0; t < total * n_hkv * dh; ++t) dk[t] = dv[t] = 0.0;
+  for (int64_t t = 0; t < total; ++t) ds[t] = 0.0;
+  for (int h = 0; h < n_hq; ++h) dgain[h] = dtau[h] = 0.0;
+  auto at = [&](const void* p, int64_t row, int nh, int h, int c) {
+    return load_elem(p, dtype, (row * nh + h) * (int64_t)dh + c);
+  };
+  for (int b = 0; b < batch; ++b) {
+    const int64_t j0 = cu_kept[b], j1 = cu_kept[b + 1];
+    for (int hq = 0; hq < n_hq; ++hq) {
+      const int kv = hq / group;
+      const double g = (double)gain[hq], tq = (double)tau[hq];
+      const double c = 1.0 / (std::sqrt((double)dh) * tq);
+      for (int64_t i = j0; i < j1; ++i) {
+        const int64_t n = i - j0 + 1;
+        std::vector<double> qk(n), z(n), p(n), dp(n);
+        double zmax = -INFINITY;
+        for (int64_t j = j0; j <= i; ++j) {
+          double dot = 0.0;
+          for (int e = 0; e < dh; ++e) dot += at(q, i, n_hq, hq, e) * at(k, j, n_hkv, kv, e);
+          qk[j - j0] = dot;
+          z[j - j0] = c * dot + g * (double)s_kept[j];
+          zmax = std::max(zmax, z[j - j0]);
+        }
+        double den = 0.0;
+        for (int64_t u = 0; u < n; ++u) den += (p[u] = std::exp(z[u] - zmax));
+        for (int64_t u = 0; u < n; ++u) p[u] /= den;
+        double D = 0.0;
+        for (int64_t j = j0; j <= i; ++j) {
+          double dot = 0.0;
+          for (int e = 0; e < dh; ++e) dot += at(dout, i, n_hq, hq, e) * at(v, j, n_hkv, kv, e);
+          dp[j - j0] = dot;
+          D += p[j - j0] * dot;
+        }
+        for (int64_t j = j0; j <= i; ++j) {
+          const int64_t u = j - j0;
+          const double dz = p[u] * (dp[u] - D);
+          for (int e = 0; e < dh; ++e) {
+            dq[(i * n_hq + hq) * dh + e] += c * dz * at(k, j, n_hkv, kv, e);
+            dk[(j * n_hkv + kv) * dh + e] += c * dz * at(q, i, n_hq, hq, e);
+            dv[(j * n_hkv + kv) * dh + e] += p[u] * at(dout, i, n_hq, hq, e);
+          }
+          ds[j] += g * dz;
+          dgain[hq] += dz * (double)s_kept[j];
+          dtau[hq] += dz * (-qk[u] / (std::sqrt((double)dh) * tq * tq));
+        }
+      }
+    }
+  }
+}
+
 // Decode over the compacted cache (MarkTechPost page, section "Comment déployer
 // TokenGate ?": generation runs on the cache the pruned prefill left behind, with
 // max_kept_prefill_tokens bounding it; section "Qu'est-ce que l'attention gérée
