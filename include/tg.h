@@ -144,6 +144,8 @@ tg_status tg_compact_kv(const void* const* src, void* const* dst, const int64_t*
  *   s_kept [total_kept] f32 (from tg_select_topk), gain, tau [n_hq] f32
  *   cu_kept [batch+1] int32 device; max_kept >= every cu_kept[b+1]-cu_kept[b]
  *   out  [total_kept, n_hq, head_dim]  dtype output
+ *   lse  [n_hq, total_kept] f32 output, may be NULL: each row's log-sum-exp
+ *        log(sum_j exp(z_j)) (natural log), which the backward reads
  * A sequence whose kept range is not inside [0, total_kept] or is longer than
  * max_kept is skipped (its out rows are left as they were) and TG_ERR_DEVICE_CHECK
  * is recorded.
@@ -153,7 +155,36 @@ tg_status tg_compact_kv(const void* const* src, void* const* dst, const int64_t*
 tg_status tg_gated_attention(const void* q, const void* k, const void* v, tg_dtype dtype,
                              const float* s_kept, const float* gain, const float* tau,
                              const int32_t* cu_kept, int batch, int64_t total_kept, int max_kept,
-                             int n_hq, int n_hkv, int head_dim, void* out, tg_stream_t stream);
+                             int n_hq, int n_hkv, int head_dim, void* out, float* lse,
+                             tg_stream_t stream);
+
+/*
+ * Backward of tg_gated_attention (MarkTechPost page on TokenGate, section "Qu'est-ce
+ * que l'attention gérée par des tokens ?": the key score enters the logits as a bias
+ * so that gradients reach the scorer; gain and temperature are learned per head).
+ * Given dout = dL/dout for a forward call (same q, k, v, s_kept, gain, tau, cu_kept)
+ * and that call's out and lse, with c_h = 1 / (sqrt(head_dim) tau[h]),
+ * P = softmax_j(z), dZ_ij = P_ij (dout_i . v_j - dout_i . out_i):
+ *   dq [total_kept, n_hq, head_dim]  dtype   c_h sum_j dZ_ij k_j
+ *   dk, dv [total_kept, n_hkv, head_dim] dtype   sum over the group's heads of
+ *                                     c_h sum_i dZ_ij q_i and sum_i P_ij dout_i
+ *   ds [total_kept] f32               dL/ds_j = sum_h gain[h] sum_i dZ_ij
+ *   dgain, dtau [n_hq] f32            sum_ij dZ_ij s_j and -(c_h/tau_h) sum_ij dZ_ij q_i.k_j
+ * Every output is overwritten. workspace: caller-owned device scratch of at least
+ * tg_gated_attention_bwd_workspace_size(...) bytes, 16-byte aligned, no initial
+ * value needed (too small: TG_ERR_WORKSPACE). TG_BF16: head_dim == 128 (tensor
+ * cores), pointers 16-byte aligned; TG_F32: head_dim <= 256 (exact SIMT path).
+ * Sequences whose kept range is invalid are skipped and TG_ERR_DEVICE_CHECK recorded.
+ */
+size_t tg_gated_attention_bwd_workspace_size(tg_dtype dtype, int batch, int64_t total_kept,
+                                             int max_kept, int n_hq, int n_hkv, int head_dim);
+tg_status tg_gated_attention_bwd(const void* q, const void* k, const void* v, const void* out,
+                                 const void* dout, tg_dtype dtype, const float* lse,
+                                 const float* s_kept, const float* gain, const float* tau,
+                                 const int32_t* cu_kept, int batch, int64_t total_kept,
+                                 int max_kept, int n_hq, int n_hkv, int head_dim, void* dq,
+                                 void* dk, void* dv, float* ds, float* dgain, float* dtau,
+                                 void* workspace, size_t workspace_bytes, tg_stream_t stream);
 
 /*
  * The kept tokens' q/k/v projections for the layers above the gate layer, so the

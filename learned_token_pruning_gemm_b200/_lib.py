@@ -24,7 +24,10 @@ SIGNATURES = {
     "tg_gate_score": (INT, [P, INT, I64, INT, P, P, P, F32, INT, P, P]),
     "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P, P]),
     "tg_compact_kv": (INT, [P, P, P, INT, P, I64, I64, P]),
-    "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P]),
+    "tg_gated_attention": (INT, [P, P, P, INT, P, P, P, P, INT, I64, INT, INT, INT, INT, P, P, P]),
+    "tg_gated_attention_bwd_workspace_size": (ctypes.c_size_t, [INT, INT, I64, INT, INT, INT, INT]),
+    "tg_gated_attention_bwd": (INT, [P, P, P, P, P, INT, P, P, P, P, P, INT, I64, INT, INT, INT,
+                                     INT, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
     "tg_qkv_rope": (INT, [P, I64, INT, P, INT, INT, INT, F32, P, P, P, P, P]),
     "tg_cache_append": (INT, [P, P, P, INT, INT, INT, INT, P, P, P, P, P]),
     "tg_gated_decode_workspace_size": (ctypes.c_size_t, [INT, INT, INT, INT]),

@@ -137,8 +137,10 @@ def compact_rows(srcs: Sequence[torch.Tensor], kept_idx: torch.Tensor,
 
 def gated_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s_kept: torch.Tensor,
                     gain: torch.Tensor, tau: torch.Tensor, cu_kept: torch.Tensor, max_kept: int,
-                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Token-gated causal GQA attention. q [K,Hq,dh], k/v [K,Hkv,dh] (same dtype)."""
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Token-gated causal GQA attention. q [K,Hq,dh], k/v [K,Hkv,dh] (same dtype).
+    If `lse` ([Hq, K] f32) is given, each row's log-sum-exp is written there."""
     K, hq, dh = q.shape
     hkv = k.shape[1]
     if k.shape != (K, hkv, dh) or v.shape != k.shape or not (q.dtype == k.dtype == v.dtype):
@@ -153,14 +155,65 @@ def gated_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s_kept: t
     if out is None:
         out = torch.empty_like(q)
     _shape(out, q.shape, "out", q.dtype)
+    if lse is not None:
+        _shape(lse, (hq, K), "lse", torch.float32)
     B = cu_kept.numel() - 1
     st = _lib.load().tg_gated_attention(
         _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _DT[q.dtype],
         _cuda(s_kept, "s_kept", torch.float32), _cuda(gain, "gain", torch.float32),
         _cuda(tau, "tau", torch.float32), _cuda(cu_kept, "cu_kept", torch.int32), B, K,
-        int(max_kept), hq, hkv, dh, _cuda(out, "out"), _stream(stream))
+        int(max_kept), hq, hkv, dh, _cuda(out, "out"),
+        _cuda(lse, "lse") if lse is not None else None, _stream(stream))
     check(st, "tg_gated_attention")
     return out
+
+
+def gated_attention_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                        dout: torch.Tensor, lse: torch.Tensor, s_kept: torch.Tensor,
+                        gain: torch.Tensor, tau: torch.Tensor, cu_kept: torch.Tensor,
+                        max_kept: int, grads=None, workspace: Optional[torch.Tensor] = None,
+                        stream=None):
+    """Gradients of gated_attention: returns (dq, dk, dv, ds, dgain, dtau) for upstream
+    dout, from the forward's out and lse ([Hq, K] f32)."""
+    K, hq, dh = q.shape
+    hkv = k.shape[1]
+    if k.shape != (K, hkv, dh) or v.shape != k.shape or not (q.dtype == k.dtype == v.dtype):
+        raise TokenGateError("gated_attention_bwd: q [K,Hq,dh], k/v [K,Hkv,dh] with one dtype")
+    if q.dtype not in _DT:
+        raise TokenGateError(f"gated_attention_bwd: unsupported dtype {q.dtype}")
+    _shape(out, q.shape, "out", q.dtype)
+    _shape(dout, q.shape, "dout", q.dtype)
+    _shape(lse, (hq, K), "lse", torch.float32)
+    _numel(s_kept, K, "s_kept")
+    _numel(gain, hq, "gain")
+    _numel(tau, hq, "tau")
+    B = cu_kept.numel() - 1
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty(K, **f32), torch.empty(hq, **f32), torch.empty(hq, **f32))
+    dq, dk, dv, ds, dg, dt = grads
+    _shape(dq, q.shape, "dq", q.dtype)
+    _shape(dk, k.shape, "dk", q.dtype)
+    _shape(dv, k.shape, "dv", q.dtype)
+    _shape(ds, (K,), "ds", torch.float32)
+    _shape(dg, (hq,), "dgain", torch.float32)
+    _shape(dt, (hq,), "dtau", torch.float32)
+    lib = _lib.load()
+    need = int(lib.tg_gated_attention_bwd_workspace_size(_DT[q.dtype], B, K, int(max_kept), hq,
+                                                           hkv, dh))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    nb = workspace.numel() * workspace.element_size()
+    st = lib.tg_gated_attention_bwd(
+        _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(out, "out"), _cuda(dout, "dout"),
+        _DT[q.dtype], _cuda(lse, "lse"), _cuda(s_kept, "s_kept", torch.float32),
+        _cuda(gain, "gain", torch.float32), _cuda(tau, "tau", torch.float32),
+        _cuda(cu_kept, "cu_kept", torch.int32), B, K, int(max_kept), hq, hkv, dh, _cuda(dq, "dq"),
+        _cuda(dk, "dk"), _cuda(dv, "dv"), _cuda(ds, "ds"), _cuda(dg, "dgain"), _cuda(dt, "dtau"),
+        _cuda(workspace, "workspace"), nb, _stream(stream))
+    check(st, "tg_gated_attention_bwd")
+    return dq, dk, dv, ds, dg, dt
 
 
 def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: torch.Tensor,

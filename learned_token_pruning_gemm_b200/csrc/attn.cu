@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const float* __restrict__ s_kept, const float* __restrict__ gain,
                            const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
                            int total, int max_kept, int n_hq, int n_hkv,
-                           __nv_bfloat16* __restrict__ out, int* status) {
+                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                           int* status) {
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
   const int z = blockIdx.z;
@@ -518,6 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) tg::mbar_arrive(&S.o_free);   // O may now be overwritten
       const float ia = 1.f / la, ib = 1.f / lb;
       const int ga = t * kBM + ra, gb = t * kBM + rb;
+      if (lse && cq == 0) {   // log-sum-exp of each row's logits (natural log), [n_hq, total]
+        constexpr float kLn2 = 0.69314718055994531f;
+        if (ga < len) lse[static_cast<int64_t>(hq) * total + seq0 + ga] = (ma + __log2f(la)) * kLn2;
+        if (gb < len) lse[static_cast<int64_t>(hq) * total + seq0 + gb] = (mb + __log2f(lb)) * kLn2;
+      }
       if (ga < len) {
         uint32_t* orow = reinterpret_cast<uint32_t*>(
             out + (static_cast<int64_t>(seq0 + ga) * n_hq + hq) * kD + cq);
@@ -557,7 +563,8 @@ __global__ void __launch_bounds__(kF32Warps * 32)
                           const float* __restrict__ v, const float* __restrict__ s_kept,
                           const float* __restrict__ gain, const float* __restrict__ tau,
                           const int32_t* __restrict__ cu_kept, int batch, int64_t total,
-                          int n_hq, int n_hkv, int dh, float* __restrict__ out, int* status) {
+                          int n_hq, int n_hkv, int dh, float* __restrict__ out,
+                          float* __restrict__ lse, int* status) {
   tg::pdl_launch_dependents();
   tg::pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -606,6 +613,7 @@ __global__ void __launch_bounds__(kF32Warps * 32)
     }
     m = m_new;
   }
+  if (lse && lane == 0) lse[static_cast<int64_t>(hq) * total + i] = m + logf(l);
   float* oi = out + (i * n_hq + hq) * dh;
 #pragma unroll
   for (int e = 0; e < kMaxPerLane; ++e) {
@@ -617,7 +625,7 @@ __global__ void __launch_bounds__(kF32Warps * 32)
 tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const float* s_kept,
                            const float* gain, const float* tau, const int32_t* cu_kept, int batch,
                            int64_t total, int max_kept, int n_hq, int n_hkv, void* out,
-                           cudaStream_t st) {
+                           float* lse, cudaStream_t st) {
   int* status = tg::status_word();
   if (!status) return TG_ERR_CUDA;
   CUtensorMap tq, tk, tv;
@@ -641,7 +649,7 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
   dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
   return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv, s_kept,
                     gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
-                    static_cast<__nv_bfloat16*>(out), status);
+                    static_cast<__nv_bfloat16*>(out), lse, status);
 }
 
 }  // namespace
@@ -650,7 +658,7 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
                                         tg_dtype dtype, const float* s_kept, const float* gain,
                                         const float* tau, const int32_t* cu_kept, int batch,
                                         int64_t total_kept, int max_kept, int n_hq, int n_hkv,
-                                        int head_dim, void* out, tg_stream_t stream) {
+                                        int head_dim, void* out, float* lse, tg_stream_t stream) {
   tg::NvtxRange nvtx_range("tg_gated_attention");
   if (batch < 0 || total_kept < 0 || max_kept < 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0)
     return TG_ERR_INVALID_ARG;
@@ -665,7 +673,7 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
     if (!tg::aligned16(q) || !tg::aligned16(k) || !tg::aligned16(v) || !tg::aligned16(out))
       return TG_ERR_MISALIGNED;
     return launch_attn_bf16(q, k, v, s_kept, gain, tau, cu_kept, batch, total_kept, max_kept, n_hq,
-                            n_hkv, out, stream);
+                            n_hkv, out, lse, stream);
   }
   if (dtype == TG_F32) {
     if (head_dim > 256) return TG_ERR_UNSUPPORTED;
@@ -677,7 +685,7 @@ extern "C" tg_status tg_gated_attention(const void* q, const void* k, const void
     return tg::launch(gated_attn_f32_kernel, grid, dim3(kF32Warps * 32), 0, stream, 0,
                       static_cast<const float*>(q), static_cast<const float*>(k),
                       static_cast<const float*>(v), s_kept, gain, tau, cu_kept, batch, total_kept,
-                      n_hq, n_hkv, head_dim, static_cast<float*>(out), status);
+                      n_hq, n_hkv, head_dim, static_cast<float*>(out), lse, status);
   }
   return TG_ERR_UNSUPPORTED;
 }

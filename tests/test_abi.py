@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.tg_abi_version() == 2
+    assert lib.tg_abi_version() == 3
     for code, name in [(0, "TG_OK"), (1, "TG_ERR_INVALID_ARG"), (3, "TG_ERR_MISALIGNED"),
                        (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (99, "TG_ERR_UNKNOWN")]:
         assert lib.tg_status_string(code).decode() == name
@@ -73,12 +73,12 @@ def test_validation_returns_status_without_gpu(lib):
     assert lib.tg_compact_kv(arr, arr, rb, 1, fake, 0, 10, None) == 0
     # attention: GQA divisibility, head dim, max_kept > total, alignment
     args = [fake, fake, fake, 1, fake, fake, fake, fake, 1, 256, 256]
-    assert lib.tg_gated_attention(*args, 16, 6, 128, fake, None) == INVALID
-    assert lib.tg_gated_attention(*args, 16, 8, 64, fake, None) == UNSUP
-    assert lib.tg_gated_attention(*args[:-1], 300, 16, 8, 128, fake, None) == INVALID
-    assert lib.tg_gated_attention(*args, 16, 8, 128, odd, None) == MIS
+    assert lib.tg_gated_attention(*args, 16, 6, 128, fake, None, None) == INVALID
+    assert lib.tg_gated_attention(*args, 16, 8, 64, fake, None, None) == UNSUP
+    assert lib.tg_gated_attention(*args[:-1], 300, 16, 8, 128, fake, None, None) == INVALID
+    assert lib.tg_gated_attention(*args, 16, 8, 128, odd, None, None) == MIS
     assert lib.tg_gated_attention(fake, fake, fake, 1, fake, fake, fake, fake, 1, 256, 256, 16, 8,
-                                  300, fake, None) == UNSUP
+                                  300, fake, None, None) == UNSUP
     # self test bounds
     assert lib.tg_selftest_bounded_wait(10, None) == INVALID
     # q/k/v projection: head_dim 128 only, even head total, d % 64, rope_base > 1,
@@ -230,3 +230,29 @@ def test_binding_decode_checks_shapes():
     _raises(lambda: api.gated_decode(q, kc, kc, sc, ln, torch.zeros(3), g, 50), "gain must have 4")
     _raises(lambda: api.cache_append(kc[:, 0], kc[:, 0], torch.zeros(3), kc, kc, sc, ln),
             "s_new must")
+
+
+def test_backward_validation_without_gpu(lib):
+    INVALID, UNSUP, MIS, WS = 1, 2, 3, 4
+    P = ctypes.c_void_p
+    fake, odd = P(0x10000), P(0x10004)
+    size = lib.tg_gated_attention_bwd_workspace_size
+    assert size(1, 1, 1868, 1868, 16, 8, 128) > 0
+    assert size(1, 1, 1868, 1868, 16, 6, 128) == 0
+    need = size(1, 1, 1000, 1000, 16, 8, 128)
+
+    def bwd(dtype=1, hq=16, hkv=8, dh=128, ws=fake, nb=None, q=fake, total=1000, mk=1000):
+        return lib.tg_gated_attention_bwd(q, fake, fake, fake, fake, dtype, fake, fake, fake, fake,
+                                          fake, 1, total, mk, hq, hkv, dh, fake, fake, fake, fake,
+                                          fake, fake, ws, need if nb is None else nb, None)
+    assert bwd(hkv=6) == INVALID
+    assert bwd(mk=1001) == INVALID
+    assert bwd(dh=64) == UNSUP
+    assert bwd(dtype=0, dh=512) == UNSUP
+    assert bwd(dtype=5) == UNSUP
+    assert bwd(nb=need - 1) == WS
+    assert bwd(ws=None) == WS
+    assert bwd(ws=odd) == MIS
+    assert bwd(q=odd) == MIS
+    assert bwd(q=None) == INVALID
+    assert bwd(total=0) == 0
