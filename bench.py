@@ -373,6 +373,58 @@ def _time_decode(gp, wl, steps, warmup, rep, flush, stream, hbm_peak):
                     "K, V and scores read once, q and out"}
 
 
+def _time_backward(gp, wl, steps, warmup, rep, flush, stream, tf_peak):
+    """The backward of the gated attention on the measured layer's kept rows: the
+    forward once (with its log-sum-exp), then `steps` backward calls for a seeded
+    upstream gradient, captured as one CUDA graph (five launches), L2 flushed before
+    each. Algorithmic flops: the five causal contractions S, dP, dV, dK, dQ, i.e.
+    2.5 times the forward's."""
+    from learned_token_pruning_gemm_b200 import api
+    K = gp.total_kept
+    lse = torch.empty(wl.hq, K, device=gp.q.device)
+    out = api.gated_attention(gp.q, gp.k, gp.v, gp.kept_scores, gp.gain, gp.tau, gp.cu_kept,
+                              gp.max_kept, lse=lse)
+    g = torch.Generator(device="cpu").manual_seed(9)
+    dout = torch.randn(out.shape, generator=g).to(out.dtype).to(out.device)
+    grads = api.gated_attention_bwd(gp.q, gp.k, gp.v, out, dout, lse, gp.kept_scores, gp.gain,
+                                    gp.tau, gp.cu_kept, gp.max_kept)
+    need = api._lib.load().tg_gated_attention_bwd_workspace_size(1, wl.batch, K, gp.max_kept,
+                                                                  wl.hq, wl.hkv, wl.dh)
+    ws = torch.empty(need, dtype=torch.uint8, device=gp.q.device)
+
+    def step():
+        api.gated_attention_bwd(gp.q, gp.k, gp.v, out, dout, lse, gp.kept_scores, gp.gain,
+                                gp.tau, gp.cu_kept, gp.max_kept, grads=grads, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    rep.barrier()
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    rep.barrier()
+    if api.device_status(reset=True) != 0:
+        raise RuntimeError("device status set by the backward")
+    ms = rep.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
+    flops = 2.5 * _work(wl)["attn_flops"]
+    return {"us": ms * 1e3, "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_tc": flops / (ms / 1e3) / 1e12 / tf_peak, "launches_per_step": 5,
+            "note": "dQ, dK, dV, score, gain and temperature gradients; flops = 2.5 x the "
+                    "forward's causal flops (S, dP, dV, dK, dQ)"}
+
+
 def run_ours(args, rep):
     ws, rank = rep.world, rep.rank
     from learned_token_pruning_gemm_b200 import pipeline, synth
@@ -411,6 +463,10 @@ def run_ours(args, rep):
     if wl.dtype == "bf16" and wl.dh == 128 and not args.no_decode:
         decode = _time_decode(gp, wl, args.steps, args.warmup, rep, flush, stream, hbm_peak)
 
+    backward = None
+    if wl.dtype == "bf16" and wl.dh == 128 and not args.no_backward:
+        backward = _time_backward(gp, wl, args.steps, args.warmup, rep, flush, stream, tf_peak)
+
     # ---- the other single-GPU workloads of the metric (16k-128k): same measurement ----
     others = {}
     for name in ([] if args.no_extra_workloads else args.extra_workloads.split(",")):
@@ -428,6 +484,9 @@ def run_ours(args, rep):
         if not args.no_decode and owl.dtype == "bf16" and owl.dh == 128:
             others[name]["decode"] = _time_decode(ogp, owl, args.steps, args.warmup, rep, flush,
                                                   stream, hbm_peak)
+        if not args.no_backward and owl.dtype == "bf16" and owl.dh == 128:
+            others[name]["backward"] = _time_backward(ogp, owl, args.steps, args.warmup, rep, flush,
+                                                      stream, tf_peak)
         del ogp, owl
         torch.cuda.empty_cache()
     clocks.stop()
@@ -499,6 +558,7 @@ def run_ours(args, rep):
             "e2e": e2e,
             "with_projection": with_proj,
             "decode": decode,
+            "backward": backward,
             "workloads": others,
             "cpu_baseline": cpu,
         }
@@ -533,6 +593,7 @@ def main():
                     help="other workloads measured the same way, reported under 'workloads'")
     ap.add_argument("--no-extra-workloads", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
