@@ -6,9 +6,13 @@
 //     z_ij = q_i . k_j / (sqrt(dh) tau_h) + g_h s_j,  j <= i;  O_i = softmax_j(z) V
 //
 // bf16 path (dh = 128). Causal work grows with the query tile index t (tile t
-// meets t+1 key tiles), so each CTA takes the pair of query tiles t and n-1-t of
-// one (query head, sequence): every CTA then does n+1 key tiles and the grid is
-// balanced. Per CTA, pipelines run across both query tiles:
+// meets t+1 key tiles). Two schedules: with few tiles per SM each CTA takes the
+// pair of query tiles t and n-1-t of one (query head, sequence), so every CTA does
+// n+1 key tiles and one wave holds the grid; with many, each CTA takes one query
+// tile and the grid is numbered longest tile first (blockIdx.x -> tile, sequence,
+// head), so the hardware, which starts CTAs in index order as SMs free up, packs
+// them greedily and no wave of equal-length CTAs leaves SMs idle at the end.
+// Per CTA, pipelines run across its query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
 //                ring. A K stage is free as soon as S_j is computed; with S issued
 //                three tiles ahead, each K load has about three tile periods to land.
@@ -136,12 +140,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const __grid_constant__ CUtensorMap tm_v,
                            const float* __restrict__ s_kept, const float* __restrict__ gain,
                            const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
-                           int total, int max_kept, int n_hq, int n_hkv,
-                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                           int* status) {
-  const int hq = blockIdx.x;
-  const int b = blockIdx.y;
-  const int z = blockIdx.z;
+                           int total, int max_kept, int n_hq, int n_hkv, int batch,
+                           int lpt_tiles, __nv_bfloat16* __restrict__ out,
+                           float* __restrict__ lse, int* status) {
+  // lpt_tiles > 0: one query tile per CTA, blockIdx.x = item in longest-first order
+  // (tile lpt_tiles-1 of every sequence and head first); 0: grid (head, sequence,
+  // pair z) and the pair of tiles n-1-z, z
+  int hq, b, z;
+  if (lpt_tiles > 0) {
+    const int i = blockIdx.x;
+    hq = i % n_hq;
+    b = (i / n_hq) % batch;
+    z = lpt_tiles - 1 - i / (n_hq * batch);   // the CTA's query tile
+  } else {
+    hq = blockIdx.x;
+    b = blockIdx.y;
+    z = blockIdx.z;
+  }
   const int kvh = hq / (n_hq / n_hkv);
 
   extern __shared__ uint8_t smem_raw[];
@@ -192,16 +207,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // a kept range outside [0, total] or longer than max_kept (the grid covers
   // max_kept rows per sequence) is not attended: record it and skip the sequence
   const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
-  if (bad && z == 0 && hq == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+  if (bad && hq == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
   const int len = bad ? 0 : seq1 - seq0;
   const int n_t = (len + kBM - 1) / kBM;
-  if (2 * z >= n_t) {           // uniform: this sequence has no pair z
+  if ((lpt_tiles > 0 ? z : 2 * z) >= n_t) {   // uniform: this sequence has no such tile
     if (warp == 2) tg::tmem_dealloc(tmem, kTmemCols);
     return;
   }
   // the CTA's query tiles: the long one first, then its partner (if distinct)
-  const int tiles[2] = {n_t - 1 - z, z};
-  const int nq = (tiles[1] < tiles[0]) ? 2 : 1;
+  const int tiles[2] = {lpt_tiles > 0 ? z : n_t - 1 - z, lpt_tiles > 0 ? z : z};
+  const int nq = (lpt_tiles == 0 && tiles[1] < tiles[0]) ? 2 : 1;
 
   if (warp == 0) {
     // ---------------- TMA producer: Q and K tiles ----------------
@@ -646,9 +661,21 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
                        static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const int n_qt = (max_kept + kBM - 1) / kBM;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return TG_ERR_CUDA;
+  const int64_t pairs = static_cast<int64_t>(n_hq) * batch * ((n_qt + 1) / 2);
+  if (pairs > sms && static_cast<int64_t>(n_qt) * batch * n_hq <= INT32_MAX) {
+    // more than one wave of pairs: one tile per CTA, longest first
+    dim3 grid(static_cast<unsigned>(static_cast<int64_t>(n_qt) * batch * n_hq));
+    return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv,
+                      s_kept, gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
+                      batch, n_qt, static_cast<__nv_bfloat16*>(out), lse, status);
+  }
   dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
   return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv, s_kept,
-                    gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
+                    gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv, batch, 0,
                     static_cast<__nv_bfloat16*>(out), lse, status);
 }
 
