@@ -59,6 +59,9 @@ def lib():
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, P, P, P, P, P, P]
         L.oracle_gated_attention_bwd.restype = None
+        L.oracle_gated_delta_rule.argtypes = [P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        L.oracle_gated_delta_rule.restype = None
         _lib = L
     return _lib
 
@@ -213,3 +216,21 @@ def gated_attention_bwd(q, k, v, dout, s_kept, gain, tau, cu_kept):
                                      _ptr(t), _ptr(cu), len(cu) - 1, hq, hkv, dh, _ptr(dq),
                                      _ptr(dk), _ptr(dv), _ptr(ds), _ptr(dg), _ptr(dtau))
     return dq, dk, dv, ds, dg, dtau
+
+
+def gated_delta_rule(q, k, v, alpha, beta, cu_seqlens) -> np.ndarray:
+    """Gated delta rule per sequence and head (state reset at each sequence):
+    q, k [T, H, dk], v [T, H, dv], alpha/beta [T, H] -> o [T, H, dv] fp64."""
+    qr, dt = _raw(q)
+    kr, dt2 = _raw(k)
+    vr, dt3 = _raw(v)
+    assert dt == dt2 == dt3
+    T, H, dk = qr.shape
+    dv = vr.shape[2]
+    a = _f32(alpha).reshape(T, H)
+    b = _f32(beta).reshape(T, H)
+    cu = _i32(cu_seqlens)
+    out = np.zeros((T, H, dv), np.float64)
+    lib().oracle_gated_delta_rule(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(a), _ptr(b), _ptr(cu),
+                                  len(cu) - 1, H, dk, dv, _ptr(out))
+    return out

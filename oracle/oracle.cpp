@@ -314,6 +314,50 @@ void oracle_gated_attention_bwd(const void* q, const void* k, const void* v, con
   }
 }
 
+// Gated delta rule over the kept tokens (MarkTechPost page, section "Est-ce que cela
+// fonctionne avec les modèles d'attention hybrides ?" and its comparison table: the
+// hybrid model's Gated DeltaNet layers are pruned too, i.e. above the gate layer
+// they run over the kept tokens only). For each sequence and head, a state
+// S in R^{dk x dv} starts at zero and, for the sequence's tokens t in order,
+//   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+//   o_t = S_t^T q_t
+// q, k [total, H, dk], v [total, H, dv] in `dtype`; alpha, beta [total, H] f32;
+// out [total, H, dv] fp64.
+void oracle_gated_delta_rule(const void* q, const void* k, const void* v, int dtype,
+                             const float* alpha, const float* beta, const int32_t* cu_seqlens,
+                             int batch, int n_heads, int dk, int dv, double* out) {
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int b = 0; b < batch; ++b) {
+    for (int h = 0; h < n_heads; ++h) {
+      std::vector<double> S((size_t)dk * dv, 0.0), kt(dk), qt(dk), vt(dv), ks(dv);
+      for (int64_t t = cu_seqlens[b]; t < cu_seqlens[b + 1]; ++t) {
+        for (int i = 0; i < dk; ++i) {
+          kt[i] = load_elem(k, dtype, (t * n_heads + h) * (int64_t)dk + i);
+          qt[i] = load_elem(q, dtype, (t * n_heads + h) * (int64_t)dk + i);
+        }
+        for (int c = 0; c < dv; ++c) vt[c] = load_elem(v, dtype, (t * n_heads + h) * (int64_t)dv + c);
+        const double a = alpha[t * n_heads + h], be = beta[t * n_heads + h];
+        // ks = k_t^T S_{t-1}
+        for (int c = 0; c < dv; ++c) {
+          double acc = 0.0;
+          for (int i = 0; i < dk; ++i) acc += kt[i] * S[(size_t)i * dv + c];
+          ks[c] = acc;
+        }
+        // S_t = a (S - be k (k^T S)) + be k v^T
+        for (int i = 0; i < dk; ++i)
+          for (int c = 0; c < dv; ++c)
+            S[(size_t)i * dv + c] = a * (S[(size_t)i * dv + c] - be * kt[i] * ks[c]) + be * kt[i] * vt[c];
+        // o_t = S_t^T q_t
+        for (int c = 0; c < dv; ++c) {
+          double acc = 0.0;
+          for (int i = 0; i < dk; ++i) acc += S[(size_t)i * dv + c] * qt[i];
+          out[(t * n_heads + h) * (int64_t)dv + c] = acc;
+        }
+      }
+    }
+  }
+}
+
 // Decode over the compacted cache (MarkTechPost page, section "Comment déployer
 // TokenGate ?": generation runs on the cache the pruned prefill left behind, with
 // max_kept_prefill_tokens bounding it; section "Qu'est-ce que l'attention gérée
