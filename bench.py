@@ -425,6 +425,54 @@ def _time_backward(gp, wl, steps, warmup, rep, flush, stream, tf_peak):
                     "forward's causal flops (S, dP, dV, dK, dQ)"}
 
 
+FP32_FMA_PER_CLK_PER_SM = 128   # B200: 4 sub-partitions x 32 fp32 FMA lanes
+
+
+def _time_deltanet(gp, wl, steps, warmup, rep, flush, stream, sm_mhz_max, n_sm):
+    """A Gated DeltaNet layer's recurrence over the layer's kept rows (row f3): the
+    workload's seeded DeltaNet inputs, one launch per step in a CUDA graph, L2 flushed
+    before each. The recurrence is sequential in the tokens, so its bound is the
+    per-token latency of the fp32 SIMT update, not a roofline of bytes or tensor
+    flops; the fraction is of the fp32 FMA peak (SMs x 128 lanes x 2 flops x clock)."""
+    from learned_token_pruning_gemm_b200 import api, synth
+    q, k, v, a, b = (t.to(gp.q.device) for t in synth.deltanet_inputs(wl))
+    cu = gp.cu_kept
+    out = torch.empty_like(v)
+
+    def step():
+        api.gated_delta_rule(q, k, v, a, b, cu, out=out)
+
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(warmup):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    rep.barrier()
+    for e0, e1 in ev:
+        flush()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    rep.barrier()
+    if api.device_status(reset=True) != 0:
+        raise RuntimeError("device status set by the delta rule")
+    ms = rep.max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev))
+    K, H, d = q.shape
+    flops = 6.0 * K * H * d * v.shape[2]   # k.s, the update, q.s: 3 x (multiply + add) per state entry
+    peak = n_sm * FP32_FMA_PER_CLK_PER_SM * 2 * sm_mhz_max * 1e6 / 1e12
+    return {"us": ms * 1e3, "tokens_per_s": K / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12,
+            "bound": "alu", "peak_tflops_fp32": peak,
+            "frac_alu": flops / (ms / 1e3) / 1e12 / peak, "launches_per_step": 1,
+            "note": "sequential in the tokens: one CTA per (16 value columns, head, sequence)"}
+
+
 def run_ours(args, rep):
     ws, rank = rep.world, rep.rank
     from learned_token_pruning_gemm_b200 import pipeline, synth
@@ -462,6 +510,13 @@ def run_ours(args, rep):
     decode = None
     if wl.dtype == "bf16" and wl.dh == 128 and not args.no_decode:
         decode = _time_decode(gp, wl, args.steps, args.warmup, rep, flush, stream, hbm_peak)
+
+    deltanet = None
+    if wl.dtype == "bf16" and wl.dh == 128 and not args.no_deltanet:
+        props = torch.cuda.get_device_properties(dev_index)
+        sm_max = clocks.max_mhz if clocks.error is None else peaks.get("sm_max_mhz", 1965.0)
+        deltanet = _time_deltanet(gp, wl, args.steps, args.warmup, rep, flush, stream, sm_max,
+                                  props.multi_processor_count)
 
     backward = None
     if wl.dtype == "bf16" and wl.dh == 128 and not args.no_backward:
@@ -559,6 +614,7 @@ def run_ours(args, rep):
             "with_projection": with_proj,
             "decode": decode,
             "backward": backward,
+            "deltanet": deltanet,
             "workloads": others,
             "cpu_baseline": cpu,
         }
@@ -594,6 +650,7 @@ def main():
     ap.add_argument("--no-extra-workloads", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-deltanet", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -278,6 +278,29 @@ tg_status tg_gated_decode_noalloc(const void* q, const void* k_cache, const void
                                   tg_stream_t stream);
 
 /*
+ * Gated delta rule over the kept tokens: the recurrence of the hybrid model's Gated
+ * DeltaNet layers, which TokenGate also prunes (MarkTechPost page on TokenGate,
+ * section "Est-ce que cela fonctionne avec les modèles d'attention hybrides ?" and
+ * the comparison table). For each sequence b (rows [cu_seqlens[b], cu_seqlens[b+1])
+ * of the packed kept rows) and head h, a state S (head_dim_k x head_dim_v) starts at
+ * zero and, for the sequence's rows t in order,
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     out_t = S_t^T q_t
+ *   q, k  [total, n_heads, head_dim_k] bf16 (the caller normalises k; with |k| = 1
+ *         and alpha, beta in [0, 1] the state stays bounded)
+ *   v     [total, n_heads, head_dim_v] bf16
+ *   alpha, beta [total, n_heads] f32 (decay and write strength per token and head)
+ *   out   [total, n_heads, head_dim_v] bf16 output
+ * TG_BF16 only; head_dim_k == 128, head_dim_v a multiple of 16 up to 1024; q, k, v,
+ * out 16-byte aligned. A sequence outside [0, total] is skipped and
+ * TG_ERR_DEVICE_CHECK recorded.
+ */
+tg_status tg_gated_delta_rule(const void* q, const void* k, const void* v, tg_dtype dtype,
+                              const float* alpha, const float* beta, const int32_t* cu_seqlens,
+                              int batch, int64_t total, int n_heads, int head_dim_k,
+                              int head_dim_v, void* out, tg_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the first error any kernel recorded on the
  * current device since the last reset (TG_OK if none). reset != 0 clears it.
  */

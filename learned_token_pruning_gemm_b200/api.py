@@ -216,6 +216,32 @@ def gated_attention_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: 
     return dq, dk, dv, ds, dg, dt
 
 
+def gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                     beta: torch.Tensor, cu_seqlens: torch.Tensor,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Gated delta rule per sequence and head over packed rows: q, k [T,H,dk], v [T,H,dv]
+    bf16, alpha/beta [T,H] f32 -> out [T,H,dv] bf16 (state reset per sequence)."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    _shape(k, q.shape, "k", q.dtype)
+    _shape(v, (T, H, dv), "v", q.dtype)
+    _shape(alpha, (T, H), "alpha", torch.float32)
+    _shape(beta, (T, H), "beta", torch.float32)
+    if cu_seqlens.numel() < 1:
+        raise TokenGateError("cu_seqlens must have batch+1 >= 1 elements")
+    if q.dtype not in _DT:
+        raise TokenGateError(f"gated_delta_rule: unsupported dtype {q.dtype}")
+    if out is None:
+        out = torch.empty_like(v)
+    _shape(out, v.shape, "out", v.dtype)
+    st = _lib.load().tg_gated_delta_rule(
+        _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _DT[q.dtype], _cuda(alpha, "alpha"),
+        _cuda(beta, "beta"), _cuda(cu_seqlens, "cu_seqlens", torch.int32),
+        cu_seqlens.numel() - 1, T, H, dk, dv, _cuda(out, "out"), _stream(stream))
+    check(st, "tg_gated_delta_rule")
+    return out
+
+
 def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: torch.Tensor,
              rope_base: float = 1e6, out=None, stream=None):
     """The kept rows' projections: (q [K,Hq,dh], k [K,Hkv,dh], v [K,Hkv,dh]) bf16 from

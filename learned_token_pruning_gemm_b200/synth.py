@@ -26,6 +26,7 @@ import torch
 _TID = {
     "x": 1, "w1": 2, "b1": 3, "w2": 4, "b2": 5, "gain": 6, "tau": 7,
     "q": 8, "k": 9, "v": 10, "plant": 11, "dup": 12, "tscore": 13, "lens": 14,
+    "dn_q": 15, "dn_k": 16, "dn_v": 17, "dn_a": 18, "dn_b": 19,
 }
 
 
@@ -255,3 +256,20 @@ def qkv_weights(wl: Workload, seed: int = 11) -> torch.Tensor:
     g = np.random.Generator(np.random.Philox(key=[wl.seed, 100 + seed]))
     n = (wl.hq + 2 * wl.hkv) * wl.dh
     return _as_dtype(g.standard_normal((n, wl.d)) / math.sqrt(wl.d), wl.dtype)
+
+
+def deltanet_inputs(wl: Workload):
+    """Inputs of a Gated DeltaNet layer over the workload's kept rows (one row per
+    kept token, the workload's query-head count and head size): q, k drawn N(0,1)
+    and scaled to unit length per head (the layer normalises them before the rule),
+    v ~ N(0,1), decay alpha ~ U(0.9, 1), write strength beta ~ U(0, 1)."""
+    K, H, d = wl.total_kept, wl.hq, wl.dh
+    def unit(name):
+        a = _rng(wl.seed, name).standard_normal((K, H, d))
+        return a / np.linalg.norm(a, axis=-1, keepdims=True)
+    q, k = unit("dn_q"), unit("dn_k")
+    v = _rng(wl.seed, "dn_v").standard_normal((K, H, d))
+    alpha = _rng(wl.seed, "dn_a").uniform(0.9, 1.0, (K, H)).astype(np.float32)
+    beta = _rng(wl.seed, "dn_b").uniform(0.0, 1.0, (K, H)).astype(np.float32)
+    return (_as_dtype(q, "bf16"), _as_dtype(k, "bf16"), _as_dtype(v, "bf16"),
+            torch.from_numpy(alpha), torch.from_numpy(beta))

@@ -256,3 +256,21 @@ def test_backward_validation_without_gpu(lib):
     assert bwd(q=odd) == MIS
     assert bwd(q=None) == INVALID
     assert bwd(total=0) == 0
+
+
+def test_delta_rule_validation_without_gpu(lib):
+    INVALID, UNSUP, MIS = 1, 2, 3
+    P = ctypes.c_void_p
+    fake, odd = P(0x10000), P(0x10004)
+
+    def dn(dtype=1, dk=128, dv=128, q=fake, a=fake, total=10, batch=1):
+        return lib.tg_gated_delta_rule(q, fake, fake, dtype, a, fake, fake, batch, total, 4, dk,
+                                       dv, fake, None)
+    assert dn(dtype=0) == UNSUP
+    assert dn(dk=64) == UNSUP
+    assert dn(dv=100) == UNSUP
+    assert dn(q=odd) == MIS
+    assert dn(a=P(0x10002)) == MIS
+    assert dn(q=None) == INVALID
+    assert dn(total=0) == 0 and dn(batch=0) == 0
+    assert dn(total=-1) == INVALID

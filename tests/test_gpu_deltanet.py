@@ -1,0 +1,67 @@
+"""GPU parity of the gated delta rule over the kept tokens (tg_gated_delta_rule)
+against the fp64 oracle, through the C ABI (MarkTechPost page on TokenGate, section
+"Est-ce que cela fonctionne avec les modèles d'attention hybrides ?": the hybrid
+model's Gated DeltaNet layers are pruned too).
+
+Tolerance: the outputs are bf16 like the attention's, so the bf16 bar of
+tests/helpers.py (1e-2 max-abs, 5e-3 relative L2); the fp32 state is updated once
+per token, and with unit keys and alpha <= 1 each update is a contraction, so the
+rounding does not grow with the sequence length."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_attn_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from learned_token_pruning_gemm_b200 import api, build
+    build.build()
+    api.device_status(reset=True)
+    return api
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors(api):
+    yield
+    assert api.device_status(reset=True) == 0, "a kernel recorded a device-side error"
+
+
+def _case(seed, lens, H, dv=128):
+    g = torch.Generator().manual_seed(seed)
+    T = sum(lens)
+    q = torch.nn.functional.normalize(torch.randn(T, H, 128, generator=g), dim=-1).to(torch.bfloat16)
+    k = torch.nn.functional.normalize(torch.randn(T, H, 128, generator=g), dim=-1).to(torch.bfloat16)
+    v = torch.randn(T, H, dv, generator=g).to(torch.bfloat16)
+    a = 0.9 + 0.1 * torch.rand(T, H, generator=g)
+    b = torch.rand(T, H, generator=g)
+    cu = np.r_[0, np.cumsum(lens)].astype(np.int32)
+    return q, k, v, a, b, cu
+
+
+@pytest.mark.parametrize("lens,H,dv", [([100], 2, 128), ([33, 1, 70, 0, 200], 3, 128),
+                                       ([64], 1, 48), ([1868], 16, 128)])
+def test_delta_rule_vs_oracle(api, orc, lens, H, dv):
+    q, k, v, a, b, cu = _case(sum(lens) + H, lens, H, dv)
+    out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                               torch.tensor(cu, device="cuda"))
+    ref = orc.gated_delta_rule(q, k, v, a, b, cu)
+    max_abs, rl2 = assert_attn_close(out, ref, torch.bfloat16, what=f"delta rule lens={lens}")
+    print(f"delta rule lens={lens} H={H}: max|O| {np.abs(ref).max():.3f} max_abs {max_abs:.2e} "
+          f"rel_l2 {rl2:.2e}")
+
+
+def test_delta_rule_on_the_16k_layers_kept_rows(api, orc):
+    # the workload's own DeltaNet inputs over its 1868 kept rows, sampled heads
+    from learned_token_pruning_gemm_b200 import synth
+    wl = synth.qwen16k()
+    q, k, v, a, b = synth.deltanet_inputs(wl)
+    cu = np.array([0, wl.total_kept], np.int32)
+    out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                               torch.tensor(cu, device="cuda"))
+    heads = [0, 7, 15]
+    ref = orc.gated_delta_rule(q[:, heads], k[:, heads], v[:, heads], a[:, heads], b[:, heads], cu)
+    assert_attn_close(out[:, heads].contiguous(), ref, torch.bfloat16, what="16k kept rows")
