@@ -8,10 +8,12 @@
 //
 // Column c of S evolves on its own: s' = alpha s + beta k (v_c - alpha k.s). So a
 // CTA takes 16 value columns of one (head, sequence) and keeps them in registers:
-// four adjacent lanes share a column, each holding 32 of its 128 key entries, so
-// the two dot products per token (k.s before the update, q.s after it) are a
-// partial sum plus two shuffles. The recurrence is sequential in t; what the
-// kernel does in parallel is the columns (dv / 16 CTAs per head) and the heads.
+// eight adjacent lanes share a column, each holding 16 of its 128 key entries, so a
+// dot product is a partial sum plus three shuffles. After token t's update the
+// same state gives both o_t = q_t.s and the next token's k_{t+1}.s, so the two are
+// reduced together: one round of shuffles per token on the sequential chain. The
+// recurrence is sequential in t; what the kernel does in parallel is the columns
+// (dv / 16 CTAs per head) and the heads.
 // Each CTA stages 32 tokens at a time (k, q, its v columns, alpha, beta) in
 // shared memory with cp.async, double-buffered so the next chunk loads while this
 // one runs, and writes its outputs 32 tokens at a time.
@@ -21,7 +23,7 @@ namespace {
 
 constexpr int kDk = 128;
 constexpr int kCols = 16;           // value columns per CTA
-constexpr int kParts = 4;           // lanes per column
+constexpr int kParts = 8;           // lanes per column
 constexpr int kPer = kDk / kParts;  // key entries per lane
 constexpr int kThreads = kCols * kParts;
 constexpr int kChunk = 32;          // tokens staged per buffer
@@ -95,8 +97,30 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int i = 0; i < kPer; ++i) s[i] = 0.f;
 
+  // this lane's 16 entries of a staged bf16 row, widened to fp32
+  auto row16 = [&](const __nv_bfloat16* src, float* f) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + part * kPer);
+#pragma unroll
+    for (int u = 0; u < kPer / 8; ++u) {
+      const uint4 w4 = p[u];
+      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        f[8 * u + 2 * e] = __uint_as_float(w[e] << 16);
+        f[8 * u + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+  };
+  auto col_sum = [&](float x) {   // over the column's eight lanes
+    x += __shfl_xor_sync(0xFFFFFFFFu, x, 1);
+    x += __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+    x += __shfl_xor_sync(0xFFFFFFFFu, x, 4);
+    return x;
+  };
+
   if (n > 0) stage(0, 0);
   int buf = 0;
+  float dot = 0.f;   // k_t . s_{t-1} for the next token (zero state: zero)
   for (int64_t tb = 0; tb < n; tb += kChunk, buf ^= 1) {
     const int rows = static_cast<int>(n - tb < kChunk ? n - tb : kChunk);
     if (tb + kChunk < n) {
@@ -106,42 +130,39 @@ __global__ void __launch_bounds__(kThreads)
       cp_async_wait_all();
     }
     __syncthreads();
-    for (int r = 0; r < rows; ++r) {
-      const uint4* kr = reinterpret_cast<const uint4*>(&S.k[buf][r][part * kPer]);
-      const uint4* qr = reinterpret_cast<const uint4*>(&S.q[buf][r][part * kPer]);
-      float kf[kPer], qf[kPer];
-#pragma unroll
-      for (int u = 0; u < kPer / 8; ++u) {
-        const uint4 kk = kr[u], qq = qr[u];
-        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w}, qw[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kf[8 * u + 2 * e] = __uint_as_float(kw[e] << 16);
-          kf[8 * u + 2 * e + 1] = __uint_as_float(kw[e] & 0xFFFF0000u);
-          qf[8 * u + 2 * e] = __uint_as_float(qw[e] << 16);
-          qf[8 * u + 2 * e + 1] = __uint_as_float(qw[e] & 0xFFFF0000u);
-        }
-      }
-      // k.s over this column (four partial sums, then the column's four lanes)
+    if (tb > 0) {   // the first token of a chunk: its k.s was not formed with the last output
+      float kf[kPer];
+      row16(S.k[buf][0], kf);
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < kPer; ++i) d4[i & 3] = fmaf(kf[i], s[i], d4[i & 3]);
-      float dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 2);
+      dot = col_sum((d4[0] + d4[1]) + (d4[2] + d4[3]));
+    }
+    for (int r = 0; r < rows; ++r) {
+      float kf[kPer], qf[kPer], kn[kPer];
+      row16(S.k[buf][r], kf);
+      row16(S.q[buf][r], qf);
+      const bool has_next = r + 1 < rows;
+      if (has_next) row16(S.k[buf][r + 1], kn);
       const float a = S.a[buf][r], be = S.b[buf][r];
       const float vc = __bfloat162float(S.v[buf][r][col]);
       const float w = be * (vc - a * dot);
-      // s <- a s + w k ; then o = q.s
-      float o4[4] = {0.f, 0.f, 0.f, 0.f};
+      // s <- a s + w k; then o_t = q_t . s and the next token's k . s, reduced together
+      float o4[4] = {0.f, 0.f, 0.f, 0.f}, n4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         s[i] = fmaf(a, s[i], w * kf[i]);
         o4[i & 3] = fmaf(qf[i], s[i], o4[i & 3]);
+        if (has_next) n4[i & 3] = fmaf(kn[i], s[i], n4[i & 3]);
       }
       float o = (o4[0] + o4[1]) + (o4[2] + o4[3]);
-      o += __shfl_xor_sync(0xFFFFFFFFu, o, 1);
-      o += __shfl_xor_sync(0xFFFFFFFFu, o, 2);
+      float dn = (n4[0] + n4[1]) + (n4[2] + n4[3]);
+#pragma unroll
+      for (int off = 1; off < kParts; off <<= 1) {
+        o += __shfl_xor_sync(0xFFFFFFFFu, o, off);
+        dn += __shfl_xor_sync(0xFFFFFFFFu, dn, off);
+      }
+      dot = dn;
       if (part == 0) S.o[r][col] = __float2bfloat16_rn(o);
     }
     __syncthreads();   // the chunk's outputs are in shared memory; its buffer may be reused
