@@ -15,11 +15,13 @@
 // (64-key chunk, KV head, sequence) loads the chunk's K and V rows of that KV
 // head with two TMA boxes each (64 dims x 64 rows, 128-byte swizzle, 32 KB in
 // all) and serves every query head of the GQA group from them: logits in fp32
-// (log2 domain), the chunk's max m and sum l of 2^(z - m), and the unnormalised
-// sum of 2^(z - m) v, written as one partial per (sequence, query head, chunk)
-// to a caller-provided workspace. A second kernel merges a row's partials in
-// chunk order (a fixed order: the result does not depend on timing) and writes
-// O = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c in bf16.
+// (log2 domain), the running max m and sum l of 2^(z - m), and the unnormalised
+// sum of 2^(z - m) v. With many chunks per KV head (large batches) one CTA walks
+// several consecutive chunks through a two-stage TMA ring and folds them with an
+// online max, so the grid stays near two CTAs per SM. Each CTA writes one partial
+// per (sequence, query head, span) to a caller-provided workspace. A second kernel
+// merges a row's partials in span order (a fixed order: the result does not depend
+// on timing) and writes O = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c in bf16.
 #include <mutex>
 
 #include "common.cuh"
@@ -34,13 +36,14 @@ constexpr int kPartial = kDh + 2;     // o[dh], m, l (fp32)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecSmem {
-  uint8_t k[2][kChunk * 64 * 2];      // two 64-dim halves of the chunk's K rows (8 KB each)
-  uint8_t v[2][kChunk * 64 * 2];
+  uint8_t k[2][2][kChunk * 64 * 2];   // [stage][dh half]: the chunk's K rows (8 KB per half)
+  uint8_t v[2][2][kChunk * 64 * 2];
   float q[kMaxGroup][kDh];
   float p[kMaxGroup][kChunk];         // logits, then 2^(z - m)
-  float m[kMaxGroup];
-  float l[kMaxGroup];
-  uint64_t full;
+  float m[kMaxGroup];                 // running max over this CTA's chunks
+  float l[kMaxGroup];                 // running sum of 2^(z - m)
+  float alpha[kMaxGroup];             // 2^(m_old - m_new) of the current chunk
+  uint64_t full[2];
   int abort_flag;
 };
 
@@ -53,12 +56,14 @@ __device__ __forceinline__ uint32_t sw_off(int j, int e) {
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
+// One CTA per (span of `cpc` 64-key chunks, KV head, sequence): the chunks stream
+// through a two-stage TMA ring and fold into one partial with an online max.
 __global__ void __launch_bounds__(kThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __nv_bfloat16* __restrict__ q, const float* __restrict__ s_cache,
                         const int32_t* __restrict__ cache_len, int cap, int max_len, int n_hq,
                         int n_hkv, const float* __restrict__ gain, const float* __restrict__ tau,
-                        float* __restrict__ partial, int n_split, int* status) {
+                        float* __restrict__ partial, int n_split, int cpc, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
@@ -66,11 +71,16 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = n_hq / n_hkv;
   if (tid == 0) {
-    tg::mbar_init(&S.full, 1);
+    tg::mbar_init(&S.full[0], 1);
+    tg::mbar_init(&S.full[1], 1);
     S.abort_flag = 0;
     tg::fence_barrier_init();
     tg::tma_prefetch_desc(&tm_k);
     tg::tma_prefetch_desc(&tm_v);
+  }
+  if (tid < kMaxGroup) {
+    S.m[tid] = -INFINITY;
+    S.l[tid] = 0.f;
   }
   __syncthreads();
   tg::pdl_launch_dependents();
@@ -80,18 +90,19 @@ __global__ void __launch_bounds__(kThreads)
   if (len < 0 || len > cap || len > max_len) {   // the combine kernel records it
     return;
   }
-  const int j0 = split * kChunk;
-  if (j0 >= len) return;                          // this chunk is past the cache's end
-  const int nv = min(kChunk, len - j0);           // valid rows of the chunk
+  const int c_begin = split * cpc;
+  const int c_end = min((len + kChunk - 1) / kChunk, c_begin + cpc);
+  if (c_begin >= c_end) return;   // this span is past the cache's end
 
-  if (tid == 0) {
-    const int row = b * cap + j0;                 // token coordinate in the (dh, heads, rows) view
-    tg::mbar_arrive_expect_tx(&S.full, 4 * kChunk * 64 * 2);
-    tg::tma_load_3d(S.k[0], &tm_k, &S.full, 0, kvh, row);
-    tg::tma_load_3d(S.k[1], &tm_k, &S.full, 64, kvh, row);
-    tg::tma_load_3d(S.v[0], &tm_v, &S.full, 0, kvh, row);
-    tg::tma_load_3d(S.v[1], &tm_v, &S.full, 64, kvh, row);
-  }
+  auto load = [&](int c, int stage) {
+    const int row = b * cap + c * kChunk;   // token coordinate in the (dh, heads, rows) view
+    tg::mbar_arrive_expect_tx(&S.full[stage], 4 * kChunk * 64 * 2);
+    tg::tma_load_3d(S.k[stage][0], &tm_k, &S.full[stage], 0, kvh, row);
+    tg::tma_load_3d(S.k[stage][1], &tm_k, &S.full[stage], 64, kvh, row);
+    tg::tma_load_3d(S.v[stage][0], &tm_v, &S.full[stage], 0, kvh, row);
+    tg::tma_load_3d(S.v[stage][1], &tm_v, &S.full[stage], 64, kvh, row);
+  };
+  if (tid == 0) load(c_begin, 0);
   // the group's queries, scaled so that the logits come out in the log2 domain
   for (int i = tid; i < G * kDh; i += kThreads) {
     const int h = i / kDh, d = i % kDh;
@@ -99,121 +110,146 @@ __global__ void __launch_bounds__(kThreads)
     const float c = kLog2e / (sqrtf(static_cast<float>(kDh)) * tau[hq]);
     S.q[h][d] = __bfloat162float(q[(static_cast<int64_t>(b) * n_hq + hq) * kDh + d]) * c;
   }
-  __syncthreads();
-  const bool ok = tg::mbar_wait(&S.full, 0, status, &S.abort_flag);
-  if (!ok) return;   // uniform: every thread waited on the same phase (the copies have landed or timed out)
-
-  // ---- logits: thread t takes key j = t % 64 and heads h = t / 64, t / 64 + 2, ... ----
-  {
-    const int j = tid & (kChunk - 1);
-    const uint8_t* kb = S.k[0];
-    float acc[kMaxGroup / 2];
+  // this thread's output dims 2(t % 64), +1 of heads t/64, t/64 + 2, ...
+  const int e = 2 * (tid & 63);
+  float o0[kMaxGroup / 2], o1[kMaxGroup / 2];
 #pragma unroll
-    for (int u = 0; u < kMaxGroup / 2; ++u) acc[u] = 0.f;
+  for (int u = 0; u < kMaxGroup / 2; ++u) o0[u] = o1[u] = 0.f;
+  __syncthreads();
+
+  for (int c = c_begin; c < c_end; ++c) {
+    const int i = c - c_begin, st = i & 1;
+    // the other stage was released by the barrier that ended the previous chunk
+    if (tid == 0 && c + 1 < c_end) load(c + 1, st ^ 1);
+    const bool ok = tg::mbar_wait(&S.full[st], (i >> 1) & 1, status, &S.abort_flag);
+    if (!__syncthreads_and(ok)) {   // a copy that never landed: leave after the others
+      if (tid == 0 && c + 1 < c_end)
+        tg::mbar_wait(&S.full[st ^ 1], ((i + 1) >> 1) & 1, status, nullptr);
+      return;
+    }
+    const int j0 = c * kChunk;
+    const int nv = min(kChunk, len - j0);   // valid rows of the chunk
+
+    // ---- logits: thread t takes key j = t % 64 and heads h = t / 64, t / 64 + 2, ... ----
+    {
+      const int j = tid & (kChunk - 1);
+      const uint8_t* kb = S.k[st][0];
+      float acc[kMaxGroup / 2];
+#pragma unroll
+      for (int u = 0; u < kMaxGroup / 2; ++u) acc[u] = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < kDh / 8; ++c) {
-      const uint4 kk = *reinterpret_cast<const uint4*>(kb + sw_off(j, 8 * c));
-      const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
-                           bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
+      for (int cc = 0; cc < kDh / 8; ++cc) {
+        const uint4 kk = *reinterpret_cast<const uint4*>(kb + sw_off(j, 8 * cc));
+        const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
+                             bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
+#pragma unroll
+        for (int u = 0; u < kMaxGroup / 2; ++u) {
+          const int h = (tid >> 6) + 2 * u;
+          if (h < G) {
+            const float4 q0 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc]);
+            const float4 q1 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc + 4]);
+            float a = acc[u];
+            a = fmaf(q0.x, kf[0], a); a = fmaf(q0.y, kf[1], a);
+            a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+            a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a);
+            a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
+            acc[u] = a;
+          }
+        }
+      }
+      const float sv = j < nv ? s_cache[static_cast<int64_t>(b) * cap + j0 + j] : 0.f;
 #pragma unroll
       for (int u = 0; u < kMaxGroup / 2; ++u) {
         const int h = (tid >> 6) + 2 * u;
         if (h < G) {
-          const float4 q0 = *reinterpret_cast<const float4*>(&S.q[h][8 * c]);
-          const float4 q1 = *reinterpret_cast<const float4*>(&S.q[h][8 * c + 4]);
-          float a = acc[u];
-          a = fmaf(q0.x, kf[0], a); a = fmaf(q0.y, kf[1], a);
-          a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
-          a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a);
-          a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
-          acc[u] = a;
+          const float bias = gain[kvh * G + h] * kLog2e * sv;
+          S.p[h][j] = j < nv ? acc[u] + bias : -INFINITY;
         }
       }
     }
-    const float s = j < nv ? s_cache[static_cast<int64_t>(b) * cap + j0 + j] : 0.f;
+    __syncthreads();
+
+    // ---- per head: the running max moves to cover this chunk; weights and their sum ----
+    for (int h = warp; h < G; h += kThreads / 32) {
+      const float z0 = S.p[h][lane], z1 = S.p[h][lane + 32];
+      float mc = fmaxf(z0, z1);
 #pragma unroll
-    for (int u = 0; u < kMaxGroup / 2; ++u) {
-      const int h = (tid >> 6) + 2 * u;
-      if (h < G) {
-        const float bias = gain[kvh * G + h] * kLog2e * s;
-        S.p[h][j] = j < nv ? acc[u] + bias : -INFINITY;
+      for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xFFFFFFFFu, mc, off));
+      const float m_old = S.m[h];
+      const float m_new = fmaxf(m_old, mc);   // finite: row 0 of every chunk is valid
+      const float p0 = tg::exp2_approx(z0 - m_new), p1 = tg::exp2_approx(z1 - m_new);
+      S.p[h][lane] = p0;
+      S.p[h][lane + 32] = p1;
+      float lc = p0 + p1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) lc += __shfl_xor_sync(0xFFFFFFFFu, lc, off);
+      __syncwarp();
+      if (lane == 0) {
+        const float al = tg::exp2_approx(m_old - m_new);   // 0 for the first chunk
+        S.alpha[h] = al;
+        S.m[h] = m_new;
+        S.l[h] = S.l[h] * al + lc;
       }
     }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // ---- per head: chunk max, weights 2^(z - m), their sum (warp w: heads w, w + 4) ----
-  for (int h = warp; h < G; h += kThreads / 32) {
-    const float z0 = S.p[h][lane], z1 = S.p[h][lane + 32];
-    float m = fmaxf(z0, z1);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const float p0 = tg::exp2_approx(z0 - m), p1 = tg::exp2_approx(z1 - m);   // row 0 is valid: m finite
-    S.p[h][lane] = p0;
-    S.p[h][lane + 32] = p1;
-    float l = p0 + p1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, o);
-    if (lane == 0) {
-      S.m[h] = m;
-      S.l[h] = l;
-    }
-  }
-  __syncthreads();
-
-  // ---- unnormalised sum of p v: thread t takes dims 2(t % 64), +1 of heads t/64, +2, ... ----
-  {
-    const int e = 2 * (tid & 63);
-    float o0[kMaxGroup / 2], o1[kMaxGroup / 2];
-#pragma unroll
-    for (int u = 0; u < kMaxGroup / 2; ++u) o0[u] = o1[u] = 0.f;
-    const uint8_t* vb = S.v[0];
-    for (int j = 0; j < nv; ++j) {
-      const uint32_t vv = *reinterpret_cast<const uint32_t*>(vb + sw_off(j, e));
-      const float v0 = bf16_lo(vv), v1 = bf16_hi(vv);
+    // ---- o = alpha o + sum_j p_j v_j ----
+    {
+      const uint8_t* vb = S.v[st][0];
 #pragma unroll
       for (int u = 0; u < kMaxGroup / 2; ++u) {
         const int h = (tid >> 6) + 2 * u;
         if (h < G) {
-          const float pj = S.p[h][j];
-          o0[u] = fmaf(pj, v0, o0[u]);
-          o1[u] = fmaf(pj, v1, o1[u]);
+          const float al = S.alpha[h];
+          o0[u] *= al;
+          o1[u] *= al;
+        }
+      }
+#pragma unroll 4
+      for (int j = 0; j < nv; ++j) {
+        const uint32_t vv = *reinterpret_cast<const uint32_t*>(vb + sw_off(j, e));
+        const float v0 = bf16_lo(vv), v1 = bf16_hi(vv);
+#pragma unroll
+        for (int u = 0; u < kMaxGroup / 2; ++u) {
+          const int h = (tid >> 6) + 2 * u;
+          if (h < G) {
+            const float pj = S.p[h][j];
+            o0[u] = fmaf(pj, v0, o0[u]);
+            o1[u] = fmaf(pj, v1, o1[u]);
+          }
         }
       }
     }
+    __syncthreads();   // stage st, S.p and S.alpha are free for the next chunk
+  }
 #pragma unroll
-    for (int u = 0; u < kMaxGroup / 2; ++u) {
-      const int h = (tid >> 6) + 2 * u;
-      if (h < G) {
-        const int hq = kvh * G + h;
-        float* pr = partial + ((static_cast<int64_t>(b) * n_hq + hq) * n_split + split) * kPartial;
-        *reinterpret_cast<float2*>(pr + e) = make_float2(o0[u], o1[u]);
-        if ((tid & 63) == 0) {
-          pr[kDh] = S.m[h];
-          pr[kDh + 1] = S.l[h];
-        }
+  for (int u = 0; u < kMaxGroup / 2; ++u) {
+    const int h = (tid >> 6) + 2 * u;
+    if (h < G) {
+      const int hq = kvh * G + h;
+      float* pr = partial + ((static_cast<int64_t>(b) * n_hq + hq) * n_split + split) * kPartial;
+      *reinterpret_cast<float2*>(pr + e) = make_float2(o0[u], o1[u]);
+      if ((tid & 63) == 0) {
+        pr[kDh] = S.m[h];
+        pr[kDh + 1] = S.l[h];
       }
     }
   }
 }
 
-// Merge one row's chunk partials in chunk order; thread d writes dimension d. The
-// chunks' maxima and sums are read by all threads at once into shared memory
-// (weights 2^(m_c - M) there), then every thread sums its dimension over the
-// chunks with independent loads (eight in flight), so no step waits on a chain
-// of global loads.
-constexpr int kCombineMaxChunks = 4096;   // shared-memory weights; longer caches loop in blocks
+// Merge one row's span partials in span order; thread d writes dimension d. One
+// round of global loads: the spans' maxima and sums go to shared memory while every
+// thread's own output loads (up to 32 spans at a time) are already in flight.
+constexpr int kCombineBlock = 32;
 
 __global__ void __launch_bounds__(kThreads)
     decode_combine_kernel(const float* __restrict__ partial, const int32_t* __restrict__ cache_len,
-                          int cap, int max_len, int n_hq, int n_split,
+                          int cap, int max_len, int n_hq, int n_split, int cpc,
                           __nv_bfloat16* __restrict__ out, int* status) {
-  __shared__ float w[kCombineMaxChunks];
-  __shared__ float red[kThreads / 32 + 1];   // block partials; red[0] keeps the max across blocks
+  __shared__ float sm[kThreads], sl[kThreads];
   tg::pdl_launch_dependents();
   tg::pdl_wait();
   const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const int lane = d & 31, warp = d >> 5;
   const int len = cache_len[b];
   __nv_bfloat16* o = out + (static_cast<int64_t>(b) * n_hq + hq) * kDh;
   if (len < 0 || len > cap || len > max_len) {
@@ -224,55 +260,40 @@ __global__ void __launch_bounds__(kThreads)
     o[d] = __float2bfloat16_rn(0.f);
     return;
   }
-  const int nc = (len + kChunk - 1) / kChunk;
+  const int nsp = ((len + kChunk - 1) / kChunk + cpc - 1) / cpc;   // spans holding a partial
   const float* pr = partial + (static_cast<int64_t>(b) * n_hq + hq) * n_split * kPartial;
-  auto block_reduce = [&](float v, bool is_max) {
-    for (int off = 16; off > 0; off >>= 1) {
-      const float x = __shfl_xor_sync(0xFFFFFFFFu, v, off);
-      v = is_max ? fmaxf(v, x) : v + x;
-    }
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    v = red[0];
-    for (int i = 1; i < kThreads / 32; ++i) v = is_max ? fmaxf(v, red[i]) : v + red[i];
-    return v;
-  };
-  float acc = 0.f, L = 0.f;
-  for (int c0 = 0; c0 < nc; c0 += kCombineMaxChunks) {
-    const int cn = min(kCombineMaxChunks, nc - c0);
-    // the overall max first (over every chunk, so the weights of all blocks agree)
-    float mloc = -INFINITY;
-    if (c0 == 0)
-      for (int c = d; c < nc; c += kThreads) mloc = fmaxf(mloc, pr[c * kPartial + kDh]);
-    const float M = c0 == 0 ? block_reduce(mloc, true) : red[0];
-    if (c0 == 0) {
-      __syncthreads();
-      if (d == 0) red[0] = M;   // kept for the later blocks
-    }
-    float lloc = 0.f;
-    for (int c = d; c < cn; c += kThreads) {
-      const float* pc = pr + (c0 + c) * kPartial;
-      const float wc = tg::exp2_approx(pc[kDh] - M);
-      w[c] = wc;
-      lloc = fmaf(wc, pc[kDh + 1], lloc);
-    }
-    __syncthreads();   // weights in shared memory
-    // block sums of l in a fixed order: warp shuffles, then warps in index order
-    for (int off = 16; off > 0; off >>= 1) lloc += __shfl_xor_sync(0xFFFFFFFFu, lloc, off);
-    if (lane == 0) red[1 + warp] = lloc;   // red[0] holds M
-    __syncthreads();
-    for (int i = 0; i < kThreads / 32; ++i) L += red[1 + i];
-    int c = 0;
-    for (; c + 8 <= cn; c += 8) {
-      float v[8];
+  float acc = 0.f, L = 0.f, M = -INFINITY;
+  for (int s0 = 0; s0 < nsp; s0 += kThreads) {   // blocks of up to 128 spans (one block below 8k keys)
+    const int ns = min(kThreads, nsp - s0);
+    float v[kCombineBlock];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = pr[(c0 + c + u) * kPartial + d];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc = fmaf(w[c + u], v[u], acc);
+    for (int u = 0; u < kCombineBlock; ++u)
+      v[u] = u < ns ? pr[(s0 + u) * kPartial + d] : 0.f;
+    if (d < ns) {
+      sm[d] = pr[(s0 + d) * kPartial + kDh];
+      sl[d] = pr[(s0 + d) * kPartial + kDh + 1];
     }
-    for (; c < cn; ++c) acc = fmaf(w[c], pr[(c0 + c) * kPartial + d], acc);
-    __syncthreads();   // w and red are rewritten by the next block
+    __syncthreads();
+    float mb = M;
+    for (int u = 0; u < ns; ++u) mb = fmaxf(mb, sm[u]);
+    const float scale = tg::exp2_approx(M - mb);   // the earlier blocks, onto the new max
+    acc *= scale;
+    L *= scale;
+    M = mb;
+#pragma unroll
+    for (int u = 0; u < kCombineBlock; ++u) {
+      if (u < ns) {
+        const float w = tg::exp2_approx(sm[u] - M);
+        L = fmaf(w, sl[u], L);
+        acc = fmaf(w, v[u], acc);
+      }
+    }
+    for (int u = kCombineBlock; u < ns; ++u) {   // spans past the first 32 of a block
+      const float w = tg::exp2_approx(sm[u] - M);
+      L = fmaf(w, sl[u], L);
+      acc = fmaf(w, pr[(s0 + u) * kPartial + d], acc);
+    }
+    __syncthreads();   // sm, sl are rewritten by the next block
   }
   o[d] = __float2bfloat16_rn(acc / L);
 }
@@ -303,6 +324,13 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 inline int n_splits(int max_len) { return (max_len + kChunk - 1) / kChunk; }
+
+// chunks per split CTA: one while the grid stays below two CTAs per SM, more beyond
+inline int chunks_per_cta(int batch, int n_hkv, int max_len, int sms) {
+  const int64_t ctas = static_cast<int64_t>(batch) * n_hkv * n_splits(max_len);
+  const int64_t target = 2 * static_cast<int64_t>(sms);
+  return ctas <= target ? 1 : static_cast<int>((ctas + target - 1) / target);
+}
 
 }  // namespace
 
@@ -371,16 +399,22 @@ extern "C" tg_status tg_gated_decode(const void* q, const void* k_cache, const v
   const size_t smem = sizeof(DecSmem) + 1024;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(decode_split_kernel), static_cast<int>(smem)))
     return TG_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return TG_ERR_CUDA;
+  const int cpc = chunks_per_cta(batch, n_hkv, max_len > 0 ? max_len : 1, sms);
+  const int n_span = (ns + cpc - 1) / cpc;   // split CTAs per (KV head, sequence)
   float* part = static_cast<float*>(workspace);
   tg_status r = TG_OK;
   if (max_len > 0) {
-    r = tg::launch(decode_split_kernel, dim3(ns, n_hkv, batch), dim3(kThreads), smem, stream, 0, tk,
-                   tv, static_cast<const __nv_bfloat16*>(q), s_cache, cache_len, cap, max_len, n_hq,
-                   n_hkv, gain, tau, part, ns, st);
+    r = tg::launch(decode_split_kernel, dim3(n_span, n_hkv, batch), dim3(kThreads), smem, stream, 0,
+                   tk, tv, static_cast<const __nv_bfloat16*>(q), s_cache, cache_len, cap, max_len,
+                   n_hq, n_hkv, gain, tau, part, ns, cpc, st);
     if (r != TG_OK) return r;
   }
   return tg::launch(decode_combine_kernel, dim3(n_hq, batch), dim3(kThreads), 0, stream, 0,
-                    static_cast<const float*>(part), cache_len, cap, max_len, n_hq, ns,
+                    static_cast<const float*>(part), cache_len, cap, max_len, n_hq, ns, cpc,
                     static_cast<__nv_bfloat16*>(out), st);
 }
 

@@ -50,6 +50,8 @@ struct alignas(16) SelectSmem {
   uint32_t warp_eq_off[kWarps];
   uint32_t cta_eq;               // published to peers
   uint32_t cta_keep;             // published to peers
+  uint32_t peer_eq[kMaxCluster]; // every CTA's published counts, fetched once
+  uint32_t peer_keep[kMaxCluster];
   uint32_t digit;
   uint32_t remaining;
   uint32_t cta_eq_off;
@@ -249,8 +251,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // thread t holds digit d = 255 - t; an inclusive prefix over t is the
         // count of matching document keys with digit >= d
         const int d = 255 - tid;
+        // every peer's count at once (independent remote loads in flight), then
+        // summed in rank order
+        uint32_t pc[kMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r)
+          pc[r] = r < static_cast<int>(csize) ? cluster.map_shared_rank(h, r)[d] : 0u;
         uint32_t cnt = 0;
-        for (unsigned r = 0; r < csize; ++r) cnt += cluster.map_shared_rank(h, r)[d];
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r) cnt += pc[r];
         uint32_t inc = warp_incl_scan(cnt, lane);
         if (lane == 31) S.scan[warp] = inc;
         tg::named_barrier(1, 256);   // warps 0-7 only
@@ -307,13 +316,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.cta_keep = tb;   // published: this CTA's tie count and tie-independent count
     }
     cluster.sync();
+    if (tid < static_cast<int>(csize)) {   // every peer's two counts, fetched in parallel
+      S.peer_eq[tid] = *cluster.map_shared_rank(&S.cta_eq, tid);
+      S.peer_keep[tid] = *cluster.map_shared_rank(&S.cta_keep, tid);
+    }
+    __syncthreads();
+    // this CTA reads no peer's shared memory after this point: announce it now and
+    // wait for the peers only before exiting, so the barrier overlaps pass 2
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     if (tid == 0) {
       // ties kept before a point = min(need, ties before it); this gives every
       // CTA's and every warp's output offset from (tie, tie-independent) counts
       uint32_t eq_before = 0, keep_before = 0, keep_total = 0;
       for (unsigned r = 0; r < csize; ++r) {
-        const uint32_t er = *cluster.map_shared_rank(&S.cta_eq, r);
-        const uint32_t br = *cluster.map_shared_rank(&S.cta_keep, r);
+        const uint32_t er = S.peer_eq[r];
+        const uint32_t br = S.peer_keep[r];
         const uint32_t kr = br + (need > eq_before ? min(need - eq_before, er) : 0u);
         if (r == rank) {
           S.cta_eq_off = eq_before;
@@ -385,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     cu_kept[b + 1] = (int32_t)(out_base + expect);
     if (b == batch - 1 && out_base + expect != total_kept) tg::set_status(status, TG_ERR_DEVICE_CHECK);
   }
-  cluster.sync();   // peers may read this CTA's shared memory until here
+  // peers may read this CTA's shared memory until they have arrived above
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 }  // namespace
