@@ -16,12 +16,16 @@
 // head with two TMA boxes each (64 dims x 64 rows, 128-byte swizzle, 32 KB in
 // all) and serves every query head of the GQA group from them: logits in fp32
 // (log2 domain), the running max m and sum l of 2^(z - m), and the unnormalised
-// sum of 2^(z - m) v. With many chunks per KV head (large batches) one CTA walks
-// several consecutive chunks through a two-stage TMA ring and folds them with an
-// online max, so the grid stays near two CTAs per SM. Each CTA writes one partial
-// per (sequence, query head, span) to a caller-provided workspace. A second kernel
-// merges a row's partials in span order (a fixed order: the result does not depend
-// on timing) and writes O = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c in bf16.
+// sum of 2^(z - m) v. Everything a CTA reads besides the chunk (the cache
+// length, the chunk's scores, the group's queries, gains and temperatures) is
+// requested at once, and the TMA copy goes out as soon as the length is known.
+// Each CTA writes one partial per (sequence, query head, chunk) to a
+// caller-provided workspace. A second kernel merges a row's partials in chunk
+// order (a fixed order: the result does not depend on timing) and writes
+// O = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c in bf16.
+// (A CTA walking several chunks through a TMA ring measured slower at every
+// batch and length tried, up to 16 sequences of 16k keys: fewer CTAs per SM hold
+// fewer bytes in flight.)
 #include <mutex>
 
 #include "common.cuh"
@@ -35,17 +39,18 @@ constexpr int kMaxGroup = 8;          // query heads per KV head
 constexpr int kPartial = kDh + 2;     // o[dh], m, l (fp32)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Shared memory: this header, then the chunk's 32 KB (K then V, each two
+// 64-column halves of 64 rows x 128 B, 128B-swizzled, 1024-byte aligned).
 struct DecSmem {
-  uint8_t k[2][2][kChunk * 64 * 2];   // [stage][dh half]: the chunk's K rows (8 KB per half)
-  uint8_t v[2][2][kChunk * 64 * 2];
-  float q[kMaxGroup][kDh];
+  float q[kMaxGroup][kDh];            // the group's queries, scaled into the log2 domain
   float p[kMaxGroup][kChunk];         // logits, then 2^(z - m)
-  float m[kMaxGroup];                 // running max over this CTA's chunks
-  float l[kMaxGroup];                 // running sum of 2^(z - m)
-  float alpha[kMaxGroup];             // 2^(m_old - m_new) of the current chunk
-  uint64_t full[2];
+  uint64_t full;
   int abort_flag;
 };
+constexpr uint32_t kHalfBytes = kChunk * 64 * 2;                            // 8 KB
+constexpr uint32_t kTileBytes = 4 * kHalfBytes;                             // K and V
+constexpr uint32_t kHeadBytes = (sizeof(DecSmem) + 1023) / 1024 * 1024;
+constexpr size_t kDecodeSmem = 1024 + kHeadBytes + kTileBytes;
 
 // byte offset of element e (0..127) of row j inside a [2][64 rows x 128 B] swizzled tile
 __device__ __forceinline__ uint32_t sw_off(int j, int e) {
@@ -56,220 +61,193 @@ __device__ __forceinline__ uint32_t sw_off(int j, int e) {
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-// One CTA per (span of `cpc` 64-key chunks, KV head, sequence): the chunks stream
-// through a two-stage TMA ring and fold into one partial with an online max.
+// One CTA per (64-key chunk, KV head, sequence).
 __global__ void __launch_bounds__(kThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __nv_bfloat16* __restrict__ q, const float* __restrict__ s_cache,
                         const int32_t* __restrict__ cache_len, int cap, int max_len, int n_hq,
                         int n_hkv, const float* __restrict__ gain, const float* __restrict__ tau,
-                        float* __restrict__ partial, int n_split, int cpc, int* status) {
+                        float* __restrict__ partial, int n_split, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
+  uint8_t* const kt = smem_raw + pad + kHeadBytes;   // K halves, then V halves
+  uint8_t* const vt = kt + 2 * kHalfBytes;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = n_hq / n_hkv;
   if (tid == 0) {
-    tg::mbar_init(&S.full[0], 1);
-    tg::mbar_init(&S.full[1], 1);
+    tg::mbar_init(&S.full, 1);
     S.abort_flag = 0;
     tg::fence_barrier_init();
     tg::tma_prefetch_desc(&tm_k);
     tg::tma_prefetch_desc(&tm_v);
   }
-  if (tid < kMaxGroup) {
-    S.m[tid] = -INFINITY;
-    S.l[tid] = 0.f;
-  }
   __syncthreads();
   tg::pdl_launch_dependents();
   tg::pdl_wait();   // global memory only from here on
 
+  // every independent load at once: the length, key j's score, this thread's
+  // query element d = tid of each head of the group, the heads' gains and tau
+  const int j0 = split * kChunk;
+  const int j = tid & (kChunk - 1);
   const int len = cache_len[b];
-  if (len < 0 || len > cap || len > max_len) {   // the combine kernel records it
-    return;
-  }
-  const int c_begin = split * cpc;
-  const int c_end = min((len + kChunk - 1) / kChunk, c_begin + cpc);
-  if (c_begin >= c_end) return;   // this span is past the cache's end
-
-  auto load = [&](int c, int stage) {
-    const int row = b * cap + c * kChunk;   // token coordinate in the (dh, heads, rows) view
-    tg::mbar_arrive_expect_tx(&S.full[stage], 4 * kChunk * 64 * 2);
-    tg::tma_load_3d(S.k[stage][0], &tm_k, &S.full[stage], 0, kvh, row);
-    tg::tma_load_3d(S.k[stage][1], &tm_k, &S.full[stage], 64, kvh, row);
-    tg::tma_load_3d(S.v[stage][0], &tm_v, &S.full[stage], 0, kvh, row);
-    tg::tma_load_3d(S.v[stage][1], &tm_v, &S.full[stage], 64, kvh, row);
-  };
-  if (tid == 0) load(c_begin, 0);
-  // the group's queries, scaled so that the logits come out in the log2 domain
-  for (int i = tid; i < G * kDh; i += kThreads) {
-    const int h = i / kDh, d = i % kDh;
+  const float sv_raw = j0 + j < cap ? s_cache[static_cast<int64_t>(b) * cap + j0 + j] : 0.f;
+  static_assert(kThreads == kDh, "thread d loads query element d");
+  float qv[kMaxGroup], cv[kMaxGroup], gv[kMaxGroup / 2];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
     const int hq = kvh * G + h;
-    const float c = kLog2e / (sqrtf(static_cast<float>(kDh)) * tau[hq]);
-    S.q[h][d] = __bfloat162float(q[(static_cast<int64_t>(b) * n_hq + hq) * kDh + d]) * c;
+    qv[h] = h < G ? __bfloat162float(q[(static_cast<int64_t>(b) * n_hq + hq) * kDh + tid]) : 0.f;
+    cv[h] = h < G ? tau[hq] : 1.f;
   }
-  // this thread's output dims 2(t % 64), +1 of heads t/64, t/64 + 2, ...
-  const int e = 2 * (tid & 63);
+#pragma unroll
+  for (int u = 0; u < kMaxGroup / 2; ++u) {
+    const int h = (tid >> 6) + 2 * u;
+    gv[u] = h < G ? gain[kvh * G + h] * kLog2e : 0.f;
+  }
+  if (len < 0 || len > cap || len > max_len) return;   // the combine kernel records it
+  if (j0 >= len) return;                                // this chunk is past the cache's end
+  if (tid == 0) {
+    const int row = b * cap + j0;   // token coordinate in the (dh, heads, rows) view
+    tg::mbar_arrive_expect_tx(&S.full, kTileBytes);
+    tg::tma_load_3d(kt, &tm_k, &S.full, 0, kvh, row);
+    tg::tma_load_3d(kt + kHalfBytes, &tm_k, &S.full, 64, kvh, row);
+    tg::tma_load_3d(vt, &tm_v, &S.full, 0, kvh, row);
+    tg::tma_load_3d(vt + kHalfBytes, &tm_v, &S.full, 64, kvh, row);
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h)
+    if (h < G) S.q[h][tid] = qv[h] * (kLog2e / (sqrtf(static_cast<float>(kDh)) * cv[h]));
+  const int nv = min(kChunk, len - j0);   // valid rows of the chunk
+  const int e = 2 * (tid & 63);           // this thread's output dims e, e + 1
   float o0[kMaxGroup / 2], o1[kMaxGroup / 2];
 #pragma unroll
   for (int u = 0; u < kMaxGroup / 2; ++u) o0[u] = o1[u] = 0.f;
   __syncthreads();
+  const bool ok = tg::mbar_wait(&S.full, 0, status, &S.abort_flag);
+  if (!__syncthreads_and(ok)) return;   // the copy never landed (recorded in the status)
 
-  for (int c = c_begin; c < c_end; ++c) {
-    const int i = c - c_begin, st = i & 1;
-    // the other stage was released by the barrier that ended the previous chunk
-    if (tid == 0 && c + 1 < c_end) load(c + 1, st ^ 1);
-    const bool ok = tg::mbar_wait(&S.full[st], (i >> 1) & 1, status, &S.abort_flag);
-    if (!__syncthreads_and(ok)) {   // a copy that never landed: leave after the others
-      if (tid == 0 && c + 1 < c_end)
-        tg::mbar_wait(&S.full[st ^ 1], ((i + 1) >> 1) & 1, status, nullptr);
-      return;
-    }
-    const int j0 = c * kChunk;
-    const int nv = min(kChunk, len - j0);   // valid rows of the chunk
-
-    // ---- logits: thread t takes key j = t % 64 and heads h = t / 64, t / 64 + 2, ... ----
-    {
-      const int j = tid & (kChunk - 1);
-      const uint8_t* kb = S.k[st][0];
-      float acc[kMaxGroup / 2];
+  // ---- logits: thread t takes key j = t % 64 and heads h = t / 64, t / 64 + 2, ... ----
+  {
+    float acc[kMaxGroup / 2];
 #pragma unroll
-      for (int u = 0; u < kMaxGroup / 2; ++u) acc[u] = 0.f;
+    for (int u = 0; u < kMaxGroup / 2; ++u) acc[u] = 0.f;
 #pragma unroll 4
-      for (int cc = 0; cc < kDh / 8; ++cc) {
-        const uint4 kk = *reinterpret_cast<const uint4*>(kb + sw_off(j, 8 * cc));
-        const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
-                             bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
-#pragma unroll
-        for (int u = 0; u < kMaxGroup / 2; ++u) {
-          const int h = (tid >> 6) + 2 * u;
-          if (h < G) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc + 4]);
-            float a = acc[u];
-            a = fmaf(q0.x, kf[0], a); a = fmaf(q0.y, kf[1], a);
-            a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
-            a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a);
-            a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
-            acc[u] = a;
-          }
-        }
-      }
-      const float sv = j < nv ? s_cache[static_cast<int64_t>(b) * cap + j0 + j] : 0.f;
+    for (int cc = 0; cc < kDh / 8; ++cc) {
+      const uint4 kk = *reinterpret_cast<const uint4*>(kt + sw_off(j, 8 * cc));
+      const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
+                           bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
 #pragma unroll
       for (int u = 0; u < kMaxGroup / 2; ++u) {
         const int h = (tid >> 6) + 2 * u;
         if (h < G) {
-          const float bias = gain[kvh * G + h] * kLog2e * sv;
-          S.p[h][j] = j < nv ? acc[u] + bias : -INFINITY;
+          const float4 q0 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc]);
+          const float4 q1 = *reinterpret_cast<const float4*>(&S.q[h][8 * cc + 4]);
+          float a = acc[u];
+          a = fmaf(q0.x, kf[0], a); a = fmaf(q0.y, kf[1], a);
+          a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+          a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a);
+          a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
+          acc[u] = a;
         }
       }
     }
-    __syncthreads();
-
-    // ---- per head: the running max moves to cover this chunk; weights and their sum ----
-    for (int h = warp; h < G; h += kThreads / 32) {
-      const float z0 = S.p[h][lane], z1 = S.p[h][lane + 32];
-      float mc = fmaxf(z0, z1);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xFFFFFFFFu, mc, off));
-      const float m_old = S.m[h];
-      const float m_new = fmaxf(m_old, mc);   // finite: row 0 of every chunk is valid
-      const float p0 = tg::exp2_approx(z0 - m_new), p1 = tg::exp2_approx(z1 - m_new);
-      S.p[h][lane] = p0;
-      S.p[h][lane + 32] = p1;
-      float lc = p0 + p1;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) lc += __shfl_xor_sync(0xFFFFFFFFu, lc, off);
-      __syncwarp();
-      if (lane == 0) {
-        const float al = tg::exp2_approx(m_old - m_new);   // 0 for the first chunk
-        S.alpha[h] = al;
-        S.m[h] = m_new;
-        S.l[h] = S.l[h] * al + lc;
-      }
+    for (int u = 0; u < kMaxGroup / 2; ++u) {
+      const int h = (tid >> 6) + 2 * u;
+      if (h < G) S.p[h][j] = j < nv ? acc[u] + gv[u] * sv_raw : -INFINITY;
     }
-    __syncthreads();
+  }
+  __syncthreads();
 
-    // ---- o = alpha o + sum_j p_j v_j ----
-    {
-      const uint8_t* vb = S.v[st][0];
+  // ---- per head: chunk max and weights; warp h writes the head's m and l ----
+  for (int h = warp; h < G; h += kThreads / 32) {
+    const float z0 = S.p[h][lane], z1 = S.p[h][lane + 32];
+    float mc = fmaxf(z0, z1);
 #pragma unroll
-      for (int u = 0; u < kMaxGroup / 2; ++u) {
-        const int h = (tid >> 6) + 2 * u;
-        if (h < G) {
-          const float al = S.alpha[h];
-          o0[u] *= al;
-          o1[u] *= al;
-        }
-      }
+    for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xFFFFFFFFu, mc, off));
+    // mc is finite: row 0 of every chunk is valid
+    const float p0 = tg::exp2_approx(z0 - mc), p1 = tg::exp2_approx(z1 - mc);
+    S.p[h][lane] = p0;
+    S.p[h][lane + 32] = p1;
+    float lc = p0 + p1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lc += __shfl_xor_sync(0xFFFFFFFFu, lc, off);
+    if (lane == 0) {
+      float* pr = partial + ((static_cast<int64_t>(b) * n_hq + kvh * G + h) * n_split + split) * kPartial;
+      pr[kDh] = mc;
+      pr[kDh + 1] = lc;
+    }
+  }
+  __syncthreads();
+
+  // ---- o = sum_j p_j v_j ----
 #pragma unroll 4
-      for (int j = 0; j < nv; ++j) {
-        const uint32_t vv = *reinterpret_cast<const uint32_t*>(vb + sw_off(j, e));
-        const float v0 = bf16_lo(vv), v1 = bf16_hi(vv);
+  for (int jj = 0; jj < nv; ++jj) {
+    const uint32_t vv = *reinterpret_cast<const uint32_t*>(vt + sw_off(jj, e));
+    const float v0 = bf16_lo(vv), v1 = bf16_hi(vv);
 #pragma unroll
-        for (int u = 0; u < kMaxGroup / 2; ++u) {
-          const int h = (tid >> 6) + 2 * u;
-          if (h < G) {
-            const float pj = S.p[h][j];
-            o0[u] = fmaf(pj, v0, o0[u]);
-            o1[u] = fmaf(pj, v1, o1[u]);
-          }
-        }
+    for (int u = 0; u < kMaxGroup / 2; ++u) {
+      const int h = (tid >> 6) + 2 * u;
+      if (h < G) {
+        const float pj = S.p[h][jj];
+        o0[u] = fmaf(pj, v0, o0[u]);
+        o1[u] = fmaf(pj, v1, o1[u]);
       }
     }
-    __syncthreads();   // stage st, S.p and S.alpha are free for the next chunk
   }
 #pragma unroll
   for (int u = 0; u < kMaxGroup / 2; ++u) {
     const int h = (tid >> 6) + 2 * u;
     if (h < G) {
-      const int hq = kvh * G + h;
-      float* pr = partial + ((static_cast<int64_t>(b) * n_hq + hq) * n_split + split) * kPartial;
+      float* pr = partial + ((static_cast<int64_t>(b) * n_hq + kvh * G + h) * n_split + split) * kPartial;
       *reinterpret_cast<float2*>(pr + e) = make_float2(o0[u], o1[u]);
-      if ((tid & 63) == 0) {
-        pr[kDh] = S.m[h];
-        pr[kDh + 1] = S.l[h];
-      }
     }
   }
 }
 
-// Merge one row's span partials in span order; thread d writes dimension d. One
-// round of global loads: the spans' maxima and sums go to shared memory while every
-// thread's own output loads (up to 32 spans at a time) are already in flight.
+// Merge one row's chunk partials. Chunks come in blocks of 128: thread d of group 0
+// loads chunk d's max and sum into shared memory, every thread takes the block's
+// max, and group g (threads 128g .. 128g + 127, thread d of it owning output
+// dimension d) folds the block's chunks 32g .. 32g + 31 with all 32 loads in
+// flight. Every group scales by the same running max, so the groups' sums add at
+// the end.
 constexpr int kCombineBlock = 32;
+constexpr int kCombineGroups = 4;
+constexpr int kCombineThreads = kCombineGroups * kDh;
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kCombineThreads)
     decode_combine_kernel(const float* __restrict__ partial, const int32_t* __restrict__ cache_len,
-                          int cap, int max_len, int n_hq, int n_split, int cpc,
+                          int cap, int max_len, int n_hq, int n_split,
                           __nv_bfloat16* __restrict__ out, int* status) {
-  __shared__ float sm[kThreads], sl[kThreads];
+  __shared__ float sm[kDh], sl[kDh];
+  __shared__ float racc[kCombineGroups - 1][kDh], rl[kCombineGroups - 1][kDh];
   tg::pdl_launch_dependents();
   tg::pdl_wait();
-  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int grp = threadIdx.x / kDh, d = threadIdx.x % kDh;
   const int len = cache_len[b];
   __nv_bfloat16* o = out + (static_cast<int64_t>(b) * n_hq + hq) * kDh;
   if (len < 0 || len > cap || len > max_len) {
-    if (d == 0 && hq == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    if (threadIdx.x == 0 && hq == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
     return;
   }
   if (len == 0) {   // an empty cache attends to nothing
-    o[d] = __float2bfloat16_rn(0.f);
+    if (grp == 0) o[d] = __float2bfloat16_rn(0.f);
     return;
   }
-  const int nsp = ((len + kChunk - 1) / kChunk + cpc - 1) / cpc;   // spans holding a partial
+  const int nsp = (len + kChunk - 1) / kChunk;   // chunks holding a partial
   const float* pr = partial + (static_cast<int64_t>(b) * n_hq + hq) * n_split * kPartial;
   float acc = 0.f, L = 0.f, M = -INFINITY;
-  for (int s0 = 0; s0 < nsp; s0 += kThreads) {   // blocks of up to 128 spans (one block below 8k keys)
-    const int ns = min(kThreads, nsp - s0);
+  for (int s0 = 0; s0 < nsp; s0 += kDh) {   // blocks of up to 128 chunks (one block below 8k keys)
+    const int ns = min(kDh, nsp - s0);
+    const int u0 = grp * kCombineBlock;   // this group's 32 chunks of the block
     float v[kCombineBlock];
 #pragma unroll
     for (int u = 0; u < kCombineBlock; ++u)
-      v[u] = u < ns ? pr[(s0 + u) * kPartial + d] : 0.f;
-    if (d < ns) {
+      v[u] = u0 + u < ns ? pr[(s0 + u0 + u) * kPartial + d] : 0.f;
+    if (grp == 0 && d < ns) {
       sm[d] = pr[(s0 + d) * kPartial + kDh];
       sl[d] = pr[(s0 + d) * kPartial + kDh + 1];
     }
@@ -282,20 +260,27 @@ __global__ void __launch_bounds__(kThreads)
     M = mb;
 #pragma unroll
     for (int u = 0; u < kCombineBlock; ++u) {
-      if (u < ns) {
-        const float w = tg::exp2_approx(sm[u] - M);
-        L = fmaf(w, sl[u], L);
+      if (u0 + u < ns) {
+        const float w = tg::exp2_approx(sm[u0 + u] - M);
+        L = fmaf(w, sl[u0 + u], L);
         acc = fmaf(w, v[u], acc);
       }
     }
-    for (int u = kCombineBlock; u < ns; ++u) {   // spans past the first 32 of a block
-      const float w = tg::exp2_approx(sm[u] - M);
-      L = fmaf(w, sl[u], L);
-      acc = fmaf(w, pr[(s0 + u) * kPartial + d], acc);
-    }
     __syncthreads();   // sm, sl are rewritten by the next block
   }
-  o[d] = __float2bfloat16_rn(acc / L);
+  if (grp > 0) {
+    racc[grp - 1][d] = acc;
+    rl[grp - 1][d] = L;
+  }
+  __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int g = 0; g < kCombineGroups - 1; ++g) {
+      acc += racc[g][d];
+      L += rl[g][d];
+    }
+    o[d] = __float2bfloat16_rn(acc / L);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -324,13 +309,6 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 inline int n_splits(int max_len) { return (max_len + kChunk - 1) / kChunk; }
-
-// chunks per split CTA: one while the grid stays below two CTAs per SM, more beyond
-inline int chunks_per_cta(int batch, int n_hkv, int max_len, int sms) {
-  const int64_t ctas = static_cast<int64_t>(batch) * n_hkv * n_splits(max_len);
-  const int64_t target = 2 * static_cast<int64_t>(sms);
-  return ctas <= target ? 1 : static_cast<int>((ctas + target - 1) / target);
-}
 
 }  // namespace
 
@@ -396,25 +374,18 @@ extern "C" tg_status tg_gated_decode(const void* q, const void* k_cache, const v
       !tg::encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v_cache, dims, strides, box,
                        CU_TENSOR_MAP_SWIZZLE_128B))
     return TG_ERR_CUDA;
-  const size_t smem = sizeof(DecSmem) + 1024;
-  if (!tg::ensure_smem(reinterpret_cast<const void*>(decode_split_kernel), static_cast<int>(smem)))
+  if (!tg::ensure_smem(reinterpret_cast<const void*>(decode_split_kernel), static_cast<int>(kDecodeSmem)))
     return TG_ERR_CUDA;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return TG_ERR_CUDA;
-  const int cpc = chunks_per_cta(batch, n_hkv, max_len > 0 ? max_len : 1, sms);
-  const int n_span = (ns + cpc - 1) / cpc;   // split CTAs per (KV head, sequence)
   float* part = static_cast<float*>(workspace);
   tg_status r = TG_OK;
   if (max_len > 0) {
-    r = tg::launch(decode_split_kernel, dim3(n_span, n_hkv, batch), dim3(kThreads), smem, stream, 0,
+    r = tg::launch(decode_split_kernel, dim3(ns, n_hkv, batch), dim3(kThreads), kDecodeSmem, stream, 0,
                    tk, tv, static_cast<const __nv_bfloat16*>(q), s_cache, cache_len, cap, max_len,
-                   n_hq, n_hkv, gain, tau, part, ns, cpc, st);
+                   n_hq, n_hkv, gain, tau, part, ns, st);
     if (r != TG_OK) return r;
   }
-  return tg::launch(decode_combine_kernel, dim3(n_hq, batch), dim3(kThreads), 0, stream, 0,
-                    static_cast<const float*>(part), cache_len, cap, max_len, n_hq, ns, cpc,
+  return tg::launch(decode_combine_kernel, dim3(n_hq, batch), dim3(kCombineThreads), 0, stream, 0,
+                    static_cast<const float*>(part), cache_len, cap, max_len, n_hq, ns,
                     static_cast<__nv_bfloat16*>(out), st);
 }
 
