@@ -86,26 +86,44 @@ def _select_both(api, orc, scores, lens, db, de, kd):
     want_idx, want_cu = orc.select_topk(scores, cu, db, de, kd)
     dev = lambda a: torch.tensor(np.asarray(a, np.int32), device="cuda")
     st = torch.tensor(scores, device="cuda")
-    idx, ks, cuk = api.select_topk(st, dev(cu), dev(db), dev(de), dev(kd), len(want_idx),
-                                   max(lens) if lens else 0)
+    idx, ks, cuk, pos = api.select_topk(st, dev(cu), dev(db), dev(de), dev(kd), len(want_idx),
+                                        max(lens) if lens else 0, want_pos=True)
     np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
     np.testing.assert_array_equal(cuk.cpu().numpy(), want_cu)
     np.testing.assert_array_equal(ks.cpu().numpy().view(np.int32),
                                   scores[want_idx].view(np.int32))
+    # a kept row's position is its offset from its sequence's first row
+    seq = np.searchsorted(cu, want_idx, side="right") - 1
+    np.testing.assert_array_equal(pos.cpu().numpy(), want_idx - cu[seq])
     return want_idx
 
 
-def test_select_ties_and_specials(api, orc):
+# up to 16384 tokens one CTA selects a sequence; longer ones go to a CTA cluster:
+# lengths on both sides of that boundary
+@pytest.mark.parametrize("n", [5000, 16384, 16385])
+def test_select_ties_and_specials(api, orc, n):
     rng = np.random.default_rng(0)
-    n = 5000
     s = (rng.integers(-40, 40, n) / 4).astype(np.float32)          # heavy exact ties
     s[rng.integers(0, n, 50)] = np.nan
     s[rng.integers(0, n, 20)] = np.inf
     s[rng.integers(0, n, 20)] = -np.inf
     s[rng.integers(0, n, 30)] = -0.0
     s[rng.integers(0, n, 30)] = 0.0
-    for k in [0, 1, 7, 999, 2500, 4700, 4744, 4745, 10 ** 6]:
-        _select_both(api, orc, s, [n], [0], [n - 256], [k])
+    nd = n - 256
+    for k in [0, 1, 7, nd // 5, nd // 2, nd - 44, nd - 1, nd, 10 ** 6]:
+        _select_both(api, orc, s, [n], [0], [nd], [k])
+
+
+def test_select_ragged_up_to_one_cta(api, orc):
+    # a batch whose longest sequence is exactly the one-CTA limit
+    rng = np.random.default_rng(5)
+    lens = rng.integers(1, 16384, 11).tolist() + [16384]
+    s = rng.standard_normal(sum(lens)).astype(np.float32)
+    db = [int(rng.integers(0, 50)) for _ in lens]
+    db = [min(d, l) for d, l in zip(db, lens)]
+    de = [max(d, l - int(rng.integers(0, 300))) for d, l in zip(db, lens)]
+    kd = [int(rng.integers(0, e - d + 2)) for d, e in zip(db, de)]
+    _select_both(api, orc, s, lens, db, de, kd)
 
 
 def test_select_doc_in_middle_and_degenerate_spans(api, orc):
@@ -139,10 +157,10 @@ def test_select_max_seqlen(api, orc):
     _select_both(api, orc, s, [n], [0], [n - 512], [15000])
 
 
-def test_select_threshold_ties_straddle(api, orc):
+@pytest.mark.parametrize("n", [16384, 32768])
+def test_select_threshold_ties_straddle(api, orc, n):
     # many copies of the K-th value on both sides of the cut
     rng = np.random.default_rng(4)
-    n = 32768
     s = rng.standard_normal(n).astype(np.float32)
     k = 3225
     kth = np.sort(s[: n - 512])[::-1][k - 1]
