@@ -98,8 +98,8 @@ def _select_both(api, orc, scores, lens, db, de, kd):
     return want_idx
 
 
-# up to 16384 tokens one CTA selects a sequence; longer ones go to a CTA cluster:
-# lengths on both sides of that boundary
+# a sequence's cluster has one CTA per 4096 tokens: one CTA, then 4 CTAs with
+# every slice full, then 5 CTAs with a one-token last slice
 @pytest.mark.parametrize("n", [5000, 16384, 16385])
 def test_select_ties_and_specials(api, orc, n):
     rng = np.random.default_rng(0)
@@ -114,8 +114,8 @@ def test_select_ties_and_specials(api, orc, n):
         _select_both(api, orc, s, [n], [0], [nd], [k])
 
 
-def test_select_ragged_up_to_one_cta(api, orc):
-    # a batch whose longest sequence is exactly the one-CTA limit
+def test_select_ragged_up_to_16384(api, orc):
+    # a batch whose longest sequence fills a 4-CTA cluster exactly
     rng = np.random.default_rng(5)
     lens = rng.integers(1, 16384, 11).tolist() + [16384]
     s = rng.standard_normal(sum(lens)).astype(np.float32)
