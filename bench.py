@@ -425,22 +425,26 @@ def _time_backward(gp, wl, steps, warmup, rep, flush, stream, tf_peak):
                     "forward's causal flops (S, dP, dV, dK, dQ)"}
 
 
-FP32_FMA_PER_CLK_PER_SM = 128   # B200: 4 sub-partitions x 32 fp32 FMA lanes
-
-
-def _time_deltanet(gp, wl, steps, warmup, rep, flush, stream, sm_mhz_max, n_sm):
-    """A Gated DeltaNet layer's recurrence over the layer's kept rows (row f3): the
-    workload's seeded DeltaNet inputs, one launch per step in a CUDA graph, L2 flushed
-    before each. The recurrence is sequential in the tokens, so its bound is the
-    per-token latency of the fp32 SIMT update, not a roofline of bytes or tensor
-    flops; the fraction is of the fp32 FMA peak (SMs x 128 lanes x 2 flops x clock)."""
+def _time_deltanet(gp, wl, steps, warmup, rep, flush, stream, tf_peak, hbm_peak):
+    """A Gated DeltaNet layer's gated delta rule over the layer's kept rows (row f3):
+    the workload's seeded DeltaNet inputs, one call (two launches) per step in a CUDA
+    graph, L2 flushed before each. The rule is computed in 64-token chunks: a parallel
+    per-chunk pass, then each sequence's chunks in order, so its time is set by that
+    chain of chunk steps, not by bytes or tensor throughput. Reported: the rule's
+    algorithmic flops (6 dk dv per token and head: k.s, the update, q.s) against the
+    bf16 tensor peak, its algorithmic bytes (q, k, v, alpha, beta read, out written)
+    against the HBM peak, and the time per chunk step."""
     from learned_token_pruning_gemm_b200 import api, synth
     q, k, v, a, b = (t.to(gp.q.device) for t in synth.deltanet_inputs(wl))
     cu = gp.cu_kept
     out = torch.empty_like(v)
+    max_len = max(wl.kept_counts)
+    ws = torch.empty(api.gated_delta_rule_workspace_size(wl.batch, q.shape[0], q.shape[1],
+                                                         v.shape[2]), dtype=torch.uint8,
+                     device=q.device)
 
     def step():
-        api.gated_delta_rule(q, k, v, a, b, cu, out=out)
+        api.gated_delta_rule(q, k, v, a, b, cu, max_len, out=out, workspace=ws)
 
     step()
     torch.cuda.synchronize()
@@ -465,12 +469,19 @@ def _time_deltanet(gp, wl, steps, warmup, rep, flush, stream, sm_mhz_max, n_sm):
         raise RuntimeError("device status set by the delta rule")
     ms = rep.max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev))
     K, H, d = q.shape
-    flops = 6.0 * K * H * d * v.shape[2]   # k.s, the update, q.s: 3 x (multiply + add) per state entry
-    peak = n_sm * FP32_FMA_PER_CLK_PER_SM * 2 * sm_mhz_max * 1e6 / 1e12
-    return {"us": ms * 1e3, "tokens_per_s": K / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12,
-            "bound": "alu", "peak_tflops_fp32": peak,
-            "frac_alu": flops / (ms / 1e3) / 1e12 / peak, "launches_per_step": 1,
-            "note": "sequential in the tokens: one CTA per (16 value columns, head, sequence)"}
+    dv = v.shape[2]
+    flops = 6.0 * K * H * d * dv
+    nbytes = K * H * (2 * d + 2 * dv) * 2 + K * H * 8   # q, k, v, out (bf16); alpha, beta
+    chunks = max((n + 63) // 64 for n in wl.kept_counts)
+    tflops = flops / (ms / 1e3) / 1e12
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"us": ms * 1e3, "tokens_per_s": K / (ms / 1e3), "tflops": tflops,
+            "frac_tensor": tflops / tf_peak, "gbs": gbs, "frac_hbm": gbs / hbm_peak,
+            "bound": "sequential chunk steps", "chunk_steps": chunks,
+            "us_per_chunk_step": ms * 1e3 / chunks, "launches_per_step": 2,
+            "note": "chunked gated delta rule: per-chunk pass (T = (I + A)^-1, W, U~, masked "
+                    "Q K^T) in parallel, then each sequence's 64-token chunks in order with "
+                    "the state; mma.sync with split bf16 operands"}
 
 
 def run_ours(args, rep):
@@ -513,10 +524,8 @@ def run_ours(args, rep):
 
     deltanet = None
     if wl.dtype == "bf16" and wl.dh == 128 and not args.no_deltanet:
-        props = torch.cuda.get_device_properties(dev_index)
-        sm_max = clocks.max_mhz if clocks.error is None else peaks.get("sm_max_mhz", 1965.0)
-        deltanet = _time_deltanet(gp, wl, args.steps, args.warmup, rep, flush, stream, sm_max,
-                                  props.multi_processor_count)
+        deltanet = _time_deltanet(gp, wl, args.steps, args.warmup, rep, flush, stream, tf_peak,
+                                  hbm_peak)
 
     backward = None
     if wl.dtype == "bf16" and wl.dh == 128 and not args.no_backward:

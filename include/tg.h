@@ -286,19 +286,29 @@ tg_status tg_gated_decode_noalloc(const void* q, const void* k_cache, const void
  * zero and, for the sequence's rows t in order,
  *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
  *     out_t = S_t^T q_t
+ * computed in chunks of 64 rows (a parallel per-chunk pass, then one sequential
+ * pass over each sequence's chunks).
  *   q, k  [total, n_heads, head_dim_k] bf16 (the caller normalises k; with |k| = 1
  *         and alpha, beta in [0, 1] the state stays bounded)
  *   v     [total, n_heads, head_dim_v] bf16
  *   alpha, beta [total, n_heads] f32 (decay and write strength per token and head)
+ *   max_seqlen  bounds every sequence's length (host value; sizes the grid)
  *   out   [total, n_heads, head_dim_v] bf16 output
+ *   workspace   caller-owned device scratch of at least
+ *               tg_gated_delta_rule_workspace_size(...) bytes, 16-byte aligned
+ *               (per 64-row chunk and head: the chunk's products that do not depend
+ *               on the state)
  * TG_BF16 only; head_dim_k == 128, head_dim_v a multiple of 16 up to 1024; q, k, v,
- * out 16-byte aligned. A sequence outside [0, total] is skipped and
- * TG_ERR_DEVICE_CHECK recorded.
+ * out 16-byte aligned. A sequence outside [0, total] or longer than max_seqlen is
+ * skipped (its rows of out are not written) and TG_ERR_DEVICE_CHECK recorded.
  */
+size_t tg_gated_delta_rule_workspace_size(int batch, int64_t total, int n_heads,
+                                          int head_dim_v);
 tg_status tg_gated_delta_rule(const void* q, const void* k, const void* v, tg_dtype dtype,
                               const float* alpha, const float* beta, const int32_t* cu_seqlens,
-                              int batch, int64_t total, int n_heads, int head_dim_k,
-                              int head_dim_v, void* out, tg_stream_t stream);
+                              int batch, int64_t total, int max_seqlen, int n_heads,
+                              int head_dim_k, int head_dim_v, void* out, void* workspace,
+                              size_t workspace_bytes, tg_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns the first error any kernel recorded on the

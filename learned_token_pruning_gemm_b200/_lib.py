@@ -34,7 +34,9 @@ SIGNATURES = {
     "tg_gated_decode": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P,
                               ctypes.c_size_t, P]),
     "tg_gated_decode_noalloc": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P]),
-    "tg_gated_delta_rule": (INT, [P, P, P, INT, P, P, P, INT, I64, INT, INT, INT, P, P]),
+    "tg_gated_delta_rule_workspace_size": (ctypes.c_size_t, [INT, I64, INT, INT]),
+    "tg_gated_delta_rule": (INT, [P, P, P, INT, P, P, P, INT, I64, INT, INT, INT, INT, P, P,
+                                  ctypes.c_size_t, P]),
     "tg_device_status": (INT, [P, INT]),
     "tg_selftest_bounded_wait": (INT, [I64, P]),
 }

@@ -216,11 +216,19 @@ def gated_attention_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: 
     return dq, dk, dv, ds, dg, dt
 
 
+def gated_delta_rule_workspace_size(batch: int, total: int, n_heads: int, head_dim_v: int) -> int:
+    return int(_lib.load().tg_gated_delta_rule_workspace_size(batch, total, n_heads, head_dim_v))
+
+
 def gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
-                     beta: torch.Tensor, cu_seqlens: torch.Tensor,
-                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                     beta: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: Optional[int] = None,
+                     out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
     """Gated delta rule per sequence and head over packed rows: q, k [T,H,dk], v [T,H,dv]
-    bf16, alpha/beta [T,H] f32 -> out [T,H,dv] bf16 (state reset per sequence)."""
+    bf16, alpha/beta [T,H] f32 -> out [T,H,dv] bf16 (state reset per sequence).
+    max_seqlen bounds every sequence's length; when None it is read from cu_seqlens
+    (a device-to-host copy). workspace: uint8 of at least gated_delta_rule_workspace_size
+    bytes, allocated here when None."""
     T, H, dk = q.shape
     dv = v.shape[2]
     _shape(k, q.shape, "k", q.dtype)
@@ -231,13 +239,23 @@ def gated_delta_rule(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: t
         raise TokenGateError("cu_seqlens must have batch+1 >= 1 elements")
     if q.dtype not in _DT:
         raise TokenGateError(f"gated_delta_rule: unsupported dtype {q.dtype}")
+    B = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        cu_h = cu_seqlens.detach().to("cpu", torch.int64)
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if B > 0 else 0
     if out is None:
         out = torch.empty_like(v)
     _shape(out, v.shape, "out", v.dtype)
+    need = gated_delta_rule_workspace_size(B, T, H, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if workspace.dtype != torch.uint8 or workspace.numel() < need:
+        raise TokenGateError(f"gated_delta_rule: workspace needs {need} bytes (uint8)")
     st = _lib.load().tg_gated_delta_rule(
         _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _DT[q.dtype], _cuda(alpha, "alpha"),
         _cuda(beta, "beta"), _cuda(cu_seqlens, "cu_seqlens", torch.int32),
-        cu_seqlens.numel() - 1, T, H, dk, dv, _cuda(out, "out"), _stream(stream))
+        B, T, int(max_seqlen), H, dk, dv, _cuda(out, "out"), _cuda(workspace, "workspace"),
+        workspace.numel(), _stream(stream))
     check(st, "tg_gated_delta_rule")
     return out
 

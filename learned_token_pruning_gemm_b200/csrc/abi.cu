@@ -110,7 +110,7 @@ __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
 
 extern "C" {
 
-int tg_abi_version(void) { return 3; }
+int tg_abi_version(void) { return 4; }
 
 const char* tg_status_string(tg_status s) {
   switch (s) {

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.tg_abi_version() == 3
+    assert lib.tg_abi_version() == 4
     for code, name in [(0, "TG_OK"), (1, "TG_ERR_INVALID_ARG"), (3, "TG_ERR_MISALIGNED"),
                        (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (99, "TG_ERR_UNKNOWN")]:
         assert lib.tg_status_string(code).decode() == name
@@ -259,18 +259,28 @@ def test_backward_validation_without_gpu(lib):
 
 
 def test_delta_rule_validation_without_gpu(lib):
-    INVALID, UNSUP, MIS = 1, 2, 3
+    INVALID, UNSUP, MIS, WS = 1, 2, 3, 4
     P = ctypes.c_void_p
     fake, odd = P(0x10000), P(0x10004)
+    big = 1 << 30
 
-    def dn(dtype=1, dk=128, dv=128, q=fake, a=fake, total=10, batch=1):
-        return lib.tg_gated_delta_rule(q, fake, fake, dtype, a, fake, fake, batch, total, 4, dk,
-                                       dv, fake, None)
+    def dn(dtype=1, dk=128, dv=128, q=fake, a=fake, total=10, batch=1, max_len=10, ws=fake,
+           ws_bytes=big):
+        return lib.tg_gated_delta_rule(q, fake, fake, dtype, a, fake, fake, batch, total, max_len,
+                                       4, dk, dv, fake, ws, ws_bytes, None)
     assert dn(dtype=0) == UNSUP
     assert dn(dk=64) == UNSUP
     assert dn(dv=100) == UNSUP
     assert dn(q=odd) == MIS
     assert dn(a=P(0x10002)) == MIS
     assert dn(q=None) == INVALID
-    assert dn(total=0) == 0 and dn(batch=0) == 0
+    assert dn(total=0) == 0 and dn(batch=0) == 0 and dn(max_len=0) == 0
     assert dn(total=-1) == INVALID
+    assert dn(max_len=-1) == INVALID
+    assert dn(ws=None) == WS
+    assert dn(ws=odd) == MIS
+    # one record per (64-row chunk slot, head): floor(total / 64) + batch slots
+    need = lib.tg_gated_delta_rule_workspace_size(3, 1000, 4, 128)
+    assert need == (1000 // 64 + 3) * 4 * (53760 + 256 * 128)
+    assert dn(total=1000, batch=3, ws_bytes=need - 1) == WS
+    assert lib.tg_gated_delta_rule_workspace_size(0, 10, 4, 128) == 0

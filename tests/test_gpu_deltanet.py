@@ -3,10 +3,13 @@ against the fp64 oracle, through the C ABI (MarkTechPost page on TokenGate, sect
 "Est-ce que cela fonctionne avec les modèles d'attention hybrides ?": the hybrid
 model's Gated DeltaNet layers are pruned too).
 
-Tolerance: the outputs are bf16 like the attention's, so the bf16 bar of
-tests/helpers.py (1e-2 max-abs, 5e-3 relative L2); the fp32 state is updated once
-per token, and with unit keys and alpha <= 1 each update is a contraction, so the
-rounding does not grow with the sequence length."""
+The GPU runs the rule in chunks of 64 tokens (a per-chunk pass with a triangular
+solve, then a pass over each sequence's chunks with the state); the oracle runs it
+token by token. Tolerance: the outputs are bf16 like the attention's, so the bf16
+bar of tests/helpers.py (1e-2 max-abs, 5e-3 relative L2). The GPU's products carry
+16 significant bits per operand with fp32 accumulation; with unit keys and
+alpha <= 1 each update is a contraction, so rounding does not grow with the
+sequence length (the 16k layer's 1868 rows and a 5000-row sequence check it)."""
 import numpy as np
 import pytest
 import torch
@@ -43,7 +46,9 @@ def _case(seed, lens, H, dv=128):
 
 
 @pytest.mark.parametrize("lens,H,dv", [([100], 2, 128), ([33, 1, 70, 0, 200], 3, 128),
-                                       ([64], 1, 48), ([1868], 16, 128)])
+                                       ([64], 1, 48), ([1868], 16, 128),
+                                       ([63, 64, 65, 127, 128, 129], 2, 128),
+                                       ([300, 17], 2, 272), ([5000], 1, 32)])
 def test_delta_rule_vs_oracle(api, orc, lens, H, dv):
     q, k, v, a, b, cu = _case(sum(lens) + H, lens, H, dv)
     out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
@@ -65,3 +70,29 @@ def test_delta_rule_on_the_16k_layers_kept_rows(api, orc):
     heads = [0, 7, 15]
     ref = orc.gated_delta_rule(q[:, heads], k[:, heads], v[:, heads], a[:, heads], b[:, heads], cu)
     assert_attn_close(out[:, heads].contiguous(), ref, torch.bfloat16, what="16k kept rows")
+
+
+def test_delta_rule_strong_decay_and_repeated_keys(api, orc):
+    # decays down to 0.05 (decay products over a chunk reach 1e-80 and underflow to
+    # zero) and every fourth key a copy of the previous one written with beta = 1
+    # (the overwrite case: the triangular solve's entries reach +-1)
+    q, k, v, a, b, cu = _case(11, [150, 90], 2)
+    g = torch.Generator().manual_seed(12)
+    a = 0.05 + 0.95 * torch.rand(a.shape, generator=g)
+    k[3::4] = k[2::4][: k[3::4].shape[0]]
+    b[3::4] = 1.0
+    out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                               torch.tensor(cu, device="cuda"))
+    ref = orc.gated_delta_rule(q, k, v, a, b, cu)
+    assert_attn_close(out, ref, torch.bfloat16, what="strong decay, repeated keys")
+
+
+def test_delta_rule_sequence_longer_than_max_seqlen_is_reported(api):
+    q, k, v, a, b, cu = _case(13, [70, 40], 1)
+    out = torch.full(v.shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                         torch.tensor(cu, device="cuda"), max_seqlen=64, out=out)
+    assert api.device_status(reset=True) == 7          # TG_ERR_DEVICE_CHECK
+    o = out.float().cpu()
+    assert torch.all(o[:70] == 7.0)                     # the 70-row sequence is skipped
+    assert not torch.all(o[70:] == 7.0)                 # the 40-row one is computed
