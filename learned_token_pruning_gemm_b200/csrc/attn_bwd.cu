@@ -47,10 +47,18 @@ __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, uint
 struct BwdWs {
   float* D;      // [n_hq, total]
   float* lse2;   // [n_hq, total]   log-sum-exp in log2 units
-  float* ds;     // [n_hkv, total]  per-KV-head partial score gradients
+  float* ds;     // partial score gradients: bf16 [2 halves, n_hkv, total], f32 [n_hkv, total]
   float* gt;     // gain / temperature partials: bf16 [n_cta, group, 4 warps, 2],
                  // f32 [total, n_hq, 1, 2]
+  float* dkv;    // bf16: dK and dV partials [2 halves][2 (dk, dv)][total, n_hkv, dh] fp32
 };
+// With at most kSplitMaxUnits (key tile, KV head, sequence) units the grid is one
+// wave and the longest units set the time: each is then split between kKvSplit CTAs
+// (halves of its items) that write fp32 partials, summed by the reduction. With more
+// units they run whole and write dK and dV directly.
+constexpr int kKvSplit = 2;
+constexpr int kSplitMaxUnits = 128;
+inline int kv_split(int64_t units) { return units <= kSplitMaxUnits ? kKvSplit : 1; }
 
 // D_i = dO_i . O_i and lse2 = lse * log2(e); one warp per (row, head)
 template <typename T>
@@ -343,14 +351,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const float* __restrict__ s_kept, const float* __restrict__ gain,
                     const float* __restrict__ tau, const int32_t* __restrict__ cu_kept, int total,
                     int max_kept, int n_hq, int n_hkv, const float* __restrict__ D,
-                    const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dk,
-                    __nv_bfloat16* __restrict__ dv, float* __restrict__ ds_part,
+                    const float* __restrict__ lse2, int batch, int nsplit,
+                    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    float* __restrict__ dkv_part, float* __restrict__ ds_part,
                     float* __restrict__ gt_part, int* status) {
-  const int jt = blockIdx.x;   // key tile: tile 0 meets the most query tiles, it starts first
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
+  // blockIdx.x = ((jt * batch + b) * n_hkv + kvh) * nsplit + half: key tile 0, which
+  // meets the most query tiles, for every sequence and head first (longest first)
+  const int cta = blockIdx.x;
+  const int half = cta % nsplit;
+  const int kvh = (cta / nsplit) % n_hkv;
+  const int b = (cta / nsplit / n_hkv) % batch;
+  const int jt = cta / nsplit / n_hkv / batch;
   const int G = n_hq / n_hkv;
-  const int cta = (b * n_hkv + kvh) * static_cast<int>(gridDim.x) + jt;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   DkvSmem& S = *reinterpret_cast<DkvSmem*>(smem_raw + pad);
@@ -390,14 +402,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
   if (bad && kvh == 0 && jt == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
   const int len = bad ? 0 : seq1 - seq0;
-  if (jt * kBN >= len) {   // no key of this tile: zero partials (the reduction reads them all)
-    for (int e = tid; e < G * 4 * 2; e += kBwdThreads) gt_part[static_cast<int64_t>(cta) * G * 8 + e] = 0.f;
+  // the reduction reads every gain/temperature slot of every CTA: start at zero
+  for (int e = tid; e < G * 4 * 2; e += kBwdThreads) gt_part[static_cast<int64_t>(cta) * G * 8 + e] = 0.f;
+  if (jt * kBN >= len) {   // no key of this tile
     if (warp == 7) tg::tmem_dealloc(tmem, 512);
     return;
   }
   const int n_qt = (len + kBM - 1) / kBM;
   const int per_head = n_qt - jt;   // query tiles jt..n_qt-1
-  const int n_items = G * per_head;   // (head, query tile) pairs, head-major
+  const int n_all = G * per_head;   // (head, query tile) items of the unit, head-major
+  const int it0 = n_all * half / nsplit, it1 = n_all * (half + 1) / nsplit;
+  const int n_items = it1 - it0;    // this CTA's items it0 .. it1-1 (local index it - it0)
+  // split units: this half's dK and dV partials, fp32 [total, n_hkv, dh] each
+  float* const dk_part = dkv_part + static_cast<int64_t>(half * 2) * total * n_hkv * kD;
+  float* const dv_part = dkv_part + static_cast<int64_t>(half * 2 + 1) * total * n_hkv * kD;
+  __syncthreads();   // the slots are zero before any warp writes its own
+  if (n_items == 0) {   // nothing to add: zero partials for this tile's keys
+    if (warp < 4) {
+      const int krow = jt * kBN + warp * 32 + lane;
+      if (krow < len) {
+        const int64_t o = (static_cast<int64_t>(seq0 + krow) * n_hkv + kvh) * kD;
+        for (int d = 0; d < kD; d += 4) {
+          *reinterpret_cast<float4*>(dk_part + o + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(dv_part + o + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        ds_part[(static_cast<int64_t>(half) * n_hkv + kvh) * total + seq0 + krow] = 0.f;
+      }
+    }
+    if (warp == 7) tg::tmem_dealloc(tmem, 512);
+    return;
+  }
 
   if (warp == 4) {
     // ---- TMA: K_j and V_j once, then the (Q_i, dO_i) ring ----
@@ -410,7 +444,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int it = 0;
       for (; it < n_items; ++it) {
         const int st = it & 1;
-        const int h = kvh * G + it / per_head, i = jt + it % per_head;
+        const int h = kvh * G + (it0 + it) / per_head, i = jt + (it0 + it) % per_head;
         if (it >= 2 && !tg::mbar_wait(&S.qd_empty[st], ((it >> 1) - 1) & 1, status, &S.abort_flag)) break;
         tg::mbar_arrive_expect_tx(&S.qd_full[st], 2 * kBM * kD * 2);
         for (int hh = 0; hh < 2; ++hh) {
@@ -471,7 +505,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ---- each item's query rows: lse2 and D (plain loads; row offsets are arbitrary) ----
     for (int it = 0; it < n_items; ++it) {
       const int st = it & 1;
-      const int h = kvh * G + it / per_head, i = jt + it % per_head;
+      const int h = kvh * G + (it0 + it) / per_head, i = jt + (it0 + it) % per_head;
       if (it >= 2 && !__all_sync(0xFFFFFFFFu, tg::mbar_wait(&S.ld_empty[st], ((it >> 1) - 1) & 1,
                                                             status, &S.abort_flag)))
         break;
@@ -496,7 +530,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool alive = true;
     for (int it = 0; it < n_items; ++it) {
       const int st = it & 1;
-      const int hl = it / per_head, h = kvh * G + hl, i = jt + it % per_head;
+      const int hl = (it0 + it) / per_head, h = kvh * G + hl, i = jt + (it0 + it) % per_head;
       const float th = tau[h];
       const float c = 1.f / (sqrtf(static_cast<float>(kD)) * th);
       const float c2 = c * kLog2e;
@@ -543,10 +577,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tg::mbar_arrive(&S.pd_full);
         tg::mbar_arrive(&S.ld_empty[st]);
       }
-      if (it % per_head == per_head - 1) {
-        // this head is done: its score-gradient share, and this warp's gain and
-        // temperature partials for it (summed over the CTA's warps by the reduction,
-        // so no barrier between the warps is needed here)
+      if ((it0 + it) % per_head == per_head - 1 || it == n_items - 1) {
+        // this head's items in this CTA are done: its score-gradient share, and this
+        // warp's gain and temperature partials for it (summed over the CTA's warps and
+        // the unit's two CTAs by the reduction, so no barrier between warps is needed)
         ds_acc = fmaf(gain[h], dz_h, ds_acc);
         float gsum = dz_h * sk, tsum = tz_h;
         for (int off = 16; off > 0; off >>= 1) {
@@ -562,28 +596,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tz_h = 0.f;
       }
     }
-    if (kvalid && alive) ds_part[static_cast<int64_t>(kvh) * total + seq0 + krow] = ds_acc;
+    if (kvalid && alive) ds_part[(static_cast<int64_t>(half) * n_hkv + kvh) * total + seq0 + krow] = ds_acc;
     if (alive) alive = tg::mbar_wait(&S.acc_done, 0, status, &S.abort_flag);
     if (__all_sync(0xFFFFFFFFu, alive)) {
       tg::tc_fence_after();
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t aa = tmem_lane_addr(tmem, warp, which ? kColDK : kColDV);
-        __nv_bfloat16* dst_base = which ? dk : dv;
+        float* dst_base = which ? dk_part : dv_part;
+        __nv_bfloat16* out_base = which ? dk : dv;
 #pragma unroll 1
         for (int ch = 0; ch < kD / 32; ++ch) {
           uint32_t a[32];
           tg::tmem_ld32(aa + 32 * ch, a);
           tg::tmem_ld_wait();
-          if (kvalid) {
+          if (kvalid && nsplit == 1) {   // the whole unit: dK, dV rows in bf16
             uint4* dst = reinterpret_cast<uint4*>(
-                dst_base + (static_cast<int64_t>(seq0 + krow) * n_hkv + kvh) * kD + 32 * ch);
+                out_base + (static_cast<int64_t>(seq0 + krow) * n_hkv + kvh) * kD + 32 * ch);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               dst[u] = make_uint4(tg::pack_bf16x2(__uint_as_float(a[8 * u]), __uint_as_float(a[8 * u + 1])),
                                   tg::pack_bf16x2(__uint_as_float(a[8 * u + 2]), __uint_as_float(a[8 * u + 3])),
                                   tg::pack_bf16x2(__uint_as_float(a[8 * u + 4]), __uint_as_float(a[8 * u + 5])),
                                   tg::pack_bf16x2(__uint_as_float(a[8 * u + 6]), __uint_as_float(a[8 * u + 7])));
+          } else if (kvalid) {
+            float4* dst = reinterpret_cast<float4*>(
+                dst_base + (static_cast<int64_t>(seq0 + krow) * n_hkv + kvh) * kD + 32 * ch);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              dst[u] = make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
+                                   __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3]));
           }
         }
       }
@@ -775,6 +817,48 @@ __global__ void __launch_bounds__(256)
   ds[j] = a;
 }
 
+// bf16 path: for each key row of a valid sequence, ds = the sum over halves and KV
+// heads of the shares and, for split units, dK and dV = half 0 + half 1 of the
+// partials, in that fixed order. Rows of a sequence that failed the device check are
+// left alone (their partials were never written). One warp per key row.
+__global__ void __launch_bounds__(256)
+    bwd_reduce_dkv_ds_kernel(const float* __restrict__ dkv_part, const float* __restrict__ ds_part,
+                             const int32_t* __restrict__ cu_kept, int batch, int64_t total,
+                             int max_kept, int n_hkv, int nsplit, __nv_bfloat16* __restrict__ dk,
+                             __nv_bfloat16* __restrict__ dv, float* __restrict__ ds) {
+  tg::pdl_launch_dependents();
+  tg::pdl_wait();
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= total) return;
+  int lo = 0, hi = batch;   // the sequence holding row j: cu_kept[b] <= j < cu_kept[b + 1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if (cu_kept[mid] <= j) lo = mid;
+    else hi = mid;
+  }
+  const int64_t s0 = cu_kept[lo], s1 = cu_kept[lo + 1];
+  if (s0 < 0 || s1 < s0 || s1 > total || s1 - s0 > max_kept || j < s0 || j >= s1) return;
+  const int64_t plane = total * n_hkv * kD;
+  for (int kv = 0; kv < (nsplit > 1 ? n_hkv : 0); ++kv) {
+    const int64_t o = (j * n_hkv + kv) * kD + 4 * lane;
+    const float4 k0 = *reinterpret_cast<const float4*>(dkv_part + o);
+    const float4 v0 = *reinterpret_cast<const float4*>(dkv_part + plane + o);
+    const float4 k1 = *reinterpret_cast<const float4*>(dkv_part + 2 * plane + o);
+    const float4 v1 = *reinterpret_cast<const float4*>(dkv_part + 3 * plane + o);
+    *reinterpret_cast<uint2*>(dk + o) =
+        make_uint2(tg::pack_bf16x2(k0.x + k1.x, k0.y + k1.y), tg::pack_bf16x2(k0.z + k1.z, k0.w + k1.w));
+    *reinterpret_cast<uint2*>(dv + o) =
+        make_uint2(tg::pack_bf16x2(v0.x + v1.x, v0.y + v1.y), tg::pack_bf16x2(v0.z + v1.z, v0.w + v1.w));
+  }
+  if (lane == 0) {
+    float a = 0.f;
+    for (int h2 = 0; h2 < nsplit; ++h2)
+      for (int kv = 0; kv < n_hkv; ++kv) a += ds_part[(static_cast<int64_t>(h2) * n_hkv + kv) * total + j];
+    ds[j] = a;
+  }
+}
+
 // one block per query head: dg_h and dtau_h summed over the partials in a fixed
 // order. Partials are [n_units][unit_heads][W][2]: bf16, a unit is a dK/dV CTA
 // (b, kvh, key tile), its heads are the group's and W = 4 (one per elementwise
@@ -831,17 +915,20 @@ size_t ws_bytes(int batch, int64_t total, int max_kept, int n_hq, int n_hkv, int
   // partials: bf16 per CTA and group head, f32 per key and head
   const int n_kt = (max_kept + kBN - 1) / kBN;
   const int G = n_hkv > 0 ? n_hq / n_hkv : 0;
-  const int64_t gt = dt == TG_BF16 ? static_cast<int64_t>(n_kt) * n_hkv * batch * G * 4 * 2
-                                   : total * n_hq * 2;
-  const int64_t floats[4] = {n_hq * total, n_hq * total, n_hkv * total, gt};
+  const bool bf = dt == TG_BF16;
+  const int ns = bf ? kv_split(static_cast<int64_t>(n_kt) * batch * n_hkv) : 1;
+  const int64_t gt = bf ? static_cast<int64_t>(n_kt) * ns * n_hkv * batch * G * 4 * 2
+                        : total * n_hq * 2;
+  const int64_t floats[5] = {n_hq * total, n_hq * total, ns * n_hkv * total, gt,
+                             ns > 1 ? static_cast<int64_t>(ns) * 2 * total * n_hkv * kD : 0};
   size_t off = 0;
-  float* ptrs[4];
-  for (int i = 0; i < 4; ++i) {
+  float* ptrs[5];
+  for (int i = 0; i < 5; ++i) {
     ptrs[i] = base ? reinterpret_cast<float*>(base + off) : nullptr;
     off += (static_cast<size_t>(floats[i]) * 4 + 255) / 256 * 256;
   }
   (void)head_dim;
-  if (ws) *ws = BwdWs{ptrs[0], ptrs[1], ptrs[2], ptrs[3]};
+  if (ws) *ws = BwdWs{ptrs[0], ptrs[1], ptrs[2], ptrs[3], ptrs[4]};
   return off;
 }
 
@@ -917,19 +1004,26 @@ extern "C" tg_status tg_gated_attention_bwd(
                    n_hq, n_hkv, static_cast<const float*>(ws.D), static_cast<const float*>(ws.lse2),
                    static_cast<__nv_bfloat16*>(dq), st);
     if (r != TG_OK) return r;
-    r = tg::launch(bwd_dkdv_kernel, dim3(n_t, n_hkv, batch), dim3(kBwdThreads), smem_kv, stream, 0,
-                   tq, tk, tv, tdo, s_kept, gain, tau, cu_kept, static_cast<int>(total_kept),
-                   max_kept, n_hq, n_hkv, static_cast<const float*>(ws.D),
-                   static_cast<const float*>(ws.lse2), static_cast<__nv_bfloat16*>(dk),
-                   static_cast<__nv_bfloat16*>(dv), ws.ds, ws.gt, st);
+    const int64_t units = static_cast<int64_t>(n_t) * batch * n_hkv;
+    const int nsplit = kv_split(units);
+    const int64_t kv_ctas = units * nsplit;
+    if (kv_ctas > INT32_MAX) return TG_ERR_UNSUPPORTED;
+    r = tg::launch(bwd_dkdv_kernel, dim3(static_cast<unsigned>(kv_ctas)), dim3(kBwdThreads), smem_kv,
+                   stream, 0, tq, tk, tv, tdo, s_kept, gain, tau, cu_kept,
+                   static_cast<int>(total_kept), max_kept, n_hq, n_hkv,
+                   static_cast<const float*>(ws.D), static_cast<const float*>(ws.lse2), batch,
+                   nsplit, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), ws.dkv,
+                   ws.ds, ws.gt, st);
     if (r != TG_OK) return r;
-    r = tg::launch(bwd_reduce_ds_kernel, dim3(static_cast<unsigned>((total_kept + 255) / 256)),
-                   dim3(256), 0, stream, 0, static_cast<const float*>(ws.ds), total_kept, n_hkv, ds);
+    r = tg::launch(bwd_reduce_dkv_ds_kernel, dim3(static_cast<unsigned>((total_kept + 7) / 8)),
+                   dim3(256), 0, stream, 0, static_cast<const float*>(ws.dkv),
+                   static_cast<const float*>(ws.ds), cu_kept, batch, total_kept, max_kept, n_hkv,
+                   nsplit, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), ds);
     if (r != TG_OK) return r;
-    // CTA units (b, kvh, jt): units_per_group = n_t (consecutive jt share a KV head)
+    // CTA units ((jt, b, kvh), half): units_per_group = nsplit (a unit's CTAs share a KV head)
     return tg::launch(bwd_reduce_gt_kernel, dim3(n_hq), dim3(256), 0, stream, 0,
-                      static_cast<const float*>(ws.gt),
-                      static_cast<int64_t>(n_t) * n_hkv * batch, G, 4, n_t, n_hq, G, dgain, dtau);
+                      static_cast<const float*>(ws.gt), kv_ctas, G, 4, nsplit, n_hq, G, dgain,
+                      dtau);
   }
   // f32
   r = tg::launch(bwd_prep_kernel<float>, dim3(static_cast<unsigned>(prep_blocks)), dim3(256), 0,

@@ -94,8 +94,11 @@ def test_backward_f32_tiny_config(api, orc):
         assert err <= 1e-4 * max(1.0, np.abs(w).max()), f"{name}: {err:.3e}"
 
 
+# up to 128 (key tile, KV head, sequence) units each unit's items are split between
+# two CTAs whose fp32 partials are summed afterwards; the last case has 240 units,
+# which run whole
 @pytest.mark.parametrize("lens,hq,hkv", [([128], 4, 2), ([300], 4, 2), ([513, 1, 129], 4, 2),
-                                         ([260], 8, 2), ([250], 3, 3)])
+                                         ([260], 8, 2), ([250], 3, 3), ([600] * 12, 8, 4)])
 def test_backward_bf16_vs_oracle(api, orc, lens, hq, hkv):
     args = _case(sum(lens) * 7 + hq, lens, hq, hkv, 128, torch.bfloat16)
     got = _run(api, *args)
