@@ -127,3 +127,21 @@ def test_backward_bf16_16k_shape_properties(api):
     for kvh in range(8):
         want = do[:, [2 * kvh, 2 * kvh + 1]].sum(axis=(0, 1))
         np.testing.assert_allclose(dv[:, kvh].sum(0), want, rtol=2e-2, atol=0.5)
+
+
+def test_backward_bf16_128k_shape_properties(api):
+    # the 128k layer's attention shape (K = 10721, 16/8 heads; 672 units, run whole):
+    # the score gradients sum to zero, and with all values equal only dv is non-zero
+    args = list(_case(6, [10721], 16, 8, 128, torch.bfloat16))
+    dq, dk, dv, ds, dg, dt = _run(api, *args)
+    assert abs(ds.sum()) <= 1e-3 * np.abs(ds).sum()
+    for a in (dq, dk, dv):
+        assert np.isfinite(a).all()
+    args[2] = torch.full_like(args[2], 0.5)
+    dq, dk, dv, ds, dg, dt = _run(api, *args)
+    for name, a in zip(["dq", "dk", "ds", "dgain", "dtau"], (dq, dk, ds, dg, dt)):
+        assert np.abs(a).max() <= 2e-3, name
+    do = args[3].double().numpy()
+    for kvh in range(8):
+        want = do[:, [2 * kvh, 2 * kvh + 1]].sum(axis=(0, 1))
+        np.testing.assert_allclose(dv[:, kvh].sum(0), want, rtol=2e-2, atol=1.0)

@@ -135,3 +135,37 @@ def test_decode_of_last_kept_token_matches_prefill_row(api, orc):
     assert_attn_close(out, ref, torch.bfloat16, what="decode of the last kept token")
     diff = (out[0].float() - gp.out[K - 1].float()).abs().max().item()
     assert diff <= 2e-2, diff    # two bf16 results of the same row, each within 1e-2
+
+
+@pytest.mark.parametrize("name", ["long128k", "ragged8"])
+def test_decode_step_on_the_benchmark_caches(api, orc, name):
+    # the decode step the benchmark times on its other layers: each sequence's kept
+    # rows (k, v, scores of the measured prefill) are its cache, capacity K_b + 64;
+    # one new token per sequence is appended and attends over the grown cache
+    from learned_token_pruning_gemm_b200 import pipeline, synth
+    wl = synth.WORKLOADS[name]()
+    gp = pipeline.GatedPrefill(wl)
+    gp.step()
+    torch.cuda.synchronize()
+    counts = wl.kept_counts
+    B, cap = wl.batch, max(counts) + 64
+    kc = torch.zeros(B, cap, wl.hkv, wl.dh, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    sc = torch.zeros(B, cap, device="cuda")
+    cu = gp.cu_kept.cpu().tolist()
+    for b in range(B):
+        kc[b, :counts[b]] = gp.k[cu[b]:cu[b + 1]]
+        vc[b, :counts[b]] = gp.v[cu[b]:cu[b + 1]]
+        sc[b, :counts[b]] = gp.kept_scores[cu[b]:cu[b + 1]]
+    g = torch.Generator().manual_seed(3)
+    qn = torch.randn(B, wl.hq, wl.dh, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, wl.hkv, wl.dh, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, wl.hkv, wl.dh, generator=g).to(torch.bfloat16)
+    sn = torch.randn(B, generator=g)
+    ln = torch.tensor(counts, dtype=torch.int32, device="cuda")
+    api.cache_append(kn.cuda(), vn.cuda(), sn.cuda(), kc, vc, sc, ln)
+    out = api.gated_decode(qn.cuda(), kc, vc, sc, ln, gp.gain, gp.tau, cap)
+    torch.cuda.synchronize()
+    assert ln.cpu().tolist() == [c + 1 for c in counts]
+    ref = orc.gated_decode(qn, kc.cpu(), vc.cpu(), sc.cpu(), [c + 1 for c in counts], wl.gain, wl.tau)
+    assert_attn_close(out, ref, torch.bfloat16, what=f"decode step on {name}")

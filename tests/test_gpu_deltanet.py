@@ -96,3 +96,29 @@ def test_delta_rule_sequence_longer_than_max_seqlen_is_reported(api):
     o = out.float().cpu()
     assert torch.all(o[:70] == 7.0)                     # the 70-row sequence is skipped
     assert not torch.all(o[70:] == 7.0)                 # the 40-row one is computed
+
+
+def test_delta_rule_on_the_128k_layers_kept_rows(api, orc):
+    # the 128k layer's 10721 kept rows (168 chunks of 64 in one sequence), sampled heads
+    from learned_token_pruning_gemm_b200 import synth
+    wl = synth.long128k()
+    q, k, v, a, b = synth.deltanet_inputs(wl)
+    cu = np.array([0, wl.total_kept], np.int32)
+    out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                               torch.tensor(cu, device="cuda"), wl.total_kept)
+    heads = [0, 9]
+    ref = orc.gated_delta_rule(q[:, heads], k[:, heads], v[:, heads], a[:, heads], b[:, heads], cu)
+    assert_attn_close(out[:, heads].contiguous(), ref, torch.bfloat16, what="128k kept rows")
+
+
+def test_delta_rule_on_the_ragged_layers_kept_rows(api, orc):
+    # the ragged layer's 8 sequences of kept rows (1385 to 3493 each), sampled heads
+    from learned_token_pruning_gemm_b200 import synth
+    wl = synth.ragged8()
+    q, k, v, a, b = synth.deltanet_inputs(wl)
+    cu = np.r_[0, np.cumsum(wl.kept_counts)].astype(np.int32)
+    out = api.gated_delta_rule(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(),
+                               torch.tensor(cu, device="cuda"), max(wl.kept_counts))
+    heads = [3, 12]
+    ref = orc.gated_delta_rule(q[:, heads], k[:, heads], v[:, heads], a[:, heads], b[:, heads], cu)
+    assert_attn_close(out[:, heads].contiguous(), ref, torch.bfloat16, what="ragged kept rows")
