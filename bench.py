@@ -104,7 +104,7 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside), "sampled_over": where}
 
 
-def _work(wl):
+def _algorithmic_work(wl):
     """Algorithmic work of one step (bytes / flops the method must move / do)."""
     N, d, h, dh, hq = wl.n_tokens, wl.d, wl.h, wl.dh, wl.hq
     esz = 2 if wl.dtype == "bf16" else 4
@@ -418,7 +418,7 @@ def _time_backward(gp, wl, steps, warmup, rep, flush, stream, tf_peak):
     if api.device_status(reset=True) != 0:
         raise RuntimeError("device status set by the backward")
     ms = rep.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
-    flops = 2.5 * _work(wl)["attn_flops"]
+    flops = 2.5 * _algorithmic_work(wl)["attn_flops"]
     return {"us": ms * 1e3, "tflops": flops / (ms / 1e3) / 1e12,
             "frac_tc": flops / (ms / 1e3) / 1e12 / tf_peak, "launches_per_step": 5,
             "note": "dQ, dK, dV, score, gain and temperature gradients; flops = 2.5 x the "
@@ -496,7 +496,7 @@ def run_ours(args, rep):
 
     wl = synth.WORKLOADS[args.workload]()
     gp = pipeline.GatedPrefill(wl)
-    work = _work(wl)
+    work = _algorithmic_work(wl)
     clocks = ClockSampler(dev_index)
     clocks.start()
     ms, stage_ms, clk = _time_layer(gp, args.steps, args.warmup, rep, flush, stream, clocks)
@@ -538,7 +538,7 @@ def run_ours(args, rep):
             continue
         owl = synth.WORKLOADS[name]()
         ogp = pipeline.GatedPrefill(owl)
-        owork = _work(owl)
+        owork = _algorithmic_work(owl)
         oms, ostage, _ = _time_layer(ogp, args.steps, args.warmup, rep, flush, stream)
         others[name] = {
             "value": ws * owl.n_tokens / (oms / 1e3), "unit": "tokens/s", "ms_per_step": oms,
