@@ -39,6 +39,12 @@
 // Because P_j lives in S_j's buffer, softmax(j+1) runs while the tensor core does
 // PV_j and S_{j+3}; the only cross-tile waits are the rare O rescale and, between
 // the two query tiles, the epilogue's read of O before it is overwritten.
+// P_j is reported on p_full[j % 3] and PV_j completes on o_done[j % 3]. Softmax
+// warps run up to two tiles apart, each bounded by what it has seen: a warp that
+// has seen S_j knows PV_{j-3} complete (S_j was issued after it), hence phase j-3 of
+// p_full[j % 3] too, so its arrival for tile j counts toward tile j; and PV_{j+1}
+// cannot start before the warp's own P_{j+1}, so at tile j the barrier that holds
+// PV_{j-1} is at most one phase short of it and a parity wait on it is exact.
 //
 // f32 path: exact fp32 SIMT kernel (one warp per query row and head).
 #include "common.cuh"
@@ -64,19 +70,6 @@ constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
 constexpr float kExp2C3 = 0.0551716685295105f;
 
-// exp2 on the FMA pipe: n = rint(x) via the 1.5*2^23 shift, 2^f by the polynomial,
-// 2^n added to the exponent field. Inputs below -125 return ~2^-125 (P is bf16;
-// such a weight is zero for every purpose here); inputs are <= 8 by construction.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  const int ni = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (ni << 23));
-}
-
 struct AttnSmem {
   uint8_t q[2][kBM * 64 * 2];               // Q tile as two 64-column halves (16 KB each)
   uint8_t k[kKStages][2][kBN * 64 * 2];
@@ -91,8 +84,8 @@ struct AttnSmem {
   uint64_t v_full[kVStages];
   uint64_t v_empty[kVStages];
   uint64_t s_full[kSBufs];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t p_full[kSBufs];                  // P_g stored by every softmax warp, on p_full[g % kSBufs]
+  uint64_t o_done[kSBufs];                  // PV_g complete, on o_done[g % kSBufs]
   uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
   uint32_t tmem_base;
   int abort_flag;
@@ -120,10 +113,45 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
-// the two bf16 halves of a packed pair, widened exactly to fp32
-__device__ __forceinline__ float bf16x2_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16x2_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-
+__device__ __forceinline__ void fsub2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// exp2 on the FMA pipe, two lanes at once (packed f32x2 additions and FMAs):
+// n = rint(x) via the 1.5*2^23 shift, 2^f by the polynomial, 2^n added to the
+// exponent field as t << 23 (t = x + 1.5*2^23 holds n in its low mantissa bits;
+// the shift's own bits, 0x4B400000, have nine zero low bits and vanish modulo
+// 2^32). Inputs below -125 return ~2^-125 (P is bf16; such a weight is zero for
+// every purpose here); inputs are <= 8 by construction.
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0, t1, x0, x1, 12582912.0f, 12582912.0f);
+  fsub2(n0, n1, t0, t1, 12582912.0f, 12582912.0f);
+  fsub2(f0, f1, x0, x1, n0, n1);
+  ffma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+  ffma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+  ffma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+// acc += the low (lo) or high (hi) bf16 half of a packed pair, widened exactly
+// (one mixed-precision add; the same value and rounding as an fp32 add)
+__device__ __forceinline__ void add_bf16_lo(float& acc, uint32_t u) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, l, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(u));
+}
+__device__ __forceinline__ void add_bf16_hi(float& acc, uint32_t u) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(u));
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -180,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mbar_init(&S.v_empty[s], 1);
     }
     for (int s = 0; s < kSBufs; ++s) tg::mbar_init(&S.s_full[s], 1);
-    tg::mbar_init(&S.p_full, kSoftmaxWarps);
-    tg::mbar_init(&S.o_done, 1);
+    for (int s = 0; s < kSBufs; ++s) tg::mbar_init(&S.p_full[s], kSoftmaxWarps);
+    for (int s = 0; s < kSBufs; ++s) tg::mbar_init(&S.o_done[s], 1);
     tg::mbar_init(&S.o_free, kSoftmaxWarps);
     S.abort_flag = 0;
     tg::fence_barrier_init();
@@ -339,7 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (alive && nt <= kSBufs) tg::mma_commit(&S.q_empty);   // every S of the tile issued
         for (int j = 0; j < nt && alive; ++j) {
           const int g = g0 + j;
-          if (!tg::mbar_wait(&S.p_full, g & 1, status, &S.abort_flag)) { alive = false; break; }
+          if (!tg::mbar_wait(&S.p_full[g % kSBufs], (g / kSBufs) & 1, status, &S.abort_flag)) {
+            alive = false;
+            break;
+          }
           const int s = g % kVStages;
           if (!tg::mbar_wait(&S.v_full[s], (g / kVStages) & 1, status, &S.abort_flag)) {
             alive = false;
@@ -361,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tg::mma_bf16_ts(tmem + kColO, tmem + kColS0 + 128u * (g % kSBufs) + kk * 8, bdesc,
                             idesc_o, (j | kk) != 0);
           }
-          tg::mma_commit(&S.o_done);
+          tg::mma_commit(&S.o_done[g % kSBufs]);
           tg::mma_commit(&S.v_empty[s]);
           // S_{g+3} goes into the buffer that held P_g (PV_g is ahead of it in the pipe)
           if (j + kSBufs < nt) {
@@ -465,27 +496,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sa[2] = {0.f, 0.f}, sb[2] = {0.f, 0.f};
         const float nma = -ma, nmb = -mb;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1, x2, x3;
-          fadd2(x0, x1, z[4 * i], z[4 * i + 1], nma, nma);
-          fadd2(x2, x3, z[4 * i + 2], z[4 * i + 3], nmb, nmb);
-          const float p0 = exp2_fma(x0);   // one key in four on the FMA pipe
-          const float p1 = tg::exp2_approx(x1);
-          const float p2 = tg::exp2_approx(x2);
-          const float p3 = tg::exp2_approx(x3);
-          pk[2 * i] = tg::pack_bf16x2(p0, p1);       // row ra, packed column 4i + l%4
-          pk[2 * i + 1] = tg::pack_bf16x2(p2, p3);   // row rb, the same column
-          // the row sums add the bf16 weights that the PV MMA multiplies: numerator
-          // and denominator then carry the same rounding, so a key that dominates
-          // its row contributes its v exactly, whatever weight the lagging max left it
-          fadd2(sa[0], sa[1], sa[0], sa[1], bf16x2_lo(pk[2 * i]), bf16x2_hi(pk[2 * i]));
-          fadd2(sb[0], sb[1], sb[0], sb[1], bf16x2_lo(pk[2 * i + 1]), bf16x2_hi(pk[2 * i + 1]));
+        for (int i = 0; i < 16; i += 2) {
+          float x[8];
+          fadd2(x[0], x[1], z[4 * i], z[4 * i + 1], nma, nma);
+          fadd2(x[2], x[3], z[4 * i + 2], z[4 * i + 3], nmb, nmb);
+          fadd2(x[4], x[5], z[4 * i + 4], z[4 * i + 5], nma, nma);
+          fadd2(x[6], x[7], z[4 * i + 6], z[4 * i + 7], nmb, nmb);
+          float q0, q4;
+          exp2_fma2(q0, q4, x[0], x[4]);   // one key in four on the FMA pipe, two at a time
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int ii = i + h;
+            const float p0 = h == 0 ? q0 : q4;
+            const float p1 = tg::exp2_approx(x[4 * h + 1]);
+            const float p2 = tg::exp2_approx(x[4 * h + 2]);
+            const float p3 = tg::exp2_approx(x[4 * h + 3]);
+            pk[2 * ii] = tg::pack_bf16x2(p0, p1);       // row ra, packed column 4i + l%4
+            pk[2 * ii + 1] = tg::pack_bf16x2(p2, p3);   // row rb, the same column
+            // the row sums add the bf16 weights that the PV MMA multiplies: numerator
+            // and denominator then carry the same rounding, so a key that dominates
+            // its row contributes its v exactly, whatever weight the lagging max left it
+            add_bf16_lo(sa[0], pk[2 * ii]);
+            add_bf16_hi(sa[1], pk[2 * ii]);
+            add_bf16_lo(sb[0], pk[2 * ii + 1]);
+            add_bf16_hi(sb[1], pk[2 * ii + 1]);
+          }
         }
         la = la * alpha_a + (sa[0] + sa[1]);
         lb = lb * alpha_b + (sb[0] + sb[1]);
         if (__any_sync(0xFFFFFFFFu, rescale)) {
-          // O must hold PV_{g-1} before it is scaled (phases <= g-2 are confirmed)
-          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
+          // O must hold PV_{g-1} before it is scaled
+          alive = tg::mbar_wait(&S.o_done[(g - 1) % kSBufs], ((g - 1) / kSBufs) & 1, status,
+                                &S.abort_flag);
           if (!all_alive(alive)) { alive = false; break; }
           tg::tc_fence_after();
 #pragma unroll
@@ -507,14 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P_g over S_g: packed bf16 pairs, 64 columns (every S read of these rows is done)
         tg::tmem_st_16x128b_x16(sbuf, pk);
         tg::tmem_st_wait();
-        // confirm PV_{g-1} (keeps the o_done phase tracking exact; normally complete)
-        if (j > 0) {
-          alive = tg::mbar_wait(&S.o_done, (g - 1) & 1, status, &S.abort_flag);
-          if (!all_alive(alive)) { alive = false; break; }
-        }
         tg::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tg::mbar_arrive(&S.p_full);
+        if (lane == 0) tg::mbar_arrive(&S.p_full[g % kSBufs]);
       }
       if (!alive) break;
       // ---------------- epilogue of this query tile: O / l -> bf16 ----------------
@@ -523,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       la += __shfl_xor_sync(0xFFFFFFFFu, la, 2);
       lb += __shfl_xor_sync(0xFFFFFFFFu, lb, 2);
       const int g_last = g0 + nt - 1;
-      alive = tg::mbar_wait(&S.o_done, g_last & 1, status, &S.abort_flag);
+      alive = tg::mbar_wait(&S.o_done[g_last % kSBufs], (g_last / kSBufs) & 1, status,
+                            &S.abort_flag);
       if (!all_alive(alive)) { alive = false; break; }
       tg::tc_fence_after();
       uint32_t o[64];

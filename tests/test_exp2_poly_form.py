@@ -42,8 +42,12 @@ def _exp2_fma_fp32(x):
     p = (c3 * fr + c2).astype(np.float32)     # fmaf rounds once; two roundings here are
     p = (p * fr + c1).astype(np.float32)      # within 2^-23 relative of it
     p = (p * fr + c0).astype(np.float32)
-    ni = t.view(np.int32) - np.int32(0x4B400000)
-    return (p.view(np.int32) + (ni << 23)).view(np.float32)
+    # n sits in t's low mantissa bits; shifting t's bits by 23 puts it in the
+    # exponent field (the shift constant's bits vanish modulo 2^32)
+    tb = t.view(np.uint32)
+    ni = tb.astype(np.int64) - 0x4B400000
+    assert np.array_equal((ni << 23) & 0xFFFFFFFF, (tb.astype(np.int64) << 23) & 0xFFFFFFFF)
+    return (p.view(np.uint32) + (tb << np.uint32(23))).view(np.float32)
 
 
 def test_fp32_sequence_matches_exp2():
