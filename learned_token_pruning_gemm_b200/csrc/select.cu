@@ -50,12 +50,8 @@ struct alignas(16) SelectSmem {
   uint32_t warp_eq_off[kWarps];
   uint32_t cta_eq;               // published to peers
   uint32_t cta_keep;             // published to peers
-  uint32_t peer_eq[kMaxCluster]; // every CTA's published counts, fetched once
-  uint32_t peer_keep[kMaxCluster];
   uint32_t digit;
   uint32_t remaining;
-  uint32_t cta_eq_off;
-  uint32_t cta_keep_off;
   uint32_t seq_keep;
   int64_t out_base;
   int64_t red[kWarps];
@@ -189,20 +185,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ld0 = clampl(db - c0), ld1 = clampl(de - c0);
   const uint32_t excl_local = (uint32_t)(chunk - (ld1 - ld0));   // keys forced to 0
 
-  // ---- load (8 loads in flight per thread) ----
-  for (int i0 = tid; i0 < chunk; i0 += 8 * kThreads) {
-    float v[8];
+  // ---- load: raw scores and keys into shared memory; when a radix select is
+  //      needed, the first pass's per-warp histograms (digit = key >> 24) are
+  //      filled on the way (16 loads in flight per thread) ----
+  const bool radix = k_eff > 0 && k_eff < nd;
+  {
+    uint32_t* wh = S.whist[warp];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads;
-      v[u] = i < n_local ? scores[base + c0 + i] : 0.f;
-    }
+    for (int i = lane; i < 256; i += 32) wh[i] = 0u;
+    __syncwarp();
+    for (int i0 = tid; i0 < chunk; i0 += 16 * kThreads) {
+      float v[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads;
-      if (i < chunk) {
-        raw[i] = v[u];
-        keys[i] = (i >= ld0 && i < ld1) ? score_key(v[u]) : 0u;
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = i < n_local ? scores[base + c0 + i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < chunk) {
+          const uint32_t key = (i >= ld0 && i < ld1) ? score_key(v[u]) : 0u;
+          raw[i] = v[u];
+          keys[i] = key;
+          if (radix) atomicAdd(&wh[key >> 24], 1u);
+        }
       }
     }
   }
@@ -218,27 +225,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (k_eff == 0) {
     T = 0xFFFFFFFFu;   // above every key (the largest key, +inf, is 0xFF800000)
     need = 0;
-  } else if (k_eff == nd) {
-    T = 0u;            // everything is kept
+  } else if (!radix) {
+    T = 0u;            // k_eff == nd: everything is kept
     need = (uint32_t)nd;
   } else {
     uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k_eff;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       uint32_t* h = S.hist[pass & 1];
-      uint32_t* wh = S.whist[warp];
+      if (pass > 0) {   // the first pass's histograms were filled by the load
+        uint32_t* wh = S.whist[warp];
 #pragma unroll
-      for (int i = lane; i < 256; i += 32) wh[i] = 0u;
-      __syncwarp();
-      for (int st = 0; st < nsteps; ++st) {
-        const uint4 kk = k4[st * 32 + lane];
+        for (int i = lane; i < 256; i += 32) wh[i] = 0u;
+        __syncwarp();
+        for (int st = 0; st < nsteps; ++st) {
+          const uint4 kk = k4[st * 32 + lane];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t key = key_at(kk, e);
-          if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t key = key_at(kk, e);
+            if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & 0xFFu], 1u);
+          }
         }
+        __syncthreads();
       }
-      __syncthreads();
       if (tid < 256) {
         uint32_t c = 0;
 #pragma unroll 8
@@ -306,51 +315,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       S.warp_base[warp] = cbase;
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t te = 0, tb = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        te += S.warp_tot[w];
-        tb += S.warp_base[w];
+    if (warp == 0) {   // this CTA's two counts, published to the peers
+      uint32_t te = lane < kWarps ? S.warp_tot[lane] : 0u;
+      uint32_t tb = lane < kWarps ? S.warp_base[lane] : 0u;
+      for (int o = 16; o > 0; o >>= 1) {
+        te += __shfl_xor_sync(full, te, o);
+        tb += __shfl_xor_sync(full, tb, o);
       }
-      S.cta_eq = te;
-      S.cta_keep = tb;   // published: this CTA's tie count and tie-independent count
+      if (lane == 0) {
+        S.cta_eq = te;
+        S.cta_keep = tb;
+      }
     }
     cluster.sync();
-    if (tid < static_cast<int>(csize)) {   // every peer's two counts, fetched in parallel
-      S.peer_eq[tid] = *cluster.map_shared_rank(&S.cta_eq, tid);
-      S.peer_keep[tid] = *cluster.map_shared_rank(&S.cta_keep, tid);
+    if (warp == 0) {
+      // Ties kept before a point = min(need, ties before it): from every CTA's and
+      // every warp's (tie, tie-independent) counts, exclusive scans in rank and warp
+      // order give each CTA's and warp's output offset. Lane r reads peer r.
+      const bool peer = lane < static_cast<int>(csize);
+      const uint32_t er = peer ? *cluster.map_shared_rank(&S.cta_eq, lane) : 0u;
+      const uint32_t br = peer ? *cluster.map_shared_rank(&S.cta_keep, lane) : 0u;
+      __syncwarp();   // reconverge before the shuffles (without it this block took ~3 us)
+      const uint32_t eq_before = warp_incl_scan(er, lane) - er;
+      const uint32_t kr = br + (need > eq_before ? min(need - eq_before, er) : 0u);
+      const uint32_t kr_incl = warp_incl_scan(kr, lane);
+      const uint32_t keep_total = __shfl_sync(full, kr_incl, 31);
+      const uint32_t cta_eq_off = __shfl_sync(full, eq_before, rank);
+      const uint32_t cta_keep_off = __shfl_sync(full, kr_incl - kr, rank);
+      const uint32_t ew = lane < kWarps ? S.warp_tot[lane] : 0u;
+      const uint32_t bw = lane < kWarps ? S.warp_base[lane] : 0u;
+      const uint32_t e_off = cta_eq_off + warp_incl_scan(ew, lane) - ew;
+      const uint32_t kw = bw + (need > e_off ? min(need - e_off, ew) : 0u);
+      const uint32_t k_off = cta_keep_off + warp_incl_scan(kw, lane) - kw;
+      if (lane < kWarps) {
+        S.warp_eq_off[lane] = e_off;
+        S.warp_off[lane] = k_off;
+      }
+      if (lane == 0) S.seq_keep = keep_total;
     }
     __syncthreads();
     // this CTA reads no peer's shared memory after this point: announce it now and
     // wait for the peers only before exiting, so the barrier overlaps pass 2
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    if (tid == 0) {
-      // ties kept before a point = min(need, ties before it); this gives every
-      // CTA's and every warp's output offset from (tie, tie-independent) counts
-      uint32_t eq_before = 0, keep_before = 0, keep_total = 0;
-      for (unsigned r = 0; r < csize; ++r) {
-        const uint32_t er = S.peer_eq[r];
-        const uint32_t br = S.peer_keep[r];
-        const uint32_t kr = br + (need > eq_before ? min(need - eq_before, er) : 0u);
-        if (r == rank) {
-          S.cta_eq_off = eq_before;
-          S.cta_keep_off = keep_before;
-        }
-        if (r < rank) keep_before += kr;
-        keep_total += kr;
-        eq_before += er;
-      }
-      S.seq_keep = keep_total;
-      uint32_t e_off = S.cta_eq_off, k_off = S.cta_keep_off;
-      for (int w = 0; w < kWarps; ++w) {
-        const uint32_t ew = S.warp_tot[w];
-        S.warp_eq_off[w] = e_off;
-        S.warp_off[w] = k_off;
-        k_off += S.warp_base[w] + (need > e_off ? min(need - e_off, ew) : 0u);
-        e_off += ew;
-      }
-    }
-    __syncthreads();
   }
 
   // ---- pass 2: keep decisions and output, ascending ----
@@ -363,12 +369,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < nsteps; ++st) {
       const uint4 kk = k4[st * 32 + lane];
       const int i4 = seg0 + st * 128 + lane * 4;
-      uint32_t ce = 0;
+      // per lane: ties (document keys == T) and tokens kept regardless of ties;
+      // one scan of both counts packed in 16-bit halves (each total <= 128)
+      uint32_t ce = 0, cb = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) ce += (i4 + e >= ld0 && i4 + e < ld1 && key_at(kk, e) == T);
-      const uint32_t incl_e = warp_incl_scan(ce, lane);
-      uint32_t rk = run_eq + incl_e - ce;
-      uint32_t nib = 0;
+      for (int e = 0; e < 4; ++e) {
+        const int i = i4 + e;
+        const bool in_doc = i >= ld0 && i < ld1;
+        const uint32_t key = key_at(kk, e);
+        ce += in_doc && key == T;
+        cb += i < n_local && (!in_doc || key > T);
+      }
+      const uint32_t packed = (ce << 16) | cb;
+      const uint32_t incl = warp_incl_scan(packed, lane);
+      const uint32_t tot = __shfl_sync(full, incl, 31);
+      const uint32_t ex_e = (incl >> 16) - ce, ex_b = (incl & 0xFFFFu) - cb;
+      // ties are kept in position order while fewer than `need` have been kept
+      uint32_t rk = run_eq + ex_e;
+      int64_t o = run_out + ex_b + (min(need, rk) - min(need, run_eq));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = i4 + e;
@@ -377,22 +395,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool eq = in_doc && key == T;
         const bool keep = i < n_local && (!in_doc || key > T || (eq && rk < need));
         rk += eq;
-        nib |= (uint32_t)keep << e;
-      }
-      const uint32_t c = __popc(nib);
-      const uint32_t incl_k = warp_incl_scan(c, lane);
-      int64_t o = run_out + incl_k - c;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if ((nib >> e) & 1u) {
-          kept_idx[o] = (int32_t)(base + c0 + i4 + e);
-          if (kept_scores) kept_scores[o] = raw[i4 + e];
-          if (kept_pos) kept_pos[o] = (int32_t)(c0 + i4 + e);
+        if (keep) {
+          kept_idx[o] = (int32_t)(base + c0 + i);
+          if (kept_scores) kept_scores[o] = raw[i];
+          if (kept_pos) kept_pos[o] = (int32_t)(c0 + i);
           ++o;
         }
       }
-      run_eq += __shfl_sync(full, incl_e, 31);
-      run_out += __shfl_sync(full, incl_k, 31);
+      const uint32_t te = tot >> 16, tb = tot & 0xFFFFu;
+      run_out += tb + (min(need, run_eq + te) - min(need, run_eq));
+      run_eq += te;
     }
   }
   if (!ok) {
