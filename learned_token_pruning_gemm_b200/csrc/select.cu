@@ -53,7 +53,6 @@ struct alignas(16) SelectSmem {
   uint32_t digit;
   uint32_t remaining;
   uint32_t seq_keep;
-  int64_t out_base;
   int64_t red[kWarps];
   // followed by: uint32_t keys[chunk]; float raw[chunk];
 };
@@ -128,27 +127,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const unsigned full = 0xFFFFFFFFu;
 
   // ---- output offset: the earlier sequences' kept counts (clamped the same way
-  //      for every sequence, so a rejected sequence still has a defined extent) ----
+  //      for every sequence, so a rejected sequence still has a defined extent).
+  //      Per-warp sums here; the block sum is read after the next block barrier,
+  //      so these loads overlap the score loads ----
   {
     int64_t acc = 0;
     for (int p = tid; p < b; p += kThreads) acc += seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, p);
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(full, acc, o);
     if (lane == 0) S.red[warp] = acc;
   }
-  __syncthreads();
-  if (tid == 0) {
+  auto block_out_base = [&]() {   // valid after a __syncthreads that follows the sums
     int64_t t = 0;
+#pragma unroll
     for (int w = 0; w < kWarps; ++w) t += S.red[w];
-    S.out_base = t;
-  }
-  __syncthreads();
-  const int64_t out_base = S.out_base;
+    return t;
+  };
 
   // Rejected sequence (or an inconsistent total found below): its output rows
   // get row id -1, score 0 and position -1, and cu_kept still advances by the
   // clamped count, clipped to total_kept, so the kernels that read these outputs
   // next see in-range offsets and an index the compaction rejects.
-  auto reject = [&](int64_t count) {
+  auto reject = [&](int64_t out_base, int64_t count) {
     const int64_t o0 = out_base < total_kept ? out_base : total_kept;
     const int64_t o1 = out_base + count < total_kept ? out_base + count : total_kept;
     for (int64_t r = o0 + (int64_t)rank * kThreads + tid; r < o1; r += (int64_t)csize * kThreads) {
@@ -170,7 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool bad = base < 0 || len < 0 || base + len > total_tokens ||
                    len > (int64_t)chunk * csize || db < 0 || de < db || de > len;
   if (bad) {
-    reject(seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, b));
+    __syncthreads();
+    reject(block_out_base(), seq_kept(cu_seqlens, doc_begin, doc_end, k_doc, b));
     return;   // uniform across the cluster: nobody reaches a cluster barrier
   }
   const int64_t nd = de - db;
@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
+  const int64_t out_base = block_out_base();
 
   const int seg = chunk / kWarps;                 // multiple of 128
   const int seg0 = warp * seg;
@@ -234,10 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int shift = 24 - 8 * pass;
       uint32_t* h = S.hist[pass & 1];
       if (pass > 0) {   // the first pass's histograms were filled by the load
-        uint32_t* wh = S.whist[warp];
-#pragma unroll
-        for (int i = lane; i < 256; i += 32) wh[i] = 0u;
-        __syncwarp();
+        uint32_t* wh = S.whist[warp];   // zeroed by the previous pass's reduction
         for (int st = 0; st < nsteps; ++st) {
           const uint4 kk = k4[st * 32 + lane];
 #pragma unroll
@@ -251,7 +249,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid < 256) {
         uint32_t c = 0;
 #pragma unroll 8
-        for (int w = 0; w < kWarps; ++w) c += S.whist[w][tid];
+        for (int w = 0; w < kWarps; ++w) {
+          c += S.whist[w][tid];
+          S.whist[w][tid] = 0u;   // ready for the next pass
+        }
         if (tid == 0 && prefix == 0) c -= excl_local;   // forced-zero keys are not document keys
         h[tid] = c;
       }
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (!ok) {
-    reject(expect);
+    reject(out_base, expect);
   } else if (rank == 0 && tid == 0) {
     if (b == 0) cu_kept[0] = 0;
     cu_kept[b + 1] = (int32_t)(out_base + expect);
