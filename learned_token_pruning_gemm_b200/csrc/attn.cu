@@ -8,10 +8,11 @@
 // bf16 path (dh = 128). Causal work grows with the query tile index t (tile t
 // meets t+1 key tiles). Two schedules: with few tiles per SM each CTA takes the
 // pair of query tiles t and n-1-t of one (query head, sequence), so every CTA does
-// n+1 key tiles and one wave holds the grid; with many, each CTA takes one query
-// tile and the grid is numbered longest tile first (blockIdx.x -> tile, sequence,
-// head), so the hardware, which starts CTAs in index order as SMs free up, packs
-// them greedily and no wave of equal-length CTAs leaves SMs idle at the end.
+// n+1 key tiles and one wave holds the grid; with many, one CTA per SM walks a list
+// of query tiles: the (tile, sequence, head) items numbered longest tile first and
+// dealt to the CTAs as a snake (c, 2G-1-c, 2G+c, ...), so every CTA's list sums to
+// about the same number of key tiles, and each next tile's loads and first S MMAs
+// run under the tail of the one before (a CTA per tile paid ~4 us of start-up each).
 // Per CTA, pipelines run across its query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
 //                ring. A K stage is free as soon as S_j is computed; with S issued
@@ -58,6 +59,7 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 constexpr int kSBufs = 3;                              // S/P buffers in TMEM
 constexpr int kBiasStages = 4;                         // per-key bias ring (beside the K ring)
+constexpr int kMaxItems = 128;                         // query tiles one CTA walks, at most
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
 constexpr float kLog2e = 1.4426950408889634f;
@@ -87,6 +89,8 @@ struct AttnSmem {
   uint64_t p_full[kSBufs];                  // P_g stored by every softmax warp, on p_full[g % kSBufs]
   uint64_t o_done[kSBufs];                  // PV_g complete, on o_done[g % kSBufs]
   uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
+  int4 item[kMaxItems];                     // the CTA's query tiles: (head, tile, seq0, len)
+  int n_items;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -171,22 +175,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                            int total, int max_kept, int n_hq, int n_hkv, int batch,
                            int lpt_tiles, __nv_bfloat16* __restrict__ out,
                            float* __restrict__ lse, int* status) {
-  // lpt_tiles > 0: one query tile per CTA, blockIdx.x = item in longest-first order
-  // (tile lpt_tiles-1 of every sequence and head first); 0: grid (head, sequence,
-  // pair z) and the pair of tiles n-1-z, z
-  int hq, b, z;
-  if (lpt_tiles > 0) {
-    const int i = blockIdx.x;
-    hq = i % n_hq;
-    b = (i / n_hq) % batch;
-    z = lpt_tiles - 1 - i / (n_hq * batch);   // the CTA's query tile
-  } else {
-    hq = blockIdx.x;
-    b = blockIdx.y;
-    z = blockIdx.z;
-  }
-  const int kvh = hq / (n_hq / n_hkv);
-
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   AttnSmem& S = *reinterpret_cast<AttnSmem*>(smem_raw + pad);
@@ -230,33 +218,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   tg::pdl_launch_dependents();
   tg::pdl_wait();   // global memory only from here on
 
-  const int seq0 = cu_kept[b];
-  const int seq1 = cu_kept[b + 1];
-  // a kept range outside [0, total] or longer than max_kept (the grid covers
-  // max_kept rows per sequence) is not attended: record it and skip the sequence
-  const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
-  if (bad && hq == 0 && tid == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
-  const int len = bad ? 0 : seq1 - seq0;
-  const int n_t = (len + kBM - 1) / kBM;
-  if ((lpt_tiles > 0 ? z : 2 * z) >= n_t) {   // uniform: this sequence has no such tile
+  // The CTA's query tiles, in the order every role walks them, listed once by one
+  // thread. Paired schedule (lpt_tiles == 0): grid (head, sequence, z), tiles n-1-z
+  // then z (if distinct). Persistent schedule (lpt_tiles > 0): the items (tile,
+  // sequence, head) numbered longest tile first, dealt to the G CTAs as a snake (c,
+  // 2G-1-c, 2G+c, ...) so that long and short items pair up; an item beyond its
+  // sequence's tiles is skipped. A sequence whose kept range lies outside [0, total]
+  // or is longer than max_kept (the grid covers max_kept rows per sequence) is not
+  // attended: it is recorded and skipped.
+  if (tid == 0) {
+    int n = 0;
+    auto add = [&](int hq, int b, int z, int r) {   // r: 0 long tile, 1 partner, -1 item
+      const int seq0 = cu_kept[b];
+      const int seq1 = cu_kept[b + 1];
+      const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
+      if (bad && hq == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+      const int len = bad ? 0 : seq1 - seq0;
+      const int n_t = (len + kBM - 1) / kBM;
+      int t = z;
+      if (r >= 0) {
+        if (2 * z >= n_t) return;                      // no such pair in this sequence
+        t = r == 0 ? n_t - 1 - z : z;
+        if (r == 1 && z >= n_t - 1 - z) return;       // the pair is one tile
+      } else if (z >= n_t) {
+        return;
+      }
+      if (n < kMaxItems) S.item[n++] = make_int4(hq, t, seq0, len);
+    };
+    if (lpt_tiles > 0) {
+      const int64_t G = gridDim.x;
+      const int64_t n_items = static_cast<int64_t>(lpt_tiles) * batch * n_hq;
+      for (int64_t r = 0;; ++r) {
+        const int64_t i = r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
+        if (i >= n_items) break;   // rounds fill in order: nothing after a short one
+        add(static_cast<int>(i % n_hq), static_cast<int>((i / n_hq) % batch),
+            lpt_tiles - 1 - static_cast<int>(i / (static_cast<int64_t>(n_hq) * batch)), -1);
+      }
+    } else {
+      add(blockIdx.x, blockIdx.y, blockIdx.z, 0);
+      add(blockIdx.x, blockIdx.y, blockIdx.z, 1);
+    }
+    S.n_items = n;
+  }
+  __syncthreads();
+  const int nq = S.n_items;
+  if (nq == 0) {   // uniform: no query tile here
     if (warp == 2) tg::tmem_dealloc(tmem, kTmemCols);
     return;
   }
-  // the CTA's query tiles: the long one first, then its partner (if distinct)
-  const int tiles[2] = {lpt_tiles > 0 ? z : n_t - 1 - z, lpt_tiles > 0 ? z : z};
-  const int nq = (lpt_tiles == 0 && tiles[1] < tiles[0]) ? 2 : 1;
 
   if (warp == 0) {
     // ---------------- TMA producer: Q and K tiles ----------------
     if (lane == 0) {
-      int g = 0;
+      int g = 0, q_issued = 0;
       bool go = true;
       for (int qi = 0; qi < nq && go; ++qi) {
-        const int t = tiles[qi];
-        if (qi > 0 && !tg::mbar_wait(&S.q_empty, 0, status, &S.abort_flag)) break;
+        const int4 itm = S.item[qi];
+        const int hq = itm.x, t = itm.y, seq0 = itm.z, kvh = hq / (n_hq / n_hkv);
+        if (qi > 0 && !tg::mbar_wait(&S.q_empty, (qi - 1) & 1, status, &S.abort_flag)) break;
         tg::mbar_arrive_expect_tx(&S.q_full, kBM * kD * 2);
         tg::tma_load_3d(S.q[0], &tm_q, &S.q_full, 0, hq, seq0 + t * kBM);
         tg::tma_load_3d(S.q[1], &tm_q, &S.q_full, 64, hq, seq0 + t * kBM);
+        ++q_issued;
         for (int j = 0; j <= t; ++j, ++g) {
           const int s = g % kKStages;
           if (g >= kKStages &&
@@ -271,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (S.abort_flag) {   // let copies in flight land before the CTA exits
-        tg::mbar_wait(&S.q_full, 0, status, nullptr);
+        if (q_issued > 0) tg::mbar_wait(&S.q_full, (q_issued - 1) & 1, status, nullptr);
         for (int j = g > kKStages ? g - kKStages : 0; j < g; ++j)
           tg::mbar_wait(&S.k_full[j % kKStages], (j / kKStages) & 1, status, nullptr);
       }
@@ -281,20 +304,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- bias staging (32 arrivals per K stage) ----------------
     // A register ring keeps the loads of the next kKStages tiles in flight, so the
     // staging keeps pace with the K ring instead of waiting one load per tile.
-    const float gl2 = gain[hq] * kLog2e;
-    const int n_tiles = (tiles[0] + 1) + (nq > 1 ? tiles[1] + 1 : 0);
-    auto tile_j = [&](int g) { return g <= tiles[0] ? g : g - (tiles[0] + 1); };
-    auto load = [&](int g, float* v) {
+    // A lookahead cursor walks (query tile, key tile) in the K ring's order.
+    int la_q = 0, la_j = 0, n_tiles = 0;
+    for (int q = 0; q < nq; ++q) n_tiles += S.item[q].y + 1;
+    auto load_next = [&](float* v) {   // the scaled bias of the tile under the cursor
+      if (la_q < nq) {
+        const int4 itm = S.item[la_q];
+        const float gl2 = gain[itm.x] * kLog2e;
 #pragma unroll
-      for (int u = 0; u < kBN / 32; ++u) {
-        const int kp = tile_j(g) * kBN + lane + 32 * u;
-        v[u] = (g < n_tiles && kp < len) ? s_kept[seq0 + kp] : 0.f;
+        for (int u = 0; u < kBN / 32; ++u) {
+          const int kp = la_j * kBN + lane + 32 * u;
+          v[u] = kp < itm.w ? gl2 * s_kept[itm.z + kp] : 0.f;
+        }
+        if (++la_j > itm.y) {
+          la_j = 0;
+          ++la_q;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < kBN / 32; ++u) v[u] = 0.f;
       }
     };
     float v0[kBN / 32], v1[kBN / 32], v2[kBN / 32];
-    load(0, v0);
-    load(1, v1);
-    load(2, v2);
+    load_next(v0);
+    load_next(v1);
+    load_next(v2);
     for (int g = 0; g < n_tiles; ++g) {
       const int s = g % kBiasStages;
       if (g >= kBiasStages &&
@@ -302,14 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    &S.abort_flag)))
         break;
 #pragma unroll
-      for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = gl2 * v0[u];
+      for (int u = 0; u < kBN / 32; ++u) S.bias[s][lane + 32 * u] = v0[u];
       tg::mbar_arrive(&S.b_full[s]);
 #pragma unroll
       for (int u = 0; u < kBN / 32; ++u) {
         v0[u] = v1[u];
         v1[u] = v2[u];
       }
-      load(g + 3, v2);
+      load_next(v2);
     }
   } else if (warp == 3) {
     // ---------------- TMA producer: V tiles ----------------
@@ -317,7 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0;
       bool go = true;
       for (int qi = 0; qi < nq && go; ++qi) {
-        for (int j = 0; j <= tiles[qi]; ++j, ++g) {
+        const int4 itm = S.item[qi];
+        const int seq0 = itm.z, kvh = itm.x / (n_hq / n_hkv);
+        for (int j = 0; j <= itm.y; ++j, ++g) {
           const int s = g % kVStages;
           if (g >= kVStages &&
               !tg::mbar_wait(&S.v_empty[s], ((g / kVStages) - 1) & 1, status, &S.abort_flag)) {
@@ -361,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool alive = true;
       int g0 = 0;
       for (int qi = 0; qi < nq && alive; ++qi) {
-        const int nt = tiles[qi] + 1;
+        const int nt = S.item[qi].y + 1;
         alive = tg::mbar_wait(&S.q_full, qi & 1, status, &S.abort_flag);
         for (int j = 0; j < kSBufs && j < nt && alive; ++j) alive = issue_s(g0 + j);
         if (alive && nt <= kSBufs) tg::mma_commit(&S.q_empty);   // every S of the tile issued
@@ -416,11 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ra = row0 + (lane >> 2), rb = ra + 8;   // rows within the tile == TMEM lanes
     const int cq = 2 * (lane & 3);                    // first column within each group of 8
     const uint32_t lane_base = static_cast<uint32_t>(row0) << 16;
-    const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
     bool alive = true;
     int g0 = 0;
     for (int qi = 0; qi < nq && alive; ++qi) {
-      const int t = tiles[qi];
+      const int4 itm = S.item[qi];
+      const int hq = itm.x, t = itm.y, seq0 = itm.z, len = itm.w;
+      const float c_h = kLog2e / (sqrtf(static_cast<float>(kD)) * tau[hq]);
       const int nt = t + 1;
       float ma = -INFINITY, mb = -INFINITY;   // running maxima of rows ra, rb
       float la = 0.f, lb = 0.f;               // this thread's share of their sums
@@ -705,8 +742,12 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
     return TG_ERR_CUDA;
   const int64_t pairs = static_cast<int64_t>(n_hq) * batch * ((n_qt + 1) / 2);
   if (pairs > sms && static_cast<int64_t>(n_qt) * batch * n_hq <= INT32_MAX) {
-    // more than one wave of pairs: one tile per CTA, longest first
-    dim3 grid(static_cast<unsigned>(static_cast<int64_t>(n_qt) * batch * n_hq));
+    // more than one wave of pairs: one CTA per SM walking query tiles longest first
+    // (more CTAs only when an SM's share would exceed kMaxItems tiles)
+    const int64_t items = static_cast<int64_t>(n_qt) * batch * n_hq;
+    int64_t ctas = items < sms ? items : sms;
+    if (ctas * kMaxItems < items) ctas = (items + kMaxItems - 1) / kMaxItems;
+    dim3 grid(static_cast<unsigned>(ctas));
     return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv,
                       s_kept, gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
                       batch, n_qt, static_cast<__nv_bfloat16*>(out), lse, status);
