@@ -6,13 +6,13 @@
 //     z_ij = q_i . k_j / (sqrt(dh) tau_h) + g_h s_j,  j <= i;  O_i = softmax_j(z) V
 //
 // bf16 path (dh = 128). Causal work grows with the query tile index t (tile t
-// meets t+1 key tiles). Two schedules: with few tiles per SM each CTA takes the
-// pair of query tiles t and n-1-t of one (query head, sequence), so every CTA does
-// n+1 key tiles and one wave holds the grid; with many, one CTA per SM walks a list
-// of query tiles: the (tile, sequence, head) items numbered longest tile first and
-// dealt to the CTAs as a snake (c, 2G-1-c, 2G+c, ...), so every CTA's list sums to
-// about the same number of key tiles, and each next tile's loads and first S MMAs
-// run under the tail of the one before (a CTA per tile paid ~4 us of start-up each).
+// meets t+1 key tiles). One CTA per SM walks a list of query tiles: the (tile,
+// sequence, head) items numbered longest tile first and dealt to the CTAs as a snake
+// (c, 2G-1-c, 2G+c, ...), so every CTA's list sums to about the same number of key
+// tiles and no CTA carries more than the longest tile plus what balances it; each
+// next tile's loads and first S MMAs run under the tail of the one before (a CTA
+// per tile paid ~4 us of start-up each, and pairs of tiles t, n-1-t per CTA left
+// the longest tile's CTA one tile and one epilogue more than it needs).
 // Per CTA, pipelines run across its query tiles:
 //   warp 0       TMA producer of Q and of K tiles (128 keys) through a 3-stage
 //                ring. A K stage is free as soon as S_j is computed; with S issued
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const float* __restrict__ s_kept, const float* __restrict__ gain,
                            const float* __restrict__ tau, const int32_t* __restrict__ cu_kept,
                            int total, int max_kept, int n_hq, int n_hkv, int batch,
-                           int lpt_tiles, __nv_bfloat16* __restrict__ out,
+                           int n_qt, int walk, __nv_bfloat16* __restrict__ out,
                            float* __restrict__ lse, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -219,44 +219,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   tg::pdl_wait();   // global memory only from here on
 
   // The CTA's query tiles, in the order every role walks them, listed once by one
-  // thread. Paired schedule (lpt_tiles == 0): grid (head, sequence, z), tiles n-1-z
-  // then z (if distinct). Persistent schedule (lpt_tiles > 0): the items (tile,
-  // sequence, head) numbered longest tile first, dealt to the G CTAs as a snake (c,
-  // 2G-1-c, 2G+c, ...) so that long and short items pair up; an item beyond its
-  // sequence's tiles is skipped. A sequence whose kept range lies outside [0, total]
-  // or is longer than max_kept (the grid covers max_kept rows per sequence) is not
-  // attended: it is recorded and skipped.
+  // thread. The items (tile, sequence, head) are numbered longest tile first (tile
+  // n_qt-1 of every sequence and head first). walk != 0: they are dealt to the G
+  // CTAs as a snake (c, 2G-1-c, 2G+c, ...) so that long and short items pair up;
+  // walk == 0: CTA c takes item c alone (for ragged batches, where the hardware's
+  // in-order start of CTAs as SMs free up also balances around the items that
+  // fall beyond a shorter sequence). An item beyond its sequence's tiles is
+  // skipped. A sequence whose kept range lies outside [0, total] or is longer than
+  // max_kept (n_qt covers max_kept rows) is not attended: it is recorded and skipped.
   if (tid == 0) {
     int n = 0;
-    auto add = [&](int hq, int b, int z, int r) {   // r: 0 long tile, 1 partner, -1 item
+    const int64_t G = gridDim.x;
+    const int64_t n_items = static_cast<int64_t>(n_qt) * batch * n_hq;
+    for (int64_t r = 0; r == 0 || walk; ++r) {
+      const int64_t i = r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
+      if (i >= n_items) break;   // rounds fill in order: nothing after a short one
+      const int hq = static_cast<int>(i % n_hq);
+      const int b = static_cast<int>((i / n_hq) % batch);
+      const int t = n_qt - 1 - static_cast<int>(i / (static_cast<int64_t>(n_hq) * batch));
       const int seq0 = cu_kept[b];
       const int seq1 = cu_kept[b + 1];
       const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
       if (bad && hq == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
       const int len = bad ? 0 : seq1 - seq0;
-      const int n_t = (len + kBM - 1) / kBM;
-      int t = z;
-      if (r >= 0) {
-        if (2 * z >= n_t) return;                      // no such pair in this sequence
-        t = r == 0 ? n_t - 1 - z : z;
-        if (r == 1 && z >= n_t - 1 - z) return;       // the pair is one tile
-      } else if (z >= n_t) {
-        return;
-      }
-      if (n < kMaxItems) S.item[n++] = make_int4(hq, t, seq0, len);
-    };
-    if (lpt_tiles > 0) {
-      const int64_t G = gridDim.x;
-      const int64_t n_items = static_cast<int64_t>(lpt_tiles) * batch * n_hq;
-      for (int64_t r = 0;; ++r) {
-        const int64_t i = r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
-        if (i >= n_items) break;   // rounds fill in order: nothing after a short one
-        add(static_cast<int>(i % n_hq), static_cast<int>((i / n_hq) % batch),
-            lpt_tiles - 1 - static_cast<int>(i / (static_cast<int64_t>(n_hq) * batch)), -1);
-      }
-    } else {
-      add(blockIdx.x, blockIdx.y, blockIdx.z, 0);
-      add(blockIdx.x, blockIdx.y, blockIdx.z, 1);
+      if (t * kBM < len && n < kMaxItems) S.item[n++] = make_int4(hq, t, seq0, len);
     }
     S.n_items = n;
   }
@@ -740,22 +726,20 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return TG_ERR_CUDA;
-  const int64_t pairs = static_cast<int64_t>(n_hq) * batch * ((n_qt + 1) / 2);
-  if (pairs > sms && static_cast<int64_t>(n_qt) * batch * n_hq <= INT32_MAX) {
-    // more than one wave of pairs: one CTA per SM walking query tiles longest first
-    // (more CTAs only when an SM's share would exceed kMaxItems tiles)
-    const int64_t items = static_cast<int64_t>(n_qt) * batch * n_hq;
-    int64_t ctas = items < sms ? items : sms;
+  // one sequence: one CTA per SM walking query tiles longest first (more CTAs only
+  // when an SM's share would exceed kMaxItems tiles); a ragged batch: one CTA per
+  // (tile, sequence, head), longest first
+  const int64_t items = static_cast<int64_t>(n_qt) * batch * n_hq;
+  const int walk = batch == 1 ? 1 : 0;
+  int64_t ctas = items;
+  if (walk) {
+    ctas = items < sms ? items : sms;
     if (ctas * kMaxItems < items) ctas = (items + kMaxItems - 1) / kMaxItems;
-    dim3 grid(static_cast<unsigned>(ctas));
-    return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv,
-                      s_kept, gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv,
-                      batch, n_qt, static_cast<__nv_bfloat16*>(out), lse, status);
   }
-  dim3 grid(n_hq, batch, (n_qt + 1) / 2);   // one CTA per pair of query tiles
-  return tg::launch(gated_attn_bf16_kernel, grid, dim3(kThreads), smem, st, 0, tq, tk, tv, s_kept,
-                    gain, tau, cu_kept, static_cast<int>(total), max_kept, n_hq, n_hkv, batch, 0,
-                    static_cast<__nv_bfloat16*>(out), lse, status);
+  if (ctas > INT32_MAX) return TG_ERR_UNSUPPORTED;
+  return tg::launch(gated_attn_bf16_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem,
+                    st, 0, tq, tk, tv, s_kept, gain, tau, cu_kept, static_cast<int>(total), max_kept,
+                    n_hq, n_hkv, batch, n_qt, walk, static_cast<__nv_bfloat16*>(out), lse, status);
 }
 
 }  // namespace
