@@ -60,6 +60,8 @@ constexpr int kVStages = 2;
 constexpr int kSBufs = 3;                              // S/P buffers in TMEM
 constexpr int kBiasStages = 4;                         // per-key bias ring (beside the K ring)
 constexpr int kMaxItems = 128;                         // query tiles one CTA walks, at most
+constexpr int kMaxWalkBatch = 256;                     // sequences a walking grid handles
+constexpr int kMaxWalkTiles = 2048;                    // query tiles per sequence, likewise
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
 constexpr float kLog2e = 1.4426950408889634f;
@@ -90,6 +92,8 @@ struct AttnSmem {
   uint64_t o_done[kSBufs];                  // PV_g complete, on o_done[g % kSBufs]
   uint64_t o_free;                          // the epilogue has read O (next query tile may overwrite)
   int4 item[kMaxItems];                     // the CTA's query tiles: (head, tile, seq0, len)
+  int2 seq[kMaxWalkBatch];                  // walking grid: each sequence's (first row, length)
+  int above[kMaxWalkTiles + 1];             // walking grid: items with a tile above t, at t + 1
   int n_items;
   uint32_t tmem_base;
   int abort_flag;
@@ -218,33 +222,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   tg::pdl_launch_dependents();
   tg::pdl_wait();   // global memory only from here on
 
-  // The CTA's query tiles, in the order every role walks them, listed once by one
-  // thread. The items (tile, sequence, head) are numbered longest tile first (tile
-  // n_qt-1 of every sequence and head first). walk != 0: they are dealt to the G
-  // CTAs as a snake (c, 2G-1-c, 2G+c, ...) so that long and short items pair up;
-  // walk == 0: CTA c takes item c alone (for ragged batches, where the hardware's
-  // in-order start of CTAs as SMs free up also balances around the items that
-  // fall beyond a shorter sequence). An item beyond its sequence's tiles is
-  // skipped. A sequence whose kept range lies outside [0, total] or is longer than
-  // max_kept (n_qt covers max_kept rows) is not attended: it is recorded and skipped.
-  if (tid == 0) {
-    int n = 0;
-    const int64_t G = gridDim.x;
-    const int64_t n_items = static_cast<int64_t>(n_qt) * batch * n_hq;
-    for (int64_t r = 0; r == 0 || walk; ++r) {
-      const int64_t i = r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
-      if (i >= n_items) break;   // rounds fill in order: nothing after a short one
-      const int hq = static_cast<int>(i % n_hq);
-      const int b = static_cast<int>((i / n_hq) % batch);
-      const int t = n_qt - 1 - static_cast<int>(i / (static_cast<int64_t>(n_hq) * batch));
-      const int seq0 = cu_kept[b];
-      const int seq1 = cu_kept[b + 1];
-      const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
-      if (bad && hq == 0) tg::set_status(status, TG_ERR_DEVICE_CHECK);
-      const int len = bad ? 0 : seq1 - seq0;
-      if (t * kBM < len && n < kMaxItems) S.item[n++] = make_int4(hq, t, seq0, len);
+  // The CTA's query tiles, in the order every role walks them. The items (tile,
+  // sequence, head) that exist are numbered longest tile first: tile n_qt-1 of every
+  // sequence long enough for it and every head, then the next tile down. walk != 0:
+  // item v goes to CTA c for v = c, 2G-1-c, 2G+c, ... (a snake, so that long and
+  // short items pair up and every CTA's list sums to about the same number of key
+  // tiles); thread r finds the CTA's r-th item from the per-sequence tile counts (a
+  // binary search over the items-above-tile counts, then the sequence). walk == 0:
+  // CTA c takes item c of the numbering over all (tile, sequence, head), skipped when
+  // the tile lies beyond its sequence. A sequence whose kept range lies outside
+  // [0, total] or is longer than max_kept (n_qt covers max_kept rows) is not
+  // attended: it is recorded and gets no tile.
+  auto seq_geom = [&](int b) -> int2 {
+    const int seq0 = cu_kept[b];
+    const int seq1 = cu_kept[b + 1];
+    const bool bad = seq0 < 0 || seq1 < seq0 || seq1 > total || seq1 - seq0 > max_kept;
+    if (bad) tg::set_status(status, TG_ERR_DEVICE_CHECK);
+    return make_int2(seq0, bad ? 0 : seq1 - seq0);
+  };
+  if (walk) {
+    for (int b = tid; b < batch; b += kThreads) S.seq[b] = seq_geom(b);
+    __syncthreads();
+    for (int t = tid - 1; t < n_qt; t += kThreads) {
+      int c = 0;
+      for (int b = 0; b < batch; ++b) {
+        const int nt = (S.seq[b].y + kBM - 1) / kBM;
+        c += nt - 1 - t > 0 ? nt - 1 - t : 0;
+      }
+      S.above[t + 1] = c * n_hq;
     }
-    S.n_items = n;
+    __syncthreads();
+    int found = 0;
+    if (tid < kMaxItems) {
+      const int64_t G = gridDim.x;
+      const int64_t v = tid * G + ((tid & 1) ? G - 1 - blockIdx.x : blockIdx.x);
+      if (v < S.above[0]) {
+        int lo = 0, hi = n_qt - 1;   // the first tile t with at most v items above it
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (S.above[mid + 1] <= v) hi = mid; else lo = mid + 1;
+        }
+        const int k = static_cast<int>(v) - S.above[lo + 1];   // index within tile lo's items
+        const int j = k / n_hq;                               // the j-th sequence long enough
+        int b = 0;
+        for (int seen = 0; b < batch; ++b) {
+          if (S.seq[b].y > lo * kBM) {
+            if (seen == j) break;
+            ++seen;
+          }
+        }
+        S.item[tid] = make_int4(k % n_hq, lo, S.seq[b].x, S.seq[b].y);
+        found = 1;
+      }
+    }
+    // a CTA's items are v = c, 2G-1-c, ... in increasing order: the first r past the
+    // last item ends the list
+    const int n = __syncthreads_count(found);
+    if (tid == 0) S.n_items = n;
+  } else if (tid == 0) {
+    const int64_t i = blockIdx.x;
+    const int hq = static_cast<int>(i % n_hq);
+    const int b = static_cast<int>((i / n_hq) % batch);
+    const int t = n_qt - 1 - static_cast<int>(i / (static_cast<int64_t>(n_hq) * batch));
+    const int2 g = seq_geom(b);
+    S.n_items = t * kBM < g.y ? 1 : 0;
+    S.item[0] = make_int4(hq, t, g.x, g.y);
   }
   __syncthreads();
   const int nq = S.n_items;
@@ -726,11 +768,11 @@ tg_status launch_attn_bf16(const void* q, const void* k, const void* v, const fl
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return TG_ERR_CUDA;
-  // one sequence: one CTA per SM walking query tiles longest first (more CTAs only
-  // when an SM's share would exceed kMaxItems tiles); a ragged batch: one CTA per
-  // (tile, sequence, head), longest first
+  // one CTA per SM walking query tiles longest first (more CTAs only when an SM's
+  // share would exceed kMaxItems tiles); beyond kMaxWalkBatch sequences or
+  // kMaxWalkTiles tiles, one CTA per (tile, sequence, head), longest first
   const int64_t items = static_cast<int64_t>(n_qt) * batch * n_hq;
-  const int walk = batch == 1 ? 1 : 0;
+  const int walk = batch <= kMaxWalkBatch && n_qt <= kMaxWalkTiles ? 1 : 0;
   int64_t ctas = items;
   if (walk) {
     ctas = items < sms ? items : sms;
