@@ -252,6 +252,27 @@ def test_attention_bf16_head_groups(api, orc, hq, hkv, lens):
     assert_attn_close(out, ref, torch.bfloat16, what=f"heads {hq}/{hkv} lens={lens}")
 
 
+def test_attention_bf16_schedule_fallback_matches_walk(api, orc):
+    # Up to 256 sequences the CTAs walk lists of query tiles; beyond, one CTA takes
+    # one tile. 300 ragged sequences (some of one row) take the second path; their
+    # first 200 alone take the first. A row's arithmetic does not depend on which
+    # CTA runs it, so the shared rows must agree bit for bit, and the oracle checks
+    # a sample of the 300-sequence run. V is drawn uniform (|v| <= 1.74): rows of a
+    # few keys carry single values of v, and with N(0,1) values near 4 the bf16
+    # rounding of the output alone reaches 2^-7.
+    lens = [int(x) for x in np.random.default_rng(7).integers(1, 400, 300)]
+    lens[5] = 1
+    q, k, v, s, gain, tau, cu = _attn_case(300, lens, 16, 8, 128, torch.bfloat16,
+                                           v_dist="uniform")
+    out_all = _run_attn(api, q, k, v, s, gain, tau, cu)
+    n200 = int(cu[200])
+    out_200 = _run_attn(api, q[:n200], k[:n200], v[:n200], s[:n200], gain, tau, cu[:201])
+    assert torch.equal(out_all[:n200], out_200)
+    rows = sample_rows(cu, 96)
+    ref = orc.gated_attention(q, k, v, s, gain, tau, cu, rows=rows)
+    assert_attn_close(out_all, ref, torch.bfloat16, rows, what="300 sequences")
+
+
 def test_attention_bf16_16k_shape_all_rows_normal_v(api, orc):
     # the 16k layer's attention shape (K = 1868, 16/8 heads) with V ~ N(0,1), every row
     q, k, v, s, gain, tau, cu = _attn_case(1868, [1868], 16, 8, 128, torch.bfloat16)
