@@ -106,7 +106,7 @@ struct DqSmem {
   uint64_t qd_full;
   uint64_t kv_full[2], kv_empty[2];
   uint64_t b_full[2], b_empty[2];
-  uint64_t sp_full, ds_full, dq_done;
+  uint64_t sp_full[2], ds_full[2], dq_done;   // per 64-key half of the key tile
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -135,8 +135,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tg::mbar_init(&S.b_full[i], 32);
       tg::mbar_init(&S.b_empty[i], 4);
     }
-    tg::mbar_init(&S.sp_full, 1);
-    tg::mbar_init(&S.ds_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      tg::mbar_init(&S.sp_full[i], 1);
+      tg::mbar_init(&S.ds_full[i], 4);
+    }
     tg::mbar_init(&S.dq_done, 1);
     S.abort_flag = 0;
     tg::fence_barrier_init();
@@ -195,41 +197,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else if (warp == 5) {
-    // ---- MMA: S = Q K^T, dP = dO V^T, then dQ += dS K ----
+    // ---- MMA: S = Q K^T, dP = dO V^T, then dQ += dS K, by 64-key halves ----
+    // Order S_lo dP_lo, S_hi dP_hi, dQ_lo, [next tile] S_lo dP_lo, dQ_hi, S_hi dP_hi,
+    // dQ_lo, ...: the elementwise warps work on one half while the tensor core
+    // computes the other. A half's S and dP are rewritten only after the dQ MMA that
+    // reads its dS was issued (the pipe runs in order) and its dP was read.
     if (lane == 0) {
-      constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_h = tg::idesc_bf16_f32(kBM, kBN / 2, false, false);
       constexpr uint32_t idesc_q = tg::idesc_bf16_f32(kBM, kD, false, true);
       bool alive = tg::mbar_wait(&S.qd_full, 0, status, &S.abort_flag);
       const uint32_t q0 = tg::smem_u32(S.q[0]), d0 = tg::smem_u32(S.dout[0]);
-      for (int j = 0; j < nt && alive; ++j) {
+      // S and dP of half h of key tile j (keys 64h .. 64h+63: rows 64h of the
+      // 128-byte-swizzled K and V tiles, 8 KB into each 64-dim half)
+      auto issue_sp = [&](int j, int h) -> bool {
         const int st = j & 1;
-        if (!tg::mbar_wait(&S.kv_full[st], (j >> 1) & 1, status, &S.abort_flag)) break;
+        if (h == 0 && !tg::mbar_wait(&S.kv_full[st], (j >> 1) & 1, status, &S.abort_flag))
+          return false;
         tg::tc_fence_after();
-        const uint32_t k0 = tg::smem_u32(S.k[st][0]), v0 = tg::smem_u32(S.v[st][0]);
+        const uint32_t k0 = tg::smem_u32(S.k[st][0]) + h * (kBN / 2) * 128;
+        const uint32_t v0 = tg::smem_u32(S.v[st][0]) + h * (kBN / 2) * 128;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          tg::mma_bf16_ss(tmem + kColS, tg::smem_desc_sw128(q0 + off, 16, 1024),
-                          tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
+          tg::mma_bf16_ss(tmem + kColS + 64 * h, tg::smem_desc_sw128(q0 + off, 16, 1024),
+                          tg::smem_desc_sw128(k0 + off, 16, 1024), idesc_h, kk != 0);
         }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          tg::mma_bf16_ss(tmem + kColDP, tg::smem_desc_sw128(d0 + off, 16, 1024),
-                          tg::smem_desc_sw128(v0 + off, 16, 1024), idesc_s, kk != 0);
+          tg::mma_bf16_ss(tmem + kColDP + 64 * h, tg::smem_desc_sw128(d0 + off, 16, 1024),
+                          tg::smem_desc_sw128(v0 + off, 16, 1024), idesc_h, kk != 0);
         }
-        tg::mma_commit(&S.sp_full);
-        if (!tg::mbar_wait(&S.ds_full, j & 1, status, &S.abort_flag)) break;
+        tg::mma_commit(&S.sp_full[h]);
+        return true;
+      };
+      // dQ += dS_h K_h: A = dS of half h (packed bf16 at columns 64h .. 64h+31 of S,
+      // 8 columns per 16 keys), B = K rows 64h + 16kk .. as an MN-major operand
+      auto issue_dq = [&](int j, int h) -> bool {
+        if (!tg::mbar_wait(&S.ds_full[h], j & 1, status, &S.abort_flag)) return false;
         tg::tc_fence_after();
+        const uint32_t k0 = tg::smem_u32(S.k[j & 1][0]);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = dS (packed bf16 over S, 8 columns per 16 keys), B = K_j rows
-          // 16kk..16kk+15 as an MN-major operand (dh halves 16 KB apart)
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
           const uint64_t bdesc = tg::smem_desc_sw128(k0 + kk * 16 * 128, kBN * 64 * 2, 1024);
-          tg::mma_bf16_ts(tmem + kColAcc, tmem + kColS + kk * 8, bdesc, idesc_q, (j | kk) != 0);
+          tg::mma_bf16_ts(tmem + kColAcc, tmem + kColS + 64 * h + (kk - 4 * h) * 8, bdesc, idesc_q,
+                          (j | kk) != 0);
         }
-        tg::mma_commit(&S.kv_empty[st]);
-        if (j == nt - 1) tg::mma_commit(&S.dq_done);
+        if (h == 1) tg::mma_commit(&S.kv_empty[j & 1]);
+        if (h == 1 && j == nt - 1) tg::mma_commit(&S.dq_done);
+        return true;
+      };
+      if (alive) alive = issue_sp(0, 0) && issue_sp(0, 1);
+      for (int j = 0; j < nt && alive; ++j) {
+        alive = issue_dq(j, 0);
+        if (alive && j + 1 < nt) alive = issue_sp(j + 1, 0);
+        if (alive) alive = issue_dq(j, 1);
+        if (alive && j + 1 < nt) alive = issue_sp(j + 1, 1);
       }
     }
     __syncwarp();
@@ -260,15 +283,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float Dr = valid ? D[static_cast<int64_t>(hq) * total + seq0 + qrow] : 0.f;
     const uint32_t sa = tmem_lane_addr(tmem, warp, kColS), da = tmem_lane_addr(tmem, warp, kColDP);
     bool alive = true;
-    for (int j = 0; j < nt; ++j) {
+    for (int j = 0; j < nt && alive; ++j) {
       const int st = j & 1;
-      alive = tg::mbar_wait(&S.sp_full, j & 1, status, &S.abort_flag);
-      if (alive) alive = tg::mbar_wait(&S.b_full[st], (j >> 1) & 1, status, &S.abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
-      tg::tc_fence_after();
+      alive = tg::mbar_wait(&S.b_full[st], (j >> 1) & 1, status, &S.abort_flag);
       const bool diag = (j == t);
 #pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
+      for (int h = 0; h < 2; ++h) {   // 64-key halves, each as soon as its S and dP land
+      if (alive) alive = tg::mbar_wait(&S.sp_full[h], j & 1, status, &S.abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
+      tg::tc_fence_after();
+#pragma unroll 1
+      for (int ch = 2 * h; ch < 2 * h + 2; ++ch) {
         uint32_t sv[32], pv[32], pk[16];
         tg::tmem_ld32(sa + 32 * ch, sv);
         tg::tmem_ld32(da + 32 * ch, pv);
@@ -285,16 +310,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           pk[e / 2] = tg::pack_bf16x2(d2[0], d2[1]);
         }
-        // packed columns 16ch..16ch+15 of S: this thread has read them already
-        tg::tmem_st16(sa + 16 * ch, pk);
+        // packed columns 64h + 16(ch-2h) .. +15 of S, inside this half's own 64
+        // columns (which this thread has read already)
+        tg::tmem_st16(sa + 64 * h + 16 * (ch - 2 * h), pk);
       }
       tg::tmem_st_wait();
       tg::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        tg::mbar_arrive(&S.ds_full);
-        tg::mbar_arrive(&S.b_empty[st]);
+      if (lane == 0) tg::mbar_arrive(&S.ds_full[h]);
       }
+      if (!alive) break;
+      if (lane == 0) tg::mbar_arrive(&S.b_empty[st]);
     }
     if (alive) alive = tg::mbar_wait(&S.dq_done, 0, status, &S.abort_flag);
     if (__all_sync(0xFFFFFFFFu, alive)) {
