@@ -365,7 +365,7 @@ struct DkvSmem {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
   uint64_t ld_full[2], ld_empty[2];
-  uint64_t st_full, pd_full, acc_done;
+  uint64_t st_full[2], pd_full[2], acc_done;   // per 64-query half of the item
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -401,8 +401,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tg::mbar_init(&S.ld_full[i], 32);
       tg::mbar_init(&S.ld_empty[i], 4);
     }
-    tg::mbar_init(&S.st_full, 1);
-    tg::mbar_init(&S.pd_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      tg::mbar_init(&S.st_full[i], 1);
+      tg::mbar_init(&S.pd_full[i], 4);
+    }
     tg::mbar_init(&S.acc_done, 1);
     S.abort_flag = 0;
     tg::fence_barrier_init();
@@ -487,43 +489,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ---- MMA: S^T = K Q^T, dP^T = V dO^T; then dV += P^T dO, dK += dS^T Q ----
+    // By 64-query halves, in the order ST_lo dPT_lo, ST_hi dPT_hi, dV_lo dK_lo, (next
+    // item) ST_lo dPT_lo, dV_hi dK_hi, ST_hi dPT_hi, ...: the elementwise warps work on
+    // one half while the tensor core computes the other. A half's S^T and dP^T are
+    // rewritten only after the dV/dK MMAs reading its P^T and dS^T were issued.
     if (lane == 0) {
-      constexpr uint32_t idesc_s = tg::idesc_bf16_f32(kBN, kBM, false, false);
+      constexpr uint32_t idesc_h = tg::idesc_bf16_f32(kBN, kBM / 2, false, false);
       constexpr uint32_t idesc_o = tg::idesc_bf16_f32(kBN, kD, false, true);
       bool alive = tg::mbar_wait(&S.kv_full, 0, status, &S.abort_flag);
       const uint32_t k0 = tg::smem_u32(S.k[0]), v0 = tg::smem_u32(S.v[0]);
-      for (int it = 0; it < n_items && alive; ++it) {
+      // S^T and dP^T of half h of item it (queries 64h .. 64h+63: rows 64h of the
+      // 128-byte-swizzled Q and dO tiles, 8 KB into each 64-dim half)
+      auto issue_sp = [&](int it, int h) -> bool {
         const int st = it & 1;
-        if (!tg::mbar_wait(&S.qd_full[st], (it >> 1) & 1, status, &S.abort_flag)) break;
+        if (h == 0 && !tg::mbar_wait(&S.qd_full[st], (it >> 1) & 1, status, &S.abort_flag))
+          return false;
         tg::tc_fence_after();
+        const uint32_t q0 = tg::smem_u32(S.q[st][0]) + h * (kBM / 2) * 128;
+        const uint32_t d0 = tg::smem_u32(S.dout[st][0]) + h * (kBM / 2) * 128;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
+          tg::mma_bf16_ss(tmem + kColST + 64 * h, tg::smem_desc_sw128(k0 + off, 16, 1024),
+                          tg::smem_desc_sw128(q0 + off, 16, 1024), idesc_h, kk != 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
+          tg::mma_bf16_ss(tmem + kColDPT + 64 * h, tg::smem_desc_sw128(v0 + off, 16, 1024),
+                          tg::smem_desc_sw128(d0 + off, 16, 1024), idesc_h, kk != 0);
+        }
+        tg::mma_commit(&S.st_full[h]);
+        return true;
+      };
+      // dV += P^T_h dO_h, dK += dS^T_h Q_h: A = the half's packed bf16 at columns
+      // 64h .. 64h+31 (8 columns per 16 queries); B = dO_i / Q_i rows 64h + 16kk ..
+      // as MN-major operands
+      auto issue_acc = [&](int it, int h) -> bool {
+        if (!tg::mbar_wait(&S.pd_full[h], it & 1, status, &S.abort_flag)) return false;
+        tg::tc_fence_after();
+        const int st = it & 1;
         const uint32_t q0 = tg::smem_u32(S.q[st][0]), d0 = tg::smem_u32(S.dout[st][0]);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          tg::mma_bf16_ss(tmem + kColST, tg::smem_desc_sw128(k0 + off, 16, 1024),
-                          tg::smem_desc_sw128(q0 + off, 16, 1024), idesc_s, kk != 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 64 * 2) + (kk & 3) * 32;
-          tg::mma_bf16_ss(tmem + kColDPT, tg::smem_desc_sw128(v0 + off, 16, 1024),
-                          tg::smem_desc_sw128(d0 + off, 16, 1024), idesc_s, kk != 0);
-        }
-        tg::mma_commit(&S.st_full);
-        if (!tg::mbar_wait(&S.pd_full, it & 1, status, &S.abort_flag)) break;
-        tg::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {
-          // A = P^T / c dS^T in TMEM (8 packed columns per 16 queries); B = dO_i or
-          // Q_i rows 16kk..16kk+15 as an MN-major operand
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
           const uint32_t acc = (it | kk) != 0;
-          tg::mma_bf16_ts(tmem + kColDV, tmem + kColST + kk * 8,
+          const uint32_t a_col = 64 * h + (kk - 4 * h) * 8;
+          tg::mma_bf16_ts(tmem + kColDV, tmem + kColST + a_col,
                           tg::smem_desc_sw128(d0 + kk * 16 * 128, kBM * 64 * 2, 1024), idesc_o, acc);
-          tg::mma_bf16_ts(tmem + kColDK, tmem + kColDPT + kk * 8,
+          tg::mma_bf16_ts(tmem + kColDK, tmem + kColDPT + a_col,
                           tg::smem_desc_sw128(q0 + kk * 16 * 128, kBM * 64 * 2, 1024), idesc_o, acc);
         }
-        tg::mma_commit(&S.qd_empty[st]);
-        if (it == n_items - 1) tg::mma_commit(&S.acc_done);
+        if (h == 1) tg::mma_commit(&S.qd_empty[st]);
+        if (h == 1 && it == n_items - 1) tg::mma_commit(&S.acc_done);
+        return true;
+      };
+      if (alive) alive = issue_sp(0, 0) && issue_sp(0, 1);
+      for (int it = 0; it < n_items && alive; ++it) {
+        alive = issue_acc(it, 0);
+        if (alive && it + 1 < n_items) alive = issue_sp(it + 1, 0);
+        if (alive) alive = issue_acc(it, 1);
+        if (alive && it + 1 < n_items) alive = issue_sp(it + 1, 1);
       }
     }
     __syncwarp();
@@ -561,14 +586,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float c = 1.f / (sqrtf(static_cast<float>(kD)) * th);
       const float c2 = c * kLog2e;
       const float b2 = gain[h] * kLog2e * sk;
-      alive = tg::mbar_wait(&S.st_full, it & 1, status, &S.abort_flag);
-      if (alive) alive = tg::mbar_wait(&S.ld_full[st], (it >> 1) & 1, status, &S.abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
-      tg::tc_fence_after();
+      alive = tg::mbar_wait(&S.ld_full[st], (it >> 1) & 1, status, &S.abort_flag);
       const bool diag = (i == jt);
       const int qlim = len - i * kBM;   // query rows of this tile inside the sequence
 #pragma unroll 1
-      for (int ch = 0; ch < kBM / 32; ++ch) {
+      for (int hq2 = 0; hq2 < 2; ++hq2) {   // 64-query halves, each as its S^T and dP^T land
+      if (alive) alive = tg::mbar_wait(&S.st_full[hq2], it & 1, status, &S.abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, alive)) { alive = false; break; }
+      tg::tc_fence_after();
+#pragma unroll 1
+      for (int ch = 2 * hq2; ch < 2 * hq2 + 2; ++ch) {
         uint32_t sv[32], pv[32], pp[16], pd[16];
         tg::tmem_ld32(sa + 32 * ch, sv);
         tg::tmem_ld32(da + 32 * ch, pv);
@@ -592,17 +619,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pp[e / 2] = tg::pack_bf16x2(p2[0], p2[1]);
           pd[e / 2] = tg::pack_bf16x2(d2[0], d2[1]);
         }
-        // packed columns 16ch..16ch+15 of S^T / dP^T: this thread has read them already
-        tg::tmem_st16(sa + 16 * ch, pp);
-        tg::tmem_st16(da + 16 * ch, pd);
+        // packed columns 64h + 16(ch-2h) .. +15 of S^T / dP^T, inside this half's
+        // own 64 columns (which this thread has read already)
+        tg::tmem_st16(sa + 64 * hq2 + 16 * (ch - 2 * hq2), pp);
+        tg::tmem_st16(da + 64 * hq2 + 16 * (ch - 2 * hq2), pd);
       }
       tg::tmem_st_wait();
       tg::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        tg::mbar_arrive(&S.pd_full);
-        tg::mbar_arrive(&S.ld_empty[st]);
+      if (lane == 0) tg::mbar_arrive(&S.pd_full[hq2]);
       }
+      if (!alive) break;
+      if (lane == 0) tg::mbar_arrive(&S.ld_empty[st]);
       if ((it0 + it) % per_head == per_head - 1 || it == n_items - 1) {
         // this head's items in this CTA are done: its score-gradient share, and this
         // warp's gain and temperature partials for it (summed over the CTA's warps and
