@@ -6,8 +6,8 @@
 // budget).
 //
 // One thread-block cluster per sequence, one launch for the whole batch. The
-// cluster has enough CTAs (1..8) for about 4096 keys each (at most 24576), so the
-// passes below stay short. Each CTA holds a contiguous slice of the sequence in
+// cluster has enough CTAs (1..16, where the device runs 16-CTA clusters, else
+// 1..8) for about 4096 keys each (at most 24576), so the passes below stay short. Each CTA holds a contiguous slice of the sequence in
 // shared memory twice: the raw fp32 scores (for the kept-score output) and
 // order-preserving 32-bit keys (NaN lowest, -0 == +0). Tokens outside the
 // document (and padding) get key 0; their count is subtracted from bin 0 so the
@@ -27,17 +27,20 @@
 // the sequence. No global scratch.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;     // 16 where the device runs such clusters (else 8)
+constexpr int kPortableCluster = 8;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kKeysTarget = 4096;                                    // keys per CTA aimed at
-constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kMaxCluster;   // 24576
+constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kPortableCluster;   // 24576
 constexpr int kChunkQuant = kWarps * 128;                            // 128 keys per warp step
 
 struct alignas(16) SelectSmem {
@@ -57,10 +60,10 @@ struct alignas(16) SelectSmem {
   // followed by: uint32_t keys[chunk]; float raw[chunk];
 };
 
-inline int select_cluster(int max_len) {
+inline int select_cluster(int max_len, int max_cluster) {
   int c = (max_len + kKeysTarget - 1) / kKeysTarget;
   if (c < 1) c = 1;
-  if (c > kMaxCluster) c = kMaxCluster;
+  if (c > max_cluster) c = max_cluster;
   return c;
 }
 
@@ -419,6 +422,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The largest cluster this device runs for the kernel: 16 CTAs (non-portable) when a
+// 16-CTA cluster with the largest shared-memory footprint it would use can be
+// resident, else the portable 8. Probed once per device; 0 if the runtime fails.
+int max_cluster_here() {
+  constexpr int kDevices = 64;
+  static int cache[kDevices];   // 0: not probed yet
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    int best = kPortableCluster;
+    const int chunk16 = select_chunk(TG_SELECT_MAX_SEQLEN, kMaxCluster);
+    const size_t smem16 = sizeof(SelectSmem) + (size_t)chunk16 * 8;
+    if (cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1) == cudaSuccess &&
+        tg::ensure_smem(reinterpret_cast<const void*>(select_topk_kernel), (int)smem16)) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kMaxCluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(kMaxCluster, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem16;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, select_topk_kernel, &cfg) == cudaSuccess &&
+          clusters > 0)
+        best = kMaxCluster;
+    }
+    (void)cudaGetLastError();   // a refused probe leaves no error behind
+    cache[dev] = best;
+  }
+  return cache[dev];
+}
+
 }  // namespace
 
 extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens,
@@ -438,7 +480,8 @@ extern "C" tg_status tg_select_topk(const float* scores, const int32_t* cu_seqle
   if (batch > 65535) return TG_ERR_UNSUPPORTED;
   int* st = tg::status_word();
   if (!st) return TG_ERR_CUDA;
-  const int csize = select_cluster(max_seqlen);
+  const int csize = select_cluster(max_seqlen, max_cluster_here());
+  if (csize <= 0) return TG_ERR_CUDA;
   const int chunk = select_chunk(max_seqlen, csize);
   if (chunk > kMaxKeysPerCta) return TG_ERR_UNSUPPORTED;
   const size_t smem = sizeof(SelectSmem) + (size_t)chunk * 8;
