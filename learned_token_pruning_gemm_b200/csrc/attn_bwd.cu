@@ -874,7 +874,8 @@ __global__ void __launch_bounds__(256)
 // bf16 path: for each key row of a valid sequence, ds = the sum over halves and KV
 // heads of the shares and, for split units, dK and dV = half 0 + half 1 of the
 // partials, in that fixed order. Rows of a sequence that failed the device check are
-// left alone (their partials were never written). One warp per key row.
+// left alone (their partials were never written). One warp per (key row, KV head)
+// for split units, one per key row otherwise.
 __global__ void __launch_bounds__(256)
     bwd_reduce_dkv_ds_kernel(const float* __restrict__ dkv_part, const float* __restrict__ ds_part,
                              const int32_t* __restrict__ cu_kept, int batch, int64_t total,
@@ -882,7 +883,12 @@ __global__ void __launch_bounds__(256)
                              __nv_bfloat16* __restrict__ dv, float* __restrict__ ds) {
   tg::pdl_launch_dependents();
   tg::pdl_wait();
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  // split units: one warp per (row j, KV head kv), its four 512-byte loads all in
+  // flight at once; whole units: one warp per row (the score gradient only)
+  const int per_row = nsplit > 1 ? n_hkv : 1;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t j = w / per_row;
+  const int kv = static_cast<int>(w % per_row);
   const int lane = threadIdx.x & 31;
   if (j >= total) return;
   int lo = 0, hi = batch;   // the sequence holding row j: cu_kept[b] <= j < cu_kept[b + 1]
@@ -894,7 +900,7 @@ __global__ void __launch_bounds__(256)
   const int64_t s0 = cu_kept[lo], s1 = cu_kept[lo + 1];
   if (s0 < 0 || s1 < s0 || s1 > total || s1 - s0 > max_kept || j < s0 || j >= s1) return;
   const int64_t plane = total * n_hkv * kD;
-  for (int kv = 0; kv < (nsplit > 1 ? n_hkv : 0); ++kv) {
+  if (nsplit > 1) {
     const int64_t o = (j * n_hkv + kv) * kD + 4 * lane;
     const float4 k0 = *reinterpret_cast<const float4*>(dkv_part + o);
     const float4 v0 = *reinterpret_cast<const float4*>(dkv_part + plane + o);
@@ -905,10 +911,10 @@ __global__ void __launch_bounds__(256)
     *reinterpret_cast<uint2*>(dv + o) =
         make_uint2(tg::pack_bf16x2(v0.x + v1.x, v0.y + v1.y), tg::pack_bf16x2(v0.z + v1.z, v0.w + v1.w));
   }
-  if (lane == 0) {
+  if (kv == 0 && lane == 0) {   // the row's score gradient, in a fixed order
     float a = 0.f;
     for (int h2 = 0; h2 < nsplit; ++h2)
-      for (int kv = 0; kv < n_hkv; ++kv) a += ds_part[(static_cast<int64_t>(h2) * n_hkv + kv) * total + j];
+      for (int h = 0; h < n_hkv; ++h) a += ds_part[(static_cast<int64_t>(h2) * n_hkv + h) * total + j];
     ds[j] = a;
   }
 }
@@ -1069,7 +1075,8 @@ extern "C" tg_status tg_gated_attention_bwd(
                    nsplit, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), ws.dkv,
                    ws.ds, ws.gt, st);
     if (r != TG_OK) return r;
-    r = tg::launch(bwd_reduce_dkv_ds_kernel, dim3(static_cast<unsigned>((total_kept + 7) / 8)),
+    r = tg::launch(bwd_reduce_dkv_ds_kernel,
+                   dim3(static_cast<unsigned>((total_kept * (nsplit > 1 ? n_hkv : 1) + 7) / 8)),
                    dim3(256), 0, stream, 0, static_cast<const float*>(ws.dkv),
                    static_cast<const float*>(ws.ds), cu_kept, batch, total_kept, max_kept, n_hkv,
                    nsplit, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), ds);
