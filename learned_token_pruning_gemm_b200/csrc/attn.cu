@@ -240,7 +240,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (bad) tg::set_status(status, TG_ERR_DEVICE_CHECK);
     return make_int2(seq0, bad ? 0 : seq1 - seq0);
   };
-  if (walk) {
+  if (walk && batch == 1) {   // one sequence: item v is tile n_t-1-v/n_hq of head v%n_hq
+    if (tid == 0) {
+      const int2 g = seq_geom(0);
+      const int64_t V = static_cast<int64_t>((g.y + kBM - 1) / kBM) * n_hq;
+      const int64_t G = gridDim.x;
+      int n = 0;
+      for (int64_t r = 0; n < kMaxItems; ++r) {
+        const int64_t v = r * G + ((r & 1) ? G - 1 - blockIdx.x : blockIdx.x);
+        if (v >= V) break;
+        S.item[n++] = make_int4(static_cast<int>(v % n_hq),
+                                static_cast<int>(V / n_hq - 1 - v / n_hq), g.x, g.y);
+      }
+      S.n_items = n;
+    }
+  } else if (walk) {
     for (int b = tid; b < batch; b += kThreads) S.seq[b] = seq_geom(b);
     __syncthreads();
     for (int t = tid - 1; t < n_qt; t += kThreads) {
