@@ -65,6 +65,7 @@ constexpr int kMaxWalkTiles = 2048;                    // query tiles per sequen
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 128 + kSoftmaxWarps * 32;    // warps 0-3 roles, 4-11 softmax
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kStagePitch = 144;   // bytes per staged 64-column row (padded: no bank conflicts)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: move the max only if it grows by > 2^8
 
 // 2^f on [-1/2, 1/2], degree-3 minimax in relative error (7.5e-5), fitted by a
@@ -79,6 +80,7 @@ struct AttnSmem {
   uint8_t k[kKStages][2][kBN * 64 * 2];
   uint8_t v[kVStages][2][kBN * 64 * 2];
   float bias[kBiasStages][kBN];
+  uint8_t ostage[kSoftmaxWarps][16][kStagePitch];   // epilogue: each warp's 16 rows of O, bf16
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[kKStages];
@@ -656,21 +658,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ga < len) lse[static_cast<int64_t>(hq) * total + seq0 + ga] = (ma + __log2f(la)) * kLn2;
         if (gb < len) lse[static_cast<int64_t>(hq) * total + seq0 + gb] = (mb + __log2f(lb)) * kLn2;
       }
-      if (ga < len) {
-        uint32_t* orow = reinterpret_cast<uint32_t*>(
-            out + (static_cast<int64_t>(seq0 + ga) * n_hq + hq) * kD + cq);
+      // O / l through this warp's staging rows, 64 columns at a time: the quad
+      // layout's 4-byte pieces go to shared memory (padded rows, no bank conflicts
+      // either way), and each store to global memory writes four whole 128-byte row
+      // segments (32 full lines per warp instead of 256 partial sectors)
+      uint8_t* stg = &S.ostage[warp - 4][0][0];
+      const int qr = lane >> 2;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          orow[4 * i] = tg::pack_bf16x2(__uint_as_float(o[4 * i]) * ia,
-                                        __uint_as_float(o[4 * i + 1]) * ia);
-      }
-      if (gb < len) {
-        uint32_t* orow = reinterpret_cast<uint32_t*>(
-            out + (static_cast<int64_t>(seq0 + gb) * n_hq + hq) * kD + cq);
+      for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          orow[4 * i] = tg::pack_bf16x2(__uint_as_float(o[4 * i + 2]) * ib,
-                                        __uint_as_float(o[4 * i + 3]) * ib);
+        for (int i = 0; i < 8; ++i) {
+          const int ii = 8 * hh + i;
+          *reinterpret_cast<uint32_t*>(stg + qr * kStagePitch + (8 * i + cq) * 2) =
+              tg::pack_bf16x2(__uint_as_float(o[4 * ii]) * ia, __uint_as_float(o[4 * ii + 1]) * ia);
+          *reinterpret_cast<uint32_t*>(stg + (qr + 8) * kStagePitch + (8 * i + cq) * 2) =
+              tg::pack_bf16x2(__uint_as_float(o[4 * ii + 2]) * ib,
+                              __uint_as_float(o[4 * ii + 3]) * ib);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = 4 * k + (lane >> 3), cb = (lane & 7) * 16;
+          const uint4 val = *reinterpret_cast<const uint4*>(stg + r * kStagePitch + cb);
+          const int gr = t * kBM + row0 + r;
+          if (gr < len)
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(
+                out + (static_cast<int64_t>(seq0 + gr) * n_hq + hq) * kD + 64 * hh) + cb) = val;
+        }
+        __syncwarp();
       }
       g0 += nt;
     }
