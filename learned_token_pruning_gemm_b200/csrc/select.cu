@@ -7,8 +7,8 @@
 //
 // One thread-block cluster per sequence, one launch for the whole batch. The
 // cluster has enough CTAs (1..16, where the device runs 16-CTA clusters, else
-// 1..8) for about 4096 keys each (at most 24576), so the passes below stay short. Each CTA holds a contiguous slice of the sequence in
-// shared memory twice: the raw fp32 scores (for the kept-score output) and
+// 1..8) for about 2048 keys each (at most 24576), so the passes below stay short.
+// Each CTA holds a contiguous slice of the sequence in shared memory twice: the raw fp32 scores (for the kept-score output) and
 // order-preserving 32-bit keys (NaN lowest, -0 == +0). Tokens outside the
 // document (and padding) get key 0; their count is subtracted from bin 0 so the
 // histograms see document tokens only.
@@ -39,7 +39,7 @@ constexpr int kMaxCluster = 16;     // 16 where the device runs such clusters (e
 constexpr int kPortableCluster = 8;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kKeysTarget = 4096;                                    // keys per CTA aimed at
+constexpr int kKeysTarget = 2048;                                    // keys per CTA aimed at
 constexpr int kMaxKeysPerCta = TG_SELECT_MAX_SEQLEN / kPortableCluster;   // 24576
 constexpr int kChunkQuant = kWarps * 128;                            // 128 keys per warp step
 
