@@ -195,8 +195,9 @@ tg_status tg_gated_attention_bwd(const void* q, const void* k, const void* v, co
  * split per head; q and k heads are rotated at pos[r] (rotary embedding with the
  * rotate-half pairing (i, i + head_dim/2) and theta_i = rope_base^(-2i/head_dim), the
  * convention of the Qwen models the pages evaluate; the pages do not describe it),
- * v heads are copied. The angle pos * theta_i is formed in fp64 and reduced modulo
- * 2 pi before an fp32 sine and cosine.
+ * v heads are copied. The angle pos * theta_i is taken in turns as an integer
+ * product with theta_i / (2 pi) in 64-bit fixed point (exact modulo one turn),
+ * rounded to 2^-24 of a turn, before an fp32 sine and cosine.
  *   xc  [n_rows, d] bf16: the compacted residual rows (tg_compact_kv)
  *   pos [n_rows] int32 device, >= 0: original positions within each sequence
  *   q [n_rows, n_hq, head_dim], k and v [n_rows, n_hkv, head_dim] bf16 outputs

@@ -10,13 +10,20 @@
 // (128-byte swizzle) through a 3-stage mbarrier ring; one thread issues, per K=16
 // step, one tcgen05.mma (M=128, N=256, bf16 -> fp32) per row tile into its own
 // 256-column TMEM accumulator (512 columns in all), both with the same W operand,
-// so W is streamed once per 256 rows. Epilogue, all 16 warps, one row tile after
-// the other: warp w reads TMEM lanes 32*(w%4).. and, of head (w/4)/2 of the tile,
-// the pairs i in [32*((w/4)%2), +32) and i + 64, so every rotate-half pair is in
-// one thread. The angle p*theta_i is formed in fp64 and reduced modulo 2 pi
-// (positions reach 1e5 and more, where an fp32 product alone is off by ~1e-2 rad),
-// then the fp32 sine and cosine of the reduced angle (MUFU, absolute error about
-// 2^-21 on [-pi, pi]); the rotation and the bf16 rounding are fp32.
+// so W is streamed once per 256 rows. The rotary angles do not depend on the
+// products, so the warps that wait on the accumulators take them while the MMAs
+// run: the angle of position p and frequency i, in turns, is p * F_i mod 1 with
+// F_i = theta_i / (2 pi) held as a 64-bit fixed-point fraction (one integer
+// product, exact modulo 2^64; positions reach 1e5 and more, where an fp32 product
+// alone is off by ~1e-2 rad), rounded to 23 bits and brought to [-pi, pi) in
+// fp32, then the fp32 sine and cosine (MUFU, absolute error about 2^-21). The two
+// heads of a tile share their rows' angles: each of a pair of warps takes half of
+// them and hands its half over through the freed stage buffers. Epilogue, all 16
+// warps, one row tile after the other: warp w reads TMEM lanes 32*(w%4).. and, of
+// head (w/4)/2 of the tile, the pairs i in [32*((w/4)%2), +32) and i + 64, so
+// every rotate-half pair is in one thread; the rotation and the bf16 rounding are
+// fp32; the rows go through shared memory (16-byte pieces, XOR-swizzled across
+// the eight rows that share banks) and leave as whole 256-byte head rows.
 #include "common.cuh"
 
 namespace {
@@ -32,7 +39,7 @@ constexpr int kHalf = kDh / 2;
 struct QkvSmem {
   uint8_t a[kStages][2][kBM * kBK * 2];   // two xc tiles, 16 KB each
   uint8_t b[kStages][kBN * kBK * 2];   // W tiles, 32 KB
-  double theta[kHalf];                 // base^(-2i/dh)
+  uint64_t turn[kHalf];                // theta_i / (2 pi) in 0.64 fixed point
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full;
@@ -71,9 +78,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::tma_prefetch_desc(&tm_x);
     tg::tma_prefetch_desc(&tm_w);
   }
-  if (tid >= 64 && tid < 64 + kHalf) {   // frequencies, fp64 (no global memory)
+  if (tid >= 64 && tid < 64 + kHalf) {   // frequencies (no global memory)
     const int i = tid - 64;
-    S.theta[i] = exp(-2.0 * i / kDh * log_base);
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    S.turn[i] = __double2ull_rn(ldexp(exp(-2.0 * i / kDh * log_base) * kInvTwoPi, 64));
   }
   tg::tc_fence_before();
   __syncthreads();
@@ -81,6 +89,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
   tg::pdl_launch_dependents();
   tg::pdl_wait();   // global memory only from here on
+
+  const int lg = warp & 3, cg = warp >> 2;
+  const int hh = cg >> 1;                 // head within the tile
+  const int i0 = (cg & 1) * 32;           // this thread's pairs: i0 .. i0+31 and +64
+  const int gh0 = n0 / kDh;               // global head index of head 0 of the tile
+  const bool rope = gh0 < n_hq + n_hkv;   // head 0 (and so any head before v) is rotated
+  const int row = lg * 32 + lane;         // row within a row tile; TMEM lane
+  // this thread's half of its rows' angles: i in [i0 + 16 hh, +16), both row tiles;
+  // (c, s) = (-cos, -sin) of the angle less pi, i.e. cos and sin of the angle itself
+  float2 cs[2][16];
+  auto angles = [&]() {
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt) {
+      const int64_t r = m0 + rt * kBM + row;
+      const int p = r < n_rows ? pos[r] : 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint64_t fx = static_cast<uint64_t>(static_cast<int64_t>(p)) * S.turn[i0 + 16 * hh + e];
+        const uint32_t fr = static_cast<uint32_t>(fx >> 32);   // turns mod 1, top 32 bits
+        // to 23 bits as a float in [1, 2] (a carry out of the top wraps to 1 turn == 0)
+        const float f1 = __uint_as_float(0x3F800000u + ((fr + 256u) >> 9));
+        const float x = (f1 - 1.5f) * 6.28318530717958648f;   // 2 pi (turns - 1/2), |x| <= pi
+        float sn, cn;
+        __sincosf(x, &sn, &cn);   // |x| <= pi: absolute error ~2^-21
+        cs[rt][e] = make_float2(-cn, -sn);
+      }
+    }
+  };
+  if (rope && warp >= 2) angles();   // under the mainloop: these warps only wait on it
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----
@@ -122,50 +159,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::mma_commit(&S.acc_full);
   }
   __syncwarp();
+  if (rope && warp < 2) angles();
 
-  // ---- epilogue: all 16 warps, the two row tiles one after the other ----
-  const int lg = warp & 3, cg = warp >> 2;
-  const int hh = cg >> 1;                 // head within the tile
-  const int i0 = (cg & 1) * 32;           // this thread's pairs: i0 .. i0+31 and +64
-  const int gh = n0 / kDh + hh;           // global head index in [q heads, k heads, v heads]
+  // ---- epilogue: all 16 warps ----
+  // Once the accumulators are complete every stage has been consumed, so the stage
+  // buffers (192 KB) hold: the angle tables of the two row tiles, [i][row] float2
+  // (64 KB each), and the bf16 output rows of one row tile (64 KB).
   const bool ok = tg::mbar_wait(&S.acc_full, 0, status, &S.abort_flag);
   if (ok) tg::tc_fence_after();
+  uint8_t* const base = &S.a[0][0][0];
+  float2* const table = reinterpret_cast<float2*>(base);   // [rt][i][row]
+  if (rope && ok) {
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) table[(rt * kHalf + i0 + 16 * hh + e) * kBM + row] = cs[rt][e];
+  }
+  // where each head of the tile goes: q, k or v, and the row stride in elements
+  auto head_dst = [&](int gh, __nv_bfloat16*& ptr, int64_t& stride) {
+    if (gh < n_hq) {
+      ptr = q + static_cast<int64_t>(gh) * kDh;
+      stride = static_cast<int64_t>(n_hq) * kDh;
+    } else if (gh < n_hq + n_hkv) {
+      ptr = k + static_cast<int64_t>(gh - n_hq) * kDh;
+      stride = static_cast<int64_t>(n_hkv) * kDh;
+    } else {
+      ptr = v + static_cast<int64_t>(gh - n_hq - n_hkv) * kDh;
+      stride = static_cast<int64_t>(n_hkv) * kDh;
+    }
+  };
+  __nv_bfloat16 *hb0, *hb1;
+  int64_t hs0, hs1;
+  head_dst(gh0, hb0, hs0);
+  head_dst(gh0 + 1, hb1, hs1);
+  const bool rot = gh0 + hh < n_hq + n_hkv;   // this thread's head is q or k
+  __syncthreads();   // angle tables written
 #pragma unroll 1
-  for (int rt = 0; rt < 2 && ok; ++rt) {
-    const int64_t r = m0 + rt * kBM + lg * 32 + lane;   // row; TMEM lane lg*32 + lane
-    uint32_t ya[32], yb[32];
-    const uint32_t base =
-        tmem + (static_cast<uint32_t>(lg * 32) << 16) + rt * kBN + hh * kDh + i0;
-    tg::tmem_ld32(base, ya);
-    tg::tmem_ld32(base + kHalf, yb);
-    tg::tmem_ld_wait();
-    if (r < n_rows) {
-      __nv_bfloat16* dst;
-      if (gh < n_hq) {
-        dst = q + (r * n_hq + gh) * kDh;
-      } else if (gh < n_hq + n_hkv) {
-        dst = k + (r * n_hkv + (gh - n_hq)) * kDh;
-      } else {
-        dst = v + (r * n_hkv + (gh - n_hq - n_hkv)) * kDh;
-      }
+  for (int rt = 0; rt < 2; ++rt) {
+    // output staging: row tile 0 after the tables, row tile 1 over table 0 (read)
+    uint8_t* const stg = rt == 0 ? base + 2 * kHalf * kBM * sizeof(float2) : base;
+    if (ok) {
+      uint32_t ya[32], yb[32];
+      const uint32_t taddr =
+          tmem + (static_cast<uint32_t>(lg * 32) << 16) + rt * kBN + hh * kDh + i0;
+      tg::tmem_ld32(taddr, ya);
+      tg::tmem_ld32(taddr + kHalf, yb);
+      tg::tmem_ld_wait();
       uint32_t oa[16], ob[16];
-      if (gh < n_hq + n_hkv) {   // q or k head: rotate each (i, i + 64) pair
-        const double p = static_cast<double>(pos[r]);
-        constexpr double kTwoPi = 6.283185307179586;
-        constexpr double kInvTwoPi = 0.15915494309189535;
+      if (rot) {   // rotate each (i, i + 64) pair
+        const float2* tb = table + (rt * kHalf + i0) * kBM + row;
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float c[2], s[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const double ang = p * S.theta[i0 + e + u];
-            const float red = static_cast<float>(fma(-kTwoPi, rint(ang * kInvTwoPi), ang));
-            __sincosf(red, &s[u], &c[u]);   // |red| <= pi: absolute error ~2^-21
-          }
+          const float2 c0 = tb[e * kBM], c1 = tb[(e + 1) * kBM];
           const float y1a = __uint_as_float(ya[e]), y1b = __uint_as_float(ya[e + 1]);
           const float y2a = __uint_as_float(yb[e]), y2b = __uint_as_float(yb[e + 1]);
-          oa[e / 2] = tg::pack_bf16x2(y1a * c[0] - y2a * s[0], y1b * c[1] - y2b * s[1]);
-          ob[e / 2] = tg::pack_bf16x2(y2a * c[0] + y1a * s[0], y2b * c[1] + y1b * s[1]);
+          oa[e / 2] = tg::pack_bf16x2(y1a * c0.x - y2a * c0.y, y1b * c1.x - y2b * c1.y);
+          ob[e / 2] = tg::pack_bf16x2(y2a * c0.x + y1a * c0.y, y2b * c1.x + y1b * c1.y);
         }
       } else {
 #pragma unroll
@@ -174,12 +223,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           ob[e / 2] = tg::pack_bf16x2(__uint_as_float(yb[e]), __uint_as_float(yb[e + 1]));
         }
       }
-      uint4* da = reinterpret_cast<uint4*>(dst + i0);
-      uint4* db = reinterpret_cast<uint4*>(dst + kHalf + i0);
+      // row `row` of the staging area: 512 bytes (two heads), 16-byte piece c at
+      // c ^ (row % 8)
+      uint8_t* const srow = stg + row * 512;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        da[u] = make_uint4(oa[4 * u], oa[4 * u + 1], oa[4 * u + 2], oa[4 * u + 3]);
-        db[u] = make_uint4(ob[4 * u], ob[4 * u + 1], ob[4 * u + 2], ob[4 * u + 3]);
+        const int ca = hh * 16 + i0 / 8 + u, cb = ca + 8;
+        *reinterpret_cast<uint4*>(srow + ((ca ^ (row & 7)) << 4)) =
+            make_uint4(oa[4 * u], oa[4 * u + 1], oa[4 * u + 2], oa[4 * u + 3]);
+        *reinterpret_cast<uint4*>(srow + ((cb ^ (row & 7)) << 4)) =
+            make_uint4(ob[4 * u], ob[4 * u + 1], ob[4 * u + 2], ob[4 * u + 3]);
+      }
+    }
+    __syncthreads();   // the row tile's outputs staged
+    if (ok) {
+      // 128 rows x 2 heads x 256 bytes: 16 threads per (row, head), whole rows out
+#pragma unroll
+      for (int pss = 0; pss < 8; ++pss) {
+        const int c = pss * kThreads + tid;
+        const int seg = c >> 4, part = c & 15;
+        const int sr = seg >> 1, h = seg & 1;
+        const int64_t r = m0 + rt * kBM + sr;
+        if (r < n_rows) {
+          const uint4 val =
+              *reinterpret_cast<const uint4*>(stg + sr * 512 + (((h * 16 + part) ^ (sr & 7)) << 4));
+          *reinterpret_cast<uint4*>((h ? hb1 : hb0) + r * (h ? hs1 : hs0) + part * 8) = val;
+        }
       }
     }
   }
