@@ -45,7 +45,8 @@ typedef enum {
   TG_ERR_WORKSPACE = 4,     /* caller-provided scratch too small */
   TG_ERR_CUDA = 5,          /* a CUDA runtime call failed (launch, attribute) */
   TG_ERR_TIMEOUT = 6,       /* device: a bounded wait ran out (see tg_device_status) */
-  TG_ERR_DEVICE_CHECK = 7   /* device: a size or index check failed, work skipped */
+  TG_ERR_DEVICE_CHECK = 7,  /* device: a size or index check failed, work skipped */
+  TG_ERR_DEBUG_BOUNDS = 8   /* device, debug library only: an index outside its buffer, access skipped */
 } tg_status;
 
 typedef enum { TG_F32 = 0, TG_BF16 = 1 } tg_dtype;
@@ -54,6 +55,18 @@ typedef struct CUstream_st* tg_stream_t; /* same type as cudaStream_t */
 
 /* Version of this ABI (bumped on any signature change). */
 int tg_abi_version(void);
+
+/*
+ * 1 in the debug library (libtokengate_debug.so, compiled with TG_DEBUG), 0 in the
+ * release library. The debug library checks the index of every data-dependent
+ * global load and store (gathers through kept indices, scatters to kept rows,
+ * cache rows, the per-sequence rows of every output) against the extent of its
+ * buffer; an index outside it skips that access and records TG_ERR_DEBUG_BOUNDS
+ * in the status word (tg_device_status), so a kernel's own index arithmetic can be
+ * checked without a memory fault and without a sanitizer. The arithmetic and the
+ * results are otherwise those of the release library, bit for bit.
+ */
+int tg_debug_build(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* tg_status_string(tg_status s);

@@ -9,7 +9,10 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtokengate.so")
+# TG_DEBUG=1 in the environment selects the debug library (index checks on every
+# data-dependent global access, TG_ERR_DEBUG_BOUNDS instead of a fault)
+LIB_PATH = os.path.join(_HERE, "libtokengate_debug.so" if os.environ.get("TG_DEBUG") == "1"
+                        else "libtokengate.so")
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
@@ -20,6 +23,7 @@ INT = ctypes.c_int
 # (name, restype, argtypes) for every symbol the header declares
 SIGNATURES = {
     "tg_abi_version": (INT, []),
+    "tg_debug_build": (INT, []),
     "tg_status_string": (ctypes.c_char_p, [INT]),
     "tg_gate_score": (INT, [P, INT, I64, INT, P, P, P, F32, INT, P, P]),
     "tg_select_topk": (INT, [P, P, P, P, P, INT, I64, I64, INT, P, P, P, P, P]),

@@ -1,6 +1,8 @@
-"""Build libtokengate.so (the C-ABI library) in-tree for sm_100a with nvcc.
+"""Build libtokengate.so (the C-ABI library) in-tree for sm_100a with nvcc, and its
+debug twin libtokengate_debug.so (TG_DEBUG: every data-dependent global access checks
+its index and records TG_ERR_DEBUG_BOUNDS instead of faulting).
 
-    python -m learned_token_pruning_gemm_b200.build [--force] [-v]
+    python -m learned_token_pruning_gemm_b200.build [--force] [--debug] [-v]
 """
 from __future__ import annotations
 
@@ -16,6 +18,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtokengate.so")
+OBJDIR_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libtokengate_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -38,9 +42,9 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose):
-    obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+def _compile(src, verbose, debug=False):
+    obj = os.path.join(OBJDIR_DEBUG if debug else OBJDIR, os.path.basename(src) + ".o")
+    cmd = [NVCC, *ARCH, *FLAGS, *(["-DTG_DEBUG=1"] if debug else []), "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -49,20 +53,22 @@ def _compile(src, verbose):
     return obj, (r.stdout + r.stderr)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale(LIB, _deps()):
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib, objdir = (LIB_DEBUG, OBJDIR_DEBUG) if debug else (LIB, OBJDIR)
+    if not force and not _stale(lib, _deps()):
+        return lib
+    os.makedirs(objdir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), _sources()))
+        results = list(ex.map(lambda s: _compile(s, verbose, debug), _sources()))
     if verbose:
         for _, log in results:
             sys.stdout.write(log)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results]])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -110,7 +110,9 @@ __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
 
 extern "C" {
 
-int tg_abi_version(void) { return 4; }
+int tg_abi_version(void) { return 5; }
+
+int tg_debug_build(void) { return tg::kDebug ? 1 : 0; }
 
 const char* tg_status_string(tg_status s) {
   switch (s) {
@@ -122,6 +124,7 @@ const char* tg_status_string(tg_status s) {
     case TG_ERR_CUDA: return "TG_ERR_CUDA";
     case TG_ERR_TIMEOUT: return "TG_ERR_TIMEOUT";
     case TG_ERR_DEVICE_CHECK: return "TG_ERR_DEVICE_CHECK";
+    case TG_ERR_DEBUG_BOUNDS: return "TG_ERR_DEBUG_BOUNDS";
   }
   return "TG_ERR_UNKNOWN";
 }

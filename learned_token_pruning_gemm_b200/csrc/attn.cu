@@ -358,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < kBN / 32; ++u) {
           const int kp = la_j * kBN + lane + 32 * u;
-          v[u] = kp < itm.w ? gl2 * s_kept[itm.z + kp] : 0.f;
+          v[u] = kp < itm.w && tg::in_bounds(itm.z + kp, total, status) ? gl2 * s_kept[itm.z + kp]
+                                                                        : 0.f;
         }
         if (++la_j > itm.y) {
           la_j = 0;
@@ -655,8 +656,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ga = t * kBM + ra, gb = t * kBM + rb;
       if (lse && cq == 0) {   // log-sum-exp of each row's logits (natural log), [n_hq, total]
         constexpr float kLn2 = 0.69314718055994531f;
-        if (ga < len) lse[static_cast<int64_t>(hq) * total + seq0 + ga] = (ma + __log2f(la)) * kLn2;
-        if (gb < len) lse[static_cast<int64_t>(hq) * total + seq0 + gb] = (mb + __log2f(lb)) * kLn2;
+        if (ga < len && tg::in_bounds(seq0 + ga, total, status))
+          lse[static_cast<int64_t>(hq) * total + seq0 + ga] = (ma + __log2f(la)) * kLn2;
+        if (gb < len && tg::in_bounds(seq0 + gb, total, status))
+          lse[static_cast<int64_t>(hq) * total + seq0 + gb] = (mb + __log2f(lb)) * kLn2;
       }
       // O / l through this warp's staging rows, 64 columns at a time: the quad
       // layout's 4-byte pieces go to shared memory (padded rows, no bank conflicts
@@ -681,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = 4 * k + (lane >> 3), cb = (lane & 7) * 16;
           const uint4 val = *reinterpret_cast<const uint4*>(stg + r * kStagePitch + cb);
           const int gr = t * kBM + row0 + r;
-          if (gr < len)
+          if (gr < len && tg::in_bounds(seq0 + gr, total, status))
             *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(
                 out + (static_cast<int64_t>(seq0 + gr) * n_hq + hq) * kD + 64 * hh) + cb) = val;
         }
@@ -739,6 +742,7 @@ __global__ void __launch_bounds__(kF32Warps * 32)
   }
   float m = -INFINITY, l = 0.f;
   for (int64_t j = j0; j <= i; ++j) {
+    if (!tg::in_bounds(j, total, status)) break;
     const float* kj = k + (j * n_hkv + kvh) * dh;
     float dot = 0.f;
 #pragma unroll

@@ -267,7 +267,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int u = 0; u < kBN / 32; ++u) {
         const int kp = j * kBN + lane + 32 * u;
-        S.bias[st][lane + 32 * u] = kp < len ? g2 * s_kept[seq0 + kp] : 0.f;
+        S.bias[st][lane + 32 * u] =
+            kp < len && tg::in_bounds(seq0 + kp, total, status) ? g2 * s_kept[seq0 + kp] : 0.f;
       }
       tg::mbar_arrive(&S.b_full[st]);
     }
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t a[32];
         tg::tmem_ld32(qa + 32 * ch, a);
         tg::tmem_ld_wait();
-        if (valid) {
+        if (valid && tg::in_bounds(seq0 + qrow, total, status)) {
           uint4* dst = reinterpret_cast<uint4*>(
               dq + (static_cast<int64_t>(seq0 + qrow) * n_hq + hq) * kD + 32 * ch);
 #pragma unroll
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = warp * 32 + lane;
     const int krow = jt * kBN + r;
     const bool kvalid = krow < len;
-    const float sk = kvalid ? s_kept[seq0 + krow] : 0.f;
+    const float sk = kvalid && tg::in_bounds(seq0 + krow, total, status) ? s_kept[seq0 + krow] : 0.f;
     const uint32_t sa = tmem_lane_addr(tmem, warp, kColST), da = tmem_lane_addr(tmem, warp, kColDPT);
     float ds_acc = 0.f;      // sum_h g_h sum_i dZ for this key
     float dz_h = 0.f, tz_h = 0.f;   // this head's sum_i dZ and sum_i dZ (q.k)
@@ -650,7 +651,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tz_h = 0.f;
       }
     }
-    if (kvalid && alive) ds_part[(static_cast<int64_t>(half) * n_hkv + kvh) * total + seq0 + krow] = ds_acc;
+    if (kvalid && alive && tg::in_bounds(seq0 + krow, total, status))
+      ds_part[(static_cast<int64_t>(half) * n_hkv + kvh) * total + seq0 + krow] = ds_acc;
     if (alive) alive = tg::mbar_wait(&S.acc_done, 0, status, &S.abort_flag);
     if (__all_sync(0xFFFFFFFFu, alive)) {
       tg::tc_fence_after();
@@ -664,7 +666,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t a[32];
           tg::tmem_ld32(aa + 32 * ch, a);
           tg::tmem_ld_wait();
-          if (kvalid && nsplit == 1) {   // the whole unit: dK, dV rows in bf16
+          if (kvalid && !tg::in_bounds(seq0 + krow, total, status)) {
+            // debug library: a row outside the kept rows is not written
+          } else if (kvalid && nsplit == 1) {   // the whole unit: dK, dV rows in bf16
             uint4* dst = reinterpret_cast<uint4*>(
                 out_base + (static_cast<int64_t>(seq0 + krow) * n_hkv + kvh) * kD + 32 * ch);
 #pragma unroll
@@ -743,6 +747,7 @@ __global__ void __launch_bounds__(128)
     acc[e] = 0.f;
   }
   for (int64_t j = j0; j <= i; ++j) {
+    if (!tg::in_bounds(j, total, status)) break;
     const float* kj = k + (j * n_hkv + kv) * dh;
     const float* vj = v + (j * n_hkv + kv) * dh;
     float qk = 0.f, dp = 0.f;
@@ -812,6 +817,7 @@ __global__ void __launch_bounds__(128)
     const float g = gain[h];
     float dzs = 0.f, tzs = 0.f;
     for (int64_t i = j; i < i1; ++i) {
+      if (!tg::in_bounds(i, total, status)) break;
       const float* qi = q + (i * n_hq + h) * dh;
       const float* di = dout + (i * n_hq + h) * dh;
       float qk = 0.f, dp = 0.f;

@@ -27,6 +27,24 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+#ifdef TG_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+
+// Debug library: true iff 0 <= i < n, else TG_ERR_DEBUG_BOUNDS is recorded and the
+// caller skips the access. Release library: always true, and the test compiles away.
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t n, int* status) {
+  if constexpr (kDebug) {
+    if (i < 0 || i >= n) {
+      set_status(status, TG_ERR_DEBUG_BOUNDS);
+      return false;
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -52,11 +52,17 @@ __global__ void __launch_bounds__(kThreads) compact_rows_kernel(CompactArgs a,
       for (; v + 224 < nv; v += 256) {   // 8 loads in flight per lane before the stores
         uint4 x[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = ld_stream(s + v + 32 * u);
+        for (int u = 0; u < 8; ++u)
+          x[u] = tg::in_bounds(sr * nv + v + 32 * u, n_src * nv, status) ? ld_stream(s + v + 32 * u)
+                                                                          : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) d[v + 32 * u] = x[u];
+        for (int u = 0; u < 8; ++u)
+          if (tg::in_bounds(r * nv + v + 32 * u, n_kept * nv, status)) d[v + 32 * u] = x[u];
       }
-      for (; v < nv; v += 32) d[v] = ld_stream(s + v);
+      for (; v < nv; v += 32)
+        if (tg::in_bounds(sr * nv + v, n_src * nv, status) &&
+            tg::in_bounds(r * nv + v, n_kept * nv, status))
+          d[v] = ld_stream(s + v);
     }
   }
 }

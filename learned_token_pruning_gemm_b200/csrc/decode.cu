@@ -297,12 +297,15 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
   const int64_t dst = (static_cast<int64_t>(b) * cap + len) * row_vecs;
+  const int64_t cache_vecs = static_cast<int64_t>(gridDim.x) * cap * row_vecs;
   for (int i = threadIdx.x; i < row_vecs; i += kThreads) {
+    if (!tg::in_bounds(dst + i, cache_vecs, status)) break;
     k_cache[dst + i] = k_new[static_cast<int64_t>(b) * row_vecs + i];
     v_cache[dst + i] = v_new[static_cast<int64_t>(b) * row_vecs + i];
   }
   __syncthreads();   // every thread has read cache_len[b] before it moves
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 &&
+      tg::in_bounds(static_cast<int64_t>(b) * cap + len, static_cast<int64_t>(gridDim.x) * cap, status)) {
     s_cache[static_cast<int64_t>(b) * cap + len] = s_new[b];
     cache_len[b] = len + 1;
   }

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   // ---- stage k and q (rows past the chunk's end are zero); decays and writes ----
   for (int i = tid; i < kC * 16; i += kThreads) {
     const int r = i >> 4, p = i & 15;
-    const bool ok = r < L;
+    const bool ok = r < L && tg::in_bounds(t0 + r, total, status);
     const int64_t row = (t0 + (ok ? r : 0)) * n_heads + h;
     cp16(&S.k[r][p * 8], k + row * kDk + p * 8, ok);
     cp16(&S.qv[r][p * 8], q + row * kDk + p * 8, ok);
@@ -614,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int r = ra + 8 * hf;
-        if (r < L) {
+        if (r < L && tg::in_bounds(t0 + r, total, status)) {
           const int col = c0 + 8 * j + 2 * (lane & 3);
           *reinterpret_cast<__nv_bfloat162*>(out + ((t0 + r) * n_heads + h) * dv + col) =
               __floats2bfloat162_rn(o[j][2 * hf], o[j][2 * hf + 1]);

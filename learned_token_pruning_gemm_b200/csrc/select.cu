@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t o0 = out_base < total_kept ? out_base : total_kept;
     const int64_t o1 = out_base + count < total_kept ? out_base + count : total_kept;
     for (int64_t r = o0 + (int64_t)rank * kThreads + tid; r < o1; r += (int64_t)csize * kThreads) {
+      if (!tg::in_bounds(r, total_kept, status)) break;
       kept_idx[r] = -1;
       if (kept_scores) kept_scores[r] = 0.f;
       if (kept_pos) kept_pos[r] = -1;
@@ -202,7 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int i = i0 + u * kThreads;
-        v[u] = i < n_local ? scores[base + c0 + i] : 0.f;
+        v[u] = i < n_local && tg::in_bounds(base + c0 + i, total_tokens, status)
+                   ? scores[base + c0 + i]
+                   : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
@@ -399,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool eq = in_doc && key == T;
         const bool keep = i < n_local && (!in_doc || key > T || (eq && rk < need));
         rk += eq;
-        if (keep) {
+        if (keep && tg::in_bounds(o, total_kept, status)) {
           kept_idx[o] = (int32_t)(base + c0 + i);
           if (kept_scores) kept_scores[o] = raw[i];
           if (kept_pos) kept_pos[o] = (int32_t)(c0 + i);

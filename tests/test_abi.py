@@ -31,10 +31,25 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(_lib.SIGNATURES), "binding signatures cover the header"
 
 
+def test_debug_library_exports_the_same_abi(lib):
+    # the debug twin (device index checks) builds too and exports every declared
+    # symbol; each library says which it is
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(dbg, n), n
+    dbg.tg_debug_build.restype = ctypes.c_int
+    assert dbg.tg_debug_build() == 1
+    assert lib.tg_debug_build() == 0
+    dbg.tg_status_string.restype = ctypes.c_char_p
+    assert dbg.tg_status_string(8).decode() == "TG_ERR_DEBUG_BOUNDS"
+
+
 def test_status_strings(lib):
-    assert lib.tg_abi_version() == 4
+    assert lib.tg_abi_version() == 5
     for code, name in [(0, "TG_OK"), (1, "TG_ERR_INVALID_ARG"), (3, "TG_ERR_MISALIGNED"),
-                       (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (99, "TG_ERR_UNKNOWN")]:
+                       (6, "TG_ERR_TIMEOUT"), (7, "TG_ERR_DEVICE_CHECK"), (8, "TG_ERR_DEBUG_BOUNDS"),
+                       (99, "TG_ERR_UNKNOWN")]:
         assert lib.tg_status_string(code).decode() == name
 
 
