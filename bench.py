@@ -262,7 +262,7 @@ def _stages_report(work, stage_ms, tf_peak, hbm_peak):
             e["gbs"] = work["compact_bytes"] / t / 1e9
         elif name == "attention":
             e["tflops"] = work["attn_flops"] / t / 1e12
-        elif name == "project":
+        elif name in ("project", "compact+project"):
             e["tflops"] = work["project_flops"] / t / 1e12
         if "tflops" in e:
             e["frac_tc"] = e["tflops"] / tf_peak
@@ -279,7 +279,7 @@ def _stages_report(work, stage_ms, tf_peak, hbm_peak):
 
 def _roofline(work, stage_ms, tf_peak, hbm_peak, peak_src, workload):
     """The dominant kernel of the step against its bound."""
-    dom = max((n for n in stage_ms if n != "project"), key=stage_ms.get)
+    dom = max((n for n in stage_ms if "project" not in n), key=stage_ms.get)
     t = stage_ms[dom] / 1e3
     if dom == "attention":
         ach, peak, unit, bound = work["attn_flops"] / t / 1e12, tf_peak, "TFLOP/s", "tensor"

@@ -222,6 +222,24 @@ tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const void* w_qkv, 
                       void* k, void* v, tg_stream_t stream);
 
 /*
+ * The compaction fused into the projection (same section): tg_qkv_rope on the rows
+ * xc[r] = x[kept_idx[r]], read straight from the full residual, so the projection
+ * does not wait for a separate compaction. The compacted rows themselves are also
+ * written to xc when xc != NULL (the layers above the gate layer carry them on).
+ * q, k, v are bit-identical to tg_compact_kv followed by tg_qkv_rope.
+ *   x        [n_src, d] bf16 device: the residual rows at the gate layer
+ *   kept_idx [n_rows] int32 device: row ids into x (tg_select_topk's kept_idx); an
+ *            id outside [0, n_src) projects a zero row, leaves that xc row as it
+ *            was and records TG_ERR_DEVICE_CHECK
+ *   xc       [n_rows, d] bf16 device output, or NULL
+ *   pos, w_qkv, q, k, v, and the shape rules: as tg_qkv_rope (n_src <= INT32_MAX).
+ */
+tg_status tg_compact_qkv_rope(const void* x, int64_t n_src, int d, const int32_t* kept_idx,
+                              int64_t n_rows, void* xc, const void* w_qkv, int n_hq, int n_hkv,
+                              int head_dim, float rope_base, const int32_t* pos, void* q, void* k,
+                              void* v, tg_stream_t stream);
+
+/*
  * Decode over the compacted cache (MarkTechPost page on TokenGate, section
  * "Comment déployer TokenGate ?": generation runs on the cache the pruned prefill
  * leaves, bounded by max_kept_prefill_tokens; section "Qu'est-ce que l'attention

@@ -33,6 +33,7 @@ SIGNATURES = {
     "tg_gated_attention_bwd": (INT, [P, P, P, P, P, INT, P, P, P, P, P, INT, I64, INT, INT, INT,
                                      INT, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
     "tg_qkv_rope": (INT, [P, I64, INT, P, INT, INT, INT, F32, P, P, P, P, P]),
+    "tg_compact_qkv_rope": (INT, [P, I64, INT, P, I64, P, P, INT, INT, INT, F32, P, P, P, P, P]),
     "tg_cache_append": (INT, [P, P, P, INT, INT, INT, INT, P, P, P, P, P]),
     "tg_gated_decode_workspace_size": (ctypes.c_size_t, [INT, INT, INT, INT]),
     "tg_gated_decode": (INT, [P, P, P, P, P, INT, INT, INT, INT, INT, INT, P, P, P, P,

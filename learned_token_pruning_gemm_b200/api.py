@@ -286,6 +286,43 @@ def qkv_rope(xc: torch.Tensor, w_qkv: torch.Tensor, n_hq: int, n_hkv: int, pos: 
     return q, k, v
 
 
+def compact_qkv_rope(x: torch.Tensor, kept_idx: torch.Tensor, w_qkv: torch.Tensor, n_hq: int,
+                     n_hkv: int, pos: torch.Tensor, rope_base: float = 1e6, xc=None, out=None,
+                     write_xc: bool = True, stream=None):
+    """The compaction fused into the projections: xc = x[kept_idx] (written when
+    write_xc, into `xc` if given) and (q, k, v) of those rows, as qkv_rope(xc, ...)
+    would give them, in one kernel that gathers the rows from x itself. x [N,d] bf16,
+    kept_idx [K] int32. Returns (xc or None, q, k, v)."""
+    N, d = x.shape
+    K = kept_idx.numel()
+    n_out = w_qkv.shape[0]
+    if (n_out % (n_hq + 2 * n_hkv)) or w_qkv.shape[1] != d or x.dtype != w_qkv.dtype:
+        raise TokenGateError("compact_qkv_rope: w_qkv [(Hq+2Hkv)*dh, d] with the dtype of x")
+    dh = n_out // (n_hq + 2 * n_hkv)
+    _numel(pos, K, "pos")
+    if write_xc:
+        if xc is None:
+            xc = torch.empty(K, d, dtype=x.dtype, device=x.device)
+        _shape(xc, (K, d), "xc", x.dtype)
+    elif xc is not None:
+        raise TokenGateError("compact_qkv_rope: xc given with write_xc=False")
+    if out is None:
+        out = (torch.empty(K, n_hq, dh, dtype=x.dtype, device=x.device),
+               torch.empty(K, n_hkv, dh, dtype=x.dtype, device=x.device),
+               torch.empty(K, n_hkv, dh, dtype=x.dtype, device=x.device))
+    q, k, v = out
+    _shape(q, (K, n_hq, dh), "q", x.dtype)
+    _shape(k, (K, n_hkv, dh), "k", x.dtype)
+    _shape(v, (K, n_hkv, dh), "v", x.dtype)
+    st = _lib.load().tg_compact_qkv_rope(
+        _cuda(x, "x", torch.bfloat16), N, d, _cuda(kept_idx, "kept_idx", torch.int32), K,
+        _cuda(xc, "xc") if xc is not None else None, _cuda(w_qkv, "w_qkv", torch.bfloat16),
+        n_hq, n_hkv, dh, float(rope_base), _cuda(pos, "pos", torch.int32), _cuda(q, "q"),
+        _cuda(k, "k"), _cuda(v, "v"), _stream(stream))
+    check(st, "tg_compact_qkv_rope")
+    return xc, q, k, v
+
+
 def cache_append(k_new: torch.Tensor, v_new: torch.Tensor, s_new: torch.Tensor,
                  k_cache: torch.Tensor, v_cache: torch.Tensor, s_cache: torch.Tensor,
                  cache_len: torch.Tensor, stream=None) -> None:

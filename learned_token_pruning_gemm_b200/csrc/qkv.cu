@@ -24,6 +24,16 @@
 // every rotate-half pair is in one thread; the rotation and the bf16 rounding are
 // fp32; the rows go through shared memory (16-byte pieces, XOR-swizzled across
 // the eight rows that share banks) and leave as whole 256-byte head rows.
+//
+// tg_compact_qkv_rope runs the same kernel on the rows of the full residual named
+// by kept_idx, so the compaction is fused into the projection: four warps that
+// otherwise only wait on the accumulators gather each stage's 2 x 128 rows x 128
+// bytes with 16-byte cp.async copies straight into the swizzled stage layout
+// (each thread one 16-byte column of 16 rows; rows past the end are zero-filled),
+// and the stage completes on their arrivals plus the W tile's TMA bytes; the MMA
+// thread orders those generic-proxy writes before its tensor-core reads with a
+// proxy fence. The compacted rows are written out on the way: of every k-block,
+// the CTAs of one column tile load it through registers and store it to xc too.
 #include "common.cuh"
 
 namespace {
@@ -36,6 +46,23 @@ constexpr int kThreads = 512;
 constexpr int kDh = 128;
 constexpr int kHalf = kDh / 2;
 
+constexpr int kGatherWarp0 = 12;             // gather mode: warps 12..15 gather the rows
+constexpr int kGatherThreads = kThreads - kGatherWarp0 * 32;
+static_assert(kGatherThreads == 128, "one 16-byte column of 16 rows per gather thread");
+
+// 16 bytes global -> shared, or 16 zero bytes when !ok (src is not read then)
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tg::smem_u32(dst)), "l"(src),
+               "r"(ok ? 16 : 0)
+               : "memory");
+}
+// one arrival on bar once this thread's earlier cp.async copies have landed
+__device__ __forceinline__ void cp_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tg::smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 struct QkvSmem {
   uint8_t a[kStages][2][kBM * kBK * 2];   // two xc tiles, 16 KB each
   uint8_t b[kStages][kBN * kBK * 2];   // W tiles, 32 KB
@@ -47,11 +74,17 @@ struct QkvSmem {
   int abort_flag;
 };
 
+// kGather: the rows are x[kept_idx[r]] (n_src rows of x), gathered by warps 12..15,
+// and xc (if not null) receives them; otherwise tm_x maps the compacted rows.
+template <bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                     int64_t n_rows, int d, int n_hq, int n_hkv, double log_base,
                     const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ q,
-                    __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v, int* status) {
+                    __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
+                    const __nv_bfloat16* __restrict__ x, int64_t n_src,
+                    const int32_t* __restrict__ kept_idx, __nv_bfloat16* __restrict__ xc,
+                    int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (tg::smem_u32(smem_raw) & 1023u)) & 1023u;
   QkvSmem& S = *reinterpret_cast<QkvSmem*>(smem_raw + pad);
@@ -63,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tg::mbar_init(&S.full[s], 1);
+      tg::mbar_init(&S.full[s], kGather ? 1 + kGatherThreads : 1);
       tg::mbar_init(&S.empty[s], 1);
     }
     tg::mbar_init(&S.acc_full, 1);
@@ -75,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tg::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tg::tma_prefetch_desc(&tm_x);
+    if (!kGather) tg::tma_prefetch_desc(&tm_x);
     tg::tma_prefetch_desc(&tm_w);
   }
   if (tid >= 64 && tid < 64 + kHalf) {   // frequencies (no global memory)
@@ -117,7 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
-  if (rope && warp >= 2) angles();   // under the mainloop: these warps only wait on it
+  const bool gather_warp = kGather && warp >= kGatherWarp0;
+  if (rope && warp >= 2 && !gather_warp) angles();   // under the mainloop: these warps only wait
+
 
   if (warp == 0 && lane == 0) {
     // ---- TMA producer ----
@@ -127,9 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kb >= kStages &&
           !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
         break;
-      tg::mbar_arrive_expect_tx(&S.full[s], (2 * kBM + kBN) * kBK * 2);
-      tg::tma_load_2d(S.a[s][0], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
-      tg::tma_load_2d(S.a[s][1], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0 + kBM));
+      if (kGather) {   // W only: the rows come from the gather warps
+        tg::mbar_arrive_expect_tx(&S.full[s], kBN * kBK * 2);
+      } else {
+        tg::mbar_arrive_expect_tx(&S.full[s], (2 * kBM + kBN) * kBK * 2);
+        tg::tma_load_2d(S.a[s][0], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0));
+        tg::tma_load_2d(S.a[s][1], &tm_x, &S.full[s], kb * kBK, static_cast<int>(m0 + kBM));
+      }
       tg::tma_load_2d(S.b[s], &tm_w, &S.full[s], kb * kBK, n0);
       ++issued;
     }
@@ -143,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % kStages;
       if (!tg::mbar_wait(&S.full[s], (kb / kStages) & 1, status, &S.abort_flag)) break;
+      if (kGather) tg::fence_proxy_async_shared();   // the gathered rows: generic-proxy writes
       tg::tc_fence_after();
       const uint32_t a0 = tg::smem_u32(S.a[s][0]), a1 = tg::smem_u32(S.a[s][1]);
       const uint32_t b0 = tg::smem_u32(S.b[s]);
@@ -157,9 +197,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       tg::mma_commit(&S.empty[s]);
     }
     tg::mma_commit(&S.acc_full);
+  } else if (gather_warp) {
+    // ---- row gather: thread gt owns 16-byte column c of rows r0 + 16u, u < 16, of
+    //      the stage's two row tiles (a warp covers four whole 128-byte rows) ----
+    const int gt = tid - kGatherWarp0 * 32;
+    const int c = gt & 7, r0 = gt >> 3;
+    int32_t src[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int64_t r = m0 + r0 + 16 * u;
+      int32_t sr = -1;
+      if (r < n_rows) {
+        sr = kept_idx[r];
+        if (sr < 0 || sr >= n_src) {   // not a row of x: zeros, and the error recorded
+          tg::set_status(status, TG_ERR_DEVICE_CHECK);
+          sr = -1;
+        }
+      }
+      src[u] = sr;
+    }
+    const int n_ct = static_cast<int>(gridDim.y);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (kb >= kStages &&
+          !tg::mbar_wait(&S.empty[s], ((kb / kStages) - 1) & 1, status, &S.abort_flag))
+        break;
+      const int64_t col = static_cast<int64_t>(kb) * kBK + 8 * c;
+      if (xc && kb % n_ct == static_cast<int>(blockIdx.y)) {
+        // this CTA also writes k-block kb of the compacted rows: through registers
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = r0 + 16 * u, rr = r & (kBM - 1);
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (src[u] >= 0) {
+            val = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(src[u]) * d + col);
+            if (tg::in_bounds(m0 + r, n_rows, status))
+              *reinterpret_cast<uint4*>(xc + (m0 + r) * d + col) = val;
+          }
+          *reinterpret_cast<uint4*>(S.a[s][r >> 7] + rr * 128 + ((c ^ (rr & 7)) << 4)) = val;
+        }
+        tg::mbar_arrive(&S.full[s]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = r0 + 16 * u, rr = r & (kBM - 1);
+          const bool ok = src[u] >= 0;
+          cp16(S.a[s][r >> 7] + rr * 128 + ((c ^ (rr & 7)) << 4),
+               x + (ok ? static_cast<int64_t>(src[u]) * d + col : 0), ok);
+        }
+        cp_arrive(&S.full[s]);
+      }
+    }
+    cp_wait_all();   // no copy may land after the CTA has moved on
   }
   __syncwarp();
-  if (rope && warp < 2) angles();
+  if (rope && (warp < 2 || gather_warp)) angles();
 
   // ---- epilogue: all 16 warps ----
   // Once the accumulators are complete every stage has been consumed, so the stage
@@ -262,42 +354,75 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+namespace {
+
+// both entry points: validation, the W map (and the xc map unless gathering), launch
+tg_status launch_qkv(const void* xc, const void* x, int64_t n_src, const int32_t* kept_idx,
+                     void* xc_out, int64_t n_rows, int d, const void* w_qkv, int n_hq, int n_hkv,
+                     int head_dim, float rope_base, const int32_t* pos, void* q, void* k, void* v,
+                     cudaStream_t stream) {
+  const bool gather = x != nullptr;
+  if (n_rows < 0 || d <= 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0) return TG_ERR_INVALID_ARG;
+  if (gather && n_src <= 0) return TG_ERR_INVALID_ARG;
+  if (!(rope_base > 1.0f)) return TG_ERR_INVALID_ARG;
+  if (n_rows == 0) return TG_OK;
+  if ((gather ? !kept_idx : !xc) || !w_qkv || !pos || !q || !k || !v) return TG_ERR_INVALID_ARG;
+  if (head_dim != kDh || d % kBK != 0 || (n_hq + 2 * n_hkv) % 2 != 0) return TG_ERR_UNSUPPORTED;
+  if (n_rows > INT32_MAX - kBM || (n_rows + kBM - 1) / kBM > INT32_MAX) return TG_ERR_UNSUPPORTED;
+  if (gather && n_src > INT32_MAX) return TG_ERR_UNSUPPORTED;
+  const int64_t n_out = static_cast<int64_t>(n_hq + 2 * n_hkv) * kDh;
+  if (n_out / kBN > 65535) return TG_ERR_UNSUPPORTED;
+  if (!tg::aligned16(gather ? x : xc) || !tg::aligned16(w_qkv) || !tg::aligned16(q) ||
+      !tg::aligned16(k) || !tg::aligned16(v) || (xc_out && !tg::aligned16(xc_out)))
+    return TG_ERR_MISALIGNED;
+  int* status = tg::status_word();
+  if (!status) return TG_ERR_CUDA;
+  CUtensorMap tx = {}, tw;
+  const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
+  const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_out)};
+  const uint32_t bw[2] = {kBK, kBN};
+  if (!tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_qkv, dw, sx, bw,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+    return TG_ERR_CUDA;
+  if (!gather) {
+    const uint64_t dx[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_rows)};
+    const uint32_t bx[2] = {kBK, kBM};
+    if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xc, dx, sx, bx,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+      return TG_ERR_CUDA;
+  }
+  const size_t smem = sizeof(QkvSmem) + 1024;
+  auto kernel = gather ? qkv_rope_kernel<true> : qkv_rope_kernel<false>;
+  if (!tg::ensure_smem(reinterpret_cast<const void*>(kernel), static_cast<int>(smem)))
+    return TG_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((n_rows + 2 * kBM - 1) / (2 * kBM)),
+                  static_cast<unsigned>(n_out / kBN));
+  return tg::launch(kernel, grid, dim3(kThreads), smem, stream, 0, tx, tw, n_rows, d, n_hq, n_hkv,
+                    log(static_cast<double>(rope_base)), pos, static_cast<__nv_bfloat16*>(q),
+                    static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v),
+                    static_cast<const __nv_bfloat16*>(x), n_src, kept_idx,
+                    static_cast<__nv_bfloat16*>(xc_out), status);
+}
+
+}  // namespace
+
 extern "C" tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const void* w_qkv,
                                  int n_hq, int n_hkv, int head_dim, float rope_base,
                                  const int32_t* pos, void* q, void* k, void* v,
                                  tg_stream_t stream) {
   tg::NvtxRange nvtx_range("tg_qkv_rope");
-  if (n_rows < 0 || d <= 0 || n_hq <= 0 || n_hkv <= 0 || head_dim <= 0) return TG_ERR_INVALID_ARG;
-  if (!(rope_base > 1.0f)) return TG_ERR_INVALID_ARG;
-  if (n_rows == 0) return TG_OK;
-  if (!xc || !w_qkv || !pos || !q || !k || !v) return TG_ERR_INVALID_ARG;
-  if (head_dim != kDh || d % kBK != 0 || (n_hq + 2 * n_hkv) % 2 != 0) return TG_ERR_UNSUPPORTED;
-  if (n_rows > INT32_MAX - kBM || (n_rows + kBM - 1) / kBM > INT32_MAX) return TG_ERR_UNSUPPORTED;
-  const int64_t n_out = static_cast<int64_t>(n_hq + 2 * n_hkv) * kDh;
-  if (n_out / kBN > 65535) return TG_ERR_UNSUPPORTED;
-  if (!tg::aligned16(xc) || !tg::aligned16(w_qkv) || !tg::aligned16(q) || !tg::aligned16(k) ||
-      !tg::aligned16(v))
-    return TG_ERR_MISALIGNED;
-  int* status = tg::status_word();
-  if (!status) return TG_ERR_CUDA;
-  CUtensorMap tx, tw;
-  const uint64_t dx[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_rows)};
-  const uint64_t sx[1] = {static_cast<uint64_t>(d) * 2};
-  const uint32_t bx[2] = {kBK, kBM};
-  const uint64_t dw[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(n_out)};
-  const uint32_t bw[2] = {kBK, kBN};
-  if (!tg::encode_tmap(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, xc, dx, sx, bx,
-                       CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !tg::encode_tmap(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_qkv, dw, sx, bw,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
-    return TG_ERR_CUDA;
-  const size_t smem = sizeof(QkvSmem) + 1024;
-  if (!tg::ensure_smem(reinterpret_cast<const void*>(qkv_rope_kernel), static_cast<int>(smem)))
-    return TG_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>((n_rows + 2 * kBM - 1) / (2 * kBM)),
-                  static_cast<unsigned>(n_out / kBN));
-  return tg::launch(qkv_rope_kernel, grid, dim3(kThreads), smem, stream, 0, tx, tw, n_rows, d, n_hq,
-                    n_hkv, log(static_cast<double>(rope_base)), pos,
-                    static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
-                    static_cast<__nv_bfloat16*>(v), status);
+  if (!xc && n_rows > 0) return TG_ERR_INVALID_ARG;
+  return launch_qkv(xc, nullptr, 0, nullptr, nullptr, n_rows, d, w_qkv, n_hq, n_hkv, head_dim,
+                    rope_base, pos, q, k, v, stream);
+}
+
+extern "C" tg_status tg_compact_qkv_rope(const void* x, int64_t n_src, int d,
+                                         const int32_t* kept_idx, int64_t n_rows, void* xc,
+                                         const void* w_qkv, int n_hq, int n_hkv, int head_dim,
+                                         float rope_base, const int32_t* pos, void* q, void* k,
+                                         void* v, tg_stream_t stream) {
+  tg::NvtxRange nvtx_range("tg_compact_qkv_rope");
+  if (!x && n_rows > 0) return TG_ERR_INVALID_ARG;
+  return launch_qkv(nullptr, x, n_src, kept_idx, xc, n_rows, d, w_qkv, n_hq, n_hkv, head_dim,
+                    rope_base, pos, q, k, v, stream);
 }

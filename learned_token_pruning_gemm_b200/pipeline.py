@@ -9,8 +9,13 @@ Two modes. By default the attention inputs q/k/v are supplied already compacted
 selection: this is the measured metric (gate + top-K + attention). With
 `project=True` the layer above the gate layer computes them itself: the kept
 residual rows' q/k/v projections with the rotary embedding at each kept token's
-original position (tg_qkv_rope on the compacted rows), so the KV entries exist
-for the kept tokens only, and attention reads those.
+original position, so the KV entries exist for the kept tokens only, and
+attention reads those: tg_compact_kv, then tg_qkv_rope on the compacted rows.
+`fuse=True` runs the compaction fused into the projection instead
+(tg_compact_qkv_rope gathers the kept rows from the residual itself and writes the
+compacted rows on the way): the same outputs bit for bit, but slower on a B200,
+because its 16-byte row gathers feed the tensor cores less steadily than TMA
+loads of rows that the compaction has already made contiguous.
 """
 from __future__ import annotations
 
@@ -28,7 +33,7 @@ class GatedPrefill:
 
     def __init__(self, wl: Workload, device: str = "cuda", use_score_override: bool = True,
                  project: bool = False, w_qkv: Optional[torch.Tensor] = None,
-                 rope_base: float = 1e6):
+                 rope_base: float = 1e6, fuse: bool = False):
         dev = torch.device(device)
         self.wl = wl
         self.project = project
@@ -72,7 +77,9 @@ class GatedPrefill:
         else:
             self.w_qkv = None
             self.kept_pos = None
-        self.STAGES = (("gate", "select", "compact", "project", "attention") if project
+        self.fuse = project and fuse
+        self.STAGES = (("gate", "select", "compact+project", "attention") if self.fuse
+                       else ("gate", "select", "compact", "project", "attention") if project
                        else ("gate", "select", "compact", "attention"))
         self.LAUNCHES_PER_STEP = len(self.STAGES)
 
@@ -93,6 +100,11 @@ class GatedPrefill:
         api.qkv_rope(self.xc, self.w_qkv, self.wl.hq, self.wl.hkv, self.kept_pos,
                      rope_base=self.rope_base, out=(self.q, self.k, self.v), stream=stream)
 
+    def stage_compact_project(self, stream=None):
+        api.compact_qkv_rope(self.x, self.kept_idx, self.w_qkv, self.wl.hq, self.wl.hkv,
+                             self.kept_pos, rope_base=self.rope_base, xc=self.xc,
+                             out=(self.q, self.k, self.v), stream=stream)
+
     def stage_attention(self, stream=None):
         api.gated_attention(self.q, self.k, self.v, self.kept_scores, self.gain, self.tau,
                             self.cu_kept, self.max_kept, out=self.out, stream=stream)
@@ -103,7 +115,7 @@ class GatedPrefill:
         tail). If `events` is a list of len(STAGES)+1 CUDA events, they are recorded
         on the stream before, between and after the stages."""
         s = stream if stream is not None else torch.cuda.current_stream()
-        fns = [getattr(self, "stage_" + n) for n in self.STAGES]
+        fns = [getattr(self, "stage_" + n.replace("+", "_")) for n in self.STAGES]
         for i, fn in enumerate(fns):
             if events is not None:
                 events[i].record(s)

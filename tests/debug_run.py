@@ -19,9 +19,10 @@ def main(path):
     res = {"debug_build": int(lib.tg_debug_build())}
     api.device_status(reset=True)
     # the layer, bf16 with the kept rows' projections on a ragged batch, and fp32
-    for name, proj in (("ragged8", True), ("tiny_f32", False)):
-        wl = synth.WORKLOADS[name]()
-        gp = pipeline.GatedPrefill(wl, project=proj)
+    for name, proj, fuse in (("ragged8", True, False), ("ragged8_fused", True, True),
+                             ("tiny_f32", False, False)):
+        wl = synth.WORKLOADS[name.replace("_fused", "")]()
+        gp = pipeline.GatedPrefill(wl, project=proj, fuse=fuse)
         gp.step()
         torch.cuda.synchronize()
         for attr in ("scores", "kept_idx", "kept_scores", "cu_kept", "kept_pos", "xc", "q", "k",

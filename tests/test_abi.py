@@ -112,6 +112,27 @@ def test_validation_returns_status_without_gpu(lib):
                            None) == MIS
     assert lib.tg_qkv_rope(None, 0, 2048, None, 16, 8, 128, 1e6, None, None, None, None,
                            None) == 0
+    # the same rules for the fused compaction + projection, plus its own: x, kept_idx
+    # and n_src > 0 required, xc optional (and aligned when given)
+    cq = lib.tg_compact_qkv_rope
+    assert cq(fake, 4096, 2048, fake, 100, fake, fake, 16, 8, 64, 1e6, fake, fake, fake, fake,
+              None) == UNSUP
+    assert cq(fake, 4096, 2000, fake, 100, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == UNSUP
+    assert cq(fake, 0, 2048, fake, 100, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == INVALID
+    assert cq(None, 4096, 2048, fake, 100, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == INVALID
+    assert cq(fake, 4096, 2048, None, 100, fake, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == INVALID
+    assert cq(fake, 4096, 2048, fake, 100, fake, fake, 16, 8, 128, 0.5, fake, fake, fake, fake,
+              None) == INVALID
+    assert cq(fake, 4096, 2048, fake, 100, odd, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == MIS
+    assert cq(odd, 4096, 2048, fake, 100, None, fake, 16, 8, 128, 1e6, fake, fake, fake, fake,
+              None) == MIS
+    assert cq(None, 0, 2048, None, 0, None, None, 16, 8, 128, 1e6, None, None, None, None,
+              None) == 0
 
 
 

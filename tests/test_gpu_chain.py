@@ -134,3 +134,56 @@ def test_rejected_sequence_leaves_defined_outputs(mods, orc):
     api.gated_attention(q.float(), kv.float(), kv.float(), ks, g, t, d([0, -40, total]), total,
                         out=sentinel.float())
     assert api.device_status(reset=True) == 7
+
+
+@pytest.mark.parametrize("name", ["qwen16k", "ragged8"])
+def test_fused_compaction_matches_separate_kernels(mods, name):
+    # the projection gathering the kept rows itself (and writing the compacted rows)
+    # against tg_compact_kv then tg_qkv_rope: the same rows, k-blocks and order, so
+    # every output is bit-identical
+    api, pipeline, synth = mods
+    wl = synth.WORKLOADS[name]()
+    fused = pipeline.GatedPrefill(wl, project=True, fuse=True)
+    sep = pipeline.GatedPrefill(wl, project=True)
+    assert fused.STAGES == ("gate", "select", "compact+project", "attention")
+    fused.step()
+    sep.step()
+    torch.cuda.synchronize()
+    assert api.device_status(reset=True) == 0
+    for attr in ("kept_idx", "xc", "q", "k", "v", "out"):
+        assert torch.equal(getattr(fused, attr), getattr(sep, attr)), attr
+
+
+def test_fused_compaction_odd_shapes_and_bad_index(mods):
+    # 300 of 700 rows (a ragged last row tile), d = 192 (three k-blocks, fewer than the
+    # four column tiles that share the compacted rows' writes), 6 q heads and 1 KV head
+    # (a column tile holding a k head and a v head)
+    api, _, _ = mods
+    g = torch.Generator().manual_seed(5)
+    N, d, hq, hkv = 700, 192, 6, 1
+    x = torch.randn(N, d, generator=g).to(torch.bfloat16).cuda()
+    w = (torch.randn((hq + 2 * hkv) * 128, d, generator=g) / d ** 0.5).to(torch.bfloat16).cuda()
+    idx = torch.sort(torch.randperm(N, generator=g)[:300])[0].to(torch.int32).cuda()
+    pos = torch.randint(0, 100000, (300,), generator=g, dtype=torch.int32).cuda()
+    xc, q, k, v = api.compact_qkv_rope(x, idx, w, hq, hkv, pos)
+    assert api.device_status(reset=True) == 0
+    xc2 = x[idx.long()]
+    q2, k2, v2 = api.qkv_rope(xc2, w, hq, hkv, pos)
+    assert torch.equal(xc, xc2)
+    for a, b in ((q, q2), (k, k2), (v, v2)):
+        assert torch.equal(a, b)
+    # without the compacted rows written
+    xn, q3, _, _ = api.compact_qkv_rope(x, idx, w, hq, hkv, pos, write_xc=False)
+    assert xn is None and torch.equal(q3, q2)
+    # an id outside x: recorded, that row projects as zeros, its xc row is left alone
+    bad = idx.clone()
+    bad[5] = N + 3
+    xcb = torch.full((300, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    _, qb, kb, vb = api.compact_qkv_rope(x, bad, w, hq, hkv, pos, xc=xcb)
+    assert api.device_status(reset=True) == 7
+    assert (xcb[5] == 7.0).all()
+    for t in (qb, kb, vb):
+        assert (t[5] == 0).all()
+    keep = torch.ones(300, dtype=torch.bool, device="cuda")
+    keep[5] = False
+    assert torch.equal(xcb[keep], xc2[keep]) and torch.equal(qb[keep], q2[keep])
