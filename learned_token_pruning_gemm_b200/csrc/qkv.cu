@@ -22,8 +22,10 @@
 // warps, one row tile after the other: warp w reads TMEM lanes 32*(w%4).. and, of
 // head (w/4)/2 of the tile, the pairs i in [32*((w/4)%2), +32) and i + 64, so
 // every rotate-half pair is in one thread; the rotation and the bf16 rounding are
-// fp32; the rows go through shared memory (16-byte pieces, XOR-swizzled across
-// the eight rows that share banks) and leave as whole 256-byte head rows.
+// fp32; the rows are staged in shared memory as the output maps' boxes (64 columns
+// x 128 rows, 128-byte swizzle) and leave as TMA tensor stores, so the second row
+// tile's rotation runs while the first one's stores drain (rows past the last are
+// clipped by the maps).
 //
 // tg_compact_qkv_rope runs the same kernel on the rows of the full residual named
 // by kept_idx, so the compaction is fused into the projection: four warps that
@@ -79,6 +81,8 @@ struct QkvSmem {
 template <bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_oq, const __grid_constant__ CUtensorMap tm_ok,
+                    const __grid_constant__ CUtensorMap tm_ov,
                     int64_t n_rows, int d, int n_hq, int n_hkv, double log_base,
                     const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ q,
                     __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ v,
@@ -267,28 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 16; ++e) table[(rt * kHalf + i0 + 16 * hh + e) * kBM + row] = cs[rt][e];
   }
-  // where each head of the tile goes: q, k or v, and the row stride in elements
-  auto head_dst = [&](int gh, __nv_bfloat16*& ptr, int64_t& stride) {
-    if (gh < n_hq) {
-      ptr = q + static_cast<int64_t>(gh) * kDh;
-      stride = static_cast<int64_t>(n_hq) * kDh;
-    } else if (gh < n_hq + n_hkv) {
-      ptr = k + static_cast<int64_t>(gh - n_hq) * kDh;
-      stride = static_cast<int64_t>(n_hkv) * kDh;
-    } else {
-      ptr = v + static_cast<int64_t>(gh - n_hq - n_hkv) * kDh;
-      stride = static_cast<int64_t>(n_hkv) * kDh;
-    }
-  };
-  __nv_bfloat16 *hb0, *hb1;
-  int64_t hs0, hs1;
-  head_dst(gh0, hb0, hs0);
-  head_dst(gh0 + 1, hb1, hs1);
   const bool rot = gh0 + hh < n_hq + n_hkv;   // this thread's head is q or k
   __syncthreads();   // angle tables written
 #pragma unroll 1
   for (int rt = 0; rt < 2; ++rt) {
-    // output staging: row tile 0 after the tables, row tile 1 over table 0 (read)
+    // output staging, four 16 KB boxes (head h, 64-column half j) of 128 rows x 128 B,
+    // 16-byte pieces swizzled as the output maps' 128-byte swizzle expects: row tile 0
+    // after the tables, row tile 1 over table 0 (read by then)
     uint8_t* const stg = rt == 0 ? base + 2 * kHalf * kBM * sizeof(float2) : base;
     if (ok) {
       uint32_t ya[32], yb[32];
@@ -315,35 +304,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           ob[e / 2] = tg::pack_bf16x2(__uint_as_float(yb[e]), __uint_as_float(yb[e + 1]));
         }
       }
-      // row `row` of the staging area: 512 bytes (two heads), 16-byte piece c at
-      // c ^ (row % 8)
-      uint8_t* const srow = stg + row * 512;
+      // oa: columns i0.. of half 0, ob: the same of half 1; piece i0/8 + u of the row
+      uint8_t* const ra = stg + (hh * 2) * (kBM * 128) + row * 128;
+      uint8_t* const rb = ra + kBM * 128;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int ca = hh * 16 + i0 / 8 + u, cb = ca + 8;
-        *reinterpret_cast<uint4*>(srow + ((ca ^ (row & 7)) << 4)) =
+        const int off = (((i0 >> 3) + u) ^ (row & 7)) << 4;
+        *reinterpret_cast<uint4*>(ra + off) =
             make_uint4(oa[4 * u], oa[4 * u + 1], oa[4 * u + 2], oa[4 * u + 3]);
-        *reinterpret_cast<uint4*>(srow + ((cb ^ (row & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(rb + off) =
             make_uint4(ob[4 * u], ob[4 * u + 1], ob[4 * u + 2], ob[4 * u + 3]);
       }
     }
-    __syncthreads();   // the row tile's outputs staged
-    if (ok) {
-      // 128 rows x 2 heads x 256 bytes: 16 threads per (row, head), whole rows out
+    tg::fence_proxy_async_shared();   // the staged rows, to the TMA unit
+    __syncthreads();
+    if (ok && tid == 0) {
+      // four boxes out; rows past the last are clipped by the maps' extent
+      const int z = static_cast<int>(m0 + rt * kBM);
 #pragma unroll
-      for (int pss = 0; pss < 8; ++pss) {
-        const int c = pss * kThreads + tid;
-        const int seg = c >> 4, part = c & 15;
-        const int sr = seg >> 1, h = seg & 1;
-        const int64_t r = m0 + rt * kBM + sr;
-        if (r < n_rows) {
-          const uint4 val =
-              *reinterpret_cast<const uint4*>(stg + sr * 512 + (((h * 16 + part) ^ (sr & 7)) << 4));
-          *reinterpret_cast<uint4*>((h ? hb1 : hb0) + r * (h ? hs1 : hs0) + part * 8) = val;
-        }
+      for (int h = 0; h < 2; ++h) {
+        const int gh = gh0 + h;
+        const CUtensorMap* m = gh < n_hq ? &tm_oq : gh < n_hq + n_hkv ? &tm_ok : &tm_ov;
+        const int y = gh < n_hq ? gh : gh < n_hq + n_hkv ? gh - n_hq : gh - n_hq - n_hkv;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          tg::tma_store_3d(m, stg + (h * 2 + j) * (kBM * 128), 64 * j, y, z);
       }
+      tg::bulk_commit();
     }
   }
+  if (tid == 0) tg::bulk_wait_read_all();   // the boxes stay in place until read
   tg::tc_fence_before();
   __syncthreads();
   if (warp == 2) {
@@ -391,13 +381,28 @@ tg_status launch_qkv(const void* xc, const void* x, int64_t n_src, const int32_t
                          CU_TENSOR_MAP_SWIZZLE_128B))
       return TG_ERR_CUDA;
   }
+  // the outputs, [n_rows, heads, 128] each, stored as 64-column x 128-row boxes
+  CUtensorMap toq, tok, tov;
+  const uint32_t bo[3] = {64, 1, kBM};
+  const uint64_t oq_d[3] = {kDh, static_cast<uint64_t>(n_hq), static_cast<uint64_t>(n_rows)};
+  const uint64_t oq_s[2] = {kDh * 2, static_cast<uint64_t>(n_hq) * kDh * 2};
+  const uint64_t ok_d[3] = {kDh, static_cast<uint64_t>(n_hkv), static_cast<uint64_t>(n_rows)};
+  const uint64_t ok_s[2] = {kDh * 2, static_cast<uint64_t>(n_hkv) * kDh * 2};
+  if (!tg::encode_tmap(&toq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, oq_d, oq_s, bo,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tg::encode_tmap(&tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, ok_d, ok_s, bo,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tg::encode_tmap(&tov, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, ok_d, ok_s, bo,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+    return TG_ERR_CUDA;
   const size_t smem = sizeof(QkvSmem) + 1024;
   auto kernel = gather ? qkv_rope_kernel<true> : qkv_rope_kernel<false>;
   if (!tg::ensure_smem(reinterpret_cast<const void*>(kernel), static_cast<int>(smem)))
     return TG_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>((n_rows + 2 * kBM - 1) / (2 * kBM)),
                   static_cast<unsigned>(n_out / kBN));
-  return tg::launch(kernel, grid, dim3(kThreads), smem, stream, 0, tx, tw, n_rows, d, n_hq, n_hkv,
+  return tg::launch(kernel, grid, dim3(kThreads), smem, stream, 0, tx, tw, toq, tok, tov, n_rows, d,
+                    n_hq, n_hkv,
                     log(static_cast<double>(rope_base)), pos, static_cast<__nv_bfloat16*>(q),
                     static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v),
                     static_cast<const __nv_bfloat16*>(x), n_src, kept_idx,
