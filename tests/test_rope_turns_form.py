@@ -6,11 +6,16 @@ the negated sine and cosine of the angle. This repeats that sequence on the CPU
 (Python integers for the fixed point, numpy float32 for every fp32 step) and
 checks x against the angle computed in 60-digit decimal arithmetic, for positions
 up to 2^31 - 1, so a wrong shift, a dropped rounding bit or a wrong constant
-fails here rather than only through the GPU parity tests."""
+fails here rather than only through the GPU parity tests. The kernel's own lines
+(taken from qkv.cu as it stands and compiled for the host) must match the mirror
+bit for bit, so the checks hold for the code that runs."""
 import decimal
 import math
+import os
 
 import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 D = decimal.Decimal
 decimal.getcontext().prec = 60
@@ -90,3 +95,47 @@ def test_negative_positions_wrap_like_the_kernel():
         # angle(-p) = -angle(p): x2 + pi = -(x1 + pi) mod 2 pi
         d = (x2 + math.pi + x1 + math.pi) % (2 * math.pi)
         assert min(d, 2 * math.pi - d) < 2e-6
+
+
+def test_kernel_source_matches_the_mirror(tmp_path):
+    # the projection kernel's own lines (the frequency's fixed point in the prologue,
+    # then the turn, its rounding and the angle), compiled for the host, must give
+    # the mirror's x bit for bit: the accuracy checks above then hold for the kernel
+    import re
+    import shutil
+    import subprocess
+    import ctypes
+    if shutil.which("g++") is None:
+        import pytest
+        pytest.skip("g++ not available")
+    src = open(os.path.join(ROOT, "learned_token_pruning_gemm_b200", "csrc", "qkv.cu")).read()
+    inv = re.search(r"constexpr double kInvTwoPi = ([0-9.e+-]+);", src).group(1)
+    turn = re.search(r"S\.turn\[i\] = (__double2ull_rn\(.*?\));", src).group(1)
+    lines = re.search(r"(const uint64_t fx = .*?const float x = [^;]*;)", src, re.S).group(1)
+    lines = re.sub(r"S\.turn\[[^\]]*\]", "F", lines)
+    code = f"""
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+static inline float __uint_as_float(uint32_t u) {{ float f; std::memcpy(&f, &u, 4); return f; }}
+static inline unsigned long long __double2ull_rn(double d) {{ return (unsigned long long)std::nearbyint(d); }}
+constexpr int kDh = 128;
+extern "C" float kernel_x(int p, int i, double log_base) {{
+  constexpr double kInvTwoPi = {inv};
+  const uint64_t F = {turn};
+  {lines}
+  return x;
+}}
+"""
+    (tmp_path / "angle.cpp").write_text(code)
+    lib = str(tmp_path / "libangle.so")
+    subprocess.check_call(["g++", "-O2", "-ffp-contract=off", "-shared", "-fPIC", "-o", lib,
+                           str(tmp_path / "angle.cpp")])
+    f = ctypes.CDLL(lib).kernel_x
+    f.restype, f.argtypes = ctypes.c_float, [ctypes.c_int, ctypes.c_int, ctypes.c_double]
+    rng = np.random.default_rng(9)
+    pos = [0, 1, 127, 16383, 10 ** 6, 2 ** 31 - 1] + [int(v) for v in rng.integers(0, 2 ** 31 - 1, 30)]
+    for base in (1e4, 1e6):
+        for i in (0, 1, 17, 33, 63):
+            for p in pos:
+                assert np.float32(f(p, i, math.log(base))) == _kernel_x(p, i, base), (p, i, base)
