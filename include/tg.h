@@ -226,7 +226,10 @@ tg_status tg_qkv_rope(const void* xc, int64_t n_rows, int d, const void* w_qkv, 
  * xc[r] = x[kept_idx[r]], read straight from the full residual, so the projection
  * does not wait for a separate compaction. The compacted rows themselves are also
  * written to xc when xc != NULL (the layers above the gate layer carry them on).
- * q, k, v are bit-identical to tg_compact_kv followed by tg_qkv_rope.
+ * q, k, v are bit-identical to tg_compact_kv followed by tg_qkv_rope. On a B200
+ * the two calls are the faster path at every size measured (1.9k to 22k rows): the
+ * 16-byte row gathers feed the tensor cores less steadily than TMA loads of rows
+ * already compacted. This one needs no compacted-row buffer when xc is NULL.
  *   x        [n_src, d] bf16 device: the residual rows at the gate layer
  *   kept_idx [n_rows] int32 device: row ids into x (tg_select_topk's kept_idx); an
  *            id outside [0, n_src) projects a zero row, leaves that xc row as it
